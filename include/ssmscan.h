@@ -1,0 +1,200 @@
+/*
+ * ssmscan.h -- C ABI of the B200 (sm_100a) selective-scan library
+ * (libssmscan.so).
+ *
+ * Operations (each defined by the passage cited beside it):
+ *   ssm_scan_fwd      Mamba's selective scan:
+ *                     "PyTorch新手也能懂：手把手拆解Mamba-minimal中的selective_scan实现"
+ *                     §2 (signature selective_scan(u, delta, A, B, C, D) and the
+ *                     shape table), §3 (deltaA = exp(delta A) by ZOH, deltaB_u =
+ *                     delta B u by Euler), §4 (sequential loop: update the state,
+ *                     then y = C.state), §5 (y + u D); plus the gate y * silu(z)
+ *                     and delta = softplus(dt + dt_bias) of "代码连连看——mamba"
+ *                     (Mamba.step()).
+ *   ss2d_scan_fwd     VMamba's SS2D: CrossScan into four scan orders, a
+ *                     selective scan per order, CrossMerge back ("关于代码SS2D中
+ *                     的d_state设置", VMamba issue 206: the scan orders only
+ *                     arrange the sequence; d_state = 1 for throughput).
+ *   ssm_state_update  one decode step of Mamba.step() ("代码连连看——mamba",
+ *                     the SSM step: softplus(dt + bias), dA = exp(dt A),
+ *                     dB = dt B, state = state dA + x dB (in place),
+ *                     y = state.C + D x, y * act(z)).
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked "device" point to device memory of the current CUDA
+ *     device, row-major and contiguous in the layout given.  The caller owns
+ *     every buffer; the library never allocates or frees memory.
+ *   - Every call enqueues its kernels on `stream` (NULL = the legacy default
+ *     stream) and returns without synchronising.  Argument errors are
+ *     reported synchronously, before anything is enqueued; launch errors are
+ *     reported by the call that launched.  Errors found by a kernel at run
+ *     time (a bounded wait that ran out) are reported by
+ *     ssm_check_device_errors().
+ *   - A non-OK status leaves a message in ssm_last_error() (per thread).
+ *   - Outputs must not alias inputs unless stated.
+ *   - dtype: SSM_F32 or SSM_BF16 applies to every activation-sized tensor of
+ *     the call (u, delta, z, B, C, y / x, dt); A, D, dt_bias and every
+ *     recurrent state are always fp32.  Arithmetic is fp32 throughout; the
+ *     output is rounded once to `dtype`.
+ *   - d_state (N) must be one of 1, 2, 4, 8, 16, 32, 64; other values return
+ *     SSM_ERR_UNSUPPORTED.  Any b, L, d_in >= 0 is accepted; b, L or d_in of
+ *     0 is a valid empty problem.  Sizes whose element counts overflow int64
+ *     return SSM_ERR_INVALID_ARG.
+ */
+#ifndef SSMSCAN_H
+#define SSMSCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so the header needs no CUDA header. */
+typedef struct CUstream_st *ssm_stream_t;
+
+typedef enum {
+    SSM_OK = 0,
+    SSM_ERR_INVALID_ARG = 1,    /* NULL required pointer, negative size, misaligned pointer, overflow */
+    SSM_ERR_UNSUPPORTED = 2,    /* valid but not compiled: d_state not in {1,2,4,...,64}, unknown dtype */
+    SSM_ERR_WORKSPACE = 3,      /* workspace smaller than ssm_scan_fwd_workspace_bytes() */
+    SSM_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed (message has the CUDA error) */
+    SSM_ERR_DEVICE_TIMEOUT = 5  /* a kernel's bounded wait ran out (ssm_check_device_errors) */
+} ssm_status;
+
+typedef enum {
+    SSM_F32 = 0,
+    SSM_BF16 = 1
+} ssm_dtype;
+
+/*
+ * Bytes of device workspace ssm_scan_fwd needs for this problem (0 when the
+ * launch it picks needs none).  The chunked path, which splits L across
+ * thread blocks when b * d_in is too small to fill the GPU, keeps one fp32
+ * (decay, state) pair per (batch, channel, state, chunk) there.  Returns
+ * (size_t)-1 for invalid sizes.
+ */
+size_t ssm_scan_fwd_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t d_state);
+
+/*
+ * Selective scan forward.  For every batch i, channel d and state n, with the
+ * state h starting at h0[i,d,n] (or 0) and for t = 0 .. L-1:
+ *     delta = delta_softplus ? softplus(dt + dt_bias[d]) : dt + dt_bias[d]
+ *             (dt = delta[i,t,d]; softplus(x) = x for x > 20)
+ *     h[n]  = exp(delta * A[d,n]) * h[n] + delta * B[i,t,n] * u[i,t,d]
+ *     y     = sum_n C[i,t,n] * h[n] + D[d] * u[i,t,d]
+ *     y[i,t,d] = z ? y * silu(z[i,t,d]) : y
+ * and h_last[i,d,n] = h[n] after the last step.
+ *
+ *   u, delta, z   device, (b, L, d_in), dtype; z nullable (no gate)
+ *   A             device fp32 (d_in, d_state); A = -exp(A_log) as the caller forms it
+ *   B, C          device, (b, L, d_state), dtype; shared by all channels
+ *   D, dt_bias    device fp32 (d_in), nullable (0 when NULL)
+ *   h0            device fp32 (b, d_in, d_state), nullable (zero start)
+ *   h_last        device fp32 (b, d_in, d_state), nullable; may equal h0
+ *   y             device, (b, L, d_in), dtype; must not alias an input
+ *   workspace     device, >= ssm_scan_fwd_workspace_bytes(...) bytes; may be
+ *                 NULL when that is 0.  Contents on entry are ignored.
+ */
+ssm_status ssm_scan_fwd(const void *u, const void *delta, const float *A,
+                        const void *B, const void *C, const float *D,
+                        const void *z, const float *dt_bias, int delta_softplus,
+                        const float *h0, float *h_last, void *y,
+                        int64_t b, int64_t L, int64_t d_in, int64_t d_state,
+                        ssm_dtype dtype, void *workspace, size_t workspace_bytes,
+                        ssm_stream_t stream);
+
+/*
+ * SS2D forward on an H x W grid (pixels row-major, p = h W + w, L = H W).
+ * Direction k visits pixel p_k(l) at step l: k = 0 row-major (p = l),
+ * k = 1 column-major (l = w H + h), k = 2 the reverse of k = 0, k = 3 the
+ * reverse of k = 1.  Each direction runs the selective scan above on
+ * u[i, p_k(l), :] with its own delta/B/C (given in its scan order) and the
+ * rows k*d_in .. k*d_in + d_in - 1 of A, D, dt_bias, with no gate and a zero
+ * start; the output is y[i,p,d] = sum_k y_k at pixel p (fp32 sum, one
+ * rounding).  The four orders are index arithmetic: no permuted copy of u
+ * and no per-direction output is stored.
+ *
+ *   u, y          device, (b, H W, d_in), dtype
+ *   delta         device, (b, 4, H W, d_in), dtype
+ *   A             device fp32 (4 d_in, d_state)
+ *   B, C          device, (b, 4, H W, d_state), dtype
+ *   D, dt_bias    device fp32 (4 d_in), nullable
+ *   workspace     device, >= ss2d_scan_fwd_workspace_bytes(...) bytes; may be
+ *                 NULL when that is 0.  Contents on entry are ignored.
+ * d_state must be 1 (the SS2D setting of VMamba); other values return
+ * SSM_ERR_UNSUPPORTED.
+ */
+ssm_status ss2d_scan_fwd(const void *u, const void *delta, const float *A,
+                         const void *B, const void *C, const float *D,
+                         const float *dt_bias, int delta_softplus, void *y,
+                         int64_t b, int64_t H, int64_t W, int64_t d_in,
+                         int64_t d_state, ssm_dtype dtype, void *workspace,
+                         size_t workspace_bytes, ssm_stream_t stream);
+
+/*
+ * Bytes of device workspace ss2d_scan_fwd needs (0 for d_state = 1 when
+ * the fp32 accumulator of one (batch, 8-channel) tile, 32 * H * W bytes, fits
+ * in shared memory, i.e. H * W <= 6272).  Larger images keep that
+ * accumulator in the workspace: b * H * W * d_in fp32.  Returns (size_t)-1
+ * for invalid sizes.
+ */
+size_t ss2d_scan_fwd_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_in,
+                                     int64_t d_state);
+
+/*
+ * One-token state update (decode), in place on ssm_state:
+ *     delta = dt_softplus ? softplus(dt[i,d] + dt_bias[d]) : dt[i,d] + dt_bias[d]
+ *     s[i,d,n] = s[i,d,n] * exp(delta * A[d,n]) + x[i,d] * delta * B[i,n]
+ *     y[i,d]   = (sum_n s[i,d,n] * C[i,n] + D[d] * x[i,d]) * (z ? silu(z[i,d]) : 1)
+ *
+ *   ssm_state     device fp32 (b, d_in, d_state), read and written in place
+ *   x, dt, z      device, (b, d_in), dtype; z nullable
+ *   A             device fp32 (d_in, d_state)
+ *   B, C          device, (b, d_state), dtype
+ *   D, dt_bias    device fp32 (d_in), nullable
+ *   y             device, (b, d_in), dtype; must not alias an input
+ */
+ssm_status ssm_state_update(float *ssm_state, const void *x, const void *dt,
+                            const float *A, const void *B, const void *C,
+                            const float *D, const void *z, const float *dt_bias,
+                            int dt_softplus, void *y, int64_t b, int64_t d_in,
+                            int64_t d_state, ssm_dtype dtype, ssm_stream_t stream);
+
+/*
+ * CrossScan as a stored permutation, for checking the index arithmetic of
+ * ss2d_scan_fwd bit-exactly: xs[i,k,l,d] = u[i, p_k(l), d].
+ *   u   device (b, H W, d_in), dtype;   xs  device (b, 4, H W, d_in), dtype
+ */
+ssm_status ss2d_cross_scan(const void *u, void *xs, int64_t b, int64_t H,
+                           int64_t W, int64_t d_in, ssm_dtype dtype,
+                           ssm_stream_t stream);
+
+/*
+ * CrossMerge: y[i,p,d] = sum_k ys[i, k, l_k(p), d] with l_k the inverse of
+ * p_k, summed in fp32 in the order k = 0, 1, 2, 3 and rounded once.
+ *   ys  device (b, 4, H W, d_in), dtype;  y  device (b, H W, d_in), dtype
+ */
+ssm_status ss2d_cross_merge(const void *ys, void *y, int64_t b, int64_t H,
+                            int64_t W, int64_t d_in, ssm_dtype dtype,
+                            ssm_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the library's device error
+ * word on the current device.  Returns SSM_OK, SSM_ERR_DEVICE_TIMEOUT when a
+ * kernel gave up a bounded wait since the last check, or SSM_ERR_CUDA.
+ */
+ssm_status ssm_check_device_errors(ssm_stream_t stream);
+
+/* Message of the last non-OK status returned on this thread ("" if none). */
+const char *ssm_last_error(void);
+
+/* Library version, "major.minor.patch". */
+const char *ssm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSMSCAN_H */

@@ -1,0 +1,401 @@
+// ssmscan.cu -- the C ABI of libssmscan.so (include/ssmscan.h): argument
+// validation, kernel selection and launch.  Every entry point validates all
+// arguments before it touches CUDA, never allocates, never synchronises
+// (except ssm_check_device_errors) and reports failures as ssm_status with a
+// per-thread message.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "ssmscan.h"
+#include "scan_fwd.cuh"
+#include "ss2d_fwd.cuh"
+#include "state_update.cuh"
+
+// Set by a kernel whose bounded wait ran out; read by ssm_check_device_errors.
+__device__ unsigned int g_ssm_device_error = 0;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+ssm_status fail(ssm_status s, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+ssm_status ok() { return SSM_OK; }
+
+bool mul_ok(int64_t a, int64_t b, int64_t *out) { return !__builtin_mul_overflow(a, b, out); }
+
+bool supported_state(int64_t n) {
+  return n == 1 || n == 2 || n == 4 || n == 8 || n == 16 || n == 32 || n == 64;
+}
+
+size_t esize(ssm_dtype t) { return t == SSM_BF16 ? 2 : 4; }
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+ssm_status check_launch(const char *what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(SSM_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
+  return ok();
+}
+
+// Opt a kernel into > 48 KB of dynamic shared memory once per device.
+template <auto Kernel>
+ssm_status ensure_smem(int bytes, const char *what) {
+  static bool done[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return fail(SSM_ERR_CUDA, "%s: cudaGetDevice failed", what);
+  if (!done[dev]) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess)
+      return fail(SSM_ERR_CUDA, "%s: cudaFuncSetAttribute: %s", what, cudaGetErrorString(e));
+    done[dev] = true;
+  }
+  return ok();
+}
+
+// ------------------------------------------------------------ scan launch
+template <typename T, int N>
+ssm_status launch_scan(const ssm::ScanParams &p, bool staged, cudaStream_t st) {
+  if constexpr (N >= 8) {
+    if (staged) {
+      constexpr int DT = 32, TC = 64;
+      using Cfg = ssm::StagedScan<T, N, DT, TC>;
+      const dim3 grid((unsigned)((p.d_in + DT - 1) / DT), (unsigned)p.b);
+      if (p.z) {
+        constexpr auto k = ssm::scan_staged_kernel<T, N, DT, TC, true>;
+        if (ssm_status s = ensure_smem<k>(Cfg::SMEM, "ssm_scan_fwd")) return s;
+        k<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(p);
+      } else {
+        constexpr auto k = ssm::scan_staged_kernel<T, N, DT, TC, false>;
+        if (ssm_status s = ensure_smem<k>(Cfg::SMEM, "ssm_scan_fwd")) return s;
+        k<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(p);
+      }
+      return check_launch("ssm_scan_fwd");
+    }
+  }
+  const int64_t threads = p.b * p.d_in;
+  const int block = 128;
+  ssm::scan_generic_kernel<T, N><<<(unsigned)((threads + block - 1) / block), block, 0, st>>>(p);
+  return check_launch("ssm_scan_fwd");
+}
+
+template <typename T>
+ssm_status dispatch_scan_n(const ssm::ScanParams &p, int64_t N, bool staged, cudaStream_t st) {
+  switch (N) {
+    case 1: return launch_scan<T, 1>(p, staged, st);
+    case 2: return launch_scan<T, 2>(p, staged, st);
+    case 4: return launch_scan<T, 4>(p, staged, st);
+    case 8: return launch_scan<T, 8>(p, staged, st);
+    case 16: return launch_scan<T, 16>(p, staged, st);
+    case 32: return launch_scan<T, 32>(p, staged, st);
+    case 64: return launch_scan<T, 64>(p, staged, st);
+  }
+  return fail(SSM_ERR_UNSUPPORTED, "d_state %lld not compiled", (long long)N);
+}
+
+// L == 0: the last state is the start state (or zeros).
+__global__ void copy_or_zero_kernel(const float *src, float *dst, int64_t n) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    dst[i] = src ? src[i] : 0.0f;
+}
+
+// ------------------------------------------------------------ step launch
+template <typename T, int N>
+ssm_status launch_step(const ssm::StepParams &p, cudaStream_t st) {
+  const int block = 256;
+  if constexpr (N >= 4) {
+    if (aligned(p.state, 16)) {
+      const int64_t threads = p.b * p.d_in * (N / 4);
+      ssm::state_update_kernel<T, N, 4>
+          <<<(unsigned)((threads + block - 1) / block), block, 0, st>>>(p);
+      return check_launch("ssm_state_update");
+    }
+  }
+  const int64_t threads = p.b * p.d_in;
+  ssm::state_update_kernel<T, N, N><<<(unsigned)((threads + block - 1) / block), block, 0, st>>>(p);
+  return check_launch("ssm_state_update");
+}
+
+template <typename T>
+ssm_status dispatch_step_n(const ssm::StepParams &p, int64_t N, cudaStream_t st) {
+  switch (N) {
+    case 1: return launch_step<T, 1>(p, st);
+    case 2: return launch_step<T, 2>(p, st);
+    case 4: return launch_step<T, 4>(p, st);
+    case 8: return launch_step<T, 8>(p, st);
+    case 16: return launch_step<T, 16>(p, st);
+    case 32: return launch_step<T, 32>(p, st);
+    case 64: return launch_step<T, 64>(p, st);
+  }
+  return fail(SSM_ERR_UNSUPPORTED, "d_state %lld not compiled", (long long)N);
+}
+
+// ------------------------------------------------------------ SS2D launch
+constexpr int kSs2dDT = 8, kSs2dTS = 8, kSs2dWarps = 8;
+constexpr int64_t kSs2dSmemPixels = 6272;  // L * 32 bytes of fp32 accumulator in shared memory
+
+template <typename T>
+ssm_status launch_ss2d(const ssm::Ss2dParams &p, cudaStream_t st) {
+  using Cfg = ssm::Ss2dCfg<kSs2dDT, kSs2dTS, kSs2dWarps>;
+  const int64_t L = p.H * p.W;
+  const dim3 grid((unsigned)((p.d_in + kSs2dDT - 1) / kSs2dDT), (unsigned)p.b);
+  if (L <= kSs2dSmemPixels) {
+    constexpr auto k = ssm::ss2d_n1_kernel<T, kSs2dDT, kSs2dTS, kSs2dWarps, true>;
+    const int smem = Cfg::AUX_BYTES + (int)(L * kSs2dDT * sizeof(float));
+    if (ssm_status s =
+            ensure_smem<k>(Cfg::AUX_BYTES + (int)(kSs2dSmemPixels * kSs2dDT * 4), "ss2d_scan_fwd"))
+      return s;
+    k<<<grid, Cfg::THREADS, smem, st>>>(p);
+  } else {
+    constexpr auto k = ssm::ss2d_n1_kernel<T, kSs2dDT, kSs2dTS, kSs2dWarps, false>;
+    k<<<grid, Cfg::THREADS, Cfg::AUX_BYTES, st>>>(p);
+  }
+  return check_launch("ss2d_scan_fwd");
+}
+
+unsigned grid_for(int64_t n) {
+  const int64_t blocks = (n + 255) / 256;
+  return (unsigned)(blocks < 148 * 32 ? (blocks > 0 ? blocks : 1) : 148 * 32);
+}
+
+}  // namespace
+
+// ============================================================== C ABI
+extern "C" {
+
+const char *ssm_last_error(void) { return g_last_error.c_str(); }
+
+const char *ssm_version(void) { return "0.1.0"; }
+
+size_t ssm_scan_fwd_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t d_state) {
+  int64_t t;
+  if (b < 0 || L < 0 || d_in < 0 || d_state < 1 || !mul_ok(b, L, &t) || !mul_ok(t, d_in, &t) ||
+      !mul_ok(t, d_state, &t))
+    return (size_t)-1;
+  return 0;
+}
+
+ssm_status ssm_scan_fwd(const void *u, const void *delta, const float *A, const void *B,
+                        const void *C, const float *D, const void *z, const float *dt_bias,
+                        int delta_softplus, const float *h0, float *h_last, void *y, int64_t b,
+                        int64_t L, int64_t d_in, int64_t d_state, ssm_dtype dtype,
+                        void *workspace, size_t workspace_bytes, ssm_stream_t stream) {
+  (void)workspace;
+  g_last_error.clear();
+  if (b < 0 || L < 0 || d_in < 0)
+    return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd: negative size (b=%lld L=%lld d_in=%lld)",
+                (long long)b, (long long)L, (long long)d_in);
+  if (dtype != SSM_F32 && dtype != SSM_BF16)
+    return fail(SSM_ERR_UNSUPPORTED, "ssm_scan_fwd: unknown dtype %d", (int)dtype);
+  if (!supported_state(d_state))
+    return fail(SSM_ERR_UNSUPPORTED, "ssm_scan_fwd: d_state %lld not in {1,2,4,8,16,32,64}",
+                (long long)d_state);
+  int64_t n_act, n_bc, n_state;
+  if (!mul_ok(b, L, &n_act) || !mul_ok(n_act, d_in, &n_act) || !mul_ok(b, L, &n_bc) ||
+      !mul_ok(n_bc, d_state, &n_bc) || !mul_ok(b, d_in, &n_state) ||
+      !mul_ok(n_state, d_state, &n_state) || n_act > INT64_MAX / 4)
+    return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd: sizes overflow int64");
+  const size_t need = ssm_scan_fwd_workspace_bytes(b, L, d_in, d_state);
+  if (workspace_bytes < need)
+    return fail(SSM_ERR_WORKSPACE, "ssm_scan_fwd: workspace %zu bytes < %zu needed",
+                workspace_bytes, need);
+  if (b == 0 || d_in == 0) return ok();
+  if (!A) return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd: A is NULL");
+  if (L > 0 && (!u || !delta || !B || !C || !y))
+    return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd: u, delta, B, C and y are required");
+  const size_t es = esize(dtype);
+  const void *act[] = {u, delta, B, C, z, y};
+  for (const void *q : act)
+    if (q && !aligned(q, es))
+      return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd: activation pointer not %zu-byte aligned", es);
+  const void *f32[] = {A, D, dt_bias, h0, h_last};
+  for (const void *q : f32)
+    if (q && !aligned(q, 4))
+      return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd: fp32 pointer not 4-byte aligned");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (L == 0) {  // no steps: the last state is the start state (or zeros)
+    if (h_last && h_last != h0) {
+      copy_or_zero_kernel<<<grid_for(n_state), 256, 0, st>>>(h0, h_last, n_state);
+      return check_launch("ssm_scan_fwd");
+    }
+    return ok();
+  }
+  if (y == u || y == delta || y == z || y == B || y == C)
+    return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd: y must not alias an input");
+
+  ssm::ScanParams p{u, delta, A, B, C, D, z, dt_bias, h0, h_last, y, b, L, d_in, delta_softplus};
+  const bool staged = d_state >= 8 && (d_in * (int64_t)es) % 16 == 0 && aligned(u, 16) &&
+                      aligned(delta, 16) && aligned(B, 16) && aligned(C, 16) &&
+                      (!z || aligned(z, 16)) && b <= 65535;
+  if (dtype == SSM_BF16) return dispatch_scan_n<__nv_bfloat16>(p, d_state, staged, st);
+  return dispatch_scan_n<float>(p, d_state, staged, st);
+}
+
+size_t ss2d_scan_fwd_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_in,
+                                     int64_t d_state) {
+  int64_t L, t;
+  if (b < 0 || H < 0 || W < 0 || d_in < 0 || d_state < 1 || !mul_ok(H, W, &L) ||
+      !mul_ok(b, L, &t) || !mul_ok(t, d_in, &t) || !mul_ok(t, 4 * d_state, &t) ||
+      t > INT64_MAX / 8)
+    return (size_t)-1;
+  if (L <= kSs2dSmemPixels) return 0;
+  return (size_t)(b * L * d_in) * sizeof(float);
+}
+
+ssm_status ss2d_scan_fwd(const void *u, const void *delta, const float *A, const void *B,
+                         const void *C, const float *D, const float *dt_bias, int delta_softplus,
+                         void *y, int64_t b, int64_t H, int64_t W, int64_t d_in, int64_t d_state,
+                         ssm_dtype dtype, void *workspace, size_t workspace_bytes,
+                         ssm_stream_t stream) {
+  g_last_error.clear();
+  if (b < 0 || H < 0 || W < 0 || d_in < 0)
+    return fail(SSM_ERR_INVALID_ARG, "ss2d_scan_fwd: negative size");
+  if (dtype != SSM_F32 && dtype != SSM_BF16)
+    return fail(SSM_ERR_UNSUPPORTED, "ss2d_scan_fwd: unknown dtype %d", (int)dtype);
+  if (d_state != 1)
+    return fail(SSM_ERR_UNSUPPORTED, "ss2d_scan_fwd: d_state %lld (only 1 is compiled)",
+                (long long)d_state);
+  const size_t need = ss2d_scan_fwd_workspace_bytes(b, H, W, d_in, d_state);
+  if (need == (size_t)-1) return fail(SSM_ERR_INVALID_ARG, "ss2d_scan_fwd: sizes overflow int64");
+  if (workspace_bytes < need || (need > 0 && !workspace))
+    return fail(SSM_ERR_WORKSPACE, "ss2d_scan_fwd: workspace %zu bytes < %zu needed",
+                workspace_bytes, need);
+  const int64_t L = H * W;
+  if (b == 0 || d_in == 0 || L == 0) return ok();
+  if (!u || !delta || !A || !B || !C || !y)
+    return fail(SSM_ERR_INVALID_ARG, "ss2d_scan_fwd: u, delta, A, B, C and y are required");
+  if (b > 65535) return fail(SSM_ERR_UNSUPPORTED, "ss2d_scan_fwd: b > 65535");
+  const size_t es = esize(dtype);
+  const void *act[] = {u, delta, B, C, y};
+  for (const void *q : act)
+    if (!aligned(q, es))
+      return fail(SSM_ERR_INVALID_ARG, "ss2d_scan_fwd: activation pointer not %zu-byte aligned", es);
+  const void *f32[] = {A, D, dt_bias, workspace};
+  for (const void *q : f32)
+    if (q && !aligned(q, 4))
+      return fail(SSM_ERR_INVALID_ARG, "ss2d_scan_fwd: fp32 pointer not 4-byte aligned");
+  if (y == u || y == delta || y == B || y == C)
+    return fail(SSM_ERR_INVALID_ARG, "ss2d_scan_fwd: y must not alias an input");
+
+  ssm::Ss2dParams p{u, delta, A, B, C, D, dt_bias, y, static_cast<float *>(workspace),
+                    b, H, W, d_in, delta_softplus};
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == SSM_BF16) return launch_ss2d<__nv_bfloat16>(p, st);
+  return launch_ss2d<float>(p, st);
+}
+
+ssm_status ssm_state_update(float *ssm_state, const void *x, const void *dt, const float *A,
+                            const void *B, const void *C, const float *D, const void *z,
+                            const float *dt_bias, int dt_softplus, void *y, int64_t b,
+                            int64_t d_in, int64_t d_state, ssm_dtype dtype,
+                            ssm_stream_t stream) {
+  g_last_error.clear();
+  if (b < 0 || d_in < 0) return fail(SSM_ERR_INVALID_ARG, "ssm_state_update: negative size");
+  if (dtype != SSM_F32 && dtype != SSM_BF16)
+    return fail(SSM_ERR_UNSUPPORTED, "ssm_state_update: unknown dtype %d", (int)dtype);
+  if (!supported_state(d_state))
+    return fail(SSM_ERR_UNSUPPORTED, "ssm_state_update: d_state %lld not in {1,2,4,8,16,32,64}",
+                (long long)d_state);
+  int64_t t;
+  if (!mul_ok(b, d_in, &t) || !mul_ok(t, d_state, &t) || t > INT64_MAX / 8)
+    return fail(SSM_ERR_INVALID_ARG, "ssm_state_update: sizes overflow int64");
+  if (b == 0 || d_in == 0) return ok();
+  if (!ssm_state || !x || !dt || !A || !B || !C || !y)
+    return fail(SSM_ERR_INVALID_ARG,
+                "ssm_state_update: ssm_state, x, dt, A, B, C and y are required");
+  const size_t es = esize(dtype);
+  const void *act[] = {x, dt, B, C, z, y};
+  for (const void *q : act)
+    if (q && !aligned(q, es))
+      return fail(SSM_ERR_INVALID_ARG, "ssm_state_update: activation pointer not %zu-byte aligned",
+                  es);
+  const void *f32[] = {ssm_state, A, D, dt_bias};
+  for (const void *q : f32)
+    if (q && !aligned(q, 4))
+      return fail(SSM_ERR_INVALID_ARG, "ssm_state_update: fp32 pointer not 4-byte aligned");
+  if (y == x || y == dt || y == z || y == B || y == C || y == ssm_state)
+    return fail(SSM_ERR_INVALID_ARG, "ssm_state_update: y must not alias an input");
+
+  ssm::StepParams p{ssm_state, x, dt, A, B, C, D, z, dt_bias, y, b, d_in, dt_softplus};
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == SSM_BF16) return dispatch_step_n<__nv_bfloat16>(p, d_state, st);
+  return dispatch_step_n<float>(p, d_state, st);
+}
+
+ssm_status ss2d_cross_scan(const void *u, void *xs, int64_t b, int64_t H, int64_t W,
+                           int64_t d_in, ssm_dtype dtype, ssm_stream_t stream) {
+  g_last_error.clear();
+  int64_t L, n;
+  if (b < 0 || H < 0 || W < 0 || d_in < 0 || !mul_ok(H, W, &L) || !mul_ok(b, 4 * L, &n) ||
+      !mul_ok(n, d_in, &n))
+    return fail(SSM_ERR_INVALID_ARG, "ss2d_cross_scan: bad sizes");
+  if (dtype != SSM_F32 && dtype != SSM_BF16)
+    return fail(SSM_ERR_UNSUPPORTED, "ss2d_cross_scan: unknown dtype %d", (int)dtype);
+  if (n == 0) return ok();
+  if (!u || !xs) return fail(SSM_ERR_INVALID_ARG, "ss2d_cross_scan: NULL pointer");
+  if (!aligned(u, esize(dtype)) || !aligned(xs, esize(dtype)))
+    return fail(SSM_ERR_INVALID_ARG, "ss2d_cross_scan: misaligned pointer");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == SSM_BF16)
+    ssm::cross_scan_kernel<__nv_bfloat16><<<grid_for(n), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16 *>(u), static_cast<__nv_bfloat16 *>(xs), b, H, W, d_in);
+  else
+    ssm::cross_scan_kernel<float><<<grid_for(n), 256, 0, st>>>(
+        static_cast<const float *>(u), static_cast<float *>(xs), b, H, W, d_in);
+  return check_launch("ss2d_cross_scan");
+}
+
+ssm_status ss2d_cross_merge(const void *ys, void *y, int64_t b, int64_t H, int64_t W,
+                            int64_t d_in, ssm_dtype dtype, ssm_stream_t stream) {
+  g_last_error.clear();
+  int64_t L, n;
+  if (b < 0 || H < 0 || W < 0 || d_in < 0 || !mul_ok(H, W, &L) || !mul_ok(b, 4 * L, &n) ||
+      !mul_ok(n, d_in, &n))
+    return fail(SSM_ERR_INVALID_ARG, "ss2d_cross_merge: bad sizes");
+  if (dtype != SSM_F32 && dtype != SSM_BF16)
+    return fail(SSM_ERR_UNSUPPORTED, "ss2d_cross_merge: unknown dtype %d", (int)dtype);
+  if (n == 0) return ok();
+  if (!ys || !y) return fail(SSM_ERR_INVALID_ARG, "ss2d_cross_merge: NULL pointer");
+  if (!aligned(ys, esize(dtype)) || !aligned(y, esize(dtype)))
+    return fail(SSM_ERR_INVALID_ARG, "ss2d_cross_merge: misaligned pointer");
+  const int64_t m = b * L * d_in;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == SSM_BF16)
+    ssm::cross_merge_kernel<__nv_bfloat16><<<grid_for(m), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16 *>(ys), static_cast<__nv_bfloat16 *>(y), b, H, W, d_in);
+  else
+    ssm::cross_merge_kernel<float><<<grid_for(m), 256, 0, st>>>(
+        static_cast<const float *>(ys), static_cast<float *>(y), b, H, W, d_in);
+  return check_launch("ss2d_cross_merge");
+}
+
+ssm_status ssm_check_device_errors(ssm_stream_t stream) {
+  g_last_error.clear();
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess)
+    return fail(SSM_ERR_CUDA, "ssm_check_device_errors: %s", cudaGetErrorString(e));
+  unsigned int v = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&v, g_ssm_device_error, sizeof v);
+  if (e != cudaSuccess)
+    return fail(SSM_ERR_CUDA, "ssm_check_device_errors: %s", cudaGetErrorString(e));
+  if (v) {
+    cudaMemcpyToSymbol(g_ssm_device_error, &zero, sizeof zero);
+    return fail(SSM_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait ran out (code %u)", v);
+  }
+  return ok();
+}
+
+}  // extern "C"

@@ -20,7 +20,7 @@ def _oracle_built():
 
 
 @pytest.fixture(scope="session")
-def cuda():
+def ssm():
     """The CUDA binding, failing loudly when no GPU or no library is present."""
     import torch
     if not torch.cuda.is_available():

@@ -1,0 +1,133 @@
+"""Host-side tests of the C ABI (no GPU needed): the library loads, exports
+every function include/ssmscan.h declares, and rejects bad arguments with the
+documented status before anything touches CUDA.  Pointers passed here are
+fake (never dereferenced): every call below fails validation first, or is an
+empty problem that returns before any CUDA call."""
+import ctypes
+
+import pytest
+
+from selective_state_space_25_b200 import ssmscan as S
+
+L = S.lib()
+FAKE = 0x100000          # 16-byte aligned, never dereferenced
+ODD = 0x100001           # misaligned for every element type
+
+
+def test_exports_every_declared_function():
+    names = S.header_functions()
+    assert {"ssm_scan_fwd", "ss2d_scan_fwd", "ssm_state_update", "ss2d_cross_scan",
+            "ss2d_cross_merge", "ssm_last_error", "ssm_check_device_errors",
+            "ssm_scan_fwd_workspace_bytes", "ss2d_scan_fwd_workspace_bytes",
+            "ssm_version"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), f"libssmscan.so does not export {n}"
+
+
+def test_version_and_empty_error():
+    assert S.version().count(".") == 2
+    assert isinstance(S.last_error(), str)
+
+
+def scan(**kw):
+    a = dict(u=FAKE, delta=FAKE, A=FAKE, B=FAKE, C=FAKE, D=None, z=None, dt_bias=None, sp=1,
+             h0=None, h_last=None, y=FAKE + 4096, b=2, L=8, d_in=16, N=16, dtype=S.SSM_BF16,
+             ws=None, ws_bytes=0, stream=None)
+    a.update(kw)
+    return L.ssm_scan_fwd(a["u"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"], a["dt_bias"],
+                          a["sp"], a["h0"], a["h_last"], a["y"], a["b"], a["L"], a["d_in"], a["N"],
+                          a["dtype"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(b=-1), S.SSM_ERR_INVALID_ARG),
+    (dict(L=-3), S.SSM_ERR_INVALID_ARG),
+    (dict(d_in=-1), S.SSM_ERR_INVALID_ARG),
+    (dict(N=3), S.SSM_ERR_UNSUPPORTED),
+    (dict(N=128), S.SSM_ERR_UNSUPPORTED),
+    (dict(N=0), S.SSM_ERR_UNSUPPORTED),
+    (dict(dtype=7), S.SSM_ERR_UNSUPPORTED),
+    (dict(b=2 ** 40, L=2 ** 40), S.SSM_ERR_INVALID_ARG),
+    (dict(u=None), S.SSM_ERR_INVALID_ARG),
+    (dict(A=None), S.SSM_ERR_INVALID_ARG),
+    (dict(y=None), S.SSM_ERR_INVALID_ARG),
+    (dict(C=None), S.SSM_ERR_INVALID_ARG),
+    (dict(u=ODD), S.SSM_ERR_INVALID_ARG),
+    (dict(A=FAKE + 2), S.SSM_ERR_INVALID_ARG),
+    (dict(h0=FAKE + 1), S.SSM_ERR_INVALID_ARG),
+    (dict(y=FAKE), S.SSM_ERR_INVALID_ARG),            # y aliases u
+    (dict(b=0), S.SSM_OK),                            # empty problem, no CUDA call
+    (dict(d_in=0), S.SSM_OK),
+])
+def test_scan_validation(kw, status):
+    assert scan(**kw) == status
+    if status != S.SSM_OK:
+        assert S.last_error() != ""
+
+
+def test_workspace_query():
+    assert S.ssm_scan_fwd_workspace_bytes(8, 2048, 1536, 16) >= 0
+    assert L.ssm_scan_fwd_workspace_bytes(-1, 1, 1, 16) == ctypes.c_size_t(-1).value
+    assert S.ss2d_scan_fwd_workspace_bytes(32, 56, 56, 192, 1) == 0
+    big = S.ss2d_scan_fwd_workspace_bytes(2, 100, 100, 16, 1)
+    assert big == 2 * 100 * 100 * 16 * 4
+
+
+def ss2d(**kw):
+    a = dict(u=FAKE, delta=FAKE, A=FAKE, B=FAKE, C=FAKE, D=None, dt_bias=None, sp=1,
+             y=FAKE + 8192, b=2, H=4, W=5, d_in=8, N=1, dtype=S.SSM_BF16, ws=None, ws_bytes=0,
+             stream=None)
+    a.update(kw)
+    return L.ss2d_scan_fwd(a["u"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["dt_bias"],
+                           a["sp"], a["y"], a["b"], a["H"], a["W"], a["d_in"], a["N"], a["dtype"],
+                           a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(H=-1), S.SSM_ERR_INVALID_ARG),
+    (dict(N=16), S.SSM_ERR_UNSUPPORTED),
+    (dict(dtype=5), S.SSM_ERR_UNSUPPORTED),
+    (dict(delta=None), S.SSM_ERR_INVALID_ARG),
+    (dict(y=FAKE), S.SSM_ERR_INVALID_ARG),
+    (dict(B=ODD), S.SSM_ERR_INVALID_ARG),
+    (dict(H=100, W=100), S.SSM_ERR_WORKSPACE),        # accumulator needs the workspace
+    (dict(b=0), S.SSM_OK),
+    (dict(W=0), S.SSM_OK),
+])
+def test_ss2d_validation(kw, status):
+    assert ss2d(**kw) == status
+
+
+def step(**kw):
+    a = dict(state=FAKE, x=FAKE, dt=FAKE, A=FAKE, B=FAKE, C=FAKE, D=None, z=None, dt_bias=None,
+             sp=1, y=FAKE + 4096, b=2, d_in=16, N=16, dtype=S.SSM_BF16, stream=None)
+    a.update(kw)
+    return L.ssm_state_update(a["state"], a["x"], a["dt"], a["A"], a["B"], a["C"], a["D"], a["z"],
+                              a["dt_bias"], a["sp"], a["y"], a["b"], a["d_in"], a["N"], a["dtype"],
+                              a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(b=-2), S.SSM_ERR_INVALID_ARG),
+    (dict(N=5), S.SSM_ERR_UNSUPPORTED),
+    (dict(state=None), S.SSM_ERR_INVALID_ARG),
+    (dict(state=FAKE + 2), S.SSM_ERR_INVALID_ARG),
+    (dict(y=FAKE), S.SSM_ERR_INVALID_ARG),            # y aliases the state
+    (dict(x=ODD), S.SSM_ERR_INVALID_ARG),
+    (dict(b=0), S.SSM_OK),
+])
+def test_step_validation(kw, status):
+    assert step(**kw) == status
+
+
+def test_cross_permutation_validation():
+    assert L.ss2d_cross_scan(None, FAKE, 1, 2, 2, 4, S.SSM_BF16, None) == S.SSM_ERR_INVALID_ARG
+    assert L.ss2d_cross_merge(FAKE, FAKE + 64, -1, 2, 2, 4, S.SSM_BF16, None) == S.SSM_ERR_INVALID_ARG
+    assert L.ss2d_cross_scan(FAKE, FAKE + 64, 0, 2, 2, 4, S.SSM_BF16, None) == S.SSM_OK
+
+
+def test_binding_rejects_wrong_tensors():
+    import torch
+    u = torch.zeros(1, 4, 8)
+    with pytest.raises((ValueError, TypeError)):
+        S.ssm_scan_fwd(u, u, torch.zeros(8, 16), torch.zeros(1, 4, 16), torch.zeros(1, 4, 15))

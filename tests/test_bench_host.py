@@ -1,0 +1,88 @@
+"""Host logic of bench.py, on the CPU: algorithmic bytes, the derived ALU
+roofline, the traffic-figure staleness rule, the reference arm's rank rule,
+and the cross-rank aggregation (world size 2 over gloo)."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from selective_state_space_25_b200.synthetic import WORKLOADS  # noqa: E402
+
+
+def test_algorithmic_bytes():
+    # Mamba-130M-shaped scan: read u, delta, z (bf16), B, C (bf16), A, D,
+    # dt_bias (fp32); write y (bf16)
+    b, L, d, N = 8, 2048, 1536, 16
+    exp = 4 * b * L * d * 2 + 2 * b * L * N * 2 + d * N * 4 + 2 * d * 4
+    assert bench.alg_bytes(WORKLOADS["mamba130m-scan"]) == exp == 202485760
+    # decode: fp32 state read + write dominates
+    assert bench.alg_bytes(WORKLOADS["mamba-decode-step"]) > 2 * 256 * 5120 * 16 * 4
+
+
+def test_alu_roofline_bounds():
+    w = WORKLOADS["mamba130m-scan"]
+    e = bench.alu_peak_elems_per_s(w)
+    sfu_only = bench.SMS * bench.SFU_PER_CLK * bench.SM_MAX_HZ / (1 + 4 / 16)
+    fma_only = bench.SMS * bench.FMA_PER_CLK * bench.SM_MAX_HZ / 4
+    assert sfu_only < e < fma_only
+
+
+def test_traffic_is_null_when_kernels_changed(tmp_path, monkeypatch):
+    f = tmp_path / "traffic.json"
+    f.write_text(json.dumps({"w": {"dram_bytes_per_launch": 123, "source_hash": "stale"}}))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
+    assert bench.traffic_for("w") is None
+    f.write_text(json.dumps({"w": {"dram_bytes_per_launch": 123,
+                                   "source_hash": bench.source_hash()}}))
+    assert bench.traffic_for("w") == 123
+
+
+def test_reference_arm_non_zero_rank_exits_without_work():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--steps", "1", "--warmup", "0"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    sys.path.insert(0, ROOT)
+    import bench as b
+    # rank r processed (r + 1) million elements in (10 + 5 r) ms
+    q.put((rank, b.aggregate(1e6 * (rank + 1), 10.0 + 5.0 * rank, world)))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_aggregate_sums_elements_and_takes_max_time_gloo():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for r in range(world):
+        assert res[r] == (3e6, 15.0)

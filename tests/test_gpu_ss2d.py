@@ -1,0 +1,117 @@
+"""GPU parity of ss2d_scan_fwd and the CrossScan / CrossMerge permutations
+against the fp64 oracle (through the C ABI).  The permutations are checked
+bit-exactly; the fused four-direction scan within the bf16 / fp32
+tolerances."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from _helpers import TOL, rel_err, to_cuda, to64
+from selective_state_space_25_b200.synthetic import WORKLOADS, ss2d_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_ss2d(S, inp, H, W, softplus=True):
+    g = to_cuda(inp)
+    return S.ss2d_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], H, W, D=g["D"],
+                           dt_bias=g["dt_bias"], delta_softplus=softplus)
+
+
+def oracle_ss2d(inp, H, W, softplus=True):
+    return oracle.ss2d_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], H, W,
+                            D=inp["D"], dt_bias=inp["dt_bias"], delta_softplus=softplus)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("H,W", [(5, 7), (1, 9), (8, 1), (16, 16), (1, 1), (33, 17)])
+def test_cross_scan_bit_exact(ssm, dtype, H, W):
+    u = torch.randn(2, H * W, 12).to(dtype)
+    xs = ssm.ss2d_cross_scan(u.cuda(), H, W)
+    np.testing.assert_array_equal(to64(xs), oracle.cross_scan(u, H, W))
+
+
+@pytest.mark.parametrize("H,W", [(5, 7), (9, 4), (1, 6)])
+def test_cross_merge_of_cross_scan_is_4u(ssm, H, W):
+    u = torch.randn(3, H * W, 16).to(torch.bfloat16).cuda()
+    y = ssm.ss2d_cross_merge(ssm.ss2d_cross_scan(u, H, W), H, W)
+    assert torch.equal(y, 4 * u)
+
+
+@pytest.mark.parametrize("k", [0, 1, 2, 3])
+def test_cross_merge_inverse_permutation_one_hot(ssm, k):
+    """With only direction k non-zero, the merge is the exact inverse gather."""
+    H, W = 6, 11
+    ys = torch.zeros(2, 4, H * W, 8)
+    ys[:, k] = torch.randn(2, H * W, 8)
+    y = ssm.ss2d_cross_merge(ys.cuda(), H, W)
+    np.testing.assert_array_equal(to64(y), oracle.cross_merge(ys, H, W))
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("b,H,W,d_in", [
+    (2, 5, 7, 8), (2, 1, 1, 8), (1, 1, 40, 16), (1, 37, 1, 8), (2, 16, 16, 12),
+    (2, 23, 29, 24), (1, 56, 56, 16), (1, 3, 300, 8),
+])
+def test_ss2d_shapes(ssm, dtype, b, H, W, d_in):
+    dt = "bf16" if dtype == torch.bfloat16 else "fp32"
+    inp = ss2d_inputs(b, H, W, d_in, 1, dt, seed=H * 100 + W, with_dt_bias=True)
+    y = gpu_ss2d(ssm, inp, H, W)
+    assert rel_err(y, oracle_ss2d(inp, H, W)) <= TOL[dtype]
+
+
+def test_ss2d_no_softplus_no_D(ssm):
+    inp = ss2d_inputs(2, 9, 13, 16, 1, "fp32", seed=4, with_D=False)
+    inp["delta"] = inp["delta"].abs() * 0.2
+    y = gpu_ss2d(ssm, inp, 9, 13, softplus=False)
+    assert rel_err(y, oracle_ss2d(inp, 9, 13, softplus=False)) <= 1e-4
+
+
+def test_ss2d_large_image_uses_workspace(ssm):
+    """H W above the shared-memory accumulator limit: the fp32 accumulator lives
+    in the caller's workspace."""
+    H, W = 80, 81
+    assert ssm.ss2d_scan_fwd_workspace_bytes(1, H, W, 16, 1) > 0
+    inp = ss2d_inputs(1, H, W, 16, 1, "bf16", seed=8)
+    y = gpu_ss2d(ssm, inp, H, W)
+    assert rel_err(y, oracle_ss2d(inp, H, W)) <= 2e-2
+
+
+def test_ss2d_equals_composition_of_gpu_scans(ssm):
+    """Fused SS2D == CrossScan, four 1-D scans, CrossMerge, all on the GPU."""
+    b, H, W, d_in = 2, 12, 10, 16
+    L = H * W
+    inp = to_cuda(ss2d_inputs(b, H, W, d_in, 1, "fp32", seed=12, with_dt_bias=True))
+    y = ssm.ss2d_scan_fwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], H, W, D=inp["D"],
+                          dt_bias=inp["dt_bias"])
+    xs = ssm.ss2d_cross_scan(inp["u"], H, W)
+    ys = torch.empty(b, 4, L, d_in, device="cuda")
+    for i in range(b):
+        for k in range(4):
+            sl = slice(k * d_in, (k + 1) * d_in)
+            ys[i, k] = ssm.ssm_scan_fwd(xs[i, k][None].contiguous(), inp["delta"][i, k][None].contiguous(),
+                                        inp["A"][sl].contiguous(), inp["B"][i, k][None].contiguous(),
+                                        inp["C"][i, k][None].contiguous(), D=inp["D"][sl].contiguous(),
+                                        dt_bias=inp["dt_bias"][sl].contiguous())[0]
+    ref = ssm.ss2d_cross_merge(ys, H, W)
+    assert rel_err(y, ref) <= 1e-5
+
+
+def test_vmamba_ss2d_workload_sampled(ssm):
+    w = WORKLOADS["vmamba-ss2d"]
+    d = w.dims
+    H, W, d_in = d["H"], d["W"], d["d_in"]
+    inp = ss2d_inputs(d["b"], H, W, d_in, d["N"], w.dtype, w.seed)
+    y = gpu_ss2d(ssm, inp, H, W)
+    torch.cuda.synchronize()
+    bsel = [0, d["b"] - 1]
+    chans = [0, 7, 8, 95, 96, 183, 184, 191]
+    rows = [k * d_in + c for k in range(4) for c in chans]
+    ref_in = dict(u=inp["u"][bsel][:, :, chans].contiguous(),
+                  delta=inp["delta"][bsel][:, :, :, chans].contiguous(),
+                  A=inp["A"][rows], B=inp["B"][bsel], C=inp["C"][bsel], D=inp["D"][rows],
+                  dt_bias=None)
+    ref = oracle_ss2d(ref_in, H, W)
+    got = y[bsel][:, :, chans]
+    assert rel_err(got, ref) <= 2e-2
