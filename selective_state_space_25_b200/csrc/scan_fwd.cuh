@@ -78,54 +78,137 @@ __global__ void __launch_bounds__(128) scan_generic_kernel(ScanParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// Staged kernel.  A CTA owns (batch i, a tile of DT channels) for the whole
+// Fast kernel.  A CTA owns (batch i, a tile of DT channels) for the whole
 // sequence and walks it in chunks of TC steps:
 //   1. the chunk's u / delta / z tile [TC x DT] and B / C rows [TC x N] are
-//      copied global -> shared with 16-byte cp.async (issued one chunk ahead,
-//      overlapping the previous chunk's scan);
-//   2. pre-pass, one thread per (t, d): delta' = softplus(dt + bias),
-//      delta' u, u and silu(z) go to shared memory as fp32; B, C rows are
-//      widened to fp32 once for all channels;
-//   3. scan: G = N / 4 threads share a channel, each owning 4 states in
-//      registers; per step 4 x (exp2, FMUL, 2 FFMA) and a G-lane shuffle sum
-//      of the partial C.h;
-//   4. post-pass, one thread per (t, d): y = (C.h + D u) * silu(z), rounded
-//      once and stored coalesced.
-// Requires: N in {8, 16, 32, 64}; d_in * sizeof(T) a multiple of 16; u,
-// delta, z, B, C 16-byte aligned.
+//      copied global -> shared with 16-byte cp.async, issued as soon as the
+//      previous chunk's u / delta / z tile has been consumed (B / C rows,
+//      which the scan reads, are double-buffered), so the copy overlaps that
+//      chunk's scan;
+//   2. pre-pass, one thread per (channel, 4 steps): delta = softplus(dt +
+//      bias), delta u, u and silu(z) are formed once per (t, d) (not once per
+//      state) and stored channel-major ([d][t], rows padded against bank
+//      conflicts) so the scan reads 4 steps of a channel in one 16-byte
+//      load; B, C rows are widened to fp32 once for all channels, laid out
+//      so each thread's states are one contiguous run.  Steps past the end
+//      of the sequence get delta = 0, which makes them identity steps;
+//   3. scan: G = N / NPT threads share a channel, each owning NPT states in
+//      registers, and take U = G steps per pass (4 when G = 1).  Per step and
+//      state pair: a packed multiply for delta A log2 e, two SFU exp2 (the
+//      last NPOLY pairs use the FMA-pipe polynomial instead), packed
+//      delta u * B, the packed recurrence FMA and the packed C.h FMA.  The U
+//      partial C.h sums of a pass meet in a reduce-scatter over the G lanes
+//      (log2 G shuffle rounds), leaving lane g with step g's sum;
+//   4. post-pass, one thread per (channel, 4 steps): y = (C.h + D u) silu(z),
+//      rounded once and stored (a warp writes whole channel rows).
+// Requires N % NPT == 0, TC % 4 == 0, d_in * sizeof(T) a multiple of 16 and
+// u, delta, z, B, C, y 16-byte aligned (checked by the launcher).
 // ---------------------------------------------------------------------------
-template <typename T, int N, int DT, int TC>
-struct StagedScan {
-  static constexpr int NPT = 4;                 // states per thread
+// ---------------------------------------------------------------------------
+// Fast kernel.  A CTA owns (batch i, a tile of DT channels) for the whole
+// sequence and walks it in chunks of TC steps:
+//   1. the chunk's u / delta / z tile [TC x DT] and B / C rows [TC x N] are
+//      copied global -> shared with 16-byte cp.async, issued as soon as the
+//      previous chunk's u / delta / z tile has been consumed (B / C rows,
+//      which the scan reads, are double-buffered), so the copy overlaps that
+//      chunk's scan;
+//   2. pre-pass, one thread per (channel, 4 steps): delta = softplus(dt +
+//      bias), delta u, u and silu(z) are formed once per (t, d) (not once per
+//      state) and stored channel-major ([d][t], rows padded against bank
+//      conflicts) so the scan reads 4 steps of a channel in one 16-byte
+//      load.  Steps past the end of the sequence get delta = 0, which makes
+//      them identity steps;
+//   3. scan: the G = N / NPT threads of a channel split its states, NPT each,
+//      and walk the chunk 4 steps per pass: first the pass's shared-memory
+//      loads and its exponentials (which do not depend on the state), then
+//      the recurrence h = dA h + delta u B and the C.h partial sums.  B and C
+//      rows are read straight from the copied tile (bf16 words widened in
+//      registers).  Per step and state
+//      pair: a packed delta A log2 e, two exp2 (SFU, or the FMA-pipe
+//      polynomial for the last NPOLY pairs), packed delta u * B, the packed
+//      recurrence FMA and the packed C.h FMA.  Each thread writes its 4
+//      partial C.h sums of a pass as one 16-byte store, one plane per state
+//      group, so no cross-lane traffic sits on the recurrence's path;
+//   4. post-pass, one thread per (channel, 4 steps): y = (sum of the G
+//      partials + D u) silu(z), rounded once and stored (a warp writes whole
+//      channel rows).
+// Requires N % NPT == 0, TC % 8 == 0, d_in * sizeof(T) a multiple of 16 and
+// u, delta, z, B, C, y 16-byte aligned (checked by the launcher).
+// ---------------------------------------------------------------------------
+template <typename T, int N, int NPT, int DT, int TC>
+struct FastScan {
   static constexpr int G = N / NPT;             // threads per channel
+  static constexpr int U = 4;                   // steps per scan pass
   static constexpr int THREADS = DT * G;
   static constexpr int ESZ = sizeof(T);
   static constexpr int VEC = 16 / ESZ;          // elements per 16-byte granule
   static constexpr int ROW_GRAN = DT / VEC;     // granules per tile row
-  static constexpr int TILE_BYTES = TC * DT * ESZ;
   static constexpr int BC_GRAN = N / VEC;       // granules per B / C row
-  static constexpr int BC_BYTES = TC * N * ESZ;
-  // shared-memory carve-up (bytes)
+  static constexpr int TCP = TC + 4;            // padded channel-major row (floats)
+  static constexpr int TILE = TC * DT * ESZ;
+  static constexpr int BCT = TC * N * ESZ;
   static constexpr int OFF_U = 0;
-  static constexpr int OFF_DT = OFF_U + TILE_BYTES;
-  static constexpr int OFF_Z = OFF_DT + TILE_BYTES;
-  static constexpr int OFF_B = OFF_Z + TILE_BYTES;
-  static constexpr int OFF_C = OFF_B + BC_BYTES;
-  static constexpr int OFF_DTU = OFF_C + BC_BYTES;                   // float2 [TC][DT]
-  static constexpr int OFF_UG = OFF_DTU + TC * DT * 8;                // float2 [TC][DT]
-  static constexpr int OFF_BF = OFF_UG + TC * DT * 8;                 // float [TC][N]
-  static constexpr int OFF_CF = OFF_BF + TC * N * 4;                  // float [TC][N]
-  static constexpr int OFF_YS = OFF_CF + TC * N * 4;                  // float [TC][DT]
-  static constexpr int SMEM = OFF_YS + TC * DT * 4;
-  static_assert(N % NPT == 0 && G <= 32 && (32 % G) == 0, "bad N");
+  static constexpr int OFF_DT = OFF_U + TILE;
+  static constexpr int OFF_Z = OFF_DT + TILE;
+  static constexpr int OFF_B = OFF_Z + TILE;
+  static constexpr int OFF_C = OFF_B + 2 * BCT;         // B, C: two stages each
+  static constexpr int OFF_DLT = OFF_C + 2 * BCT;        // float [DT][TCP]: delta
+  static constexpr int OFF_DU = OFF_DLT + DT * TCP * 4;  // float [DT][TCP]: delta u
+  static constexpr int OFF_UF = OFF_DU + DT * TCP * 4;   // float [DT][TCP]: u
+  static constexpr int OFF_GT = OFF_UF + DT * TCP * 4;   // float [DT][TCP]: silu(z)
+  // C.h partial sums, one plane per state group g: [g][DT][TCP].  Planes
+  // are skewed so a quarter-warp's 16-byte accesses land in 8 distinct bank
+  // groups both when the scan writes and when the post-pass reads.
+  static constexpr int PADG = G >= 8 ? 4 : 32 / G;
+  static constexpr int PLANE = DT * TCP + PADG;
+  static constexpr int OFF_YS = OFF_GT + DT * TCP * 4;
+  static constexpr int SMEM = OFF_YS + G * PLANE * 4;
+  static_assert(NPT % 2 == 0 && N % NPT == 0 && G <= 32 && (32 % G) == 0, "bad NPT");
   static_assert(DT % VEC == 0 && N % VEC == 0, "tile rows must be whole granules");
-  static_assert(THREADS % 32 == 0, "whole warps");
+  static_assert(THREADS % 32 == 0 && THREADS % DT == 0, "thread count");
+  static_assert(TC % 8 == 0, "chunk length");
+  static_assert(OFF_DLT % 16 == 0 && (PLANE * 4) % 16 == 0, "alignment");
 };
 
-template <typename T, int N, int DT, int TC, bool HAS_Z>
-__global__ void __launch_bounds__(StagedScan<T, N, DT, TC>::THREADS)
-    scan_staged_kernel(ScanParams p) {
-  using S = StagedScan<T, N, DT, TC>;
+// Raw words of NPT consecutive B / C entries (bf16 pairs, or fp32 values).
+template <typename T, int NPT> struct StateWords {
+  static constexpr int W = sizeof(T) == 2 ? NPT / 2 : NPT;
+  uint32_t w[W];
+  __device__ __forceinline__ void load(const T *row) {
+    if constexpr (W == 1) {
+      w[0] = *reinterpret_cast<const uint32_t *>(row);
+    } else if constexpr (W == 2) {
+      const uint2 q = *reinterpret_cast<const uint2 *>(row);
+      w[0] = q.x; w[1] = q.y;
+    } else {
+#pragma unroll
+      for (int i = 0; i < W; i += 4) {
+        const uint4 q = *reinterpret_cast<const uint4 *>(row + i * 4 / sizeof(T));
+        w[i] = q.x; w[i + 1] = q.y; w[i + 2] = q.z; w[i + 3] = q.w;
+      }
+    }
+  }
+  // entries 2k, 2k + 1 as a packed fp32 pair
+  __device__ __forceinline__ float2 pair(int k) const {
+    if constexpr (sizeof(T) == 2)
+      return make_float2(bf16lo(w[k]), bf16hi(w[k]));
+    else
+      return make_float2(__uint_as_float(w[2 * k]), __uint_as_float(w[2 * k + 1]));
+  }
+};
+
+// Everything stage 2 of a scan pass needs, produced by stage 1.
+template <typename T, int NPT> struct PassBuf {
+  float du[4];                      // delta u of the 4 steps
+  float2 a[4][NPT / 2];             // exp2(delta A log2 e) per step and state pair
+  StateWords<T, NPT> B[4], C[4];    // B, C entries of this thread's states
+};
+
+template <typename T, int N, int NPT, int DT, int TC, bool HAS_Z, int NPOLY>
+__global__ void __launch_bounds__(FastScan<T, N, NPT, DT, TC>::THREADS)
+    scan_fast_kernel(ScanParams p) {
+  using S = FastScan<T, N, NPT, DT, TC>;
+  constexpr int G = S::G, THREADS = S::THREADS, NP2 = NPT / 2, TCP = S::TCP;
   extern __shared__ __align__(16) unsigned char smem[];
   const int tid = threadIdx.x;
   const int64_t ib = blockIdx.y;
@@ -144,15 +227,14 @@ __global__ void __launch_bounds__(StagedScan<T, N, DT, TC>::THREADS)
   T *sz = reinterpret_cast<T *>(smem + S::OFF_Z);
   T *sB = reinterpret_cast<T *>(smem + S::OFF_B);
   T *sC = reinterpret_cast<T *>(smem + S::OFF_C);
-  float2 *sdtu = reinterpret_cast<float2 *>(smem + S::OFF_DTU);
-  float2 *sug = reinterpret_cast<float2 *>(smem + S::OFF_UG);
-  float *sBf = reinterpret_cast<float *>(smem + S::OFF_BF);
-  float *sCf = reinterpret_cast<float *>(smem + S::OFF_CF);
+  float *sdl = reinterpret_cast<float *>(smem + S::OFF_DLT);
+  float *sdu = reinterpret_cast<float *>(smem + S::OFF_DU);
+  float *suf = reinterpret_cast<float *>(smem + S::OFF_UF);
+  float *sgt = reinterpret_cast<float *>(smem + S::OFF_GT);
   float *sys = reinterpret_cast<float *>(smem + S::OFF_YS);
 
-  // ---- copy chunk [t0, t0 + TC) of this CTA's tiles into shared memory
-  auto prefetch = [&](int64_t t0) {
-    for (int q = tid; q < TC * S::ROW_GRAN; q += S::THREADS) {
+  auto prefetch = [&](int64_t t0, int stage) {
+    for (int q = tid; q < TC * S::ROW_GRAN; q += THREADS) {
       const int t = q / S::ROW_GRAN, gq = q - t * S::ROW_GRAN;
       const int64_t dd = d0 + gq * S::VEC;
       const bool ok = (t0 + t < L) && (dd < d_in);
@@ -162,93 +244,155 @@ __global__ void __launch_bounds__(StagedScan<T, N, DT, TC>::THREADS)
       cp_async16(sdt + so, gdt + off, ok ? 16 : 0);
       if (HAS_Z) cp_async16(sz + so, gz + off, ok ? 16 : 0);
     }
-    for (int q = tid; q < TC * S::BC_GRAN; q += S::THREADS) {
+    for (int q = tid; q < TC * S::BC_GRAN; q += THREADS) {
       const int t = q / S::BC_GRAN, gq = q - t * S::BC_GRAN;
       const bool ok = (t0 + t < L);
       const int64_t off = ok ? ((ib * L + t0 + t) * N + gq * S::VEC) : 0;
-      const int so = t * N + gq * S::VEC;
+      const int so = stage * TC * N + t * N + gq * S::VEC;
       cp_async16(sB + so, gB + off, ok ? 16 : 0);
       cp_async16(sC + so, gC + off, ok ? 16 : 0);
     }
     cp_async_commit();
   };
 
-  // ---- per-thread scan state: channel dl, state group g
-  const int dl = tid / S::G;
-  const int g = tid - dl * S::G;
+  // ---- pre/post-pass role: channel c (fixed per thread), 4-step groups
+  const int c = tid % DT;
+  const int sg0 = tid / DT;
+  constexpr int SG_STRIDE = THREADS / DT;
+  const int64_t dc = d0 + c;
+  const bool c_ok = dc < d_in;
+  const float bias = (c_ok && p.dt_bias) ? p.dt_bias[dc] : 0.0f;
+  const float Dc = (c_ok && p.D) ? p.D[dc] : 0.0f;
+
+  // ---- scan role: channel dl, states g*NPT .. g*NPT + NPT - 1
+  const int dl = tid / G;
+  const int g = tid - dl * G;
   const int64_t d = d0 + dl;
   const bool d_ok = d < d_in;
-  float A2[S::NPT], h[S::NPT];
+  float2 A2[NP2], h[NP2];
 #pragma unroll
-  for (int j = 0; j < S::NPT; ++j) {
-    const int n = g * S::NPT + j;
-    A2[j] = d_ok ? p.A[d * N + n] * kLog2e : 0.0f;
-    h[j] = (d_ok && p.h0) ? p.h0[(ib * d_in + d) * N + n] : 0.0f;
+  for (int k = 0; k < NP2; ++k) {
+    const int n = g * NPT + 2 * k;
+    A2[k] = d_ok ? make_float2(p.A[d * N + n] * kLog2e, p.A[d * N + n + 1] * kLog2e)
+                 : make_float2(0.0f, 0.0f);
+    const float *h0 = p.h0 + (ib * d_in + d) * N + n;
+    h[k] = (d_ok && p.h0) ? make_float2(h0[0], h0[1]) : make_float2(0.0f, 0.0f);
   }
+  const float *rdl = sdl + dl * TCP;
+  const float *rdu = sdu + dl * TCP;
+  float *ys_own = sys + g * S::PLANE + dl * TCP;
+
+  // stage 1 of a pass: loads and exponentials (independent of the state)
+  auto stage1 = [&](int t, const T *cB, const T *cC, PassBuf<T, NPT> &pb) {
+    const float4 dv = *reinterpret_cast<const float4 *>(rdl + t);
+    const float4 uv = *reinterpret_cast<const float4 *>(rdu + t);
+    const float dd[4] = {dv.x, dv.y, dv.z, dv.w};
+    pb.du[0] = uv.x; pb.du[1] = uv.y; pb.du[2] = uv.z; pb.du[3] = uv.w;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      pb.B[s].load(cB + (t + s) * N + g * NPT);
+      pb.C[s].load(cC + (t + s) * N + g * NPT);
+      const float2 d2 = make_float2(dd[s], dd[s]);
+#pragma unroll
+      for (int k = 0; k < NP2; ++k) {
+        const float2 x = __fmul2_rn(d2, A2[k]);
+        pb.a[s][k] = (k >= NP2 - NPOLY) ? exp2_poly2(x) : exp2_sfu2(x);
+      }
+    }
+  };
+  // stage 2 of a pass: the recurrence and the partial C.h sums
+  auto stage2 = [&](int t, const PassBuf<T, NPT> &pb) {
+    float ys[4];
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const float2 u2 = make_float2(pb.du[s], pb.du[s]);
+      float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int k = 0; k < NP2; ++k) {
+        h[k] = __ffma2_rn(pb.a[s][k], h[k], __fmul2_rn(u2, pb.B[s].pair(k)));
+        acc = __ffma2_rn(h[k], pb.C[s].pair(k), acc);
+      }
+      ys[s] = acc.x + acc.y;
+    }
+    *reinterpret_cast<float4 *>(ys_own + t) = make_float4(ys[0], ys[1], ys[2], ys[3]);
+  };
 
   const int64_t nchunks = (L + TC - 1) / TC;
-  prefetch(0);
-  for (int64_t c = 0; c < nchunks; ++c) {
-    const int64_t t0 = c * TC;
+  prefetch(0, 0);
+  for (int64_t ch = 0; ch < nchunks; ++ch) {
+    const int stage = (int)(ch & 1);
+    const T *cB = sB + stage * TC * N;
+    const T *cC = sC + stage * TC * N;
+    const int64_t t0 = ch * TC;
     const int tc = (int)((L - t0) < (int64_t)TC ? (L - t0) : (int64_t)TC);
     cp_async_wait<0>();
-    __syncthreads();  // tiles of chunk c visible; previous post-pass done
+    __syncthreads();  // raw tiles of this chunk visible; previous post-pass done
 
-    // ---- pre-pass: per (t, d) and per (t, n)
-    for (int q = tid; q < TC * DT; q += S::THREADS) {
-      const int t = q / DT, c_ = q - t * DT;
-      const int64_t dd = d0 + c_;
-      const float bias = (p.dt_bias && dd < d_in) ? p.dt_bias[dd] : 0.0f;
-      float delta = Elem<T>::load(sdt, q) + bias;
-      if (p.delta_softplus) delta = softplus_f32(delta);
-      const float ut = Elem<T>::load(su, q);
-      sdtu[q] = make_float2(delta, delta * ut);
-      const float gate = HAS_Z ? silu_f32(Elem<T>::load(sz, q)) : 1.0f;
-      sug[q] = make_float2(ut, gate);
-    }
-    for (int q = tid; q < TC * N; q += S::THREADS) {
-      sBf[q] = Elem<T>::load(sB, q);
-      sCf[q] = Elem<T>::load(sC, q);
-    }
-    __syncthreads();  // raw tiles consumed
-
-    if (c + 1 < nchunks) prefetch(t0 + TC);  // overlaps the scan below
-
-    // ---- scan over the chunk
-    for (int t = 0; t < tc; ++t) {
-      const float2 q = sdtu[t * DT + dl];
-      const float4 bv = *reinterpret_cast<const float4 *>(sBf + t * N + g * S::NPT);
-      const float4 cv = *reinterpret_cast<const float4 *>(sCf + t * N + g * S::NPT);
-      const float bb[4] = {bv.x, bv.y, bv.z, bv.w};
-      const float cc[4] = {cv.x, cv.y, cv.z, cv.w};
-      float acc = 0.0f;
+    // ---- pre-pass: per (channel, 4 steps)
+    for (int sg = sg0; sg < TC / 4; sg += SG_STRIDE) {
+      float dv[4], duv[4], uv[4], gv[4];
 #pragma unroll
-      for (int j = 0; j < S::NPT; ++j) {
-        const float a = ex2_approx(q.x * A2[j]);
-        h[j] = fmaf(a, h[j], q.y * bb[j]);
-        acc = fmaf(h[j], cc[j], acc);
+      for (int s = 0; s < 4; ++s) {
+        const int t = sg * 4 + s;
+        const float ut = Elem<T>::load(su, t * DT + c);
+        float e = Elem<T>::load(sdt, t * DT + c) + bias;
+        if (p.delta_softplus) e = softplus_f32(e);
+        e = t < tc ? e : 0.0f;  // identity step past the end
+        dv[s] = e;
+        duv[s] = e * ut;
+        uv[s] = ut;
+        gv[s] = HAS_Z ? silu_for<T>(Elem<T>::load(sz, t * DT + c)) : 1.0f;
       }
-#pragma unroll
-      for (int m = 1; m < S::G; m <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
-      if (g == 0) sys[t * DT + dl] = acc;
+      const int o = c * TCP + sg * 4;
+      *reinterpret_cast<float4 *>(sdl + o) = make_float4(dv[0], dv[1], dv[2], dv[3]);
+      *reinterpret_cast<float4 *>(sdu + o) = make_float4(duv[0], duv[1], duv[2], duv[3]);
+      *reinterpret_cast<float4 *>(suf + o) = make_float4(uv[0], uv[1], uv[2], uv[3]);
+      *reinterpret_cast<float4 *>(sgt + o) = make_float4(gv[0], gv[1], gv[2], gv[3]);
     }
-    __syncthreads();
+    __syncthreads();  // delta, delta u, u, gate ready; u / delta / z tile consumed
 
-    // ---- post-pass: D skip, gate, one rounding, coalesced store
-    for (int q = tid; q < tc * DT; q += S::THREADS) {
-      const int t = q / DT, c_ = q - t * DT;
-      const int64_t dd = d0 + c_;
-      if (dd >= d_in) continue;
-      const float2 ug = sug[q];
-      const float Dd = p.D ? p.D[dd] : 0.0f;
-      const float yt = fmaf(Dd, ug.x, sys[q]) * ug.y;
-      Elem<T>::store(gy, (ib * L + t0 + t) * d_in + dd, yt);
+    if (ch + 1 < nchunks) prefetch(t0 + TC, stage ^ 1);  // overlaps the scan below
+
+    // ---- scan over the chunk, 4 steps per pass
+    const int tcr = (tc + 3) / 4 * 4;
+    for (int t = 0; t < tcr; t += 4) {
+      PassBuf<T, NPT> pb;
+      stage1(t, cB, cC, pb);
+      stage2(t, pb);
+    }
+    __syncthreads();  // partial sums of the chunk complete
+
+    // ---- post-pass: sum of the partials, D skip, gate, one rounding
+    if (c_ok) {
+      for (int sg = sg0; sg * 4 < tc; sg += SG_STRIDE) {
+        const int o = c * TCP + sg * 4;
+        const float4 u4 = *reinterpret_cast<const float4 *>(suf + o);
+        const float4 g4 = *reinterpret_cast<const float4 *>(sgt + o);
+        float4 y4 = *reinterpret_cast<const float4 *>(sys + o);
+#pragma unroll
+        for (int q = 1; q < G; ++q) {
+          const float4 v = *reinterpret_cast<const float4 *>(sys + q * S::PLANE + o);
+          y4.x += v.x; y4.y += v.y; y4.z += v.z; y4.w += v.w;
+        }
+        const float uu[4] = {u4.x, u4.y, u4.z, u4.w}, gg[4] = {g4.x, g4.y, g4.z, g4.w};
+        const float yy[4] = {y4.x, y4.y, y4.z, y4.w};
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          const int t = sg * 4 + s;
+          if (t < tc)
+            Elem<T>::store(gy, (ib * L + t0 + t) * d_in + dc, fmaf(Dc, uu[s], yy[s]) * gg[s]);
+        }
+      }
     }
   }
 
   if (p.h_last && d_ok) {
+    float *hl = p.h_last + (ib * d_in + d) * N + g * NPT;
 #pragma unroll
-    for (int j = 0; j < S::NPT; ++j) p.h_last[(ib * d_in + d) * N + g * S::NPT + j] = h[j];
+    for (int k = 0; k < NP2; ++k) {
+      hl[2 * k] = h[k].x;
+      hl[2 * k + 1] = h[k].y;
+    }
   }
 }
 

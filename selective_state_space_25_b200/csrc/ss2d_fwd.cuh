@@ -11,6 +11,8 @@
 // no per-direction output exists in memory.
 #pragma once
 
+#include <type_traits>
+
 #include "ssm_common.cuh"
 
 namespace ssm {
@@ -35,55 +37,170 @@ struct Ss2dParams {
   int delta_softplus;
 };
 
-// Affine map h -> A h + B of a run of steps; compose(first, then).
-struct Aff {
-  float a, b;
+// ---------------------------------------------------------------------------
+// d_state = 1 kernel.  A CTA owns (batch i, 8 channels) and runs the four
+// directions in turn, summing their outputs per pixel in an fp32
+// accumulator of the whole image (k0 + k1 + k2 + k3, one rounding at the
+// end, deterministic).  Within a direction the sequence is walked in chunks
+// of LC = 8 WARPS TS steps:
+//   1. the chunk's delta rows and the u rows of the pixels it visits (16
+//      bytes = 8 bf16 channels each) are copied global -> shared with
+//      cp.async, one chunk ahead; B / C values likewise when they are 16-byte
+//      aligned, else read directly;
+//   2. thread (segment s, channel pair cp) takes TS consecutive steps of its
+//      two channels: delta = softplus(dt + bias), dA = exp2(delta A log2 e)
+//      (FMA-pipe polynomial or SFU), delta u B, C and D u go to registers,
+//      and the segment's composed affine map h -> P h + Q is formed;
+//   3. a shuffle scan over the warp's 8 segments and a pass over the warps'
+//      totals give each segment its incoming state, the carry of the previous
+//      chunk included (the operator is (a, b) o (a', b') = (a a', a' b + b'));
+//   4. the segment replays its steps, h = dA h + delta u B, and adds
+//      y = C h + D u into the accumulator at the pixel each step visits.
+// TS is odd so the 8 segments of a warp hit distinct bank groups in the
+// staged rows; the accumulator rows are skewed (pixel (h, w) lives in row
+// h W + (w + kappa h) mod W, W + kappa odd) so both row- and column-major
+// runs spread over the banks.
+// ---------------------------------------------------------------------------
+template <typename T, int TS, int WARPS>
+struct Ss2dCfg {
+  static constexpr int DT = 8, PAIRS = 4, SPW = 8;
+  static constexpr int THREADS = 32 * WARPS;
+  static constexpr int S = SPW * WARPS;       // segments per chunk
+  static constexpr int LC = S * TS;           // steps per chunk
+  static constexpr int ESZ = sizeof(T);
+  static constexpr int ROWB = DT * ESZ;       // bytes of one staged row (8 channels)
+  static constexpr int GRAN_PER_ROW = ROWB / 16;
+  static constexpr int BC_VEC = 16 / ESZ;
+  static constexpr int BC_PAD = BC_VEC;       // room for the unaligned B / C fallback
+  static constexpr int OFF_D = 0;
+  static constexpr int OFF_U = OFF_D + LC * ROWB;
+  static constexpr int OFF_B = OFF_U + LC * ROWB;
+  static constexpr int OFF_C = OFF_B + (LC + BC_PAD) * ESZ;
+  static constexpr int OFF_AGG = (OFF_C + (LC + BC_PAD) * ESZ + 15) / 16 * 16;  // float4 [WARPS][PAIRS]
+  static constexpr int OFF_CARRY = OFF_AGG + WARPS * PAIRS * 16;              // float [8]
+  static constexpr int OFF_ACC = OFF_CARRY + 32;                               // float [L][8]
+  static constexpr int AUX_BYTES = OFF_ACC;
+  static_assert(TS % 2 == 1, "TS odd keeps the warp's segments on distinct bank groups");
+  static_assert(ROWB % 16 == 0 && (LC * ESZ) % 16 == 0, "16-byte staging");
 };
-__device__ __forceinline__ Aff aff_then(Aff first, Aff then) {
-  return Aff{then.a * first.a, fmaf(then.a, first.b, then.b)};
+
+struct Aff2 {
+  float2 a, b;  // two channels' h -> a h + b
+};
+__device__ __forceinline__ Aff2 aff2_then(Aff2 first, Aff2 then) {
+  return Aff2{__fmul2_rn(then.a, first.a), __ffma2_rn(then.a, first.b, then.b)};
 }
 
-// ---------------------------------------------------------------------------
-// d_state = 1 kernel.  CTA = (batch, DT channels), all four directions in
-// turn.  Within a direction the sequence is walked in chunks of
-// S * TS steps: thread (segment s, channel c) takes TS consecutive steps,
-// forms dA, delta B u in registers and their composed affine map; a
-// shuffle scan over the warp's segments and a shared-memory pass over the
-// warps give each segment its incoming state (the carry of the previous
-// chunk included); the segment then replays its steps and adds y into the
-// fp32 accumulator at the pixel each step visits.  Summation order per pixel
-// is k0 + k1 + k2 + k3, deterministic, rounded once at the end.
-// ---------------------------------------------------------------------------
-template <int DT, int TS, int WARPS>
-struct Ss2dCfg {
-  static constexpr int THREADS = 32 * WARPS;
-  static constexpr int SPW = 32 / DT;       // segments per warp
-  static constexpr int S = SPW * WARPS;     // segments per chunk
-  static constexpr int LC = S * TS;         // steps per chunk
-  static_assert(32 % DT == 0, "DT divides 32");
-  // shared memory besides the accumulator
-  static constexpr int AUX_BYTES = WARPS * DT * (int)sizeof(Aff) + DT * (int)sizeof(float);
+// a / b for 0 <= a < 2^24, 0 < b, from a float reciprocal and one correction
+// (the float quotient is within one of the integer one there).
+__device__ __forceinline__ int div_small(int a, int b, float inv_b) {
+  int q = (int)((float)a * inv_b);
+  const int r = a - q * b;
+  q += (r >= b) - (r < 0);
+  return q;
+}
+
+__device__ __forceinline__ int add_mod(int x, int dx, int m) {  // |dx| <= 2, 0 <= x < m
+  x += dx;
+  while (x >= m) x -= m;
+  while (x < 0) x += m;
+  return x;
+}
+
+// Walks the pixels direction k visits at consecutive steps without
+// divisions: (h, w) and sk = (kappa h) mod W for the skewed accumulator row.
+struct PixWalk {
+  int h, w, sk;
+  int H, W, kappa, skH1;  // skH1 = (kappa (H - 1)) mod W
+  __device__ __forceinline__ void init(int k, int l, int H_, int W_, float invH, float invW) {
+    H = H_;
+    W = W_;
+    kappa = (W & 1) ? 2 : 1;
+    const int ll = k >= 2 ? H * W - 1 - l : l;
+    if ((k & 1) == 0) {
+      h = div_small(ll, W, invW);
+      w = ll - h * W;
+    } else {
+      w = div_small(ll, H, invH);
+      h = ll - w * H;
+    }
+    const int kh = kappa * h;
+    sk = kh - div_small(kh, W, invW) * W;
+    const int kh1 = kappa * (H - 1);
+    skH1 = kh1 - div_small(kh1, W, invW) * W;
+  }
+  template <int k>
+  __device__ __forceinline__ void step() {
+    if constexpr ((k & 1) == 0) {  // row-major: w moves, h on wrap
+      if constexpr (k == 0) {
+        if (++w == W) { w = 0; ++h; sk = add_mod(sk, kappa, W); }
+      } else {
+        if (--w < 0) { w = W - 1; --h; sk = add_mod(sk, -kappa, W); }
+      }
+    } else {                       // column-major: h moves, w on wrap
+      if constexpr (k == 1) {
+        if (++h == H) { h = 0; ++w; sk = 0; } else { sk = add_mod(sk, kappa, W); }
+      } else {
+        if (--h < 0) { h = H - 1; --w; sk = skH1; } else { sk = add_mod(sk, -kappa, W); }
+      }
+    }
+  }
+  __device__ __forceinline__ int pix() const { return h * W + w; }
+  __device__ __forceinline__ int acc_row() const {
+    int s = w + sk;
+    if (s >= W) s -= W;
+    return h * W + s;
+  }
 };
 
-template <typename T, int DT, int TS, int WARPS, bool ACC_SMEM>
-__global__ void __launch_bounds__(Ss2dCfg<DT, TS, WARPS>::THREADS)
+// Pixel -> accumulator row (see the skew above), for one-off lookups.
+__device__ __forceinline__ int ss2d_acc_row(int pix, int W, float invW) {
+  const int h = div_small(pix, W, invW), w = pix - h * W;
+  const int kh = ((W & 1) ? 2 : 1) * h;
+  int s = w + kh - div_small(kh, W, invW) * W;
+  if (s >= W) s -= W;
+  return h * W + s;
+}
+
+// Pixel direction k visits at step l (32-bit, for one-off lookups).
+__device__ __forceinline__ int ss2d_pixel32(int k, int l, int H, int W, float invH) {
+  const int ll = k >= 2 ? H * W - 1 - l : l;
+  if ((k & 1) == 0) return ll;
+  const int w = div_small(ll, H, invH);
+  return (ll - w * H) * W + w;
+}
+
+// ROW_ASYNC: delta / u rows staged with cp.async (needs d_in a multiple of 8
+// and 16-byte aligned u, delta); otherwise with plain bounds-checked loads.
+// BC_ASYNC: B / C staged with cp.async (needs H W a multiple of 16 / sizeof(T)
+// and 16-byte aligned B, C); otherwise read from global memory per step.
+template <typename T, int TS, int WARPS, bool ACC_SMEM, bool A_POLY, bool ROW_ASYNC,
+          bool BC_ASYNC>
+__global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     ss2d_n1_kernel(Ss2dParams p) {
-  using Cfg = Ss2dCfg<DT, TS, WARPS>;
+  using Cfg = Ss2dCfg<T, TS, WARPS>;
+  constexpr int THREADS = Cfg::THREADS, LC = Cfg::LC, DT = Cfg::DT;
   extern __shared__ __align__(16) unsigned char smem[];
-  Aff *agg = reinterpret_cast<Aff *>(smem);                        // [WARPS][DT]
-  float *carry = reinterpret_cast<float *>(smem + WARPS * DT * sizeof(Aff));  // [DT]
-  float *acc_s = reinterpret_cast<float *>(smem + Cfg::AUX_BYTES);  // [L][DT]
+  T *tD = reinterpret_cast<T *>(smem + Cfg::OFF_D);
+  T *tU = reinterpret_cast<T *>(smem + Cfg::OFF_U);
+  T *tB = reinterpret_cast<T *>(smem + Cfg::OFF_B);
+  T *tC = reinterpret_cast<T *>(smem + Cfg::OFF_C);
+  float4 *agg = reinterpret_cast<float4 *>(smem + Cfg::OFF_AGG);
+  float *carry = reinterpret_cast<float *>(smem + Cfg::OFF_CARRY);
+  float *acc_s = reinterpret_cast<float *>(smem + Cfg::OFF_ACC);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int ch = lane % DT;
-  const int sl = lane / DT;
+  const int cp = lane & 3;           // channel pair
+  const int sl = lane >> 2;          // segment within the warp
   const int seg = warp * Cfg::SPW + sl;
   const int64_t ib = blockIdx.y;
   const int64_t d0 = (int64_t)blockIdx.x * DT;
-  const int64_t d = d0 + ch;
-  const bool d_ok = d < p.d_in;
   const int64_t H = p.H, W = p.W, L = H * W, d_in = p.d_in;
+  const int Hi = (int)H, Wi = (int)W, Li = (int)L;  // H W < 2^24 (checked by the launcher)
+  const float invH = 1.0f / (float)Hi, invW = 1.0f / (float)Wi;
+  const int64_t dA = d0 + 2 * cp;    // first channel of the pair
+  const bool ok0 = dA < d_in, ok1 = dA + 1 < d_in;
 
   const T *gu = static_cast<const T *>(p.u);
   const T *gdt = static_cast<const T *>(p.delta);
@@ -91,90 +208,186 @@ __global__ void __launch_bounds__(Ss2dCfg<DT, TS, WARPS>::THREADS)
   const T *gC = static_cast<const T *>(p.C);
   T *gy = static_cast<T *>(p.y);
 
-  // accumulator addressing: shared [L][DT] or global (b, L, d_in)
-  float *acc_base = ACC_SMEM ? acc_s : p.acc_global + ib * L * d_in + d0;
-  const int64_t acc_stride = ACC_SMEM ? DT : d_in;
+  float *acc_g = p.acc_global + ib * L * d_in + d0;
 
-  const int64_t nchunks = (L + Cfg::LC - 1) / Cfg::LC;
+  const int64_t nchunks = (L + LC - 1) / LC;
+  const int64_t nsteps = 4 * nchunks;  // (direction, chunk) pairs, walked in order
+
+  // stage the delta / u rows (and B / C) of step block q = k * nchunks + c
+  auto prefetch = [&](int64_t q) {
+    const int k = (int)(q / nchunks);
+    const int64_t l0 = (q - (int64_t)k * nchunks) * LC;
+    const int64_t seq = ib * 4 + k;
+    if constexpr (ROW_ASYNC) {
+      for (int r = tid; r < LC * Cfg::GRAN_PER_ROW; r += THREADS) {
+        const int row = r / Cfg::GRAN_PER_ROW, part = r - row * Cfg::GRAN_PER_ROW;
+        const int64_t l = l0 + row;
+        const bool ok = l < L;
+        const int64_t pix = ok ? ss2d_pixel32(k, (int)l, Hi, Wi, invH) : 0;
+        const int64_t offd = ok ? (seq * L + l) * d_in + d0 : 0;
+        const int64_t offu = ok ? (ib * L + pix) * d_in + d0 : 0;
+        const int so = row * DT + part * (16 / Cfg::ESZ);
+        cp_async16(tD + so, gdt + offd + part * (16 / Cfg::ESZ), ok ? 16 : 0);
+        cp_async16(tU + so, gu + offu + part * (16 / Cfg::ESZ), ok ? 16 : 0);
+      }
+    } else {
+      for (int r = tid; r < LC * DT; r += THREADS) {
+        const int row = r / DT, ch = r - row * DT;
+        const int64_t l = l0 + row;
+        const bool ok = l < L && d0 + ch < d_in;
+        const int64_t pix = ok ? ss2d_pixel32(k, (int)l, Hi, Wi, invH) : 0;
+        tD[r] = ok ? gdt[(seq * L + l) * d_in + d0 + ch] : T(0.0f);
+        tU[r] = ok ? gu[(ib * L + pix) * d_in + d0 + ch] : T(0.0f);
+      }
+    }
+    if constexpr (BC_ASYNC) {
+      for (int r = tid; r < LC / Cfg::BC_VEC; r += THREADS) {
+        const int64_t l = l0 + r * Cfg::BC_VEC;
+        const int64_t rem = L - l;
+        const int bytes = rem <= 0 ? 0 : (rem >= Cfg::BC_VEC ? 16 : (int)rem * Cfg::ESZ);
+        const int64_t off = bytes ? seq * L + l : 0;
+        cp_async16(tB + r * Cfg::BC_VEC, gB + off, bytes);
+        cp_async16(tC + r * Cfg::BC_VEC, gC + off, bytes);
+      }
+    }
+    cp_async_commit();
+  };
+
+  if (tid < DT) carry[tid] = 0.0f;  // the first direction starts from h = 0
+  prefetch(0);
+  float2 A2 = make_float2(0.0f, 0.0f), bias = A2, Dd = A2;
+
+  // one chunk of direction K (index arithmetic specialised per direction)
+  auto chunk = [&](auto kc, int64_t q, int64_t c) {
+    constexpr int K = decltype(kc)::value;
+    const int64_t l0 = c * LC;
+    const int64_t seq = ib * 4 + K;
+    cp_async_wait<0>();
+    __syncthreads();  // staged rows of this chunk visible
+
+    // ---- 1. this segment's steps into registers
+    const int64_t lb = l0 + (int64_t)seg * TS;
+    float2 a[TS], bu[TS], du[TS];
+    float cc[TS];
+    Aff2 mine{make_float2(1.0f, 1.0f), make_float2(0.0f, 0.0f)};
+#pragma unroll
+    for (int j = 0; j < TS; ++j) {
+      const int row = seg * TS + j;
+      const bool valid = lb + j < L;
+      float2 dv, uv, bc;
+      if constexpr (sizeof(T) == 2) {
+        const uint32_t wd = *reinterpret_cast<const uint32_t *>(tD + row * DT + 2 * cp);
+        const uint32_t wu = *reinterpret_cast<const uint32_t *>(tU + row * DT + 2 * cp);
+        dv = make_float2(bf16lo(wd), bf16hi(wd));
+        uv = make_float2(bf16lo(wu), bf16hi(wu));
+      } else {
+        dv = *reinterpret_cast<const float2 *>(tD + row * DT + 2 * cp);
+        uv = *reinterpret_cast<const float2 *>(tU + row * DT + 2 * cp);
+      }
+      if constexpr (BC_ASYNC) {
+        bc = make_float2(Elem<T>::load(tB, row), Elem<T>::load(tC, row));
+      } else {
+        bc = valid ? make_float2(Elem<T>::load(gB, seq * L + lb + j), Elem<T>::load(gC, seq * L + lb + j))
+                   : make_float2(0.0f, 0.0f);
+      }
+      float2 e = __fadd2_rn(dv, bias);
+      if (p.delta_softplus) e = softplus2_f32(e);
+      if (!valid) e = make_float2(0.0f, 0.0f);  // identity step past the end
+      const float2 x = __fmul2_rn(e, A2);
+      a[j] = A_POLY ? exp2_poly2(x) : exp2_sfu2(x);
+      bu[j] = __fmul2_rn(__fmul2_rn(e, uv), make_float2(bc.x, bc.x));
+      du[j] = __fmul2_rn(Dd, uv);
+      cc[j] = bc.y;
+      mine = aff2_then(mine, Aff2{a[j], bu[j]});
+    }
+    __syncthreads();  // staged rows consumed
+    if (q + 1 < nsteps) prefetch(q + 1);
+
+    // ---- 2. inclusive scan over the warp's segments (lanes cp, cp + 4, ...)
+    Aff2 inc = mine;
+#pragma unroll
+    for (int off = 1; off < Cfg::SPW; off <<= 1) {
+      Aff2 prev;
+      prev.a.x = __shfl_up_sync(0xffffffffu, inc.a.x, off * 4);
+      prev.a.y = __shfl_up_sync(0xffffffffu, inc.a.y, off * 4);
+      prev.b.x = __shfl_up_sync(0xffffffffu, inc.b.x, off * 4);
+      prev.b.y = __shfl_up_sync(0xffffffffu, inc.b.y, off * 4);
+      if (sl >= off) inc = aff2_then(prev, inc);
+    }
+    Aff2 exc;
+    exc.a.x = __shfl_up_sync(0xffffffffu, inc.a.x, 4);
+    exc.a.y = __shfl_up_sync(0xffffffffu, inc.a.y, 4);
+    exc.b.x = __shfl_up_sync(0xffffffffu, inc.b.x, 4);
+    exc.b.y = __shfl_up_sync(0xffffffffu, inc.b.y, 4);
+    if (sl == 0) exc = Aff2{make_float2(1.0f, 1.0f), make_float2(0.0f, 0.0f)};
+    if (sl == Cfg::SPW - 1) agg[warp * Cfg::PAIRS + cp] = make_float4(inc.a.x, inc.a.y, inc.b.x, inc.b.y);
+    __syncthreads();
+
+    // ---- 3. incoming state: previous chunk's carry, earlier warps, earlier segments
+    float2 h = make_float2(carry[2 * cp], carry[2 * cp + 1]);
+    for (int w = 0; w < warp; ++w) {
+      const float4 g4 = agg[w * Cfg::PAIRS + cp];
+      h = __ffma2_rn(make_float2(g4.x, g4.y), h, make_float2(g4.z, g4.w));
+    }
+    h = __ffma2_rn(exc.a, h, exc.b);
+
+    // ---- 4. replay, accumulate y at the visited pixels
+    PixWalk pw;
+    pw.init(K, (int)(lb < L ? lb : 0), Hi, Wi, invH, invW);
+#pragma unroll
+    for (int j = 0; j < TS; ++j) {
+      h = __ffma2_rn(a[j], h, bu[j]);
+      if (lb + j < L) {
+        const float2 yv = __ffma2_rn(make_float2(cc[j], cc[j]), h, du[j]);
+        float *dst = ACC_SMEM ? acc_s + pw.acc_row() * DT + 2 * cp
+                              : acc_g + (int64_t)pw.pix() * d_in + 2 * cp;
+        if (ok1) {
+          float2 *d2 = reinterpret_cast<float2 *>(dst);
+          if constexpr (K == 0)
+            *d2 = yv;
+          else
+            *d2 = __fadd2_rn(*d2, yv);
+        } else if (ok0) {
+          dst[0] = K == 0 ? yv.x : dst[0] + yv.x;
+        }
+        if (j + 1 < TS) pw.template step<K>();
+      }
+    }
+    __syncthreads();  // chunk's accumulator updates and carry reads done
+    if (warp == WARPS - 1 && sl == Cfg::SPW - 1) {
+      const bool last = c == nchunks - 1;  // the next direction starts from h = 0
+      carry[2 * cp] = last ? 0.0f : h.x;
+      carry[2 * cp + 1] = last ? 0.0f : h.y;
+    }
+  };
 
   for (int k = 0; k < 4; ++k) {
-    const int64_t pk = k * d_in + d;  // parameter row of (direction, channel)
-    const float A2 = d_ok ? p.A[pk] * kLog2e : 0.0f;
-    const float bias = (d_ok && p.dt_bias) ? p.dt_bias[pk] : 0.0f;
-    const float Dd = (d_ok && p.D) ? p.D[pk] : 0.0f;
-    const int64_t seq = ib * 4 + k;  // row block of (batch, direction) in delta / B / C
-    if (tid < DT) carry[tid] = 0.0f;
-    __syncthreads();
-
+    const int64_t pk0 = k * d_in + dA;  // parameter rows of (direction, channel pair)
+    A2 = make_float2(ok0 ? p.A[pk0] * kLog2e : 0.0f, ok1 ? p.A[pk0 + 1] * kLog2e : 0.0f);
+    bias = make_float2((ok0 && p.dt_bias) ? p.dt_bias[pk0] : 0.0f,
+                       (ok1 && p.dt_bias) ? p.dt_bias[pk0 + 1] : 0.0f);
+    Dd = make_float2((ok0 && p.D) ? p.D[pk0] : 0.0f, (ok1 && p.D) ? p.D[pk0 + 1] : 0.0f);
     for (int64_t c = 0; c < nchunks; ++c) {
-      const int64_t l_begin = c * Cfg::LC + (int64_t)seg * TS;
-      float a[TS], bu[TS], cc[TS], du[TS];
-      Aff mine{1.0f, 0.0f};
-#pragma unroll
-      for (int j = 0; j < TS; ++j) {
-        const int64_t l = l_begin + j;
-        a[j] = 1.0f;
-        bu[j] = 0.0f;
-        cc[j] = 0.0f;
-        du[j] = 0.0f;
-        if (l < L && d_ok) {
-          float delta = Elem<T>::load(gdt, (seq * L + l) * d_in + d) + bias;
-          if (p.delta_softplus) delta = softplus_f32(delta);
-          const float ut = Elem<T>::load(gu, (ib * L + ss2d_pixel(k, l, H, W)) * d_in + d);
-          a[j] = ex2_approx(delta * A2);
-          bu[j] = delta * ut * Elem<T>::load(gB, seq * L + l);
-          cc[j] = Elem<T>::load(gC, seq * L + l);
-          du[j] = Dd * ut;
-        }
-        mine = aff_then(mine, Aff{a[j], bu[j]});
+      const int64_t q = (int64_t)k * nchunks + c;
+      switch (k) {
+        case 0: chunk(std::integral_constant<int, 0>{}, q, c); break;
+        case 1: chunk(std::integral_constant<int, 1>{}, q, c); break;
+        case 2: chunk(std::integral_constant<int, 2>{}, q, c); break;
+        default: chunk(std::integral_constant<int, 3>{}, q, c); break;
       }
-      // inclusive scan over the warp's segments of this channel (lanes ch, ch+DT, ...)
-      Aff inc = mine;
-#pragma unroll
-      for (int off = 1; off < Cfg::SPW; off <<= 1) {
-        const float pa = __shfl_up_sync(0xffffffffu, inc.a, off * DT);
-        const float pb = __shfl_up_sync(0xffffffffu, inc.b, off * DT);
-        if (sl >= off) inc = aff_then(Aff{pa, pb}, inc);
-      }
-      // exclusive prefix inside the warp
-      Aff exc{__shfl_up_sync(0xffffffffu, inc.a, DT), __shfl_up_sync(0xffffffffu, inc.b, DT)};
-      if (sl == 0) exc = Aff{1.0f, 0.0f};
-      if (sl == Cfg::SPW - 1) agg[warp * DT + ch] = inc;
-      __syncthreads();
-
-      float h = carry[ch];
-      for (int w = 0; w < warp; ++w) {
-        const Aff q = agg[w * DT + ch];
-        h = fmaf(q.a, h, q.b);
-      }
-      h = fmaf(exc.a, h, exc.b);
-
-#pragma unroll
-      for (int j = 0; j < TS; ++j) {
-        const int64_t l = l_begin + j;
-        h = fmaf(a[j], h, bu[j]);
-        if (l < L && d_ok) {
-          const float yt = fmaf(cc[j], h, du[j]);
-          float *dst = acc_base + ss2d_pixel(k, l, H, W) * acc_stride + (ACC_SMEM ? ch : ch);
-          if (k == 0)
-            *dst = yt;
-          else
-            *dst += yt;
-        }
-      }
-      __syncthreads();
-      if (warp == WARPS - 1 && sl == Cfg::SPW - 1) carry[ch] = h;
-      // the next chunk reads carry only after its first barrier
     }
-    __syncthreads();
   }
+  __syncthreads();
 
-  // round once and store, channel-fastest
-  for (int64_t q = tid; q < L * DT; q += Cfg::THREADS) {
-    const int64_t pix = q / DT;
-    const int c_ = (int)(q - pix * DT);
-    if (d0 + c_ < d_in)
-      Elem<T>::store(gy, (ib * L + pix) * d_in + d0 + c_, acc_base[pix * acc_stride + c_]);
+  // ---- round once and store (a warp writes 4 pixels x 8 channels)
+  for (int r = tid; r < Li * DT; r += THREADS) {
+    const int pix = r / DT;
+    const int ch = r - pix * DT;
+    if (d0 + ch < d_in) {
+      const float v = ACC_SMEM ? acc_s[ss2d_acc_row(pix, Wi, invW) * DT + ch]
+                               : acc_g[(int64_t)pix * d_in + ch];
+      Elem<T>::store(gy, (ib * L + pix) * d_in + d0 + ch, v);
+    }
   }
 }
 

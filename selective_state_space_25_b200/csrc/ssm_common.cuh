@@ -31,25 +31,106 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return y;
 }
 
-// -------------------------------------------------------------- softplus
-// delta = softplus(x) with torch's threshold: x for x > 20, else
-// log(1 + e^x).  With e = 2^(x log2 e):
-//   e <  1/16 : log1p(e) by its alternating series to e^5 (truncation
-//               below e^6/6, i.e. < 2e-7 of the result);
-//   e >= 1/16 : ln2 * log2(1 + e) on the SFU (1 + e is then far enough
-//               from 1 that its rounding costs < 1e-6 relative).
-__device__ __forceinline__ float softplus_f32(float x) {
-  const float e = ex2_approx(x * kLog2e);
-  const float series =
-      e * fmaf(e, fmaf(e, fmaf(e, fmaf(e, 0.2f, -0.25f), 1.0f / 3.0f), -0.5f), 1.0f);
-  const float via_log = kLn2 * lg2_approx(1.0f + e);
-  const float r = e < 0.0625f ? series : via_log;
-  return x > 20.0f ? x : r;
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
-// SiLU gate: z * sigmoid(z) = z / (1 + e^-z).
+// -------------------------------------------------------------- softplus
+// delta = softplus(x) = max(x, 0) + log1p(e) with e = exp(-|x|) in (0, 1]:
+// one SFU exp2, then log1p(e) = e s(e) with s the degree-7 minimax fit of
+// log1p(e) / e on [0, 1] made by fit_polys.py (relative error 2.2e-7), so
+// the result keeps its relative accuracy where softplus(x) ~ e^x.  For
+// x > 20 this returns x exactly (e s(e) < 2.1e-9 vanishes in the sum), which
+// is torch's thresholded softplus.
+constexpr float kLog1pS0 = 9.999998212e-01f;
+constexpr float kLog1pS1 = -4.999740422e-01f;
+constexpr float kLog1pS2 = 3.327547908e-01f;
+constexpr float kLog1pS3 = -2.449546307e-01f;
+constexpr float kLog1pS4 = 1.774524003e-01f;
+constexpr float kLog1pS5 = -1.076816991e-01f;
+constexpr float kLog1pS6 = 4.408961907e-02f;
+constexpr float kLog1pS7 = -8.539204486e-03f;
+
+__device__ __forceinline__ float softplus_f32(float x) {
+  const float e = ex2_approx(-fabsf(x) * kLog2e);
+  float s = fmaf(kLog1pS7, e, kLog1pS6);
+  s = fmaf(s, e, kLog1pS5);
+  s = fmaf(s, e, kLog1pS4);
+  s = fmaf(s, e, kLog1pS3);
+  s = fmaf(s, e, kLog1pS2);
+  s = fmaf(s, e, kLog1pS1);
+  s = fmaf(s, e, kLog1pS0);
+  return fmaf(e, s, fmaxf(x, 0.0f));
+}
+
+// softplus of two values with packed fp32 arithmetic (same formula as above).
+__device__ __forceinline__ float2 softplus2_f32(float2 x) {
+  const float2 ax = make_float2(fabsf(x.x), fabsf(x.y));
+  const float2 e2 = __fmul2_rn(ax, make_float2(-kLog2e, -kLog2e));
+  const float2 e = make_float2(ex2_approx(e2.x), ex2_approx(e2.y));
+  float2 s = __ffma2_rn(make_float2(kLog1pS7, kLog1pS7), e, make_float2(kLog1pS6, kLog1pS6));
+  s = __ffma2_rn(s, e, make_float2(kLog1pS5, kLog1pS5));
+  s = __ffma2_rn(s, e, make_float2(kLog1pS4, kLog1pS4));
+  s = __ffma2_rn(s, e, make_float2(kLog1pS3, kLog1pS3));
+  s = __ffma2_rn(s, e, make_float2(kLog1pS2, kLog1pS2));
+  s = __ffma2_rn(s, e, make_float2(kLog1pS1, kLog1pS1));
+  s = __ffma2_rn(s, e, make_float2(kLog1pS0, kLog1pS0));
+  return __ffma2_rn(e, s, make_float2(fmaxf(x.x, 0.0f), fmaxf(x.y, 0.0f)));
+}
+
+// SiLU gate: z * sigmoid(z) = z / (1 + e^-z) (SFU exp2 + reciprocal).
 __device__ __forceinline__ float silu_f32(float z) {
   return z * rcp_approx(1.0f + ex2_approx(-z * kLog2e));
+}
+
+// SiLU through sigmoid(z) = (1 + tanh(z / 2)) / 2: one SFU op.  tanh.approx
+// has a relative error near 2^-11, below the 2^-9 rounding of a bf16
+// output, so bf16 paths use this form and fp32 paths the one above.
+__device__ __forceinline__ float silu_fast(float z) {
+  return z * fmaf(0.5f, tanh_approx(0.5f * z), 0.5f);
+}
+
+template <typename T> __device__ __forceinline__ float silu_for(float z) {
+  if constexpr (sizeof(T) == 2)
+    return silu_fast(z);
+  else
+    return silu_f32(z);
+}
+
+// ------------------------------------------------- exp2 on the FMA pipe
+// 2^x for two values at once, on the FP32 pipe instead of the SFU, so a
+// kernel can split its exponentials between the two units.
+// Range reduction: j = rint(x) (adding 1.5 * 2^23 rounds to an integer),
+// r = x - j in [-1/2, 1/2]; 2^r = 1 + r q(r) with q the degree-4 minimax
+// fit of (2^r - 1) / r made by fit_polys.py (relative error of 2^r
+// below 1.7e-7 and of 2^r - 1 below 4.7e-7); 2^j is added to the exponent
+// field.  x is clamped to [-126, 126] so the exponent stays a normal number.
+constexpr float kExp2Q0 = 6.931471229e-01f;
+constexpr float kExp2Q1 = 2.402235121e-01f;
+constexpr float kExp2Q2 = 5.550500378e-02f;
+constexpr float kExp2Q3 = 9.666245431e-03f;
+constexpr float kExp2Q4 = 1.333353808e-03f;
+
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fminf(fmaxf(x.x, -126.0f), 126.0f);
+  x.y = fminf(fmaxf(x.y, -126.0f), 126.0f);
+  const float2 magic = make_float2(12582912.0f, 12582912.0f);
+  const float2 t = __fadd2_rn(x, magic);                          // low bits hold rint(x)
+  const float2 j = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 r = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);   // x - j, exact
+  float2 q = __ffma2_rn(make_float2(kExp2Q4, kExp2Q4), r, make_float2(kExp2Q3, kExp2Q3));
+  q = __ffma2_rn(q, r, make_float2(kExp2Q2, kExp2Q2));
+  q = __ffma2_rn(q, r, make_float2(kExp2Q1, kExp2Q1));
+  q = __ffma2_rn(q, r, make_float2(kExp2Q0, kExp2Q0));
+  const float2 p = __ffma2_rn(q, r, make_float2(1.0f, 1.0f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
+__device__ __forceinline__ float2 exp2_sfu2(float2 x) {
+  return make_float2(ex2_approx(x.x), ex2_approx(x.y));
 }
 
 // ------------------------------------------------------- element access

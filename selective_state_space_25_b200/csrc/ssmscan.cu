@@ -66,24 +66,61 @@ ssm_status ensure_smem(int bytes, const char *what) {
 }
 
 // ------------------------------------------------------------ scan launch
+// Tile shape of the fast scan kernel: channels per CTA, steps per chunk,
+// states per thread, and how many of a thread's state pairs take the
+// FMA-pipe exp2 instead of the SFU.
+#ifndef SSM_SCAN_DT
+#define SSM_SCAN_DT 32
+#endif
+#ifndef SSM_SCAN_TC
+#define SSM_SCAN_TC 32
+#endif
+#ifndef SSM_SCAN_NPT
+#define SSM_SCAN_NPT 4
+#endif
+#ifndef SSM_SCAN_NPOLY
+#define SSM_SCAN_NPOLY 0
+#endif
+
+// States per thread: the requested count, halved until a CTA (DT channels x
+// N / NPT threads) is whole warps, and at least 2.
+constexpr int fast_npt(int n, int want, int dt) {
+  int npt = want < n ? want : n;
+  while (npt > 2 && (dt * (n / npt)) % 32 != 0) npt /= 2;
+  while (n / npt > 32) npt *= 2;
+  return npt;
+}
+
+template <typename T, int N, bool HAS_Z, int WANT_NPT>
+ssm_status launch_scan_fast_npt(const ssm::ScanParams &p, cudaStream_t st) {
+  constexpr int NPT = fast_npt(N, WANT_NPT, SSM_SCAN_DT);
+  constexpr int DT = SSM_SCAN_DT, TC = SSM_SCAN_TC;
+  constexpr int NPOLY = SSM_SCAN_NPOLY < NPT / 2 ? SSM_SCAN_NPOLY : NPT / 2;
+  using Cfg = ssm::FastScan<T, N, NPT, DT, TC>;
+  constexpr auto k = ssm::scan_fast_kernel<T, N, NPT, DT, TC, HAS_Z, NPOLY>;
+  if (ssm_status s = ensure_smem<k>(Cfg::SMEM, "ssm_scan_fwd")) return s;
+  const dim3 grid((unsigned)((p.d_in + DT - 1) / DT), (unsigned)p.b);
+  k<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(p);
+  return check_launch("ssm_scan_fwd");
+}
+
+// Fewer channels leave fewer warps per SM: split each channel's states over
+// more threads (2 per thread instead of 4) when b * d_in is below the size
+// where the measured crossover lies.
+constexpr int64_t kScanSplitChannels = 12288;
+
+template <typename T, int N, bool HAS_Z>
+ssm_status launch_scan_fast(const ssm::ScanParams &p, cudaStream_t st) {
+  if (p.b * p.d_in < kScanSplitChannels)
+    return launch_scan_fast_npt<T, N, HAS_Z, SSM_SCAN_NPT / 2>(p, st);
+  return launch_scan_fast_npt<T, N, HAS_Z, SSM_SCAN_NPT>(p, st);
+}
+
 template <typename T, int N>
-ssm_status launch_scan(const ssm::ScanParams &p, bool staged, cudaStream_t st) {
+ssm_status launch_scan(const ssm::ScanParams &p, bool fast, cudaStream_t st) {
   if constexpr (N >= 8) {
-    if (staged) {
-      constexpr int DT = 32, TC = 64;
-      using Cfg = ssm::StagedScan<T, N, DT, TC>;
-      const dim3 grid((unsigned)((p.d_in + DT - 1) / DT), (unsigned)p.b);
-      if (p.z) {
-        constexpr auto k = ssm::scan_staged_kernel<T, N, DT, TC, true>;
-        if (ssm_status s = ensure_smem<k>(Cfg::SMEM, "ssm_scan_fwd")) return s;
-        k<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(p);
-      } else {
-        constexpr auto k = ssm::scan_staged_kernel<T, N, DT, TC, false>;
-        if (ssm_status s = ensure_smem<k>(Cfg::SMEM, "ssm_scan_fwd")) return s;
-        k<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(p);
-      }
-      return check_launch("ssm_scan_fwd");
-    }
+    if (fast)
+      return p.z ? launch_scan_fast<T, N, true>(p, st) : launch_scan_fast<T, N, false>(p, st);
   }
   const int64_t threads = p.b * p.d_in;
   const int block = 128;
@@ -92,15 +129,15 @@ ssm_status launch_scan(const ssm::ScanParams &p, bool staged, cudaStream_t st) {
 }
 
 template <typename T>
-ssm_status dispatch_scan_n(const ssm::ScanParams &p, int64_t N, bool staged, cudaStream_t st) {
+ssm_status dispatch_scan_n(const ssm::ScanParams &p, int64_t N, bool fast, cudaStream_t st) {
   switch (N) {
-    case 1: return launch_scan<T, 1>(p, staged, st);
-    case 2: return launch_scan<T, 2>(p, staged, st);
-    case 4: return launch_scan<T, 4>(p, staged, st);
-    case 8: return launch_scan<T, 8>(p, staged, st);
-    case 16: return launch_scan<T, 16>(p, staged, st);
-    case 32: return launch_scan<T, 32>(p, staged, st);
-    case 64: return launch_scan<T, 64>(p, staged, st);
+    case 1: return launch_scan<T, 1>(p, fast, st);
+    case 2: return launch_scan<T, 2>(p, fast, st);
+    case 4: return launch_scan<T, 4>(p, fast, st);
+    case 8: return launch_scan<T, 8>(p, fast, st);
+    case 16: return launch_scan<T, 16>(p, fast, st);
+    case 32: return launch_scan<T, 32>(p, fast, st);
+    case 64: return launch_scan<T, 64>(p, fast, st);
   }
   return fail(SSM_ERR_UNSUPPORTED, "d_state %lld not compiled", (long long)N);
 }
@@ -144,26 +181,52 @@ ssm_status dispatch_step_n(const ssm::StepParams &p, int64_t N, cudaStream_t st)
 }
 
 // ------------------------------------------------------------ SS2D launch
-constexpr int kSs2dDT = 8, kSs2dTS = 8, kSs2dWarps = 8;
-constexpr int64_t kSs2dSmemPixels = 6272;  // L * 32 bytes of fp32 accumulator in shared memory
+// Segment length (odd), warps per CTA, and whether dA uses the FMA-pipe exp2.
+#ifndef SSM_SS2D_TS
+#define SSM_SS2D_TS 5
+#endif
+#ifndef SSM_SS2D_WARPS
+#define SSM_SS2D_WARPS 8
+#endif
+#ifndef SSM_SS2D_APOLY
+#define SSM_SS2D_APOLY 0
+#endif
+constexpr int kSs2dDT = 8;
+constexpr int64_t kSs2dSmemPixels = 6272;  // H W of the shared-memory fp32 accumulator, 32 B each
+
+template <typename T, bool ACC_SMEM, bool ROW_ASYNC, bool BC_ASYNC>
+ssm_status launch_ss2d_cfg(const ssm::Ss2dParams &p, cudaStream_t st) {
+  using Cfg = ssm::Ss2dCfg<T, SSM_SS2D_TS, SSM_SS2D_WARPS>;
+  constexpr auto k = ssm::ss2d_n1_kernel<T, SSM_SS2D_TS, SSM_SS2D_WARPS, ACC_SMEM,
+                                         SSM_SS2D_APOLY != 0, ROW_ASYNC, BC_ASYNC>;
+  const int64_t L = p.H * p.W;
+  const int smem = Cfg::AUX_BYTES + (ACC_SMEM ? (int)(L * kSs2dDT * sizeof(float)) : 0);
+  if (ssm_status s = ensure_smem<k>(Cfg::AUX_BYTES + (int)(kSs2dSmemPixels * kSs2dDT * 4),
+                                    "ss2d_scan_fwd"))
+    return s;
+  const dim3 grid((unsigned)((p.d_in + kSs2dDT - 1) / kSs2dDT), (unsigned)p.b);
+  k<<<grid, Cfg::THREADS, smem, st>>>(p);
+  return check_launch("ss2d_scan_fwd");
+}
+
+template <typename T, bool ACC_SMEM>
+ssm_status launch_ss2d_acc(const ssm::Ss2dParams &p, bool row_async, bool bc_async,
+                           cudaStream_t st) {
+  if (row_async)
+    return bc_async ? launch_ss2d_cfg<T, ACC_SMEM, true, true>(p, st)
+                    : launch_ss2d_cfg<T, ACC_SMEM, true, false>(p, st);
+  return bc_async ? launch_ss2d_cfg<T, ACC_SMEM, false, true>(p, st)
+                  : launch_ss2d_cfg<T, ACC_SMEM, false, false>(p, st);
+}
 
 template <typename T>
 ssm_status launch_ss2d(const ssm::Ss2dParams &p, cudaStream_t st) {
-  using Cfg = ssm::Ss2dCfg<kSs2dDT, kSs2dTS, kSs2dWarps>;
   const int64_t L = p.H * p.W;
-  const dim3 grid((unsigned)((p.d_in + kSs2dDT - 1) / kSs2dDT), (unsigned)p.b);
-  if (L <= kSs2dSmemPixels) {
-    constexpr auto k = ssm::ss2d_n1_kernel<T, kSs2dDT, kSs2dTS, kSs2dWarps, true>;
-    const int smem = Cfg::AUX_BYTES + (int)(L * kSs2dDT * sizeof(float));
-    if (ssm_status s =
-            ensure_smem<k>(Cfg::AUX_BYTES + (int)(kSs2dSmemPixels * kSs2dDT * 4), "ss2d_scan_fwd"))
-      return s;
-    k<<<grid, Cfg::THREADS, smem, st>>>(p);
-  } else {
-    constexpr auto k = ssm::ss2d_n1_kernel<T, kSs2dDT, kSs2dTS, kSs2dWarps, false>;
-    k<<<grid, Cfg::THREADS, Cfg::AUX_BYTES, st>>>(p);
-  }
-  return check_launch("ss2d_scan_fwd");
+  const size_t es = sizeof(T);
+  const bool row_async = (p.d_in % kSs2dDT) == 0 && aligned(p.u, 16) && aligned(p.delta, 16);
+  const bool bc_async = (L * (int64_t)es) % 16 == 0 && aligned(p.B, 16) && aligned(p.C, 16);
+  if (L <= kSs2dSmemPixels) return launch_ss2d_acc<T, true>(p, row_async, bc_async, st);
+  return launch_ss2d_acc<T, false>(p, row_async, bc_async, st);
 }
 
 unsigned grid_for(int64_t n) {
@@ -237,11 +300,11 @@ ssm_status ssm_scan_fwd(const void *u, const void *delta, const float *A, const 
     return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd: y must not alias an input");
 
   ssm::ScanParams p{u, delta, A, B, C, D, z, dt_bias, h0, h_last, y, b, L, d_in, delta_softplus};
-  const bool staged = d_state >= 8 && (d_in * (int64_t)es) % 16 == 0 && aligned(u, 16) &&
-                      aligned(delta, 16) && aligned(B, 16) && aligned(C, 16) &&
-                      (!z || aligned(z, 16)) && b <= 65535;
-  if (dtype == SSM_BF16) return dispatch_scan_n<__nv_bfloat16>(p, d_state, staged, st);
-  return dispatch_scan_n<float>(p, d_state, staged, st);
+  const bool fast = d_state >= 8 && (d_in * (int64_t)es) % 16 == 0 && aligned(u, 16) &&
+                    aligned(delta, 16) && aligned(B, 16) && aligned(C, 16) && aligned(y, 16) &&
+                    (!z || aligned(z, 16)) && b <= 65535;
+  if (dtype == SSM_BF16) return dispatch_scan_n<__nv_bfloat16>(p, d_state, fast, st);
+  return dispatch_scan_n<float>(p, d_state, fast, st);
 }
 
 size_t ss2d_scan_fwd_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_in,
@@ -275,6 +338,8 @@ ssm_status ss2d_scan_fwd(const void *u, const void *delta, const float *A, const
                 workspace_bytes, need);
   const int64_t L = H * W;
   if (b == 0 || d_in == 0 || L == 0) return ok();
+  if (L >= (int64_t(1) << 22))
+    return fail(SSM_ERR_UNSUPPORTED, "ss2d_scan_fwd: H * W = %lld >= 2^22 pixels", (long long)L);
   if (!u || !delta || !A || !B || !C || !y)
     return fail(SSM_ERR_INVALID_ARG, "ss2d_scan_fwd: u, delta, A, B, C and y are required");
   if (b > 65535) return fail(SSM_ERR_UNSUPPORTED, "ss2d_scan_fwd: b > 65535");
