@@ -144,6 +144,32 @@ size_t ss2d_scan_fwd_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_
                                      int64_t d_state);
 
 /*
+ * ss2d_scan_fwd without a workspace, for callers that cannot allocate device
+ * memory: code running inside a host framework that owns every device buffer
+ * and hands out none for scratch, and real-time loops that must not call
+ * cudaMalloc (it can synchronise the device and can fail on a fragmented
+ * heap in the middle of a run).  The pages have no counterpart; this is a
+ * packaging variant of ss2d_scan_fwd with the same arguments, layouts and
+ * results, minus workspace / workspace_bytes.
+ *
+ * Large images keep their fp32 per-pixel accumulator in a 16 MiB array that
+ * the library reserves statically on every GPU that loads it, held until
+ * the process exits.  Limit: b * H * W * d_in * 4 bytes (the value
+ * ss2d_scan_fwd_workspace_bytes returns) must not exceed 16 MiB, else
+ * SSM_ERR_WORKSPACE; images whose accumulator fits in shared memory need
+ * none of it.  The first call on a device looks the array's device address
+ * up (cudaGetSymbolAddress) and caches it; make that first call before any
+ * stream capture.  All calls on a device share the one array, which keeps
+ * the last call's contents (nothing needs clearing: every call overwrites
+ * the part it reads); calls whose kernels overlap on the GPU race on it.
+ */
+ssm_status ss2d_scan_fwd_noalloc(const void *u, const void *delta, const float *A,
+                                 const void *B, const void *C, const float *D,
+                                 const float *dt_bias, int delta_softplus, void *y,
+                                 int64_t b, int64_t H, int64_t W, int64_t d_in,
+                                 int64_t d_state, ssm_dtype dtype, ssm_stream_t stream);
+
+/*
  * One-token state update (decode), in place on ssm_state:
  *     delta = dt_softplus ? softplus(dt[i,d] + dt_bias[d]) : dt[i,d] + dt_bias[d]
  *     s[i,d,n] = s[i,d,n] * exp(delta * A[d,n]) + x[i,d] * delta * B[i,n]

@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "ssmscan.h"
@@ -445,6 +446,68 @@ ssm_status ss2d_cross_merge(const void *ys, void *y, int64_t b, int64_t H, int64
     ssm::cross_merge_kernel<float><<<grid_for(m), 256, 0, st>>>(
         static_cast<const float *>(ys), static_cast<float *>(y), b, H, W, d_in);
   return check_launch("ss2d_cross_merge");
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- no-alloc SS2D
+// Scratch of ss2d_scan_fwd_noalloc: the fp32 per-pixel accumulator of the
+// large-image SS2D path, in a file-scope device array instead of caller
+// memory.  Every GPU that loads this library holds it (16 MiB) until exit.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) float g_ss2d_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+namespace {
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+ssm_status noalloc_scratch(float **out) {
+  static std::mutex mu;
+  static float *ptr[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 64)
+    return fail(SSM_ERR_CUDA, "ss2d_scan_fwd_noalloc: cudaGetDevice failed");
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptr[dev]) {
+    void *addr = nullptr;
+    e = cudaGetSymbolAddress(&addr, g_ss2d_noalloc_scratch);
+    if (e != cudaSuccess || !addr)
+      return fail(SSM_ERR_CUDA, "ss2d_scan_fwd_noalloc: cudaGetSymbolAddress: %s",
+                  cudaGetErrorString(e));
+    ptr[dev] = static_cast<float *>(addr);
+  }
+  *out = ptr[dev];
+  return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+ssm_status ss2d_scan_fwd_noalloc(const void *u, const void *delta, const float *A,
+                                 const void *B, const void *C, const float *D,
+                                 const float *dt_bias, int delta_softplus, void *y, int64_t b,
+                                 int64_t H, int64_t W, int64_t d_in, int64_t d_state,
+                                 ssm_dtype dtype, ssm_stream_t stream) {
+  g_last_error.clear();
+  const size_t need = ss2d_scan_fwd_workspace_bytes(b, H, W, d_in, d_state);
+  if (need == (size_t)-1)
+    return fail(SSM_ERR_INVALID_ARG, "ss2d_scan_fwd_noalloc: invalid or overflowing sizes");
+  if (need > kNoAllocScratchBytes)
+    return fail(SSM_ERR_WORKSPACE,
+                "ss2d_scan_fwd_noalloc: needs %zu bytes of scratch, the static array holds %zu "
+                "(b * H * W * d_in * 4 must not exceed it); use ss2d_scan_fwd with a workspace",
+                need, kNoAllocScratchBytes);
+  float *scratch = nullptr;
+  if (need > 0) {
+    if (ssm_status s = noalloc_scratch(&scratch)) return s;
+  }
+  // The accumulator needs no clearing: the first direction stores every
+  // pixel before the others add to it.
+  return ss2d_scan_fwd(u, delta, A, B, C, D, dt_bias, delta_softplus, y, b, H, W, d_in, d_state,
+                       dtype, scratch, need, stream);
 }
 
 ssm_status ssm_check_device_errors(ssm_stream_t stream) {
