@@ -15,7 +15,8 @@ tiny-fp32-scan) measure the companion kernels.
 Timing: W untimed warm-up steps, then exactly K timed steps bracketed by a
 barrier and torch.cuda.synchronize() on both sides; each step's kernel is
 timed with CUDA events on the stream it is launched on, and L2 is flushed
-(a 256 MB write) between steps, outside the events.  The max over ranks is
+between steps, outside the events (a 256 MB write, then a read of it, so no
+dirty lines remain for the timed kernel to write back).  The max over ranks is
 taken.  Under torchrun each rank runs its own replica of the workload
 (replicas only: the path needs no collective); value = all ranks' elements /
 the slowest rank's time.
@@ -353,11 +354,16 @@ def run_ours(args, w):
     torch.cuda.synchronize()
     with ClockSampler(dev.index) as clk:
         for i in range(K):
-            flush.zero_()                      # L2 flush, outside the timed events
+            # L2 flush outside the timed events: write 256 MB (twice the L2),
+            # then read it back so no dirty lines are left for the timed
+            # kernel to write back
+            flush.zero_()
+            flush_sum = flush.sum(dtype=torch.int64)
             starts[i].record(stream)
             step()
             ends[i].record(stream)
         torch.cuda.synchronize()
+    del flush_sum
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -408,7 +414,7 @@ def run_ours(args, w):
             "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": w.name, **w.dims, "io_dtype": w.dtype,
-                       "parallelism": f"replicas{world}", "l2": "flushed between steps (256 MB write)"},
+                       "parallelism": f"replicas{world}", "l2": "flushed between steps (256 MB write, then read, outside the timed events)"},
             "gpu_launches": K,
             "roofline": roof,
             "clocks": clk.summary(),

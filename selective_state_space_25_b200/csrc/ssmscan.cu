@@ -151,10 +151,22 @@ __global__ void copy_or_zero_kernel(const float *src, float *dst, int64_t n) {
 }
 
 // ------------------------------------------------------------ step launch
+#ifndef SSM_STEP_CPT
+#define SSM_STEP_CPT 1
+#endif
+
 template <typename T, int N>
 ssm_status launch_step(const ssm::StepParams &p, cudaStream_t st) {
   const int block = 256;
   if constexpr (N >= 4) {
+    if (aligned(p.state, 16) && aligned(p.A, 16) && aligned(p.B, 16) && aligned(p.C, 16)) {
+      constexpr int CPT = SSM_STEP_CPT;
+      const int64_t per = (p.b * p.d_in + CPT - 1) / CPT;
+      const int64_t threads = per * (N / 4);
+      ssm::state_update_vec_kernel<T, N, CPT>
+          <<<(unsigned)((threads + block - 1) / block), block, 0, st>>>(p);
+      return check_launch("ssm_state_update");
+    }
     if (aligned(p.state, 16)) {
       const int64_t threads = p.b * p.d_in * (N / 4);
       ssm::state_update_kernel<T, N, 4>
