@@ -9,6 +9,8 @@
 // they are formed in registers one step at a time.
 #pragma once
 
+#include <type_traits>
+
 #include "ssm_common.cuh"
 
 namespace ssm {
@@ -135,7 +137,9 @@ __global__ void __launch_bounds__(128) scan_generic_kernel(ScanParams p) {
 // Requires N % NPT == 0, TC % 8 == 0, d_in * sizeof(T) a multiple of 16 and
 // u, delta, z, B, C, y 16-byte aligned (checked by the launcher).
 // ---------------------------------------------------------------------------
-template <typename T, int N, int NPT, int DT, int TC>
+// BCF: B and C rows widened to fp32 once per CTA in the pre-pass (instead of
+// by every thread in the scan); the raw tile is then single-buffered.
+template <typename T, int N, int NPT, int DT, int TC, bool BCF = false>
 struct FastScan {
   static constexpr int G = N / NPT;             // threads per channel
   static constexpr int U = 4;                   // steps per scan pass
@@ -151,8 +155,11 @@ struct FastScan {
   static constexpr int OFF_DT = OFF_U + TILE;
   static constexpr int OFF_Z = OFF_DT + TILE;
   static constexpr int OFF_B = OFF_Z + TILE;
-  static constexpr int OFF_C = OFF_B + 2 * BCT;         // B, C: two stages each
-  static constexpr int OFF_DLT = OFF_C + 2 * BCT;        // float [DT][TCP]: delta
+  static constexpr int STAGES = BCF ? 1 : 2;            // raw B / C stages
+  static constexpr int OFF_C = OFF_B + STAGES * BCT;
+  static constexpr int OFF_BF = OFF_C + STAGES * BCT;    // float [TC][N] B, then C (BCF)
+  static constexpr int BF_BYTES = BCF ? 2 * TC * N * 4 : 0;
+  static constexpr int OFF_DLT = (OFF_BF + BF_BYTES + 15) / 16 * 16;  // float [DT][TCP]: delta
   static constexpr int OFF_DU = OFF_DLT + DT * TCP * 4;  // float [DT][TCP]: delta u
   static constexpr int OFF_UF = OFF_DU + DT * TCP * 4;   // float [DT][TCP]: u
   static constexpr int OFF_GT = OFF_UF + DT * TCP * 4;   // float [DT][TCP]: silu(z)
@@ -204,10 +211,11 @@ template <typename T, int NPT> struct PassBuf {
   StateWords<T, NPT> B[4], C[4];    // B, C entries of this thread's states
 };
 
-template <typename T, int N, int NPT, int DT, int TC, bool HAS_Z, int NPOLY>
-__global__ void __launch_bounds__(FastScan<T, N, NPT, DT, TC>::THREADS)
+template <typename T, int N, int NPT, int DT, int TC, bool HAS_Z, int NPOLY, bool BCF>
+__global__ void __launch_bounds__(FastScan<T, N, NPT, DT, TC, BCF>::THREADS)
     scan_fast_kernel(ScanParams p) {
-  using S = FastScan<T, N, NPT, DT, TC>;
+  using S = FastScan<T, N, NPT, DT, TC, BCF>;
+  using TB = typename std::conditional<BCF, float, T>::type;  // element type the scan reads B / C in
   constexpr int G = S::G, THREADS = S::THREADS, NP2 = NPT / 2, TCP = S::TCP;
   extern __shared__ __align__(16) unsigned char smem[];
   const int tid = threadIdx.x;
@@ -232,6 +240,8 @@ __global__ void __launch_bounds__(FastScan<T, N, NPT, DT, TC>::THREADS)
   float *suf = reinterpret_cast<float *>(smem + S::OFF_UF);
   float *sgt = reinterpret_cast<float *>(smem + S::OFF_GT);
   float *sys = reinterpret_cast<float *>(smem + S::OFF_YS);
+  float *sBf = reinterpret_cast<float *>(smem + S::OFF_BF);
+  float *sCf = sBf + TC * N;
 
   auto prefetch = [&](int64_t t0, int stage) {
     for (int q = tid; q < TC * S::ROW_GRAN; q += THREADS) {
@@ -283,7 +293,7 @@ __global__ void __launch_bounds__(FastScan<T, N, NPT, DT, TC>::THREADS)
   float *ys_own = sys + g * S::PLANE + dl * TCP;
 
   // stage 1 of a pass: loads and exponentials (independent of the state)
-  auto stage1 = [&](int t, const T *cB, const T *cC, PassBuf<T, NPT> &pb) {
+  auto stage1 = [&](int t, const TB *cB, const TB *cC, PassBuf<TB, NPT> &pb) {
     const float4 dv = *reinterpret_cast<const float4 *>(rdl + t);
     const float4 uv = *reinterpret_cast<const float4 *>(rdu + t);
     const float dd[4] = {dv.x, dv.y, dv.z, dv.w};
@@ -301,7 +311,7 @@ __global__ void __launch_bounds__(FastScan<T, N, NPT, DT, TC>::THREADS)
     }
   };
   // stage 2 of a pass: the recurrence and the partial C.h sums
-  auto stage2 = [&](int t, const PassBuf<T, NPT> &pb) {
+  auto stage2 = [&](int t, const PassBuf<TB, NPT> &pb) {
     float ys[4];
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
@@ -320,9 +330,17 @@ __global__ void __launch_bounds__(FastScan<T, N, NPT, DT, TC>::THREADS)
   const int64_t nchunks = (L + TC - 1) / TC;
   prefetch(0, 0);
   for (int64_t ch = 0; ch < nchunks; ++ch) {
-    const int stage = (int)(ch & 1);
-    const T *cB = sB + stage * TC * N;
-    const T *cC = sC + stage * TC * N;
+    const int stage = S::STAGES == 2 ? (int)(ch & 1) : 0;
+    const T *rB = sB + stage * TC * N;  // raw (copied) B / C rows of this chunk
+    const T *rC = sC + stage * TC * N;
+    const TB *cB, *cC;                  // the rows the scan reads
+    if constexpr (BCF) {
+      cB = sBf;
+      cC = sCf;
+    } else {
+      cB = rB;
+      cC = rC;
+    }
     const int64_t t0 = ch * TC;
     const int tc = (int)((L - t0) < (int64_t)TC ? (L - t0) : (int64_t)TC);
     cp_async_wait<0>();
@@ -349,14 +367,22 @@ __global__ void __launch_bounds__(FastScan<T, N, NPT, DT, TC>::THREADS)
       *reinterpret_cast<float4 *>(suf + o) = make_float4(uv[0], uv[1], uv[2], uv[3]);
       *reinterpret_cast<float4 *>(sgt + o) = make_float4(gv[0], gv[1], gv[2], gv[3]);
     }
-    __syncthreads();  // delta, delta u, u, gate ready; u / delta / z tile consumed
+    if constexpr (BCF) {
+      for (int q = tid; q < TC * N / 2; q += THREADS) {
+        const uint32_t wb = reinterpret_cast<const uint32_t *>(rB)[q];
+        const uint32_t wc = reinterpret_cast<const uint32_t *>(rC)[q];
+        reinterpret_cast<float2 *>(sBf)[q] = make_float2(bf16lo(wb), bf16hi(wb));
+        reinterpret_cast<float2 *>(sCf)[q] = make_float2(bf16lo(wc), bf16hi(wc));
+      }
+    }
+    __syncthreads();  // delta, delta u, u, gate (and fp32 B / C) ready; raw tiles consumed
 
-    if (ch + 1 < nchunks) prefetch(t0 + TC, stage ^ 1);  // overlaps the scan below
+    if (ch + 1 < nchunks) prefetch(t0 + TC, S::STAGES == 2 ? stage ^ 1 : 0);  // overlaps the scan
 
     // ---- scan over the chunk, 4 steps per pass
     const int tcr = (tc + 3) / 4 * 4;
     for (int t = 0; t < tcr; t += 4) {
-      PassBuf<T, NPT> pb;
+      PassBuf<TB, NPT> pb;
       stage1(t, cB, cC, pb);
       stage2(t, pb);
     }

@@ -100,10 +100,13 @@ __device__ __forceinline__ int div_small(int a, int b, float inv_b) {
   return q;
 }
 
-__device__ __forceinline__ int add_mod(int x, int dx, int m) {  // |dx| <= 2, 0 <= x < m
+// (x + dx) mod m for 0 <= x < m and |dx| <= 2 (m = 1 gives 0), branch-free.
+__device__ __forceinline__ int add_mod(int x, int dx, int m) {
   x += dx;
-  while (x >= m) x -= m;
-  while (x < 0) x += m;
+  x -= (x >= m) ? m : 0;
+  x -= (x >= m) ? m : 0;
+  x += (x < 0) ? m : 0;
+  x += (x < 0) ? m : 0;
   return x;
 }
 
@@ -112,10 +115,12 @@ __device__ __forceinline__ int add_mod(int x, int dx, int m) {  // |dx| <= 2, 0 
 struct PixWalk {
   int h, w, sk;
   int H, W, kappa, skH1;  // skH1 = (kappa (H - 1)) mod W
-  __device__ __forceinline__ void init(int k, int l, int H_, int W_, float invH, float invW) {
+  __device__ __forceinline__ void init(int k, int l, int H_, int W_, float invH, float invW,
+                                       int skH1_) {
     H = H_;
     W = W_;
     kappa = (W & 1) ? 2 : 1;
+    skH1 = skH1_;
     const int ll = k >= 2 ? H * W - 1 - l : l;
     if ((k & 1) == 0) {
       h = div_small(ll, W, invW);
@@ -126,8 +131,6 @@ struct PixWalk {
     }
     const int kh = kappa * h;
     sk = kh - div_small(kh, W, invW) * W;
-    const int kh1 = kappa * (H - 1);
-    skH1 = kh1 - div_small(kh1, W, invW) * W;
   }
   template <int k>
   __device__ __forceinline__ void step() {
@@ -197,18 +200,22 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
   const int64_t ib = blockIdx.y;
   const int64_t d0 = (int64_t)blockIdx.x * DT;
   const int64_t H = p.H, W = p.W, L = H * W, d_in = p.d_in;
-  const int Hi = (int)H, Wi = (int)W, Li = (int)L;  // H W < 2^24 (checked by the launcher)
+  // H W < 2^22 and H W d_in < 2^31 (checked by the launcher): per-image
+  // offsets fit 32-bit integers; only the per-(batch, direction) bases are 64-bit
+  const int Hi = (int)H, Wi = (int)W, Li = (int)L, di = (int)d_in;
   const float invH = 1.0f / (float)Hi, invW = 1.0f / (float)Wi;
+  const int kappa = (Wi & 1) ? 2 : 1;
+  const int skH1 = (kappa * (Hi - 1)) % Wi;
   const int64_t dA = d0 + 2 * cp;    // first channel of the pair
   const bool ok0 = dA < d_in, ok1 = dA + 1 < d_in;
 
-  const T *gu = static_cast<const T *>(p.u);
-  const T *gdt = static_cast<const T *>(p.delta);
-  const T *gB = static_cast<const T *>(p.B);
-  const T *gC = static_cast<const T *>(p.C);
-  T *gy = static_cast<T *>(p.y);
+  const T *gu = static_cast<const T *>(p.u) + ib * L * d_in + d0;    // this image, channel d0
+  const T *gdt = static_cast<const T *>(p.delta) + ib * 4 * L * d_in + d0;
+  const T *gB = static_cast<const T *>(p.B) + ib * 4 * L;
+  const T *gC = static_cast<const T *>(p.C) + ib * 4 * L;
+  T *gy = static_cast<T *>(p.y) + ib * L * d_in + d0;
 
-  float *acc_g = p.acc_global + ib * L * d_in + d0;
+  float *acc_g = p.acc_global + ib * L * d_in + d0;  // this image, channel d0
 
   const int64_t nchunks = (L + LC - 1) / LC;
   const int64_t nsteps = 4 * nchunks;  // (direction, chunk) pairs, walked in order
@@ -216,36 +223,35 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
   // stage the delta / u rows (and B / C) of step block q = k * nchunks + c
   auto prefetch = [&](int64_t q) {
     const int k = (int)(q / nchunks);
-    const int64_t l0 = (q - (int64_t)k * nchunks) * LC;
-    const int64_t seq = ib * 4 + k;
+    const int l0 = (int)(q - (int64_t)k * nchunks) * LC;
+    const T *dk = gdt + (int64_t)k * L * d_in;  // delta rows of direction k
     if constexpr (ROW_ASYNC) {
       for (int r = tid; r < LC * Cfg::GRAN_PER_ROW; r += THREADS) {
         const int row = r / Cfg::GRAN_PER_ROW, part = r - row * Cfg::GRAN_PER_ROW;
-        const int64_t l = l0 + row;
-        const bool ok = l < L;
-        const int64_t pix = ok ? ss2d_pixel32(k, (int)l, Hi, Wi, invH) : 0;
-        const int64_t offd = ok ? (seq * L + l) * d_in + d0 : 0;
-        const int64_t offu = ok ? (ib * L + pix) * d_in + d0 : 0;
+        const int l = l0 + row;
+        const bool ok = l < Li;
+        const int pix = ok ? ss2d_pixel32(k, l, Hi, Wi, invH) : 0;
         const int so = row * DT + part * (16 / Cfg::ESZ);
-        cp_async16(tD + so, gdt + offd + part * (16 / Cfg::ESZ), ok ? 16 : 0);
-        cp_async16(tU + so, gu + offu + part * (16 / Cfg::ESZ), ok ? 16 : 0);
+        const int po = part * (16 / Cfg::ESZ);
+        cp_async16(tD + so, dk + (ok ? l * di : 0) + po, ok ? 16 : 0);
+        cp_async16(tU + so, gu + pix * di + po, ok ? 16 : 0);
       }
     } else {
       for (int r = tid; r < LC * DT; r += THREADS) {
         const int row = r / DT, ch = r - row * DT;
-        const int64_t l = l0 + row;
-        const bool ok = l < L && d0 + ch < d_in;
-        const int64_t pix = ok ? ss2d_pixel32(k, (int)l, Hi, Wi, invH) : 0;
-        tD[r] = ok ? gdt[(seq * L + l) * d_in + d0 + ch] : T(0.0f);
-        tU[r] = ok ? gu[(ib * L + pix) * d_in + d0 + ch] : T(0.0f);
+        const int l = l0 + row;
+        const bool ok = l < Li && d0 + ch < d_in;
+        const int pix = ok ? ss2d_pixel32(k, l, Hi, Wi, invH) : 0;
+        tD[r] = ok ? dk[l * di + ch] : T(0.0f);
+        tU[r] = ok ? gu[pix * di + ch] : T(0.0f);
       }
     }
     if constexpr (BC_ASYNC) {
       for (int r = tid; r < LC / Cfg::BC_VEC; r += THREADS) {
-        const int64_t l = l0 + r * Cfg::BC_VEC;
-        const int64_t rem = L - l;
-        const int bytes = rem <= 0 ? 0 : (rem >= Cfg::BC_VEC ? 16 : (int)rem * Cfg::ESZ);
-        const int64_t off = bytes ? seq * L + l : 0;
+        const int l = l0 + r * Cfg::BC_VEC;
+        const int rem = Li - l;
+        const int bytes = rem <= 0 ? 0 : (rem >= Cfg::BC_VEC ? 16 : rem * Cfg::ESZ);
+        const int64_t off = bytes ? (int64_t)k * L + l : 0;
         cp_async16(tB + r * Cfg::BC_VEC, gB + off, bytes);
         cp_async16(tC + r * Cfg::BC_VEC, gC + off, bytes);
       }
@@ -260,20 +266,20 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
   // one chunk of direction K (index arithmetic specialised per direction)
   auto chunk = [&](auto kc, int64_t q, int64_t c) {
     constexpr int K = decltype(kc)::value;
-    const int64_t l0 = c * LC;
-    const int64_t seq = ib * 4 + K;
+    const int l0 = (int)c * LC;
+    const T *Bk = gB + (int64_t)K * L, *Ck = gC + (int64_t)K * L;
     cp_async_wait<0>();
     __syncthreads();  // staged rows of this chunk visible
 
     // ---- 1. this segment's steps into registers
-    const int64_t lb = l0 + (int64_t)seg * TS;
+    const int lb = l0 + seg * TS;
     float2 a[TS], bu[TS], du[TS];
     float cc[TS];
     Aff2 mine{make_float2(1.0f, 1.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
     for (int j = 0; j < TS; ++j) {
       const int row = seg * TS + j;
-      const bool valid = lb + j < L;
+      const bool valid = lb + j < Li;
       float2 dv, uv, bc;
       if constexpr (sizeof(T) == 2) {
         const uint32_t wd = *reinterpret_cast<const uint32_t *>(tD + row * DT + 2 * cp);
@@ -287,7 +293,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
       if constexpr (BC_ASYNC) {
         bc = make_float2(Elem<T>::load(tB, row), Elem<T>::load(tC, row));
       } else {
-        bc = valid ? make_float2(Elem<T>::load(gB, seq * L + lb + j), Elem<T>::load(gC, seq * L + lb + j))
+        bc = valid ? make_float2(Elem<T>::load(Bk, lb + j), Elem<T>::load(Ck, lb + j))
                    : make_float2(0.0f, 0.0f);
       }
       float2 e = __fadd2_rn(dv, bias);
@@ -333,14 +339,14 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
 
     // ---- 4. replay, accumulate y at the visited pixels
     PixWalk pw;
-    pw.init(K, (int)(lb < L ? lb : 0), Hi, Wi, invH, invW);
+    pw.init(K, lb < Li ? lb : 0, Hi, Wi, invH, invW, skH1);
 #pragma unroll
     for (int j = 0; j < TS; ++j) {
       h = __ffma2_rn(a[j], h, bu[j]);
-      if (lb + j < L) {
+      if (lb + j < Li) {
         const float2 yv = __ffma2_rn(make_float2(cc[j], cc[j]), h, du[j]);
         float *dst = ACC_SMEM ? acc_s + pw.acc_row() * DT + 2 * cp
-                              : acc_g + (int64_t)pw.pix() * d_in + 2 * cp;
+                              : acc_g + pw.pix() * di + 2 * cp;
         if (ok1) {
           float2 *d2 = reinterpret_cast<float2 *>(dst);
           if constexpr (K == 0)
@@ -379,14 +385,20 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
   }
   __syncthreads();
 
-  // ---- round once and store (a warp writes 4 pixels x 8 channels)
-  for (int r = tid; r < Li * DT; r += THREADS) {
-    const int pix = r / DT;
-    const int ch = r - pix * DT;
-    if (d0 + ch < d_in) {
-      const float v = ACC_SMEM ? acc_s[ss2d_acc_row(pix, Wi, invW) * DT + ch]
-                               : acc_g[(int64_t)pix * d_in + ch];
-      Elem<T>::store(gy, (ib * L + pix) * d_in + d0 + ch, v);
+  // ---- round once and store: image row by image row (a warp writes 4
+  // pixels x 8 channels per instruction), the skew undone per row
+  const int ch = tid & (DT - 1);
+  if (d0 + ch < d_in) {
+    int sk = 0;  // (kappa h) mod W
+    for (int hh = 0; hh < Hi; ++hh) {
+      for (int w = tid / DT; w < Wi; w += THREADS / DT) {
+        int sc = w + sk;
+        if (sc >= Wi) sc -= Wi;
+        const int pix = hh * Wi + w;
+        const float v = ACC_SMEM ? acc_s[(hh * Wi + sc) * DT + ch] : acc_g[pix * di + ch];
+        Elem<T>::store(gy, pix * di + ch, v);
+      }
+      sk = add_mod(sk, kappa, Wi);
     }
   }
 }

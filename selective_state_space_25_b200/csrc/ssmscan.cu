@@ -92,13 +92,18 @@ constexpr int fast_npt(int n, int want, int dt) {
   return npt;
 }
 
+#ifndef SSM_SCAN_BCF
+#define SSM_SCAN_BCF 0
+#endif
+
 template <typename T, int N, bool HAS_Z, int WANT_NPT>
 ssm_status launch_scan_fast_npt(const ssm::ScanParams &p, cudaStream_t st) {
   constexpr int NPT = fast_npt(N, WANT_NPT, SSM_SCAN_DT);
   constexpr int DT = SSM_SCAN_DT, TC = SSM_SCAN_TC;
   constexpr int NPOLY = SSM_SCAN_NPOLY < NPT / 2 ? SSM_SCAN_NPOLY : NPT / 2;
-  using Cfg = ssm::FastScan<T, N, NPT, DT, TC>;
-  constexpr auto k = ssm::scan_fast_kernel<T, N, NPT, DT, TC, HAS_Z, NPOLY>;
+  constexpr bool BCF = SSM_SCAN_BCF != 0 && sizeof(T) == 2;  // widen bf16 B / C once per CTA
+  using Cfg = ssm::FastScan<T, N, NPT, DT, TC, BCF>;
+  constexpr auto k = ssm::scan_fast_kernel<T, N, NPT, DT, TC, HAS_Z, NPOLY, BCF>;
   if (ssm_status s = ensure_smem<k>(Cfg::SMEM, "ssm_scan_fwd")) return s;
   const dim3 grid((unsigned)((p.d_in + DT - 1) / DT), (unsigned)p.b);
   k<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(p);
@@ -351,8 +356,9 @@ ssm_status ss2d_scan_fwd(const void *u, const void *delta, const float *A, const
                 workspace_bytes, need);
   const int64_t L = H * W;
   if (b == 0 || d_in == 0 || L == 0) return ok();
-  if (L >= (int64_t(1) << 22))
-    return fail(SSM_ERR_UNSUPPORTED, "ss2d_scan_fwd: H * W = %lld >= 2^22 pixels", (long long)L);
+  if (L >= (int64_t(1) << 22) || L * d_in >= (int64_t(1) << 31))
+    return fail(SSM_ERR_UNSUPPORTED,
+                "ss2d_scan_fwd: H * W = %lld must be < 2^22 and H * W * d_in < 2^31", (long long)L);
   if (!u || !delta || !A || !B || !C || !y)
     return fail(SSM_ERR_INVALID_ARG, "ss2d_scan_fwd: u, delta, A, B, C and y are required");
   if (b > 65535) return fail(SSM_ERR_UNSUPPORTED, "ss2d_scan_fwd: b > 65535");
