@@ -55,11 +55,11 @@ def _load():
         lib.oracle_selective_scan.restype = None
         lib.oracle_state_update.argtypes = [P] * 9 + [ctypes.c_int, P] + [I64] * 3
         lib.oracle_state_update.restype = None
-        lib.oracle_cross_scan.argtypes = [P, P] + [I64] * 4
+        lib.oracle_cross_scan.argtypes = [P, P] + [I64] * 4 + [ctypes.c_int]
         lib.oracle_cross_scan.restype = None
-        lib.oracle_cross_merge.argtypes = [P, P] + [I64] * 4
+        lib.oracle_cross_merge.argtypes = [P, P] + [I64] * 4 + [ctypes.c_int]
         lib.oracle_cross_merge.restype = None
-        lib.oracle_ss2d_scan.argtypes = [P] * 7 + [ctypes.c_int, P] + [I64] * 5
+        lib.oracle_ss2d_scan.argtypes = [P] * 7 + [ctypes.c_int, P] + [I64] * 5 + [ctypes.c_int]
         lib.oracle_ss2d_scan.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
@@ -142,29 +142,33 @@ def state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplu
     return y, st
 
 
-def cross_scan(u, H, W):
-    """u (b, H W, d_in) -> xs (b, 4, H W, d_in)."""
+ORDERS = {"cross": 0, "snake": 1}
+
+
+def cross_scan(u, H, W, order="cross"):
+    """u (b, H W, d_in) -> xs (b, 4, H W, d_in); order "cross" or "snake"."""
     u = _f64(u)
     b, L, d_in = u.shape
     if L != H * W:
         raise ValueError("oracle.cross_scan: L != H*W")
     xs = np.empty((b, 4, L, d_in), np.float64)
-    _load().oracle_cross_scan(_ptr(u), _ptr(xs), b, H, W, d_in)
+    _load().oracle_cross_scan(_ptr(u), _ptr(xs), b, H, W, d_in, ORDERS[order])
     return xs
 
 
-def cross_merge(ys, H, W):
+def cross_merge(ys, H, W, order="cross"):
     """ys (b, 4, H W, d_in) -> y (b, H W, d_in)."""
     ys = _f64(ys)
     b, K, L, d_in = ys.shape
     if K != 4 or L != H * W:
         raise ValueError("oracle.cross_merge: bad shape")
     y = np.empty((b, L, d_in), np.float64)
-    _load().oracle_cross_merge(_ptr(ys), _ptr(y), b, H, W, d_in)
+    _load().oracle_cross_merge(_ptr(ys), _ptr(y), b, H, W, d_in, ORDERS[order])
     return y
 
 
-def ss2d_scan(u, delta, A, B, C, H, W, D=None, dt_bias=None, delta_softplus=True):
+def ss2d_scan(u, delta, A, B, C, H, W, D=None, dt_bias=None, delta_softplus=True,
+              order="cross"):
     """fp64 SS2D forward.  u: (b, H W, d_in); delta: (b, 4, H W, d_in);
     A: (4 d_in, N); B, C: (b, 4, H W, N); D, dt_bias: (4 d_in)."""
     u = _f64(u)
@@ -180,7 +184,7 @@ def ss2d_scan(u, delta, A, B, C, H, W, D=None, dt_bias=None, delta_softplus=True
     y = np.empty((b, L, d_in), np.float64)
     rc = _load().oracle_ss2d_scan(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
                                   _ptr(D), _ptr(dt_bias), int(bool(delta_softplus)),
-                                  _ptr(y), b, H, W, d_in, N)
+                                  _ptr(y), b, H, W, d_in, N, ORDERS[order])
     if rc != 0:
         raise MemoryError("oracle.ss2d_scan: allocation failed")
     return y

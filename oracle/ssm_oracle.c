@@ -30,7 +30,8 @@
  *   - the gate act(z) is SiLU: z / (1 + exp(-z)).
  *   - absent D / z / dt_bias mean D = 0, no gate, bias = 0.
  *   - SS2D directions: k0 row-major (l = h W + w), k1 column-major
- *     (l = w H + h), k2 = k0 reversed, k3 = k1 reversed; delta/B/C of
+ *     (l = w H + h), k2 = k0 reversed, k3 = k1 reversed ("cross"); the snake
+ *     variant flips every odd row of k0 and odd column of k1; delta/B/C of
  *     direction k are given in that direction's scan order; A, D, dt_bias
  *     rows of direction k are k*d_in .. k*d_in + d_in - 1; the merge is the
  *     plain sum over the four directions at each pixel.
@@ -184,31 +185,40 @@ void oracle_state_update(double *state, const double *x, const double *dt,
 /*
  * Pixel visited at step l of scan direction k on an H x W grid (pixels are
  * numbered row-major, p = h W + w).  [VMamba-206]: four orders, row-major,
- * column-major and both reversed.
+ * column-major and both reversed (order 0, "cross"); the snake scan the
+ * issue mentions (order 1) walks odd rows right to left and odd columns
+ * bottom to top, so consecutive steps stay neighbours.
  */
-static int64_t oracle_ss2d_pixel(int k, int64_t l, int64_t H, int64_t W)
+static int64_t oracle_ss2d_pixel(int k, int order, int64_t l, int64_t H, int64_t W)
 {
     const int64_t L = H * W;
     if (k >= 2)
         l = L - 1 - l;               /* k2, k3: the reverse of k0, k1 */
-    if (k == 0 || k == 2)
-        return l;                    /* row-major: l = h W + w */
+    if (k == 0 || k == 2) {
+        const int64_t h = l / W;     /* row-major: l = h W + w */
+        int64_t w = l % W;
+        if (order == 1 && h % 2 == 1)
+            w = W - 1 - w;
+        return h * W + w;
+    }
     {
-        const int64_t h = l % H;     /* column-major: l = w H + h */
+        int64_t h = l % H;           /* column-major: l = w H + h */
         const int64_t w = l / H;
+        if (order == 1 && w % 2 == 1)
+            h = H - 1 - h;
         return h * W + w;
     }
 }
 
 /* CrossScan: xs[b, k, l, d] = u[b, pixel_k(l), d]. */
 void oracle_cross_scan(const double *u, double *xs, int64_t b, int64_t H,
-                       int64_t W, int64_t d_in)
+                       int64_t W, int64_t d_in, int order)
 {
     const int64_t L = H * W;
     for (int64_t ib = 0; ib < b; ++ib)
         for (int k = 0; k < 4; ++k)
             for (int64_t l = 0; l < L; ++l) {
-                const int64_t p = oracle_ss2d_pixel(k, l, H, W);
+                const int64_t p = oracle_ss2d_pixel(k, order, l, H, W);
                 for (int64_t d = 0; d < d_in; ++d)
                     xs[((ib * 4 + k) * L + l) * d_in + d] =
                         u[(ib * L + p) * d_in + d];
@@ -217,14 +227,14 @@ void oracle_cross_scan(const double *u, double *xs, int64_t b, int64_t H,
 
 /* CrossMerge: y[b, pixel_k(l), d] = sum over k of ys[b, k, l, d]. */
 void oracle_cross_merge(const double *ys, double *y, int64_t b, int64_t H,
-                        int64_t W, int64_t d_in)
+                        int64_t W, int64_t d_in, int order)
 {
     const int64_t L = H * W;
     memset(y, 0, (size_t)(b * L * d_in) * sizeof(double));
     for (int64_t ib = 0; ib < b; ++ib)
         for (int k = 0; k < 4; ++k)
             for (int64_t l = 0; l < L; ++l) {
-                const int64_t p = oracle_ss2d_pixel(k, l, H, W);
+                const int64_t p = oracle_ss2d_pixel(k, order, l, H, W);
                 for (int64_t d = 0; d < d_in; ++d)
                     y[(ib * L + p) * d_in + d] +=
                         ys[((ib * 4 + k) * L + l) * d_in + d];
@@ -243,7 +253,8 @@ void oracle_cross_merge(const double *ys, double *y, int64_t b, int64_t H,
 int oracle_ss2d_scan(const double *u, const double *delta, const double *A,
                      const double *B, const double *C, const double *D,
                      const double *dt_bias, int delta_softplus, double *y,
-                     int64_t b, int64_t H, int64_t W, int64_t d_in, int64_t N)
+                     int64_t b, int64_t H, int64_t W, int64_t d_in, int64_t N,
+                     int order)
 {
     const int64_t L = H * W;
     const size_t n_xs = (size_t)(b * 4 * L * d_in);
@@ -254,7 +265,7 @@ int oracle_ss2d_scan(const double *u, const double *delta, const double *A,
         free(ys);
         return -1;
     }
-    oracle_cross_scan(u, xs, b, H, W, d_in);
+    oracle_cross_scan(u, xs, b, H, W, d_in, order);
     for (int64_t ib = 0; ib < b; ++ib)
         for (int k = 0; k < 4; ++k) {
             const int64_t seq = ib * 4 + k;
@@ -266,7 +277,7 @@ int oracle_ss2d_scan(const double *u, const double *delta, const double *A,
                                   delta_softplus, NULL, NULL,
                                   ys + seq * L * d_in, 1, L, d_in, N);
         }
-    oracle_cross_merge(ys, y, b, H, W, d_in);
+    oracle_cross_merge(ys, y, b, H, W, d_in, order);
     free(xs);
     free(ys);
     return 0;

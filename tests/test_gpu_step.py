@@ -9,7 +9,7 @@ import torch
 
 import oracle
 from _helpers import TOL, rel_err, to_cuda, to64
-from selective_state_space_25_b200.synthetic import WORKLOADS, step_inputs
+from selective_state_space_25_b200.synthetic import WORKLOADS, scan_inputs, step_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -81,3 +81,28 @@ def test_decode_workload_steps_1_10_1000(ssm):
     hstar = delta * to64(inp["B"])[:, None, :] * x / (1.0 - a)
     hk = hstar + a ** steps * (to64(inp["state"]) - hstar)
     assert rel_err(st, hk) <= 1e-3
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_prefill_then_decode_handoff(ssm, dtype):
+    """A prefill scan over L tokens exports h_last; one decode step from that
+    state on token L+1 equals the oracle's scan over all L+1 tokens (the
+    cached-state path of Mamba.forward in "代码连连看——mamba")."""
+    dt = "bf16" if dtype == torch.bfloat16 else "fp32"
+    b, L, d_in, N = 2, 97, 64, 16
+    inp = scan_inputs(b, L + 1, d_in, N, dt, seed=31)
+    g = to_cuda(inp)
+    pre = lambda t: t[:, :L].contiguous()
+    state = torch.empty(b, d_in, N, device="cuda")
+    y_pre = ssm.ssm_scan_fwd(pre(g["u"]), pre(g["delta"]), g["A"], pre(g["B"]), pre(g["C"]),
+                             D=g["D"], z=pre(g["z"]), dt_bias=g["dt_bias"], h_last=state)
+    last = lambda t: t[:, L].contiguous()
+    y_tok = ssm.ssm_state_update(state, last(g["u"]), last(g["delta"]), g["A"], last(g["B"]),
+                                 last(g["C"]), D=g["D"], z=last(g["z"]), dt_bias=g["dt_bias"])
+    y_ref, h_ref = oracle.selective_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"],
+                                         D=inp["D"], z=inp["z"], dt_bias=inp["dt_bias"],
+                                         return_last_state=True)
+    tol = TOL[dtype]
+    assert rel_err(y_pre, y_ref[:, :L]) <= tol
+    assert rel_err(y_tok, y_ref[:, L]) <= tol
+    assert rel_err(state, h_ref) <= max(tol, 1e-4)

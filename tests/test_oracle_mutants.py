@@ -50,10 +50,14 @@ MUTANTS = {
     # SS2D: direction k3 not reversed
     "ss2d_k3_not_reversed": ("if (k >= 2)\n        l = L - 1 - l;", "if (k == 2)\n        l = L - 1 - l;"),
     # SS2D: column-major index computed with W instead of H (square grids only agree)
-    "ss2d_colmajor_wrong": ("const int64_t h = l % H;     /* column-major: l = w H + h */\n"
+    "ss2d_colmajor_wrong": ("int64_t h = l % H;           /* column-major: l = w H + h */\n"
                             "        const int64_t w = l / H;",
-                            "const int64_t h = l / W;     /* column-major: l = w H + h */\n"
+                            "int64_t h = l / W;           /* column-major: l = w H + h */\n"
                             "        const int64_t w = l % W;"),
+    # SS2D snake: odd rows not flipped
+    "ss2d_snake_rows_unflipped": ("if (order == 1 && h % 2 == 1)", "if (order == 1 && h % 2 == 7)"),
+    # SS2D snake: even columns flipped instead of odd ones
+    "ss2d_snake_cols_wrong_parity": ("if (order == 1 && w % 2 == 1)", "if (order == 1 && w % 2 == 0)"),
 }
 
 

@@ -383,3 +383,56 @@ def test_pins_reject_zoh_B_variant():
     zoh = (math.exp(delta * A) - 1.0) / A * Bv * u
     euler = delta * Bv * u
     assert abs(zoh) < 1e-15 and abs(euler - 0.459) < 1e-12
+
+
+# --------------------------------------------------------------------------
+# SS2D snake order (the "蛇形Scan / 蛇形Merge" variant of [VMamba-206]):
+# odd rows right to left in k0, odd columns bottom to top in k1.
+# --------------------------------------------------------------------------
+def _numpy_snake_scan(u, H, W):
+    b, L, d = u.shape
+    rm = u.reshape(b, H, W, d).copy()
+    rm[:, 1::2] = rm[:, 1::2, ::-1]
+    cm = u.reshape(b, H, W, d).transpose(0, 2, 1, 3).copy()    # (b, W, H, d): columns
+    cm[:, 1::2] = cm[:, 1::2, ::-1]
+    rm, cm = rm.reshape(b, L, d), cm.reshape(b, L, d)
+    return np.stack([rm, cm, rm[:, ::-1], cm[:, ::-1]], axis=1)
+
+
+def test_ss2d_snake_orders_hand_derived():
+    # H = 2, W = 3, pixels p = h*3 + w.  Orders written out by hand.
+    u = np.arange(6, dtype=np.float64).reshape(1, 6, 1)
+    xs = oracle.cross_scan(u, 2, 3, order="snake")[0, :, :, 0]
+    assert xs[0].tolist() == [0, 1, 2, 5, 4, 3]       # rows, odd row right to left
+    assert xs[1].tolist() == [0, 3, 4, 1, 2, 5]       # columns, odd column bottom to top
+    assert xs[2].tolist() == [3, 4, 5, 2, 1, 0]       # reverse of the first
+    assert xs[3].tolist() == [5, 2, 1, 4, 3, 0]       # reverse of the second
+
+
+@pytest.mark.parametrize("H,W", [(5, 7), (1, 9), (8, 1), (4, 4), (3, 6)])
+def test_ss2d_snake_matches_numpy(H, W):
+    u = RNG.standard_normal((2, H * W, 3))
+    np.testing.assert_array_equal(oracle.cross_scan(u, H, W, order="snake"),
+                                  _numpy_snake_scan(u, H, W))
+    np.testing.assert_array_equal(
+        oracle.cross_merge(oracle.cross_scan(u, H, W, order="snake"), H, W, order="snake"), 4.0 * u)
+
+
+def test_ss2d_snake_scan_is_four_1d_scans():
+    b, H, W, d_in, N = 2, 3, 5, 4, 1
+    L = H * W
+    u = RNG.standard_normal((b, L, d_in))
+    delta = RNG.standard_normal((b, 4, L, d_in))
+    A = -RNG.uniform(0.5, 2.0, size=(4 * d_in, N))
+    B = RNG.standard_normal((b, 4, L, N))
+    C = RNG.standard_normal((b, 4, L, N))
+    D = RNG.standard_normal(4 * d_in)
+    y = oracle.ss2d_scan(u, delta, A, B, C, H, W, D=D, order="snake")
+    xs = _numpy_snake_scan(u, H, W)
+    perm = _numpy_snake_scan(np.arange(L, dtype=np.float64).reshape(1, L, 1), H, W)[0, :, :, 0]
+    ref = np.zeros_like(u)
+    for k in range(4):
+        sl = slice(k * d_in, (k + 1) * d_in)
+        yk = oracle.selective_scan(xs[:, k], delta[:, k], A[sl], B[:, k], C[:, k], D=D[sl])
+        ref[:, perm[k].astype(int)] += yk       # step l of direction k lands on pixel perm[k][l]
+    np.testing.assert_allclose(y, ref, rtol=1e-13, atol=1e-13)
