@@ -68,6 +68,12 @@ typedef enum {
     SSM_BF16 = 1
 } ssm_dtype;
 
+/* SS2D scan orders (see ss2d_scan_fwd_ex). */
+typedef enum {
+    SSM_SS2D_CROSS = 0,  /* row-major, column-major and both reversed (VMamba CrossScan) */
+    SSM_SS2D_SNAKE = 1   /* as CROSS with odd rows / odd columns walked backwards */
+} ssm_ss2d_order;
+
 /*
  * Bytes of device workspace ssm_scan_fwd needs for this problem (0 when the
  * launch it picks needs none).  The chunked path, which splits L across
@@ -134,6 +140,25 @@ ssm_status ss2d_scan_fwd(const void *u, const void *delta, const float *A,
                          size_t workspace_bytes, ssm_stream_t stream);
 
 /*
+ * ss2d_scan_fwd with a choice of scan order ("关于代码SS2D中的d_state设置",
+ * VMamba issue 206, mentions a snake scan and snake merge besides
+ * CrossScan).  SSM_SS2D_CROSS is ss2d_scan_fwd.  SSM_SS2D_SNAKE keeps the
+ * four directions but walks them boustrophedon: direction 0 visits row h
+ * left to right when h is even and right to left when h is odd; direction 1
+ * visits column w top to bottom when w is even and bottom to top when w is
+ * odd; directions 2 and 3 are the reverses of 0 and 1.  delta / B / C are
+ * given in the chosen order's step order; everything else is as in
+ * ss2d_scan_fwd.  An unknown order returns SSM_ERR_UNSUPPORTED.
+ */
+ssm_status ss2d_scan_fwd_ex(const void *u, const void *delta, const float *A,
+                            const void *B, const void *C, const float *D,
+                            const float *dt_bias, int delta_softplus, void *y,
+                            int64_t b, int64_t H, int64_t W, int64_t d_in,
+                            int64_t d_state, ssm_ss2d_order order, ssm_dtype dtype,
+                            void *workspace, size_t workspace_bytes,
+                            ssm_stream_t stream);
+
+/*
  * Bytes of device workspace ss2d_scan_fwd needs (0 for d_state = 1 when
  * the fp32 accumulator of one (batch, 8-channel) tile, 32 * H * W bytes, fits
  * in shared memory, i.e. H * W <= 6272).  Larger images keep that
@@ -196,6 +221,14 @@ ssm_status ssm_state_update(float *ssm_state, const void *x, const void *dt,
 ssm_status ss2d_cross_scan(const void *u, void *xs, int64_t b, int64_t H,
                            int64_t W, int64_t d_in, ssm_dtype dtype,
                            ssm_stream_t stream);
+
+/* ss2d_cross_scan / ss2d_cross_merge in the given scan order. */
+ssm_status ss2d_cross_scan_ex(const void *u, void *xs, int64_t b, int64_t H,
+                              int64_t W, int64_t d_in, ssm_ss2d_order order,
+                              ssm_dtype dtype, ssm_stream_t stream);
+ssm_status ss2d_cross_merge_ex(const void *ys, void *y, int64_t b, int64_t H,
+                               int64_t W, int64_t d_in, ssm_ss2d_order order,
+                               ssm_dtype dtype, ssm_stream_t stream);
 
 /*
  * CrossMerge: y[i,p,d] = sum_k ys[i, k, l_k(p), d] with l_k the inverse of

@@ -17,13 +17,37 @@
 
 namespace ssm {
 
+// Scan orders.  Cross (VMamba's CrossScan): k0 row-major, k1 column-major,
+// k2 / k3 their reverses.  Snake (the snake scan of the same thread): as
+// cross, but odd rows of k0 run right to left and odd columns of k1 bottom
+// to top, so consecutive steps stay neighbours.
+enum Ss2dOrder { kOrderCross = 0, kOrderSnake = 1 };
+
+template <int ORDER>
 __device__ __forceinline__ int64_t ss2d_pixel(int k, int64_t l, int64_t H, int64_t W) {
   const int64_t L = H * W;
   if (k >= 2) l = L - 1 - l;
-  if ((k & 1) == 0) return l;
+  if ((k & 1) == 0) {
+    if constexpr (ORDER == kOrderCross) return l;
+    const int64_t h = l / W, r = l - h * W;
+    return h * W + ((h & 1) ? W - 1 - r : r);
+  }
   const int64_t w = l / H;
-  const int64_t h = l - w * H;
+  const int64_t r = l - w * H;
+  const int64_t h = (ORDER == kOrderSnake && (w & 1)) ? H - 1 - r : r;
   return h * W + w;
+}
+
+// Step index at which direction k visits pixel (h, w): the inverse of ss2d_pixel.
+template <int ORDER>
+__device__ __forceinline__ int64_t ss2d_step_of(int k, int64_t h, int64_t w, int64_t H,
+                                                int64_t W) {
+  int64_t l;
+  if ((k & 1) == 0)
+    l = h * W + ((ORDER == kOrderSnake && (h & 1)) ? W - 1 - w : w);
+  else
+    l = w * H + ((ORDER == kOrderSnake && (w & 1)) ? H - 1 - h : h);
+  return k >= 2 ? H * W - 1 - l : l;
 }
 
 struct Ss2dParams {
@@ -112,6 +136,7 @@ __device__ __forceinline__ int add_mod(int x, int dx, int m) {
 
 // Walks the pixels direction k visits at consecutive steps without
 // divisions: (h, w) and sk = (kappa h) mod W for the skewed accumulator row.
+template <int ORDER>
 struct PixWalk {
   int h, w, sk;
   int H, W, kappa, skH1;  // skH1 = (kappa (H - 1)) mod W
@@ -125,26 +150,52 @@ struct PixWalk {
     if ((k & 1) == 0) {
       h = div_small(ll, W, invW);
       w = ll - h * W;
+      if (ORDER == kOrderSnake && (h & 1)) w = W - 1 - w;
     } else {
       w = div_small(ll, H, invH);
       h = ll - w * H;
+      if (ORDER == kOrderSnake && (w & 1)) h = H - 1 - h;
     }
     const int kh = kappa * h;
     sk = kh - div_small(kh, W, invW) * W;
   }
   template <int k>
   __device__ __forceinline__ void step() {
-    if constexpr ((k & 1) == 0) {  // row-major: w moves, h on wrap
-      if constexpr (k == 0) {
-        if (++w == W) { w = 0; ++h; sk = add_mod(sk, kappa, W); }
-      } else {
-        if (--w < 0) { w = W - 1; --h; sk = add_mod(sk, -kappa, W); }
+    if constexpr (ORDER == kOrderCross) {
+      if constexpr ((k & 1) == 0) {  // row-major: w moves, h on wrap
+        if constexpr (k == 0) {
+          if (++w == W) { w = 0; ++h; sk = add_mod(sk, kappa, W); }
+        } else {
+          if (--w < 0) { w = W - 1; --h; sk = add_mod(sk, -kappa, W); }
+        }
+      } else {                       // column-major: h moves, w on wrap
+        if constexpr (k == 1) {
+          if (++h == H) { h = 0; ++w; sk = 0; } else { sk = add_mod(sk, kappa, W); }
+        } else {
+          if (--h < 0) { h = H - 1; --w; sk = skH1; } else { sk = add_mod(sk, -kappa, W); }
+        }
       }
-    } else {                       // column-major: h moves, w on wrap
-      if constexpr (k == 1) {
-        if (++h == H) { h = 0; ++w; sk = 0; } else { sk = add_mod(sk, kappa, W); }
+    } else {  // snake: at a row (column) end the walk turns into the next one
+      if constexpr ((k & 1) == 0) {
+        // forward: even rows left to right, odd rows right to left
+        const bool right = ((h & 1) == 0) == (k == 0);
+        const bool turn = right ? w == W - 1 : w == 0;
+        if (turn) {
+          h += k == 0 ? 1 : -1;
+          sk = add_mod(sk, k == 0 ? kappa : -kappa, W);
+        } else {
+          w += right ? 1 : -1;
+        }
       } else {
-        if (--h < 0) { h = H - 1; --w; sk = skH1; } else { sk = add_mod(sk, -kappa, W); }
+        // forward: even columns top to bottom, odd columns bottom to top
+        const bool down = ((w & 1) == 0) == (k == 1);
+        const bool turn = down ? h == H - 1 : h == 0;
+        if (turn) {
+          w += k == 1 ? 1 : -1;
+        } else {
+          h += down ? 1 : -1;
+          sk = add_mod(sk, down ? kappa : -kappa, W);
+        }
       }
     }
   }
@@ -166,11 +217,18 @@ __device__ __forceinline__ int ss2d_acc_row(int pix, int W, float invW) {
 }
 
 // Pixel direction k visits at step l (32-bit, for one-off lookups).
-__device__ __forceinline__ int ss2d_pixel32(int k, int l, int H, int W, float invH) {
+template <int ORDER>
+__device__ __forceinline__ int ss2d_pixel32(int k, int l, int H, int W, float invH, float invW) {
   const int ll = k >= 2 ? H * W - 1 - l : l;
-  if ((k & 1) == 0) return ll;
+  if ((k & 1) == 0) {
+    if constexpr (ORDER == kOrderCross) return ll;
+    const int h = div_small(ll, W, invW), r = ll - h * W;
+    return h * W + ((h & 1) ? W - 1 - r : r);
+  }
   const int w = div_small(ll, H, invH);
-  return (ll - w * H) * W + w;
+  const int r = ll - w * H;
+  const int h = (ORDER == kOrderSnake && (w & 1)) ? H - 1 - r : r;
+  return h * W + w;
 }
 
 // ROW_ASYNC: delta / u rows staged with cp.async (needs d_in a multiple of 8
@@ -178,7 +236,7 @@ __device__ __forceinline__ int ss2d_pixel32(int k, int l, int H, int W, float in
 // BC_ASYNC: B / C staged with cp.async (needs H W a multiple of 16 / sizeof(T)
 // and 16-byte aligned B, C); otherwise read from global memory per step.
 template <typename T, int TS, int WARPS, bool ACC_SMEM, bool A_POLY, bool ROW_ASYNC,
-          bool BC_ASYNC>
+          bool BC_ASYNC, int ORDER>
 __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     ss2d_n1_kernel(Ss2dParams p) {
   using Cfg = Ss2dCfg<T, TS, WARPS>;
@@ -230,7 +288,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
         const int row = r / Cfg::GRAN_PER_ROW, part = r - row * Cfg::GRAN_PER_ROW;
         const int l = l0 + row;
         const bool ok = l < Li;
-        const int pix = ok ? ss2d_pixel32(k, l, Hi, Wi, invH) : 0;
+        const int pix = ok ? ss2d_pixel32<ORDER>(k, l, Hi, Wi, invH, invW) : 0;
         const int so = row * DT + part * (16 / Cfg::ESZ);
         const int po = part * (16 / Cfg::ESZ);
         cp_async16(tD + so, dk + (ok ? l * di : 0) + po, ok ? 16 : 0);
@@ -241,7 +299,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
         const int row = r / DT, ch = r - row * DT;
         const int l = l0 + row;
         const bool ok = l < Li && d0 + ch < d_in;
-        const int pix = ok ? ss2d_pixel32(k, l, Hi, Wi, invH) : 0;
+        const int pix = ok ? ss2d_pixel32<ORDER>(k, l, Hi, Wi, invH, invW) : 0;
         tD[r] = ok ? dk[l * di + ch] : T(0.0f);
         tU[r] = ok ? gu[pix * di + ch] : T(0.0f);
       }
@@ -338,7 +396,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     h = __ffma2_rn(exc.a, h, exc.b);
 
     // ---- 4. replay, accumulate y at the visited pixels
-    PixWalk pw;
+    PixWalk<ORDER> pw;
     pw.init(K, lb < Li ? lb : 0, Hi, Wi, invH, invW, skH1);
 #pragma unroll
     for (int j = 0; j < TS; ++j) {
@@ -407,7 +465,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
 // CrossScan / CrossMerge as stored permutations (for checking the index
 // arithmetic above bit-exactly).
 // ---------------------------------------------------------------------------
-template <typename T>
+template <typename T, int ORDER>
 __global__ void cross_scan_kernel(const T *u, T *xs, int64_t b, int64_t H, int64_t W,
                                   int64_t d_in) {
   const int64_t L = H * W;
@@ -418,11 +476,11 @@ __global__ void cross_scan_kernel(const T *u, T *xs, int64_t b, int64_t H, int64
     const int64_t l = (i / d_in) % L;
     const int k = (int)((i / (d_in * L)) % 4);
     const int64_t ib = i / (d_in * L * 4);
-    xs[i] = u[(ib * L + ss2d_pixel(k, l, H, W)) * d_in + d];
+    xs[i] = u[(ib * L + ss2d_pixel<ORDER>(k, l, H, W)) * d_in + d];
   }
 }
 
-template <typename T>
+template <typename T, int ORDER>
 __global__ void cross_merge_kernel(const T *ys, T *y, int64_t b, int64_t H, int64_t W,
                                    int64_t d_in) {
   const int64_t L = H * W;
@@ -432,14 +490,11 @@ __global__ void cross_merge_kernel(const T *ys, T *y, int64_t b, int64_t H, int6
     const int64_t d = i % d_in;
     const int64_t pix = (i / d_in) % L;
     const int64_t ib = i / (d_in * L);
-    // l_k(p): inverse of p_k.  Row-major index and column-major index of p.
-    const int64_t hh = pix / W, ww = pix - (pix / W) * W;
-    const int64_t l_rm = pix, l_cm = ww * H + hh;
-    const int64_t l_of[4] = {l_rm, l_cm, L - 1 - l_rm, L - 1 - l_cm};
+    const int64_t hh = pix / W, ww = pix - hh * W;
     float s = 0.0f;
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-      s += Elem<T>::load(ys, ((ib * 4 + k) * L + l_of[k]) * d_in + d);
+    for (int k = 0; k < 4; ++k)  // summed k0 + k1 + k2 + k3, rounded once
+      s += Elem<T>::load(ys, ((ib * 4 + k) * L + ss2d_step_of<ORDER>(k, hh, ww, H, W)) * d_in + d);
     Elem<T>::store(y, i, s);
   }
 }

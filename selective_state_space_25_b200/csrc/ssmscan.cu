@@ -8,6 +8,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <type_traits>
 
 #include "ssmscan.h"
 #include "scan_fwd.cuh"
@@ -212,11 +213,11 @@ ssm_status dispatch_step_n(const ssm::StepParams &p, int64_t N, cudaStream_t st)
 constexpr int kSs2dDT = 8;
 constexpr int64_t kSs2dSmemPixels = 6272;  // H W of the shared-memory fp32 accumulator, 32 B each
 
-template <typename T, bool ACC_SMEM, bool ROW_ASYNC, bool BC_ASYNC>
+template <typename T, bool ACC_SMEM, bool ROW_ASYNC, bool BC_ASYNC, int ORDER>
 ssm_status launch_ss2d_cfg(const ssm::Ss2dParams &p, cudaStream_t st) {
   using Cfg = ssm::Ss2dCfg<T, SSM_SS2D_TS, SSM_SS2D_WARPS>;
   constexpr auto k = ssm::ss2d_n1_kernel<T, SSM_SS2D_TS, SSM_SS2D_WARPS, ACC_SMEM,
-                                         SSM_SS2D_APOLY != 0, ROW_ASYNC, BC_ASYNC>;
+                                         SSM_SS2D_APOLY != 0, ROW_ASYNC, BC_ASYNC, ORDER>;
   const int64_t L = p.H * p.W;
   const int smem = Cfg::AUX_BYTES + (ACC_SMEM ? (int)(L * kSs2dDT * sizeof(float)) : 0);
   if (ssm_status s = ensure_smem<k>(Cfg::AUX_BYTES + (int)(kSs2dSmemPixels * kSs2dDT * 4),
@@ -227,24 +228,30 @@ ssm_status launch_ss2d_cfg(const ssm::Ss2dParams &p, cudaStream_t st) {
   return check_launch("ss2d_scan_fwd");
 }
 
-template <typename T, bool ACC_SMEM>
+template <typename T, bool ACC_SMEM, int ORDER>
 ssm_status launch_ss2d_acc(const ssm::Ss2dParams &p, bool row_async, bool bc_async,
                            cudaStream_t st) {
   if (row_async)
-    return bc_async ? launch_ss2d_cfg<T, ACC_SMEM, true, true>(p, st)
-                    : launch_ss2d_cfg<T, ACC_SMEM, true, false>(p, st);
-  return bc_async ? launch_ss2d_cfg<T, ACC_SMEM, false, true>(p, st)
-                  : launch_ss2d_cfg<T, ACC_SMEM, false, false>(p, st);
+    return bc_async ? launch_ss2d_cfg<T, ACC_SMEM, true, true, ORDER>(p, st)
+                    : launch_ss2d_cfg<T, ACC_SMEM, true, false, ORDER>(p, st);
+  return bc_async ? launch_ss2d_cfg<T, ACC_SMEM, false, true, ORDER>(p, st)
+                  : launch_ss2d_cfg<T, ACC_SMEM, false, false, ORDER>(p, st);
 }
 
-template <typename T>
-ssm_status launch_ss2d(const ssm::Ss2dParams &p, cudaStream_t st) {
+template <typename T, int ORDER>
+ssm_status launch_ss2d_order(const ssm::Ss2dParams &p, cudaStream_t st) {
   const int64_t L = p.H * p.W;
   const size_t es = sizeof(T);
   const bool row_async = (p.d_in % kSs2dDT) == 0 && aligned(p.u, 16) && aligned(p.delta, 16);
   const bool bc_async = (L * (int64_t)es) % 16 == 0 && aligned(p.B, 16) && aligned(p.C, 16);
-  if (L <= kSs2dSmemPixels) return launch_ss2d_acc<T, true>(p, row_async, bc_async, st);
-  return launch_ss2d_acc<T, false>(p, row_async, bc_async, st);
+  if (L <= kSs2dSmemPixels) return launch_ss2d_acc<T, true, ORDER>(p, row_async, bc_async, st);
+  return launch_ss2d_acc<T, false, ORDER>(p, row_async, bc_async, st);
+}
+
+template <typename T>
+ssm_status launch_ss2d(const ssm::Ss2dParams &p, ssm_ss2d_order order, cudaStream_t st) {
+  return order == SSM_SS2D_SNAKE ? launch_ss2d_order<T, ssm::kOrderSnake>(p, st)
+                                 : launch_ss2d_order<T, ssm::kOrderCross>(p, st);
 }
 
 unsigned grid_for(int64_t n) {
@@ -341,7 +348,18 @@ ssm_status ss2d_scan_fwd(const void *u, const void *delta, const float *A, const
                          void *y, int64_t b, int64_t H, int64_t W, int64_t d_in, int64_t d_state,
                          ssm_dtype dtype, void *workspace, size_t workspace_bytes,
                          ssm_stream_t stream) {
+  return ss2d_scan_fwd_ex(u, delta, A, B, C, D, dt_bias, delta_softplus, y, b, H, W, d_in,
+                          d_state, SSM_SS2D_CROSS, dtype, workspace, workspace_bytes, stream);
+}
+
+ssm_status ss2d_scan_fwd_ex(const void *u, const void *delta, const float *A, const void *B,
+                            const void *C, const float *D, const float *dt_bias,
+                            int delta_softplus, void *y, int64_t b, int64_t H, int64_t W,
+                            int64_t d_in, int64_t d_state, ssm_ss2d_order order, ssm_dtype dtype,
+                            void *workspace, size_t workspace_bytes, ssm_stream_t stream) {
   g_last_error.clear();
+  if (order != SSM_SS2D_CROSS && order != SSM_SS2D_SNAKE)
+    return fail(SSM_ERR_UNSUPPORTED, "ss2d_scan_fwd: unknown scan order %d", (int)order);
   if (b < 0 || H < 0 || W < 0 || d_in < 0)
     return fail(SSM_ERR_INVALID_ARG, "ss2d_scan_fwd: negative size");
   if (dtype != SSM_F32 && dtype != SSM_BF16)
@@ -377,8 +395,8 @@ ssm_status ss2d_scan_fwd(const void *u, const void *delta, const float *A, const
   ssm::Ss2dParams p{u, delta, A, B, C, D, dt_bias, y, static_cast<float *>(workspace),
                     b, H, W, d_in, delta_softplus};
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype == SSM_BF16) return launch_ss2d<__nv_bfloat16>(p, st);
-  return launch_ss2d<float>(p, st);
+  if (dtype == SSM_BF16) return launch_ss2d<__nv_bfloat16>(p, order, st);
+  return launch_ss2d<float>(p, order, st);
 }
 
 ssm_status ssm_state_update(float *ssm_state, const void *x, const void *dt, const float *A,
@@ -421,6 +439,12 @@ ssm_status ssm_state_update(float *ssm_state, const void *x, const void *dt, con
 
 ssm_status ss2d_cross_scan(const void *u, void *xs, int64_t b, int64_t H, int64_t W,
                            int64_t d_in, ssm_dtype dtype, ssm_stream_t stream) {
+  return ss2d_cross_scan_ex(u, xs, b, H, W, d_in, SSM_SS2D_CROSS, dtype, stream);
+}
+
+ssm_status ss2d_cross_scan_ex(const void *u, void *xs, int64_t b, int64_t H, int64_t W,
+                              int64_t d_in, ssm_ss2d_order order, ssm_dtype dtype,
+                              ssm_stream_t stream) {
   g_last_error.clear();
   int64_t L, n;
   if (b < 0 || H < 0 || W < 0 || d_in < 0 || !mul_ok(H, W, &L) || !mul_ok(b, 4 * L, &n) ||
@@ -428,22 +452,36 @@ ssm_status ss2d_cross_scan(const void *u, void *xs, int64_t b, int64_t H, int64_
     return fail(SSM_ERR_INVALID_ARG, "ss2d_cross_scan: bad sizes");
   if (dtype != SSM_F32 && dtype != SSM_BF16)
     return fail(SSM_ERR_UNSUPPORTED, "ss2d_cross_scan: unknown dtype %d", (int)dtype);
+  if (order != SSM_SS2D_CROSS && order != SSM_SS2D_SNAKE)
+    return fail(SSM_ERR_UNSUPPORTED, "ss2d_cross_scan: unknown scan order %d", (int)order);
   if (n == 0) return ok();
   if (!u || !xs) return fail(SSM_ERR_INVALID_ARG, "ss2d_cross_scan: NULL pointer");
   if (!aligned(u, esize(dtype)) || !aligned(xs, esize(dtype)))
     return fail(SSM_ERR_INVALID_ARG, "ss2d_cross_scan: misaligned pointer");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto run = [&](auto tag, auto ord) {
+    using T = decltype(tag);
+    constexpr int O = decltype(ord)::value;
+    ssm::cross_scan_kernel<T, O><<<grid_for(n), 256, 0, st>>>(
+        static_cast<const T *>(u), static_cast<T *>(xs), b, H, W, d_in);
+  };
+  using Cross = std::integral_constant<int, ssm::kOrderCross>;
+  using Snake = std::integral_constant<int, ssm::kOrderSnake>;
   if (dtype == SSM_BF16)
-    ssm::cross_scan_kernel<__nv_bfloat16><<<grid_for(n), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16 *>(u), static_cast<__nv_bfloat16 *>(xs), b, H, W, d_in);
+    order == SSM_SS2D_SNAKE ? run(__nv_bfloat16(), Snake()) : run(__nv_bfloat16(), Cross());
   else
-    ssm::cross_scan_kernel<float><<<grid_for(n), 256, 0, st>>>(
-        static_cast<const float *>(u), static_cast<float *>(xs), b, H, W, d_in);
+    order == SSM_SS2D_SNAKE ? run(float(), Snake()) : run(float(), Cross());
   return check_launch("ss2d_cross_scan");
 }
 
 ssm_status ss2d_cross_merge(const void *ys, void *y, int64_t b, int64_t H, int64_t W,
                             int64_t d_in, ssm_dtype dtype, ssm_stream_t stream) {
+  return ss2d_cross_merge_ex(ys, y, b, H, W, d_in, SSM_SS2D_CROSS, dtype, stream);
+}
+
+ssm_status ss2d_cross_merge_ex(const void *ys, void *y, int64_t b, int64_t H, int64_t W,
+                               int64_t d_in, ssm_ss2d_order order, ssm_dtype dtype,
+                               ssm_stream_t stream) {
   g_last_error.clear();
   int64_t L, n;
   if (b < 0 || H < 0 || W < 0 || d_in < 0 || !mul_ok(H, W, &L) || !mul_ok(b, 4 * L, &n) ||
@@ -451,18 +489,26 @@ ssm_status ss2d_cross_merge(const void *ys, void *y, int64_t b, int64_t H, int64
     return fail(SSM_ERR_INVALID_ARG, "ss2d_cross_merge: bad sizes");
   if (dtype != SSM_F32 && dtype != SSM_BF16)
     return fail(SSM_ERR_UNSUPPORTED, "ss2d_cross_merge: unknown dtype %d", (int)dtype);
+  if (order != SSM_SS2D_CROSS && order != SSM_SS2D_SNAKE)
+    return fail(SSM_ERR_UNSUPPORTED, "ss2d_cross_merge: unknown scan order %d", (int)order);
   if (n == 0) return ok();
   if (!ys || !y) return fail(SSM_ERR_INVALID_ARG, "ss2d_cross_merge: NULL pointer");
   if (!aligned(ys, esize(dtype)) || !aligned(y, esize(dtype)))
     return fail(SSM_ERR_INVALID_ARG, "ss2d_cross_merge: misaligned pointer");
   const int64_t m = b * L * d_in;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto run = [&](auto tag, auto ord) {
+    using T = decltype(tag);
+    constexpr int O = decltype(ord)::value;
+    ssm::cross_merge_kernel<T, O><<<grid_for(m), 256, 0, st>>>(
+        static_cast<const T *>(ys), static_cast<T *>(y), b, H, W, d_in);
+  };
+  using Cross = std::integral_constant<int, ssm::kOrderCross>;
+  using Snake = std::integral_constant<int, ssm::kOrderSnake>;
   if (dtype == SSM_BF16)
-    ssm::cross_merge_kernel<__nv_bfloat16><<<grid_for(m), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16 *>(ys), static_cast<__nv_bfloat16 *>(y), b, H, W, d_in);
+    order == SSM_SS2D_SNAKE ? run(__nv_bfloat16(), Snake()) : run(__nv_bfloat16(), Cross());
   else
-    ssm::cross_merge_kernel<float><<<grid_for(m), 256, 0, st>>>(
-        static_cast<const float *>(ys), static_cast<float *>(y), b, H, W, d_in);
+    order == SSM_SS2D_SNAKE ? run(float(), Snake()) : run(float(), Cross());
   return check_launch("ss2d_cross_merge");
 }
 

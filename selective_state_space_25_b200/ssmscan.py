@@ -53,6 +53,13 @@ _lib.ss2d_cross_scan.argtypes = [_P, _P] + [_I64] * 4 + [_INT, _P]
 _lib.ss2d_cross_scan.restype = _INT
 _lib.ss2d_cross_merge.argtypes = [_P, _P] + [_I64] * 4 + [_INT, _P]
 _lib.ss2d_cross_merge.restype = _INT
+_lib.ss2d_scan_fwd_ex.argtypes = [_P] * 7 + [_INT, _P] + [_I64] * 5 + [_INT, _INT, _P, _SZ, _P]
+_lib.ss2d_scan_fwd_ex.restype = _INT
+_lib.ss2d_cross_scan_ex.argtypes = [_P, _P] + [_I64] * 4 + [_INT, _INT, _P]
+_lib.ss2d_cross_scan_ex.restype = _INT
+_lib.ss2d_cross_merge_ex.argtypes = [_P, _P] + [_I64] * 4 + [_INT, _INT, _P]
+_lib.ss2d_cross_merge_ex.restype = _INT
+SS2D_ORDERS = {"cross": 0, "snake": 1}
 _lib.ssm_check_device_errors.argtypes = [_P]
 _lib.ssm_check_device_errors.restype = _INT
 
@@ -166,10 +173,10 @@ def ss2d_scan_fwd_workspace_bytes(b: int, H: int, W: int, d_in: int, d_state: in
 
 
 def ss2d_scan_fwd(u, delta, A, B, C, H, W, D=None, dt_bias=None, delta_softplus=True, y=None,
-                  workspace=None, stream=None):
+                  workspace=None, stream=None, order="cross"):
     """SS2D forward.  u: (b, H W, d_in); delta: (b, 4, H W, d_in); A: (4 d_in, N)
-    fp32; B, C: (b, 4, H W, N); D, dt_bias: (4 d_in,) fp32.  Returns y
-    (b, H W, d_in)."""
+    fp32; B, C: (b, 4, H W, N); D, dt_bias: (4 d_in,) fp32; order "cross" or
+    "snake".  Returns y (b, H W, d_in)."""
     b, L, d_in = u.shape
     N = A.shape[-1]
     if L != H * W:
@@ -188,9 +195,9 @@ def ss2d_scan_fwd(u, delta, A, B, C, H, W, D=None, dt_bias=None, delta_softplus=
     ws_bytes = ss2d_scan_fwd_workspace_bytes(b, H, W, d_in, N)
     if workspace is None and ws_bytes > 0:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    st = _lib.ss2d_scan_fwd(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
-                            _ptr(dt_bias), int(bool(delta_softplus)), _ptr(y), b, H, W, d_in, N,
-                            _dtype_code(u), _ptr(workspace),
+    st = _lib.ss2d_scan_fwd_ex(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                               _ptr(dt_bias), int(bool(delta_softplus)), _ptr(y), b, H, W, d_in, N,
+                               SS2D_ORDERS[order], _dtype_code(u), _ptr(workspace),
                             0 if workspace is None else workspace.numel() * workspace.element_size(),
                             _stream(stream))
     _check(st, "ss2d_scan_fwd")
@@ -222,27 +229,27 @@ def ssm_state_update(ssm_state, x, dt, A, B, C, D=None, z=None, dt_bias=None, dt
     return y
 
 
-def ss2d_cross_scan(u, H, W, xs=None, stream=None):
+def ss2d_cross_scan(u, H, W, xs=None, stream=None, order="cross"):
     """xs[b, k, l, d] = u[b, p_k(l), d]; u (b, H W, d_in) -> xs (b, 4, H W, d_in)."""
     b, L, d_in = u.shape
     if xs is None:
         xs = torch.empty((b, 4, L, d_in), dtype=u.dtype, device=u.device)
     _need(u, "u", (b, L, d_in), u.dtype, u.device)
     _need(xs, "xs", (b, 4, L, d_in), u.dtype, u.device)
-    _check(_lib.ss2d_cross_scan(_ptr(u), _ptr(xs), b, H, W, d_in, _dtype_code(u), _stream(stream)),
-           "ss2d_cross_scan")
+    _check(_lib.ss2d_cross_scan_ex(_ptr(u), _ptr(xs), b, H, W, d_in, SS2D_ORDERS[order],
+                                   _dtype_code(u), _stream(stream)), "ss2d_cross_scan")
     return xs
 
 
-def ss2d_cross_merge(ys, H, W, y=None, stream=None):
+def ss2d_cross_merge(ys, H, W, y=None, stream=None, order="cross"):
     """y[b, p, d] = sum_k ys[b, k, l_k(p), d]; ys (b, 4, H W, d_in) -> y (b, H W, d_in)."""
     b, K, L, d_in = ys.shape
     if y is None:
         y = torch.empty((b, L, d_in), dtype=ys.dtype, device=ys.device)
     _need(ys, "ys", (b, 4, L, d_in), ys.dtype, ys.device)
     _need(y, "y", (b, L, d_in), ys.dtype, ys.device)
-    _check(_lib.ss2d_cross_merge(_ptr(ys), _ptr(y), b, H, W, d_in, _dtype_code(ys), _stream(stream)),
-           "ss2d_cross_merge")
+    _check(_lib.ss2d_cross_merge_ex(_ptr(ys), _ptr(y), b, H, W, d_in, SS2D_ORDERS[order],
+                                    _dtype_code(ys), _stream(stream)), "ss2d_cross_merge")
     return y
 
 

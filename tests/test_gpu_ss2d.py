@@ -115,3 +115,43 @@ def test_vmamba_ss2d_workload_sampled(ssm):
     ref = oracle_ss2d(ref_in, H, W)
     got = y[bsel][:, :, chans]
     assert rel_err(got, ref) <= 2e-2
+
+
+# ------------------------------------------------------------------ snake order
+@pytest.mark.parametrize("H,W", [(5, 7), (6, 4), (1, 9), (8, 1), (2, 3)])
+def test_snake_cross_scan_and_merge_bit_exact(ssm, H, W):
+    u = torch.randn(2, H * W, 8).to(torch.bfloat16)
+    xs = ssm.ss2d_cross_scan(u.cuda(), H, W, order="snake")
+    np.testing.assert_array_equal(to64(xs), oracle.cross_scan(u, H, W, order="snake"))
+    y = ssm.ss2d_cross_merge(xs, H, W, order="snake")
+    assert torch.equal(y.cpu(), 4 * u)
+    for k in range(4):                         # one direction at a time: exact inverse gather
+        ys = torch.zeros(2, 4, H * W, 8)
+        ys[:, k] = torch.randn(2, H * W, 8)
+        ym = ssm.ss2d_cross_merge(ys.cuda(), H, W, order="snake")
+        np.testing.assert_array_equal(to64(ym), oracle.cross_merge(ys, H, W, order="snake"))
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("b,H,W,d_in", [(2, 5, 7, 8), (1, 1, 40, 16), (1, 37, 1, 8),
+                                         (2, 16, 16, 24), (1, 56, 56, 16), (2, 9, 11, 12)])
+def test_ss2d_snake_shapes(ssm, dtype, b, H, W, d_in):
+    dt = "bf16" if dtype == torch.bfloat16 else "fp32"
+    inp = ss2d_inputs(b, H, W, d_in, 1, dt, seed=H * 31 + W, with_dt_bias=True)
+    g = to_cuda(inp)
+    y = ssm.ss2d_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], H, W, D=g["D"],
+                          dt_bias=g["dt_bias"], order="snake")
+    ref = oracle.ss2d_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], H, W,
+                           D=inp["D"], dt_bias=inp["dt_bias"], order="snake")
+    assert rel_err(y, ref) <= TOL[dtype]
+
+
+def test_ss2d_snake_large_image_workspace(ssm):
+    H, W = 79, 83
+    inp = ss2d_inputs(1, H, W, 8, 1, "bf16", seed=41)
+    g = to_cuda(inp)
+    y = ssm.ss2d_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], H, W, D=g["D"],
+                          order="snake")
+    ref = oracle.ss2d_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], H, W,
+                           D=inp["D"], order="snake")
+    assert rel_err(y, ref) <= 2e-2
