@@ -61,6 +61,8 @@ def _load():
         lib.oracle_cross_merge.restype = None
         lib.oracle_ss2d_scan.argtypes = [P] * 7 + [ctypes.c_int, P] + [I64] * 5 + [ctypes.c_int]
         lib.oracle_ss2d_scan.restype = ctypes.c_int
+        lib.oracle_conv_step.argtypes = [P] * 5 + [I64] * 3
+        lib.oracle_conv_step.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
@@ -140,6 +142,20 @@ def state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplu
                                 _ptr(D), _ptr(z), _ptr(dt_bias), int(bool(dt_softplus)),
                                 _ptr(y), b, d_in, N)
     return y, st
+
+
+def conv_step(conv_state, x, weight, bias=None):
+    """fp64 causal-conv1d decode step.  conv_state (b, d_in, d_conv) -- a NEW
+    array is returned, the argument is not modified; x (b, d_in); weight
+    (d_in, d_conv); bias (d_in).  Returns (x_out (b, d_in), new_conv_state)."""
+    cs = _f64(conv_state).copy()
+    b, d_in, d_conv = cs.shape
+    x = _f64(x, (b, d_in))
+    weight = _f64(weight, (d_in, d_conv))
+    bias = _f64(bias, (d_in,))
+    out = np.empty((b, d_in), np.float64)
+    _load().oracle_conv_step(_ptr(cs), _ptr(x), _ptr(weight), _ptr(bias), _ptr(out), b, d_in, d_conv)
+    return out, cs
 
 
 ORDERS = {"cross": 0, "snake": 1}

@@ -183,6 +183,33 @@ void oracle_state_update(double *state, const double *x, const double *dt,
 }
 
 /*
+ * Causal-conv1d decode step, [Mamba-step] "Conv step" without
+ * causal_conv1d_update: conv_state = roll(conv_state, -1) along the window,
+ * conv_state[..., -1] = x, x = sum(conv_state * weight, -1) + bias,
+ * x = act(x) with act = SiLU.  conv_state (b, d_in, d_conv) is updated in
+ * place; x, x_out are (b, d_in); weight is (d_in, d_conv); bias (d_in) is
+ * nullable.
+ */
+void oracle_conv_step(double *conv_state, const double *x, const double *weight,
+                      const double *bias, double *x_out, int64_t b, int64_t d_in,
+                      int64_t d_conv)
+{
+    int64_t bd;
+#pragma omp parallel for schedule(static)
+    for (bd = 0; bd < b * d_in; ++bd) {
+        const int64_t d = bd % d_in;
+        double *cs = &conv_state[bd * d_conv];
+        for (int64_t j = 0; j + 1 < d_conv; ++j)  /* roll left by one */
+            cs[j] = cs[j + 1];
+        cs[d_conv - 1] = x[bd];
+        double acc = bias ? bias[d] : 0.0;
+        for (int64_t j = 0; j < d_conv; ++j)
+            acc += cs[j] * weight[d * d_conv + j];
+        x_out[bd] = oracle_silu(acc);
+    }
+}
+
+/*
  * Pixel visited at step l of scan direction k on an H x W grid (pixels are
  * numbered row-major, p = h W + w).  [VMamba-206]: four orders, row-major,
  * column-major and both reversed (order 0, "cross"); the snake scan the

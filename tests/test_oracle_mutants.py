@@ -54,6 +54,12 @@ MUTANTS = {
                             "        const int64_t w = l / H;",
                             "int64_t h = l / W;           /* column-major: l = w H + h */\n"
                             "        const int64_t w = l % W;"),
+    # conv step: window not rolled (the newest value overwrites the last tap only)
+    "conv_no_roll": ("for (int64_t j = 0; j + 1 < d_conv; ++j)  /* roll left by one */",
+                     "for (int64_t j = 0; j + 1 < 0; ++j)  /* roll left by one */"),
+    # conv step: weight taps reversed
+    "conv_taps_reversed": ("acc += cs[j] * weight[d * d_conv + j];",
+                           "acc += cs[j] * weight[d * d_conv + d_conv - 1 - j];"),
     # SS2D snake: odd rows not flipped
     "ss2d_snake_rows_unflipped": ("if (order == 1 && h % 2 == 1)", "if (order == 1 && h % 2 == 7)"),
     # SS2D snake: even columns flipped instead of odd ones

@@ -436,3 +436,44 @@ def test_ss2d_snake_scan_is_four_1d_scans():
         yk = oracle.selective_scan(xs[:, k], delta[:, k], A[sl], B[:, k], C[:, k], D=D[sl])
         ref[:, perm[k].astype(int)] += yk       # step l of direction k lands on pixel perm[k][l]
     np.testing.assert_allclose(y, ref, rtol=1e-13, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# Causal-conv1d decode step ("代码连连看——mamba", Mamba.step(), Conv step):
+# roll the window left, append x, dot with the weight, add the bias, SiLU.
+# --------------------------------------------------------------------------
+def test_conv_step_one_hot_taps():
+    b, d_in, K = 2, 3, 4
+    cs = RNG.standard_normal((b, d_in, K))
+    x = RNG.standard_normal((b, d_in))
+    last = np.zeros((d_in, K)); last[:, -1] = 1.0        # newest tap only
+    out, new = oracle.conv_step(cs, x, last)
+    np.testing.assert_allclose(out, x / (1.0 + np.exp(-x)), rtol=1e-15)
+    np.testing.assert_array_equal(new[..., :-1], cs[..., 1:])   # rolled left by one
+    np.testing.assert_array_equal(new[..., -1], x)              # x appended
+    first = np.zeros((d_in, K)); first[:, 0] = 1.0       # oldest tap: the old second entry
+    out0, _ = oracle.conv_step(cs, x, first, bias=np.full(d_in, 0.25))
+    v = cs[..., 1] + 0.25
+    np.testing.assert_allclose(out0, v / (1.0 + np.exp(-v)), rtol=1e-15)
+
+
+@pytest.mark.parametrize("K", [2, 3, 4])
+def test_conv_steps_equal_causal_convolution(K):
+    """T decode steps from a zero window == a causal convolution of the
+    sequence with zero left padding, written with numpy.correlate."""
+    b, d_in, T = 2, 3, 11
+    xs = RNG.standard_normal((b, T, d_in))
+    w = RNG.standard_normal((d_in, K))
+    bias = RNG.standard_normal(d_in)
+    cs = np.zeros((b, d_in, K))
+    outs = []
+    for t in range(T):
+        o, cs = oracle.conv_step(cs, xs[:, t], w, bias)
+        outs.append(o)
+    got = np.stack(outs, 1)
+    for ib in range(b):
+        for d in range(d_in):
+            padded = np.concatenate([np.zeros(K - 1), xs[ib, :, d]])
+            pre = np.correlate(padded, w[d], mode="valid") + bias[d]   # sum_j w[j] x[t-K+1+j]
+            np.testing.assert_allclose(got[ib, :, d], pre / (1.0 + np.exp(-pre)), rtol=1e-12,
+                                       atol=1e-14)
