@@ -63,6 +63,9 @@ def _load():
         lib.oracle_ss2d_scan.restype = ctypes.c_int
         lib.oracle_conv_step.argtypes = [P] * 5 + [I64] * 3
         lib.oracle_conv_step.restype = None
+        lib.oracle_selective_scan_bwd.argtypes = ([P] * 8 + [ctypes.c_int] + [P] * 12
+                                                  + [I64] * 4)
+        lib.oracle_selective_scan_bwd.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
@@ -121,6 +124,41 @@ def selective_scan(u, delta, A, B, C, D=None, z=None, dt_bias=None,
                                   _ptr(D), _ptr(z), _ptr(dt_bias), int(bool(delta_softplus)),
                                   _ptr(h0), _ptr(h_last), _ptr(y), b, L, d_in, N)
     return (y, h_last) if return_last_state else y
+
+
+def selective_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None,
+                       delta_softplus=True, h0=None, dh_last=None):
+    """fp64 gradients of sum(dout * y) + sum(dh_last * h_last) for the scan
+    of ``selective_scan``.  Returns a dict with du, ddelta (b, L, d_in); dA
+    (d_in, N); dB, dC (b, L, N); dD, ddt_bias (d_in); dz (b, L, d_in, only
+    with z); dh0 (b, d_in, N)."""
+    u = _f64(u)
+    b, L, d_in = u.shape
+    A = _f64(A)
+    N = A.shape[1]
+    delta = _f64(delta, (b, L, d_in))
+    B = _f64(B, (b, L, N))
+    C = _f64(C, (b, L, N))
+    D = _f64(D, (d_in,))
+    z = _f64(z, (b, L, d_in))
+    dt_bias = _f64(dt_bias, (d_in,))
+    h0 = _f64(h0, (b, d_in, N))
+    dout = _f64(dout, (b, L, d_in))
+    dh_last = _f64(dh_last, (b, d_in, N))
+    g = dict(du=np.empty((b, L, d_in)), ddelta=np.empty((b, L, d_in)), dA=np.empty((d_in, N)),
+             dB=np.empty((b, L, N)), dC=np.empty((b, L, N)), dD=np.empty(d_in),
+             dz=np.empty((b, L, d_in)) if z is not None else None,
+             ddt_bias=np.empty(d_in), dh0=np.empty((b, d_in, N)))
+    rc = _load().oracle_selective_scan_bwd(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
+        int(bool(delta_softplus)), _ptr(h0), _ptr(dout), _ptr(dh_last),
+        _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]),
+        _ptr(g["dD"]), _ptr(g["dz"]), _ptr(g["ddt_bias"]), _ptr(g["dh0"]), b, L, d_in, N)
+    if rc != 0:
+        raise MemoryError("oracle.selective_scan_bwd: out of memory")
+    if z is None:
+        del g["dz"]
+    return g
 
 
 def state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True):

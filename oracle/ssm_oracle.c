@@ -309,3 +309,168 @@ int oracle_ss2d_scan(const double *u, const double *delta, const double *A,
     free(ys);
     return 0;
 }
+
+/* Derivative of oracle_softplus: the logistic sigmoid below the threshold,
+ * 1 above it (the linear branch). */
+static double oracle_softplus_grad(double x)
+{
+    if (x > 20.0)
+        return 1.0;
+    return 1.0 / (1.0 + exp(-x));
+}
+
+/*
+ * Backward of oracle_selective_scan: the gradients of
+ *     loss = sum_{i,t,d} dout[i,t,d] y[i,t,d] + sum_{i,d,n} dh_last[i,d,n] h_last[i,d,n]
+ * with respect to every input, by the chain rule applied to the forward
+ * recurrence above ([Minimal-scan] §3-§5 with the gate of [Mamba-step]),
+ * walked backwards in time.  "Fast backward" is what the VMamba discussion
+ * ([VMamba-206]) asks of a scan kernel; the gradient itself is the plain
+ * definition.  For one (batch, channel), with delta_t the softplus'd step,
+ * a_t[n] = exp(delta_t A[n]) and h_t the state after step t (h_{-1} = h0):
+ *
+ *   forward:   h_t = a_t h_{t-1} + delta_t B_t u_t,   yp_t = C_t.h_t + D u_t,
+ *              y_t = yp_t silu(z_t)
+ *   backward:  g_t = dout_t silu(z_t),   dz_t = dout_t yp_t silu'(z_t)
+ *              lam <- lam + g_t C_t                 (lam = d loss / d h_t)
+ *              dC_t += g_t h_t,  dD += g_t u_t,  du_t = g_t D
+ *              ddelta_t = sum_n lam (A a_t h_{t-1} + B_t u_t)
+ *              dA += lam delta_t a_t h_{t-1},  dB_t += lam delta_t u_t,
+ *              du_t += sum_n lam delta_t B_t
+ *              lam <- lam a_t                       (now d loss / d h_{t-1})
+ *   and at the end dh0 = lam.  The gradient of the raw delta input is
+ *   ddelta_t softplus'(delta + dt_bias) (or ddelta_t without softplus), and
+ *   ddt_bias is its sum over batch and time.
+ *
+ * dB, dC sum over the channels; dA, dD, ddt_bias over batch (and time).
+ * Outputs dz, dD, ddt_bias, dh0 may be NULL (not computed); dz is only
+ * written when z is given.  dh_last may be NULL (zero).  Batches run in
+ * parallel; the sums over batch are taken afterwards in batch order.
+ * Returns 0, or -1 when scratch memory could not be allocated.
+ */
+int oracle_selective_scan_bwd(const double *u, const double *delta,
+                              const double *A, const double *B, const double *C,
+                              const double *D, const double *z,
+                              const double *dt_bias, int delta_softplus,
+                              const double *h0, const double *dout,
+                              const double *dh_last,
+                              double *du, double *ddelta, double *dA,
+                              double *dB, double *dC, double *dD, double *dz,
+                              double *ddt_bias, double *dh0,
+                              int64_t b, int64_t L, int64_t d_in, int64_t N)
+{
+    /* per-batch partial sums of the per-channel gradients */
+    double *pA = (double *)calloc((size_t)(b * d_in * N + 1), sizeof(double));
+    double *pD = (double *)calloc((size_t)(b * d_in + 1), sizeof(double));
+    double *pbias = (double *)calloc((size_t)(b * d_in + 1), sizeof(double));
+    int failed = !pA || !pD || !pbias;
+    if (!failed) {
+        memset(dB, 0, (size_t)(b * L * N) * sizeof(double));
+        memset(dC, 0, (size_t)(b * L * N) * sizeof(double));
+    }
+
+    int64_t ib;
+#pragma omp parallel for schedule(dynamic, 1) reduction(|| : failed)
+    for (ib = 0; ib < b; ++ib) {
+        if (failed)
+            continue;
+        /* states after every step, plus h0 in front: hs[(t + 1) N + n] */
+        double *hs = (double *)malloc((size_t)((L + 1) * N + 1) * sizeof(double));
+        double *dts = (double *)malloc((size_t)(L + 1) * sizeof(double));
+        double *pre = (double *)malloc((size_t)(L + 1) * sizeof(double));
+        double *yp = (double *)malloc((size_t)(L + 1) * sizeof(double));
+        double *lam = (double *)malloc((size_t)(N + 1) * sizeof(double));
+        if (!hs || !dts || !pre || !yp || !lam) {
+            failed = 1;
+            free(hs); free(dts); free(pre); free(yp); free(lam);
+            continue;
+        }
+        for (int64_t d = 0; d < d_in; ++d) {
+            const int64_t bd = ib * d_in + d;
+            /* forward, keeping what the backward needs */
+            for (int64_t n = 0; n < N; ++n)
+                hs[n] = h0 ? h0[bd * N + n] : 0.0;
+            for (int64_t t = 0; t < L; ++t) {
+                const int64_t row = ib * L + t;
+                double x = delta[row * d_in + d];
+                if (dt_bias)
+                    x += dt_bias[d];
+                pre[t] = x;
+                dts[t] = delta_softplus ? oracle_softplus(x) : x;
+                const double ut = u[row * d_in + d];
+                double acc = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    const double a = exp(dts[t] * A[d * N + n]);
+                    hs[(t + 1) * N + n] = a * hs[t * N + n] + dts[t] * B[row * N + n] * ut;
+                    acc += hs[(t + 1) * N + n] * C[row * N + n];
+                }
+                if (D)
+                    acc += ut * D[d];
+                yp[t] = acc;
+            }
+            /* backward in time */
+            for (int64_t n = 0; n < N; ++n)
+                lam[n] = dh_last ? dh_last[bd * N + n] : 0.0;
+            for (int64_t t = L - 1; t >= 0; --t) {
+                const int64_t row = ib * L + t;
+                const int64_t at = row * d_in + d;
+                const double ut = u[at];
+                double g = dout[at];
+                if (z) {
+                    const double zt = z[at];
+                    const double s = 1.0 / (1.0 + exp(-zt));
+                    if (dz)
+                        dz[at] = g * yp[t] * s * (1.0 + zt * (1.0 - s));
+                    g *= zt * s;
+                }
+                if (D)
+                    pD[bd] += g * ut;
+                double dut = D ? g * D[d] : 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    lam[n] += g * C[row * N + n];
+                    dC[row * N + n] += g * hs[(t + 1) * N + n];
+                }
+                double ddt = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    const double a = exp(dts[t] * A[d * N + n]);
+                    const double hprev = hs[t * N + n];
+                    ddt += lam[n] * (A[d * N + n] * a * hprev + B[row * N + n] * ut);
+                    pA[bd * N + n] += lam[n] * dts[t] * a * hprev;
+                    dB[row * N + n] += lam[n] * dts[t] * ut;
+                    dut += lam[n] * dts[t] * B[row * N + n];
+                    lam[n] *= a;
+                }
+                if (delta_softplus)
+                    ddt *= oracle_softplus_grad(pre[t]);
+                du[at] = dut;
+                ddelta[at] = ddt;
+                pbias[bd] += ddt;
+            }
+            if (dh0)
+                for (int64_t n = 0; n < N; ++n)
+                    dh0[bd * N + n] = lam[n];
+        }
+        free(hs); free(dts); free(pre); free(yp); free(lam);
+    }
+    if (!failed) {
+        for (int64_t d = 0; d < d_in; ++d) {
+            for (int64_t n = 0; n < N; ++n) {
+                double s = 0.0;
+                for (int64_t i = 0; i < b; ++i)
+                    s += pA[(i * d_in + d) * N + n];
+                dA[d * N + n] = s;
+            }
+            double sD = 0.0, sb = 0.0;
+            for (int64_t i = 0; i < b; ++i) {
+                sD += pD[i * d_in + d];
+                sb += pbias[i * d_in + d];
+            }
+            if (dD)
+                dD[d] = sD;
+            if (ddt_bias)
+                ddt_bias[d] = sb;
+        }
+    }
+    free(pA); free(pD); free(pbias);
+    return failed ? -1 : 0;
+}

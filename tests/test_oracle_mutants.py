@@ -64,6 +64,20 @@ MUTANTS = {
     "ss2d_snake_rows_unflipped": ("if (order == 1 && h % 2 == 1)", "if (order == 1 && h % 2 == 7)"),
     # SS2D snake: even columns flipped instead of odd ones
     "ss2d_snake_cols_wrong_parity": ("if (order == 1 && w % 2 == 1)", "if (order == 1 && w % 2 == 0)"),
+    # backward: the adjoint is not decayed on its way to the previous step
+    "bwd_lam_no_decay": ("lam[n] *= a;", "lam[n] *= 1.0;"),
+    # backward: dB misses the step size
+    "bwd_dB_no_delta": ("dB[row * N + n] += lam[n] * dts[t] * ut;", "dB[row * N + n] += lam[n] * ut;"),
+    # backward: softplus derivative dropped from the delta gradient
+    "bwd_no_softplus_grad": ("ddt *= oracle_softplus_grad(pre[t]);", "ddt *= 1.0;"),
+    # backward: the decay gradient uses h_t instead of h_{t-1}
+    "bwd_hprev_off_by_one": ("const double hprev = hs[t * N + n];",
+                             "const double hprev = hs[(t + 1) * N + n];"),
+    # backward: wrong sign inside the SiLU derivative
+    "bwd_silu_grad_sign": ("s * (1.0 + zt * (1.0 - s))", "s * (1.0 - zt * (1.0 - s))"),
+    # backward: dC takes dout past the gate without the silu(z) factor
+    "bwd_C_grad_ungated": ("dC[row * N + n] += g * hs[(t + 1) * N + n];",
+                           "dC[row * N + n] += dout[at] * hs[(t + 1) * N + n];"),
 }
 
 

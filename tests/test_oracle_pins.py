@@ -477,3 +477,102 @@ def test_conv_steps_equal_causal_convolution(K):
             pre = np.correlate(padded, w[d], mode="valid") + bias[d]   # sum_j w[j] x[t-K+1+j]
             np.testing.assert_allclose(got[ib, :, d], pre / (1.0 + np.exp(-pre)), rtol=1e-12,
                                        atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# Backward scan: gradients of sum(dout * y) + sum(dh_last * h_last).
+# Pinned to central finite differences of the (separately pinned) forward
+# oracle, and to exact linearity identities that need no differencing.
+# --------------------------------------------------------------------------
+def _bwd_problem(rng, b=2, L=6, d_in=3, N=4, z=True, h0=True):
+    u, dt, A, B, C, D, zz, bias, hh = _rand_problem(b, L, d_in, N, rng, h0=h0, z=z)
+    bias = rng.uniform(-1.5, 0.5, size=d_in)       # softplus well inside its smooth branch
+    dout = rng.standard_normal((b, L, d_in))
+    dhl = rng.standard_normal((b, d_in, N))
+    return dict(u=u, delta=dt, A=A, B=B, C=C, D=D, z=zz, dt_bias=bias, h0=hh), dout, dhl
+
+
+def _loss(args, dout, dhl, softplus=True):
+    y, hl = oracle.selective_scan(args["u"], args["delta"], args["A"], args["B"], args["C"],
+                                  D=args["D"], z=args["z"], dt_bias=args["dt_bias"],
+                                  delta_softplus=softplus, h0=args["h0"], return_last_state=True)
+    return float(np.sum(dout * y) + np.sum(dhl * hl))
+
+
+_GRAD_OF = {"u": "du", "delta": "ddelta", "A": "dA", "B": "dB", "C": "dC", "D": "dD",
+            "z": "dz", "dt_bias": "ddt_bias", "h0": "dh0"}
+
+
+@pytest.mark.parametrize("softplus", [True, False])
+def test_bwd_matches_central_differences(softplus):
+    rng = np.random.default_rng(77 + softplus)
+    args, dout, dhl = _bwd_problem(rng)
+    if not softplus:
+        args["delta"] = np.abs(args["delta"]) * 0.3 + 0.05
+        args["dt_bias"] = rng.uniform(0.0, 0.1, size=args["dt_bias"].shape)
+    g = oracle.selective_scan_bwd(args["u"], args["delta"], args["A"], args["B"], args["C"], dout,
+                                  D=args["D"], z=args["z"], dt_bias=args["dt_bias"],
+                                  delta_softplus=softplus, h0=args["h0"], dh_last=dhl)
+    eps = 1e-6
+    for name, gname in _GRAD_OF.items():
+        x = args[name]
+        fd = np.empty_like(x)
+        for idx in np.ndindex(x.shape):
+            keep = x[idx]
+            x[idx] = keep + eps
+            fp = _loss(args, dout, dhl, softplus)
+            x[idx] = keep - eps
+            fm = _loss(args, dout, dhl, softplus)
+            x[idx] = keep
+            fd[idx] = (fp - fm) / (2 * eps)
+        scale = max(1.0, float(np.max(np.abs(fd))))
+        np.testing.assert_allclose(g[gname], fd, rtol=0, atol=2e-7 * scale, err_msg=name)
+
+
+def test_bwd_linearity_identities():
+    """Exact identities (no differencing).  Without the gate, y and h_last
+    are jointly linear in (u, h0), in C, and -- with h0 = 0 -- the scan part
+    is linear in B, so the loss equals the gradient's inner product with the
+    argument (Euler's theorem for degree-1 homogeneous functions)."""
+    rng = np.random.default_rng(5)
+    args, dout, dhl = _bwd_problem(rng, b=3, L=11, d_in=4, N=5, z=False)
+    call = lambda a, dh: oracle.selective_scan_bwd(
+        a["u"], a["delta"], a["A"], a["B"], a["C"], dout, D=a["D"], dt_bias=a["dt_bias"],
+        h0=a["h0"], dh_last=dh)
+    y, hl = oracle.selective_scan(args["u"], args["delta"], args["A"], args["B"], args["C"],
+                                  D=args["D"], dt_bias=args["dt_bias"], h0=args["h0"],
+                                  return_last_state=True)
+    g = call(args, dhl)
+    F = np.sum(dout * y) + np.sum(dhl * hl)
+    assert np.sum(g["du"] * args["u"]) + np.sum(g["dh0"] * args["h0"]) == pytest.approx(F, rel=1e-12)
+    Dterm = np.sum(dout * args["u"] * args["D"][None, None, :])
+    assert np.sum(g["dC"] * args["C"]) == pytest.approx(np.sum(dout * y) - Dterm, rel=1e-12)
+    assert np.sum(g["dD"] * args["D"]) == pytest.approx(Dterm, rel=1e-12)
+    args["h0"] = None
+    y0, hl0 = oracle.selective_scan(args["u"], args["delta"], args["A"], args["B"], args["C"],
+                                    D=args["D"], dt_bias=args["dt_bias"], return_last_state=True)
+    g0 = call(args, dhl)
+    assert np.sum(g0["dB"] * args["B"]) == pytest.approx(
+        np.sum(dout * y0) - Dterm + np.sum(dhl * hl0), rel=1e-12)
+    assert np.all(g0["dh0"] == g["dh0"])     # dh0 does not depend on h0
+
+
+def test_bwd_L1_closed_form():
+    """One step from h0 with a scalar decay: every gradient by hand."""
+    u, dt, A, B, C, D, h0 = 0.7, -0.3, -2.0, 1.5, -0.8, 0.4, 0.9
+    dout, dhl = 1.3, -0.6
+    delta = _softplus_ref(dt)
+    a = math.exp(delta * A)
+    h = a * h0 + delta * B * u
+    lam = dout * C + dhl                           # d loss / d h
+    g = oracle.selective_scan_bwd(np.full((1, 1, 1), u), np.full((1, 1, 1), dt),
+                                  np.full((1, 1), A), np.full((1, 1, 1), B),
+                                  np.full((1, 1, 1), C), np.full((1, 1, 1), dout),
+                                  D=np.full(1, D), h0=np.full((1, 1, 1), h0),
+                                  dh_last=np.full((1, 1, 1), dhl))
+    sig = 1.0 / (1.0 + math.exp(-dt))
+    exp = dict(du=dout * D + lam * delta * B, dC=dout * h, dD=dout * u, dB=lam * delta * u,
+               dA=lam * delta * a * h0, dh0=lam * a,
+               ddelta=lam * (A * a * h0 + B * u) * sig)
+    for k, v in exp.items():
+        assert float(g[k].ravel()[0]) == pytest.approx(v, rel=1e-13, abs=1e-15), k
