@@ -423,8 +423,7 @@ int oracle_selective_scan_bwd(const double *u, const double *delta,
                         dz[at] = g * yp[t] * s * (1.0 + zt * (1.0 - s));
                     g *= zt * s;
                 }
-                if (D)
-                    pD[bd] += g * ut;
+                pD[bd] += g * ut;          /* defined at D = 0 when D is absent */
                 double dut = D ? g * D[d] : 0.0;
                 for (int64_t n = 0; n < N; ++n) {
                     lam[n] += g * C[row * N + n];

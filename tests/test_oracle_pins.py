@@ -576,3 +576,18 @@ def test_bwd_L1_closed_form():
                ddelta=lam * (A * a * h0 + B * u) * sig)
     for k, v in exp.items():
         assert float(g[k].ravel()[0]) == pytest.approx(v, rel=1e-13, abs=1e-15), k
+
+
+def test_bwd_absent_D_is_D_zero():
+    """Without D (and without dt_bias) the gradients are those at D = 0 (and
+    bias = 0): dD and ddt_bias are still defined and equal the explicit-zero
+    case exactly."""
+    rng = np.random.default_rng(8)
+    args, dout, dhl = _bwd_problem(rng, b=2, L=9, d_in=3, N=4)
+    base = dict(u=args["u"], delta=args["delta"], A=args["A"], B=args["B"], C=args["C"], dout=dout,
+                z=args["z"], h0=args["h0"], dh_last=dhl)
+    g_none = oracle.selective_scan_bwd(**base)
+    g_zero = oracle.selective_scan_bwd(**base, D=np.zeros(3), dt_bias=np.zeros(3))
+    for k in g_zero:
+        np.testing.assert_array_equal(g_none[k], g_zero[k], err_msg=k)
+    assert np.any(g_none["dD"] != 0)
