@@ -10,7 +10,8 @@ prefill scan (b=8, L=2048, d_in=1536, N=16, bf16 activations, fp32 state):
 the configuration the headline metric (Gelem/s = b L d_in N per second, and
 HBM GB/s as a fraction of the measured peak) is quoted on.  Other workloads
 (--workload mamba1.4b-long-scan | vmamba-ss2d | mamba-decode-step |
-tiny-fp32-scan) measure the companion kernels.
+mamba-decode-conv-step | mamba130m-scan-bwd | tiny-fp32-scan) measure the
+companion kernels.
 
 Timing: W untimed warm-up steps, then exactly K timed steps bracketed by a
 barrier and torch.cuda.synchronize() on both sides; each step's kernel is
@@ -74,11 +75,19 @@ def alg_bytes(w) -> int:
     if w.kind == "scan":
         b, L, di, N = d["b"], d["L"], d["d_in"], d["N"]
         return 4 * b * L * di * es + 2 * b * L * N * es + di * N * 4 + 2 * di * 4
+    if w.kind == "scan_bwd":
+        # read u, delta, z, dout, B, C, A, D, dt_bias; write du, ddelta, dz,
+        # dB, dC (fp32), dA, dD, ddt_bias (fp32)
+        b, L, di, N = d["b"], d["L"], d["d_in"], d["N"]
+        return (7 * b * L * di * es + 2 * b * L * N * es + 2 * b * L * N * 4
+                + 2 * (di * N * 4 + 2 * di * 4))
     if w.kind == "ss2d":
         b, L, di, N = d["b"], d["H"] * d["W"], d["d_in"], d["N"]
         return 2 * b * L * di * es + b * 4 * L * di * es + 2 * b * 4 * L * N * es + 4 * di * (N + 1) * 4
     b, di, N = d["b"], d["d_in"], d["N"]
-    return 2 * b * di * N * 4 + 4 * b * di * es + 2 * b * N * es + di * N * 4 + 2 * di * 4
+    step = 2 * b * di * N * 4 + 4 * b * di * es + 2 * b * N * es + di * N * 4 + 2 * di * 4
+    K = d.get("d_conv", 0)           # window read + written, depthwise weight and bias read
+    return step + (2 * b * di * K * es + di * K * 4 + di * 4 if K else 0)
 
 
 def alu_peak_elems_per_s(w) -> float:
@@ -95,6 +104,11 @@ def alu_peak_elems_per_s(w) -> float:
     N = w.dims["N"]
     if w.kind == "ss2d":
         X, F = 3.0, 12.0
+    elif w.kind == "scan_bwd":
+        # three passes over each element (chunk states, recompute, adjoint):
+        # 3 exps and ~18 FMA-pipe ops; per (t, d) softplus twice, its
+        # derivative once and the gate's SiLU and derivative (8 / N)
+        X, F = 3.0 + 8.0 / N, 18.0
     else:
         X, F = 1.0 + 4.0 / N, 4.0
     P = 8.0
@@ -213,14 +227,30 @@ def build_step(S, w, dev_in):
         fn = lambda: S.ss2d_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], d["H"], d["W"],
                                      D=g["D"], dt_bias=g["dt_bias"], y=y)
         return fn, y
+    if w.kind == "scan_bwd":
+        out = S.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["dout"], D=g["D"],
+                             z=g["z"], dt_bias=g["dt_bias"])
+        ws = torch.empty(S.ssm_scan_bwd_workspace_bytes(d["b"], d["L"], d["d_in"], d["N"]),
+                         dtype=torch.uint8, device=g["u"].device)
+        fn = lambda: S.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["dout"], D=g["D"],
+                                    z=g["z"], dt_bias=g["dt_bias"], workspace=ws, out=out)
+        return fn, list(out.values())
     y = torch.empty_like(g["x"])
+    if "conv_state" in g:
+        fn = lambda: S.ssm_conv_state_update(g["conv_state"], g["conv_weight"], g["state"], g["x"],
+                                             g["dt"], g["A"], g["B"], g["C"],
+                                             conv_bias=g["conv_bias"], D=g["D"], z=g["z"],
+                                             dt_bias=g["dt_bias"], y=y)
+        return fn, y
     fn = lambda: S.ssm_state_update(g["state"], g["x"], g["dt"], g["A"], g["B"], g["C"], D=g["D"],
                                     z=g["z"], dt_bias=g["dt_bias"], y=y)
     return fn, y
 
 
 def default_steps(w) -> int:
-    return {"scan": 200, "ss2d": 300, "step": 1000}[w.kind] if w.name != "mamba1.4b-long-scan" else 60
+    if w.name == "mamba1.4b-long-scan":
+        return 60
+    return {"scan": 200, "scan_bwd": 60, "ss2d": 300, "step": 1000}[w.kind]
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -235,7 +265,15 @@ def oracle_sample(w, inp, target_s: float):
 
     def run(nch):
         t0 = time.perf_counter()
-        if w.kind == "scan":
+        if w.kind == "scan_bwd":
+            sl = lambda t: t[:, :, :nch].contiguous()
+            oracle.selective_scan_bwd(sl(inp["u"]), sl(inp["delta"]), inp["A"][:nch], inp["B"],
+                                      inp["C"], sl(inp["dout"]), D=inp["D"][:nch], z=sl(inp["z"]),
+                                      dt_bias=inp["dt_bias"][:nch])
+            el = d["b"] * d["L"] * nch * d["N"]
+            desc = (f"backward, all {d['b']} batches x full L={d['L']} x first {nch} of "
+                    f"{d['d_in']} channels")
+        elif w.kind == "scan":
             sl = lambda t: t[:, :, :nch].contiguous()
             oracle.selective_scan(sl(inp["u"]), sl(inp["delta"]), inp["A"][:nch], inp["B"], inp["C"],
                                   D=inp["D"][:nch], z=sl(inp["z"]), dt_bias=inp["dt_bias"][:nch])
@@ -249,7 +287,11 @@ def oracle_sample(w, inp, target_s: float):
             desc = f"all {d['b']} images x 4 directions x first {nch} of {d['d_in']} channels"
         else:
             sl = lambda t: t[:, :nch].contiguous()
-            oracle.state_update(inp["state"][:, :nch].contiguous(), sl(inp["x"]), sl(inp["dt"]),
+            x = sl(inp["x"])
+            if "conv_state" in inp:
+                x, _ = oracle.conv_step(inp["conv_state"][:, :nch].contiguous(), x,
+                                        inp["conv_weight"][:nch], inp["conv_bias"][:nch])
+            oracle.state_update(inp["state"][:, :nch].contiguous(), x, sl(inp["dt"]),
                                 inp["A"][:nch], inp["B"], inp["C"], D=inp["D"][:nch], z=sl(inp["z"]),
                                 dt_bias=inp["dt_bias"][:nch])
             el = d["b"] * nch * d["N"]
@@ -437,20 +479,23 @@ def run_e2e(S, w, host, dev, K, W):
     dbuf = {k: (torch.empty_like(v, device=dev) if isinstance(v, torch.Tensor) else v)
             for k, v in host.items()}
     step, y = build_step(S, w, dbuf)
-    y_host = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
-    skip = {"state"} if w.kind == "step" else set()     # the decode state lives on the GPU
+    ys = y if isinstance(y, list) else [y]
+    y_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in ys]
+    skip = {"state", "conv_state"} if w.kind == "step" else set()   # decode states live on the GPU
+    skip &= pinned.keys()
     for k in skip:
         dbuf[k].copy_(pinned[k])
     h2d = sum(v.numel() * v.element_size() for k, v in pinned.items()
               if isinstance(v, torch.Tensor) and k not in skip)
-    d2h = y.numel() * y.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in ys)
 
     def one():
         for k, v in pinned.items():
             if isinstance(v, torch.Tensor) and k not in skip:
                 dbuf[k].copy_(v, non_blocking=True)
         step()
-        y_host.copy_(y, non_blocking=True)
+        for hb, t in zip(y_host, ys):
+            hb.copy_(t, non_blocking=True)
 
     for _ in range(W):
         one()

@@ -19,6 +19,11 @@
  *                     the SSM step: softplus(dt + bias), dA = exp(dt A),
  *                     dB = dt B, state = state dA + x dB (in place),
  *                     y = state.C + D x, y * act(z)).
+ *   ssm_scan_bwd      the gradients of ssm_scan_fwd by the reverse-time
+ *                     adjoint of its recurrence (same passages).
+ *   ssm_conv_state_update  the same step with the depthwise causal-conv1d
+ *                     step of Mamba.step() in front of it (roll conv_state
+ *                     left, append x, sum conv_state * weight + bias, SiLU).
  *
  * Conventions for every entry point:
  *   - Pointers marked "device" point to device memory of the current CUDA
@@ -107,6 +112,60 @@ ssm_status ssm_scan_fwd(const void *u, const void *delta, const float *A,
                         const void *B, const void *C, const float *D,
                         const void *z, const float *dt_bias, int delta_softplus,
                         const float *h0, float *h_last, void *y,
+                        int64_t b, int64_t L, int64_t d_in, int64_t d_state,
+                        ssm_dtype dtype, void *workspace, size_t workspace_bytes,
+                        ssm_stream_t stream);
+
+/*
+ * Workspace of ssm_scan_bwd: the state at the start of every 16-step chunk
+ * of the sequence, fp32: b * ceil(L / 16) * d_in * d_state * 4 bytes.
+ * Returns (size_t)-1 for invalid sizes.
+ */
+size_t ssm_scan_bwd_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t d_state);
+
+/*
+ * Selective scan backward: the gradients of
+ *     loss = sum dout[i,t,d] out[i,t,d] + sum dh_last[i,d,n] h_last[i,d,n]
+ * for the forward of ssm_scan_fwd with the same inputs, by the chain rule
+ * through its recurrence ("手把手拆解Mamba-minimal中的selective_scan实现"
+ * §3-§5 and the gate of "代码连连看——mamba", Mamba.step()), walked backwards
+ * in time.  With delta_t = softplus(dt_t + dt_bias), a_t = exp(delta_t A),
+ * g_t = dout_t silu(z_t), lam = d loss / d h_t:
+ *     lam += g_t C_t;  dC_t += g_t h_t;  dD += g_t u_t
+ *     ddelta_t = softplus'(dt_t + dt_bias) sum_n lam (A a_t h_{t-1} + B_t u_t)
+ *     dA += lam delta_t a_t h_{t-1};  dB_t += lam delta_t u_t
+ *     du_t = g_t D + delta_t sum_n lam B_t;  lam *= a_t
+ *     dz_t = dout_t (C_t.h_t + D u_t) silu'(z_t);  dh0 = lam after step 0
+ * softplus' is the logistic sigmoid, and 1 above the threshold 20.
+ * The forward states are recomputed from h0 inside the call (nothing from
+ * ssm_scan_fwd is kept).
+ *
+ *   inputs        exactly those of ssm_scan_fwd (u, delta, A, B, C, D, z,
+ *                 dt_bias, delta_softplus, h0), plus
+ *   dout          device, (b, L, d_in), dtype: gradient of the output y
+ *   dh_last       device fp32 (b, d_in, d_state), nullable (zero)
+ *   du, ddelta    device, (b, L, d_in), dtype (ddelta is the gradient of
+ *                 the raw delta input, before bias and softplus)
+ *   dz            device, (b, L, d_in), dtype, nullable; written only when
+ *                 z is given
+ *   dA            device fp32 (d_in, d_state), required (summed over b, L)
+ *   dB, dC        device fp32 (b, L, d_state) (summed over d_in)
+ *   dD, ddt_bias  device fp32 (d_in), nullable (summed over b, L); dD is
+ *                 the gradient at the given D (0 when D is NULL)
+ *   dh0           device fp32 (b, d_in, d_state), nullable
+ *   workspace     device, >= ssm_scan_bwd_workspace_bytes(...) bytes;
+ *                 contents on entry are ignored
+ * Every output is overwritten (the summed ones are zeroed on the stream
+ * first); outputs must not alias inputs or each other.  b <= 65535.
+ * Arithmetic is fp32; the sums over channels and batch are taken with fp32
+ * atomics, so their rounding order varies from run to run.
+ */
+ssm_status ssm_scan_bwd(const void *u, const void *delta, const float *A,
+                        const void *B, const void *C, const float *D,
+                        const void *z, const float *dt_bias, int delta_softplus,
+                        const float *h0, const void *dout, const float *dh_last,
+                        void *du, void *ddelta, float *dA, float *dB, float *dC,
+                        float *dD, void *dz, float *ddt_bias, float *dh0,
                         int64_t b, int64_t L, int64_t d_in, int64_t d_state,
                         ssm_dtype dtype, void *workspace, size_t workspace_bytes,
                         ssm_stream_t stream);
@@ -212,6 +271,33 @@ ssm_status ssm_state_update(float *ssm_state, const void *x, const void *dt,
                             const float *D, const void *z, const float *dt_bias,
                             int dt_softplus, void *y, int64_t b, int64_t d_in,
                             int64_t d_state, ssm_dtype dtype, ssm_stream_t stream);
+
+/*
+ * One-token decode step with the depthwise causal conv1d of Mamba.step()
+ * ("代码连连看——mamba", the conv step: the window is rolled one place left,
+ * x goes into its last slot, x_conv = sum_j window[j] * weight[d, j] + bias,
+ * then SiLU) fused in front of the state update above:
+ *     w'[i,d,j] = w[i,d,j+1] (j < d_conv-1),  w'[i,d,d_conv-1] = x[i,d]
+ *     xc[i,d]   = silu(sum_j w'[i,d,j] * conv_weight[d,j] + conv_bias[d])
+ *     then ssm_state_update with x replaced by xc (D multiplies xc too).
+ * xc stays in fp32 between the two steps (it is not rounded to dtype).
+ *
+ *   conv_state    device, (b, d_in, d_conv), dtype, read and written in place
+ *                 (the new window w'); must not alias another argument
+ *   conv_weight   device fp32 (d_in, d_conv): the depthwise kernel, tap j
+ *                 multiplying the j-th oldest entry of the window
+ *   conv_bias     device fp32 (d_in), nullable
+ *   d_conv        1 .. 8, else SSM_ERR_UNSUPPORTED
+ *   x             device, (b, d_in), dtype: the raw (pre-conv) input
+ *   every other argument as for ssm_state_update
+ */
+ssm_status ssm_conv_state_update(void *conv_state, const float *conv_weight,
+                                 const float *conv_bias, int64_t d_conv,
+                                 float *ssm_state, const void *x, const void *dt,
+                                 const float *A, const void *B, const void *C,
+                                 const float *D, const void *z, const float *dt_bias,
+                                 int dt_softplus, void *y, int64_t b, int64_t d_in,
+                                 int64_t d_state, ssm_dtype dtype, ssm_stream_t stream);
 
 /*
  * CrossScan as a stored permutation, for checking the index arithmetic of

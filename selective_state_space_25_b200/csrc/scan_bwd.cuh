@@ -1,0 +1,389 @@
+// scan_bwd.cuh -- backward of the selective scan: the reverse-time adjoint
+// of the recurrence of "手把手拆解Mamba-minimal中的selective_scan实现" §3-§5
+// with the gate of "代码连连看——mamba" (Mamba.step()); the fast backward
+// the VMamba discussion ("关于代码SS2D中的d_state设置") asks of a scan kernel.
+//
+// For one (batch, channel), with delta_t = softplus(dt_t + bias),
+// a_t = exp(delta_t A) and h_t the state after step t:
+//     lam   <- lam + g_t C_t                   g_t = dout_t silu(z_t)
+//     dC_t  += g_t h_t          dD += g_t u_t   dz_t = dout_t yp_t silu'(z_t)
+//     ddelta_t = softplus'(.) (sum_n A lam a_t h_{t-1} + u_t sum_n lam B_t)
+//     dA    += lam delta_t a_t h_{t-1}
+//     dB_t  += lam delta_t u_t  du_t = g_t D + delta_t sum_n lam B_t
+//     lam   <- lam a_t                          (dh0 = lam at the end)
+//
+// One CTA owns DT channels of one batch for the whole sequence; G = N / NPT
+// threads share a channel, NPT states each.
+//   pass 1  walks the sequence forwards and saves the state at the start of
+//           every TT-step chunk in the caller's workspace;
+//   pass 2  walks the chunks backwards.  Per chunk: recompute the states
+//           from the saved start into shared memory (with each thread's
+//           partial C.h); dC_t = sum over channels of g_t h_t as a column
+//           pass over those states; the adjoint, which overwrites each
+//           state row with lam_t and leaves each thread's partial sums of
+//           lam B and A lam a h_{t-1}; dB_t = sum over channels of
+//           lam_t delta_t u_t as a second column pass; and a pass per
+//           (step, channel) that adds the G partials and writes du, ddelta
+//           and dz.
+// Nothing in the per-step loops crosses lanes, so each step's critical
+// path is the adjoint's own FMA chain.  dB and dC rows of the chunk go to
+// the fp32 outputs with (vector) global atomics, one per CTA and row;
+// dA, dD and ddt_bias are added once per CTA at the end.
+#pragma once
+
+#include "ssm_common.cuh"
+
+namespace ssm {
+
+struct BwdParams {
+  const void *u, *delta;
+  const float *A;
+  const void *B, *C;
+  const float *D;
+  const void *z;
+  const float *dt_bias;
+  const float *h0;
+  const void *dout;
+  const float *dh_last;
+  void *du, *ddelta, *dz;
+  float *dA, *dB, *dC, *dD, *ddt_bias, *dh0;
+  float *chunk_h;  // workspace (b, n_chunks, d_in, N) fp32
+  int64_t b, L, d_in;
+  int softplus;
+  int vec_atomics;  // dB and dC 16-byte aligned: float4 atomics
+};
+
+template <int N>
+struct BwdCfg {
+  static constexpr int NPT = N < 4 ? N : 4;  // states per thread
+  static constexpr int G = N / NPT;          // threads per channel
+  static constexpr int THREADS = 128;
+  static constexpr int DT = THREADS / G;     // channels per CTA
+  static constexpr int TT = 16;              // steps per chunk
+  static constexpr int PROW = DT + 1;        // plane row (padded: column reads hit distinct banks)
+  static constexpr int PL = TT * PROW;       // one (step, channel) plane
+  static constexpr int HROW = THREADS * NPT + (NPT == 4 ? 16 : 0);  // state row, padded
+  // planes: delta, u, g, dz factor, softplus'
+  static constexpr int OFF_B = 5 * PL;
+  static constexpr int OFF_C = OFF_B + TT * N;
+  static constexpr int OFF_P1 = OFF_C + TT * N;      // partial sum_n lam B       [t][thread]
+  static constexpr int OFF_P2 = OFF_P1 + TT * THREADS;  // partial sum_n A lam a h  [t][thread]
+  static constexpr int OFF_PY = OFF_P2 + TT * THREADS;  // partial C.h              [t][thread]
+  static constexpr int OFF_H = OFF_PY + TT * THREADS;   // states, then adjoints     [t][thread][NPT]
+  static constexpr int FLOATS = OFF_H + TT * HROW;
+  static constexpr size_t SMEM = FLOATS * sizeof(float);
+  static_assert(OFF_H % 4 == 0 && HROW % 4 == 0, "state rows must be 16-byte aligned");
+  static_assert(G >= 1 && G <= 32 && 32 % G == 0 && THREADS % DT == 0, "bad N");
+};
+
+template <int NPT>
+__device__ __forceinline__ void load_vec(const float *s, float (&v)[NPT]) {
+  if constexpr (NPT == 4) {
+    const float4 w = *reinterpret_cast<const float4 *>(s);
+    v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w;
+  } else if constexpr (NPT == 2) {
+    const float2 w = *reinterpret_cast<const float2 *>(s);
+    v[0] = w.x; v[1] = w.y;
+  } else {
+#pragma unroll
+    for (int j = 0; j < NPT; ++j) v[j] = s[j];
+  }
+}
+
+template <int NPT>
+__device__ __forceinline__ void store_vec(float *s, const float (&v)[NPT]) {
+  if constexpr (NPT == 4) {
+    *reinterpret_cast<float4 *>(s) = make_float4(v[0], v[1], v[2], v[3]);
+  } else if constexpr (NPT == 2) {
+    *reinterpret_cast<float2 *>(s) = make_float2(v[0], v[1]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < NPT; ++j) s[j] = v[j];
+  }
+}
+
+// Sum of the G consecutive partials starting at s.
+template <int G>
+__device__ __forceinline__ float sum_partials(const float *s) {
+  float acc = 0.0f;
+  if constexpr (G % 4 == 0) {
+#pragma unroll
+    for (int k = 0; k < G; k += 4) {
+      const float4 w = *reinterpret_cast<const float4 *>(s + k);
+      acc += (w.x + w.y) + (w.z + w.w);
+    }
+  } else if constexpr (G == 2) {
+    const float2 w = *reinterpret_cast<const float2 *>(s);
+    acc = w.x + w.y;
+  } else {
+    acc = s[0];
+  }
+  return acc;
+}
+
+template <typename T, int N>
+__global__ void __launch_bounds__(128) scan_bwd_kernel(BwdParams p) {
+  using Cfg = BwdCfg<N>;
+  constexpr int NPT = Cfg::NPT, G = Cfg::G, DT = Cfg::DT, TT = Cfg::TT, NT = Cfg::THREADS;
+  constexpr int PROW = Cfg::PROW, PL = Cfg::PL, HROW = Cfg::HROW;
+  extern __shared__ float4 bwd_smem4[];
+  float *sm = reinterpret_cast<float *>(bwd_smem4);
+  float *sDelta = sm, *sU = sm + PL, *sG = sm + 2 * PL, *sDzf = sm + 3 * PL, *sSpg = sm + 4 * PL;
+  float *sB = sm + Cfg::OFF_B, *sC = sm + Cfg::OFF_C;
+  float *sP1 = sm + Cfg::OFF_P1, *sP2 = sm + Cfg::OFF_P2, *sPy = sm + Cfg::OFF_PY;
+  float *sH = sm + Cfg::OFF_H;
+
+  const int tid = threadIdx.x;
+  const int ch = tid / G, g = tid - (tid / G) * G;
+  const int64_t ib = blockIdx.y;
+  const int64_t d0 = (int64_t)blockIdx.x * DT;
+  const int64_t d = d0 + ch;
+  const bool active = d < p.d_in;
+  const int64_t L = p.L, d_in = p.d_in;
+  const int nC = (int)((L + TT - 1) / TT);
+  const T *gu = static_cast<const T *>(p.u);
+  const T *gdelta = static_cast<const T *>(p.delta);
+  const T *gB = static_cast<const T *>(p.B);
+  const T *gC = static_cast<const T *>(p.C);
+  const T *gz = static_cast<const T *>(p.z);
+  const T *gdout = static_cast<const T *>(p.dout);
+
+  float Av[NPT], A2[NPT];
+#pragma unroll
+  for (int j = 0; j < NPT; ++j) {
+    Av[j] = active ? p.A[d * N + g * NPT + j] : 0.0f;
+    A2[j] = Av[j] * kLog2e;
+  }
+
+  // Chunk c's (step, channel) inputs into the planes; with `full` also the
+  // gate terms and C.  Rows past the sequence and channels past d_in are 0.
+  auto stage = [&](int c, bool full) {
+    const int64_t t0 = (int64_t)c * TT;
+    const int nT = (int)(L - t0 < TT ? L - t0 : TT);
+    for (int i = tid; i < TT * DT; i += NT) {
+      const int t = i / DT, cc = i - t * DT;
+      const int64_t dd = d0 + cc;
+      float dl = 0.0f, uu = 0.0f, gg = 0.0f, dzf = 0.0f, spg = 0.0f;
+      if (t < nT && dd < d_in) {
+        const int64_t at = (ib * L + t0 + t) * d_in + dd;
+        const float pre = Elem<T>::load(gdelta, at) + (p.dt_bias ? p.dt_bias[dd] : 0.0f);
+        uu = Elem<T>::load(gu, at);
+        if (p.softplus) {
+          dl = softplus_f32(pre);
+          if (full) spg = pre > 20.0f ? 1.0f : rcp_approx(1.0f + ex2_approx(-pre * kLog2e));
+        } else {
+          dl = pre;
+          spg = 1.0f;
+        }
+        if (full) {
+          const float go = Elem<T>::load(gdout, at);
+          if (gz) {
+            const float zz = Elem<T>::load(gz, at);
+            const float sg = rcp_approx(1.0f + ex2_approx(-zz * kLog2e));
+            gg = go * zz * sg;
+            dzf = go * sg * fmaf(zz, 1.0f - sg, 1.0f);
+          } else {
+            gg = go;
+          }
+        }
+      }
+      const int s = t * PROW + cc;
+      sDelta[s] = dl;
+      sU[s] = uu;
+      if (full) {
+        sG[s] = gg;
+        sDzf[s] = dzf;
+        sSpg[s] = spg;
+      }
+    }
+    for (int i = tid; i < TT * N; i += NT) {
+      const int t = i / N;
+      const int64_t row = (ib * L + t0 + t) * N + (i - t * N);
+      sB[i] = t < nT ? Elem<T>::load(gB, row) : 0.0f;
+      if (full) sC[i] = t < nT ? Elem<T>::load(gC, row) : 0.0f;
+    }
+    return nT;
+  };
+
+  float *my_chunk_h = p.chunk_h + ((ib * nC) * d_in + d) * N + g * NPT;  // + c * d_in * N
+  float h[NPT];
+
+  // one forward step of this thread's states (pass 1 and the recompute)
+  auto fwd_step = [&](int t) -> float {
+    const float dl = sDelta[t * PROW + ch];
+    const float du = dl * sU[t * PROW + ch];
+    float bv[NPT], cv[NPT];
+    load_vec<NPT>(sB + t * N + g * NPT, bv);
+    load_vec<NPT>(sC + t * N + g * NPT, cv);
+    float yp = 0.0f;
+#pragma unroll
+    for (int j = 0; j < NPT; ++j) {
+      h[j] = fmaf(ex2_approx(dl * A2[j]), h[j], du * bv[j]);
+      yp = fmaf(h[j], cv[j], yp);
+    }
+    return yp;
+  };
+
+  // ---------------- pass 1: chunk-start states, forwards
+#pragma unroll
+  for (int j = 0; j < NPT; ++j)
+    h[j] = (active && p.h0) ? p.h0[(ib * d_in + d) * N + g * NPT + j] : 0.0f;
+  for (int c = 0; c < nC; ++c) {
+    if (active) store_vec<NPT>(my_chunk_h + (int64_t)c * d_in * N, h);
+    if (c == nC - 1) break;  // the last chunk's end state is not needed
+    __syncthreads();
+    stage(c, false);  // a chunk before the last is full
+    __syncthreads();
+#pragma unroll
+    for (int t = 0; t < TT; ++t) (void)fwd_step(t);
+  }
+
+  // ---------------- pass 2: adjoint, chunks backwards
+  float lam[NPT], dAacc[NPT];
+#pragma unroll
+  for (int j = 0; j < NPT; ++j) {
+    lam[j] = (active && p.dh_last) ? p.dh_last[(ib * d_in + d) * N + g * NPT + j] : 0.0f;
+    dAacc[j] = 0.0f;
+  }
+  // the per-(step, channel) pass keeps one channel per thread
+  const int pch = tid % DT;
+  const float pD = (d0 + pch < d_in && p.D) ? p.D[d0 + pch] : 0.0f;
+  float Dacc = 0.0f, bias_acc = 0.0f;
+
+  auto adj_step = [&](int t, const float (&hs)[NPT]) {
+    const float gt = sG[t * PROW + ch];
+    const float dl = sDelta[t * PROW + ch];
+    float hp[NPT], bv[NPT], cv[NPT], lt[NPT];
+    if (t > 0) {
+      load_vec<NPT>(sH + (t - 1) * HROW + tid * NPT, hp);
+    } else {
+#pragma unroll
+      for (int j = 0; j < NPT; ++j) hp[j] = hs[j];
+    }
+    load_vec<NPT>(sB + t * N + g * NPT, bv);
+    load_vec<NPT>(sC + t * N + g * NPT, cv);
+    float S1 = 0.0f, S2 = 0.0f;
+#pragma unroll
+    for (int j = 0; j < NPT; ++j) {
+      lam[j] = fmaf(gt, cv[j], lam[j]);
+      lt[j] = lam[j];
+      const float la = lam[j] * ex2_approx(dl * A2[j]);
+      const float q = la * hp[j];
+      S2 = fmaf(Av[j], q, S2);
+      S1 = fmaf(lam[j], bv[j], S1);
+      dAacc[j] = fmaf(q, dl, dAacc[j]);
+      lam[j] = la;
+    }
+    store_vec<NPT>(sH + t * HROW + tid * NPT, lt);
+    sP1[t * NT + tid] = S1;
+    sP2[t * NT + tid] = S2;
+  };
+
+  // sum over the CTA's channels of w[t][ch] X[t][ch][n] for every (t, n) of
+  // the chunk, X the state rows; added to out (b, L, N) rows t0 .. t0+nT-1
+  auto column_pass = [&](bool use_g, float *out, int64_t t0, int nT) {
+    for (int o = tid; o < TT * G; o += NT) {
+      const int t = o / G, gi = o - (o / G) * G;
+      float acc[NPT];
+#pragma unroll
+      for (int j = 0; j < NPT; ++j) acc[j] = 0.0f;
+      const float *xs = sH + t * HROW + gi * NPT;
+#pragma unroll 4
+      for (int cc = 0; cc < DT; ++cc) {
+        const float w = use_g ? sG[t * PROW + cc] : sDelta[t * PROW + cc] * sU[t * PROW + cc];
+        float x[NPT];
+        load_vec<NPT>(xs + cc * G * NPT, x);
+#pragma unroll
+        for (int j = 0; j < NPT; ++j) acc[j] = fmaf(w, x[j], acc[j]);
+      }
+      if (t < nT) {
+        float *dst = out + (ib * L + t0 + t) * N + gi * NPT;
+        if constexpr (NPT == 4) {
+          if (p.vec_atomics) {
+            atomicAdd(reinterpret_cast<float4 *>(dst), make_float4(acc[0], acc[1], acc[2], acc[3]));
+            continue;
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < NPT; ++j) atomicAdd(dst + j, acc[j]);
+      }
+    }
+  };
+
+  for (int c = nC - 1; c >= 0; --c) {
+    __syncthreads();  // the previous chunk's planes have been read
+    const int nT = stage(c, true);
+    const int64_t t0 = (int64_t)c * TT;
+    float hs[NPT];
+    if (active) {
+      load_vec<NPT>(my_chunk_h + (int64_t)c * d_in * N, hs);
+    } else {
+#pragma unroll
+      for (int j = 0; j < NPT; ++j) hs[j] = 0.0f;
+    }
+    __syncthreads();
+
+    // recompute the chunk's states and the partial pre-gate outputs
+#pragma unroll
+    for (int j = 0; j < NPT; ++j) h[j] = hs[j];
+    if (nT == TT) {
+#pragma unroll
+      for (int t = 0; t < TT; ++t) {
+        sPy[t * NT + tid] = fwd_step(t);
+        store_vec<NPT>(sH + t * HROW + tid * NPT, h);
+      }
+    } else {
+      for (int t = 0; t < nT; ++t) {
+        sPy[t * NT + tid] = fwd_step(t);
+        store_vec<NPT>(sH + t * HROW + tid * NPT, h);
+      }
+    }
+    __syncthreads();
+    column_pass(true, p.dC, t0, nT);  // dC_t = sum_ch g_t h_t
+    __syncthreads();
+
+    // the adjoint through the chunk (state rows become adjoint rows)
+    if (nT == TT) {
+#pragma unroll
+      for (int t = TT - 1; t >= 0; --t) adj_step(t, hs);
+    } else {
+      for (int t = nT - 1; t >= 0; --t) adj_step(t, hs);
+    }
+    __syncthreads();
+    column_pass(false, p.dB, t0, nT);  // dB_t = sum_ch lam_t delta_t u_t
+
+    // per (step, channel): add the partials, write du, ddelta, dz
+    for (int i = tid; i < TT * DT; i += NT) {
+      const int t = i / DT;  // i % DT == pch
+      const int64_t dd = d0 + pch;
+      const int s = t * PROW + pch;
+      const float S1 = sum_partials<G>(sP1 + t * NT + pch * G);
+      const float S2 = sum_partials<G>(sP2 + t * NT + pch * G);
+      const float yp = sum_partials<G>(sPy + t * NT + pch * G);
+      const float gt = sG[s], dl = sDelta[s], uu = sU[s];
+      const float ddt = fmaf(uu, S1, S2) * sSpg[s];
+      if (t < nT && dd < d_in) {
+        const int64_t at = (ib * L + t0 + t) * d_in + dd;
+        Elem<T>::store(static_cast<T *>(p.du), at, fmaf(gt, pD, dl * S1));
+        Elem<T>::store(static_cast<T *>(p.ddelta), at, ddt);
+        if (gz && p.dz) Elem<T>::store(static_cast<T *>(p.dz), at, sDzf[s] * fmaf(pD, uu, yp));
+        bias_acc += ddt;
+        Dacc = fmaf(gt, uu, Dacc);
+      }
+    }
+  }
+
+  if (active) {
+#pragma unroll
+    for (int j = 0; j < NPT; ++j) {
+      atomicAdd(p.dA + d * N + g * NPT + j, dAacc[j]);
+      if (p.dh0) p.dh0[(ib * d_in + d) * N + g * NPT + j] = lam[j];
+    }
+  }
+  if (d0 + pch < d_in) {
+    if (p.dD) atomicAdd(p.dD + d0 + pch, Dacc);
+    if (p.ddt_bias) atomicAdd(p.ddt_bias + d0 + pch, bias_acc);
+  }
+}
+
+}  // namespace ssm

@@ -325,7 +325,8 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
   auto chunk = [&](auto kc, int64_t q, int64_t c) {
     constexpr int K = decltype(kc)::value;
     const int l0 = (int)c * LC;
-    const T *Bk = gB + (int64_t)K * L, *Ck = gC + (int64_t)K * L;
+    [[maybe_unused]] const T *Bk = gB + (int64_t)K * L;
+    [[maybe_unused]] const T *Ck = gC + (int64_t)K * L;
     cp_async_wait<0>();
     __syncthreads();  // staged rows of this chunk visible
 

@@ -11,6 +11,7 @@
 #include <type_traits>
 
 #include "ssmscan.h"
+#include "scan_bwd.cuh"
 #include "scan_fwd.cuh"
 #include "ss2d_fwd.cuh"
 #include "state_update.cuh"
@@ -160,43 +161,81 @@ __global__ void copy_or_zero_kernel(const float *src, float *dst, int64_t n) {
 #ifndef SSM_STEP_CPT
 #define SSM_STEP_CPT 1
 #endif
+#ifndef SSM_CONV_STEP_CPT
+#define SSM_CONV_STEP_CPT 1
+#endif
 
-template <typename T, int N>
-ssm_status launch_step(const ssm::StepParams &p, cudaStream_t st) {
+template <typename T, int N, bool CONV>
+ssm_status launch_step(const ssm::StepParams &p, cudaStream_t st, const char *what) {
   const int block = 256;
   if constexpr (N >= 4) {
     if (aligned(p.state, 16) && aligned(p.A, 16) && aligned(p.B, 16) && aligned(p.C, 16)) {
-      constexpr int CPT = SSM_STEP_CPT;
+      constexpr int CPT = CONV ? SSM_CONV_STEP_CPT : SSM_STEP_CPT;
       const int64_t per = (p.b * p.d_in + CPT - 1) / CPT;
       const int64_t threads = per * (N / 4);
-      ssm::state_update_vec_kernel<T, N, CPT>
+      ssm::state_update_vec_kernel<T, N, CPT, CONV>
           <<<(unsigned)((threads + block - 1) / block), block, 0, st>>>(p);
-      return check_launch("ssm_state_update");
+      return check_launch(what);
     }
     if (aligned(p.state, 16)) {
       const int64_t threads = p.b * p.d_in * (N / 4);
-      ssm::state_update_kernel<T, N, 4>
+      ssm::state_update_kernel<T, N, 4, CONV>
           <<<(unsigned)((threads + block - 1) / block), block, 0, st>>>(p);
-      return check_launch("ssm_state_update");
+      return check_launch(what);
     }
   }
   const int64_t threads = p.b * p.d_in;
-  ssm::state_update_kernel<T, N, N><<<(unsigned)((threads + block - 1) / block), block, 0, st>>>(p);
-  return check_launch("ssm_state_update");
+  ssm::state_update_kernel<T, N, N, CONV>
+      <<<(unsigned)((threads + block - 1) / block), block, 0, st>>>(p);
+  return check_launch(what);
 }
 
-template <typename T>
-ssm_status dispatch_step_n(const ssm::StepParams &p, int64_t N, cudaStream_t st) {
+template <typename T, bool CONV>
+ssm_status dispatch_step_n(const ssm::StepParams &p, int64_t N, cudaStream_t st, const char *what) {
   switch (N) {
-    case 1: return launch_step<T, 1>(p, st);
-    case 2: return launch_step<T, 2>(p, st);
-    case 4: return launch_step<T, 4>(p, st);
-    case 8: return launch_step<T, 8>(p, st);
-    case 16: return launch_step<T, 16>(p, st);
-    case 32: return launch_step<T, 32>(p, st);
-    case 64: return launch_step<T, 64>(p, st);
+    case 1: return launch_step<T, 1, CONV>(p, st, what);
+    case 2: return launch_step<T, 2, CONV>(p, st, what);
+    case 4: return launch_step<T, 4, CONV>(p, st, what);
+    case 8: return launch_step<T, 8, CONV>(p, st, what);
+    case 16: return launch_step<T, 16, CONV>(p, st, what);
+    case 32: return launch_step<T, 32, CONV>(p, st, what);
+    case 64: return launch_step<T, 64, CONV>(p, st, what);
   }
-  return fail(SSM_ERR_UNSUPPORTED, "d_state %lld not compiled", (long long)N);
+  return fail(SSM_ERR_UNSUPPORTED, "%s: d_state %lld not compiled", what, (long long)N);
+}
+
+// Shared validation of ssm_state_update and ssm_conv_state_update.
+ssm_status check_step_args(const char *what, float *ssm_state, const void *x, const void *dt,
+                           const float *A, const void *B, const void *C, const float *D,
+                           const void *z, const float *dt_bias, void *y, int64_t b, int64_t d_in,
+                           int64_t d_state, ssm_dtype dtype, bool *empty) {
+  *empty = false;
+  if (b < 0 || d_in < 0) return fail(SSM_ERR_INVALID_ARG, "%s: negative size", what);
+  if (dtype != SSM_F32 && dtype != SSM_BF16)
+    return fail(SSM_ERR_UNSUPPORTED, "%s: unknown dtype %d", what, (int)dtype);
+  if (!supported_state(d_state))
+    return fail(SSM_ERR_UNSUPPORTED, "%s: d_state %lld not in {1,2,4,8,16,32,64}", what,
+                (long long)d_state);
+  int64_t t;
+  if (!mul_ok(b, d_in, &t) || !mul_ok(t, d_state, &t) || t > INT64_MAX / 8)
+    return fail(SSM_ERR_INVALID_ARG, "%s: sizes overflow int64", what);
+  if (b == 0 || d_in == 0) {
+    *empty = true;
+    return ok();
+  }
+  if (!ssm_state || !x || !dt || !A || !B || !C || !y)
+    return fail(SSM_ERR_INVALID_ARG, "%s: ssm_state, x, dt, A, B, C and y are required", what);
+  const size_t es = esize(dtype);
+  const void *act[] = {x, dt, B, C, z, y};
+  for (const void *q : act)
+    if (q && !aligned(q, es))
+      return fail(SSM_ERR_INVALID_ARG, "%s: activation pointer not %zu-byte aligned", what, es);
+  const void *f32[] = {ssm_state, A, D, dt_bias};
+  for (const void *q : f32)
+    if (q && !aligned(q, 4)) return fail(SSM_ERR_INVALID_ARG, "%s: fp32 pointer not 4-byte aligned", what);
+  if (y == x || y == dt || y == z || y == B || y == C || y == ssm_state)
+    return fail(SSM_ERR_INVALID_ARG, "%s: y must not alias an input", what);
+  return ok();
 }
 
 // ------------------------------------------------------------ SS2D launch
@@ -257,6 +296,37 @@ ssm_status launch_ss2d(const ssm::Ss2dParams &p, ssm_ss2d_order order, cudaStrea
 unsigned grid_for(int64_t n) {
   const int64_t blocks = (n + 255) / 256;
   return (unsigned)(blocks < 148 * 32 ? (blocks > 0 ? blocks : 1) : 148 * 32);
+}
+
+// ------------------------------------------------------------ backward scan
+constexpr int64_t bwd_chunk(int64_t) { return ssm::BwdCfg<16>::TT; }
+static_assert(ssm::BwdCfg<1>::TT == ssm::BwdCfg<16>::TT && ssm::BwdCfg<2>::TT == ssm::BwdCfg<16>::TT &&
+                  ssm::BwdCfg<4>::TT == ssm::BwdCfg<16>::TT && ssm::BwdCfg<8>::TT == ssm::BwdCfg<16>::TT &&
+                  ssm::BwdCfg<32>::TT == ssm::BwdCfg<16>::TT && ssm::BwdCfg<64>::TT == ssm::BwdCfg<16>::TT,
+              "bwd_chunk must match BwdCfg");
+
+template <typename T, int N>
+ssm_status launch_bwd(const ssm::BwdParams &p, cudaStream_t st) {
+  using Cfg = ssm::BwdCfg<N>;
+  constexpr auto k = ssm::scan_bwd_kernel<T, N>;
+  if (ssm_status s = ensure_smem<k>((int)Cfg::SMEM, "ssm_scan_bwd")) return s;
+  const dim3 grid((unsigned)((p.d_in + Cfg::DT - 1) / Cfg::DT), (unsigned)p.b);
+  k<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(p);
+  return check_launch("ssm_scan_bwd");
+}
+
+template <typename T>
+ssm_status dispatch_bwd_n(const ssm::BwdParams &p, int64_t N, cudaStream_t st) {
+  switch (N) {
+    case 1: return launch_bwd<T, 1>(p, st);
+    case 2: return launch_bwd<T, 2>(p, st);
+    case 4: return launch_bwd<T, 4>(p, st);
+    case 8: return launch_bwd<T, 8>(p, st);
+    case 16: return launch_bwd<T, 16>(p, st);
+    case 32: return launch_bwd<T, 32>(p, st);
+    case 64: return launch_bwd<T, 64>(p, st);
+  }
+  return fail(SSM_ERR_UNSUPPORTED, "ssm_scan_bwd: d_state %lld not compiled", (long long)N);
 }
 
 }  // namespace
@@ -332,6 +402,92 @@ ssm_status ssm_scan_fwd(const void *u, const void *delta, const float *A, const 
   return dispatch_scan_n<float>(p, d_state, fast, st);
 }
 
+size_t ssm_scan_bwd_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t d_state) {
+  int64_t t;
+  if (b < 0 || L < 0 || d_in < 0 || !supported_state(d_state)) return (size_t)-1;
+  const int64_t n_chunks = (L + bwd_chunk(d_state) - 1) / bwd_chunk(d_state);
+  if (!mul_ok(b, n_chunks, &t) || !mul_ok(t, d_in, &t) || !mul_ok(t, d_state, &t) ||
+      t > INT64_MAX / 8)
+    return (size_t)-1;
+  return (size_t)t * sizeof(float);
+}
+
+ssm_status ssm_scan_bwd(const void *u, const void *delta, const float *A, const void *B,
+                        const void *C, const float *D, const void *z, const float *dt_bias,
+                        int delta_softplus, const float *h0, const void *dout,
+                        const float *dh_last, void *du, void *ddelta, float *dA, float *dB,
+                        float *dC, float *dD, void *dz, float *ddt_bias, float *dh0, int64_t b,
+                        int64_t L, int64_t d_in, int64_t d_state, ssm_dtype dtype,
+                        void *workspace, size_t workspace_bytes, ssm_stream_t stream) {
+  g_last_error.clear();
+  const char *what = "ssm_scan_bwd";
+  if (b < 0 || L < 0 || d_in < 0)
+    return fail(SSM_ERR_INVALID_ARG, "%s: negative size (b=%lld L=%lld d_in=%lld)", what,
+                (long long)b, (long long)L, (long long)d_in);
+  if (dtype != SSM_F32 && dtype != SSM_BF16)
+    return fail(SSM_ERR_UNSUPPORTED, "%s: unknown dtype %d", what, (int)dtype);
+  if (!supported_state(d_state))
+    return fail(SSM_ERR_UNSUPPORTED, "%s: d_state %lld not in {1,2,4,8,16,32,64}", what,
+                (long long)d_state);
+  int64_t n_act, n_bc, n_state;
+  if (!mul_ok(b, L, &n_act) || !mul_ok(n_act, d_in, &n_act) || !mul_ok(b, L, &n_bc) ||
+      !mul_ok(n_bc, d_state, &n_bc) || !mul_ok(b, d_in, &n_state) ||
+      !mul_ok(n_state, d_state, &n_state) || n_act > INT64_MAX / 4 || n_bc > INT64_MAX / 4)
+    return fail(SSM_ERR_INVALID_ARG, "%s: sizes overflow int64", what);
+  const size_t need = ssm_scan_bwd_workspace_bytes(b, L, d_in, d_state);
+  if (need == (size_t)-1) return fail(SSM_ERR_INVALID_ARG, "%s: sizes overflow int64", what);
+  if (b == 0 || d_in == 0) return ok();
+  if (workspace_bytes < need || (need > 0 && !workspace))
+    return fail(SSM_ERR_WORKSPACE, "%s: workspace %zu bytes < %zu needed", what, workspace_bytes,
+                need);
+  if (b > 65535) return fail(SSM_ERR_UNSUPPORTED, "%s: b %lld > 65535", what, (long long)b);
+  if (!A || !dA) return fail(SSM_ERR_INVALID_ARG, "%s: A and dA are required", what);
+  if (L > 0 && (!u || !delta || !B || !C || !dout || !du || !ddelta || !dB || !dC))
+    return fail(SSM_ERR_INVALID_ARG,
+                "%s: u, delta, B, C, dout, du, ddelta, dB and dC are required", what);
+  const size_t es = esize(dtype);
+  const void *act[] = {u, delta, B, C, z, dout, du, ddelta, dz};
+  for (const void *q : act)
+    if (q && !aligned(q, es))
+      return fail(SSM_ERR_INVALID_ARG, "%s: activation pointer not %zu-byte aligned", what, es);
+  const void *f32[] = {A, D, dt_bias, h0, dh_last, dA, dB, dC, dD, ddt_bias, dh0, workspace};
+  for (const void *q : f32)
+    if (q && !aligned(q, 4))
+      return fail(SSM_ERR_INVALID_ARG, "%s: fp32 pointer not 4-byte aligned", what);
+  const void *outs[] = {du, ddelta, dz, dA, dB, dC, dD, ddt_bias, dh0, workspace};
+  const void *ins[] = {u, delta, A, B, C, D, z, dt_bias, h0, dout, dh_last};
+  for (const void *o : outs) {
+    if (!o) continue;
+    for (const void *i : ins)
+      if (o == i) return fail(SSM_ERR_INVALID_ARG, "%s: an output aliases an input", what);
+    int same = 0;
+    for (const void *o2 : outs) same += (o2 == o);
+    if (same > 1) return fail(SSM_ERR_INVALID_ARG, "%s: two outputs share a buffer", what);
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // the sums over channels and over the batch accumulate into zeroed outputs
+  cudaError_t e = cudaMemsetAsync(dA, 0, (size_t)(d_in * d_state) * sizeof(float), st);
+  if (e == cudaSuccess && L > 0) e = cudaMemsetAsync(dB, 0, (size_t)n_bc * sizeof(float), st);
+  if (e == cudaSuccess && L > 0) e = cudaMemsetAsync(dC, 0, (size_t)n_bc * sizeof(float), st);
+  if (e == cudaSuccess && dD) e = cudaMemsetAsync(dD, 0, (size_t)d_in * sizeof(float), st);
+  if (e == cudaSuccess && ddt_bias)
+    e = cudaMemsetAsync(ddt_bias, 0, (size_t)d_in * sizeof(float), st);
+  if (e != cudaSuccess)
+    return fail(SSM_ERR_CUDA, "%s: cudaMemsetAsync: %s", what, cudaGetErrorString(e));
+  if (L == 0) {  // no steps: the gradient reaching h0 is dh_last
+    if (dh0) {
+      copy_or_zero_kernel<<<grid_for(n_state), 256, 0, st>>>(dh_last, dh0, n_state);
+      return check_launch(what);
+    }
+    return ok();
+  }
+  ssm::BwdParams p{u, delta, A, B, C, D, z, dt_bias, h0, dout, dh_last, du, ddelta, dz,
+                   dA, dB, dC, dD, ddt_bias, dh0, static_cast<float *>(workspace),
+                   b, L, d_in, delta_softplus, aligned(dB, 16) && aligned(dC, 16)};
+  if (dtype == SSM_BF16) return dispatch_bwd_n<__nv_bfloat16>(p, d_state, st);
+  return dispatch_bwd_n<float>(p, d_state, st);
+}
+
 size_t ss2d_scan_fwd_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_in,
                                      int64_t d_state) {
   int64_t L, t;
@@ -405,36 +561,46 @@ ssm_status ssm_state_update(float *ssm_state, const void *x, const void *dt, con
                             int64_t d_in, int64_t d_state, ssm_dtype dtype,
                             ssm_stream_t stream) {
   g_last_error.clear();
-  if (b < 0 || d_in < 0) return fail(SSM_ERR_INVALID_ARG, "ssm_state_update: negative size");
-  if (dtype != SSM_F32 && dtype != SSM_BF16)
-    return fail(SSM_ERR_UNSUPPORTED, "ssm_state_update: unknown dtype %d", (int)dtype);
-  if (!supported_state(d_state))
-    return fail(SSM_ERR_UNSUPPORTED, "ssm_state_update: d_state %lld not in {1,2,4,8,16,32,64}",
-                (long long)d_state);
-  int64_t t;
-  if (!mul_ok(b, d_in, &t) || !mul_ok(t, d_state, &t) || t > INT64_MAX / 8)
-    return fail(SSM_ERR_INVALID_ARG, "ssm_state_update: sizes overflow int64");
-  if (b == 0 || d_in == 0) return ok();
-  if (!ssm_state || !x || !dt || !A || !B || !C || !y)
-    return fail(SSM_ERR_INVALID_ARG,
-                "ssm_state_update: ssm_state, x, dt, A, B, C and y are required");
-  const size_t es = esize(dtype);
-  const void *act[] = {x, dt, B, C, z, y};
-  for (const void *q : act)
-    if (q && !aligned(q, es))
-      return fail(SSM_ERR_INVALID_ARG, "ssm_state_update: activation pointer not %zu-byte aligned",
-                  es);
-  const void *f32[] = {ssm_state, A, D, dt_bias};
-  for (const void *q : f32)
-    if (q && !aligned(q, 4))
-      return fail(SSM_ERR_INVALID_ARG, "ssm_state_update: fp32 pointer not 4-byte aligned");
-  if (y == x || y == dt || y == z || y == B || y == C || y == ssm_state)
-    return fail(SSM_ERR_INVALID_ARG, "ssm_state_update: y must not alias an input");
-
-  ssm::StepParams p{ssm_state, x, dt, A, B, C, D, z, dt_bias, y, b, d_in, dt_softplus};
+  bool empty = false;
+  if (ssm_status s = check_step_args("ssm_state_update", ssm_state, x, dt, A, B, C, D, z, dt_bias,
+                                     y, b, d_in, d_state, dtype, &empty))
+    return s;
+  if (empty) return ok();
+  ssm::StepParams p{ssm_state, x, dt, A, B, C, D, z, dt_bias, y, b, d_in, dt_softplus,
+                    nullptr, nullptr, nullptr, 0};
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype == SSM_BF16) return dispatch_step_n<__nv_bfloat16>(p, d_state, st);
-  return dispatch_step_n<float>(p, d_state, st);
+  if (dtype == SSM_BF16) return dispatch_step_n<__nv_bfloat16, false>(p, d_state, st, "ssm_state_update");
+  return dispatch_step_n<float, false>(p, d_state, st, "ssm_state_update");
+}
+
+ssm_status ssm_conv_state_update(void *conv_state, const float *conv_weight, const float *conv_bias,
+                                 int64_t d_conv, float *ssm_state, const void *x, const void *dt,
+                                 const float *A, const void *B, const void *C, const float *D,
+                                 const void *z, const float *dt_bias, int dt_softplus, void *y,
+                                 int64_t b, int64_t d_in, int64_t d_state, ssm_dtype dtype,
+                                 ssm_stream_t stream) {
+  g_last_error.clear();
+  const char *what = "ssm_conv_state_update";
+  bool empty = false;
+  if (ssm_status s = check_step_args(what, ssm_state, x, dt, A, B, C, D, z, dt_bias, y, b, d_in,
+                                     d_state, dtype, &empty))
+    return s;
+  if (d_conv < 1 || d_conv > ssm::kMaxConv)
+    return fail(SSM_ERR_UNSUPPORTED, "%s: d_conv %lld not in [1, %d]", what, (long long)d_conv,
+                ssm::kMaxConv);
+  if (empty) return ok();
+  if (!conv_state || !conv_weight)
+    return fail(SSM_ERR_INVALID_ARG, "%s: conv_state and conv_weight are required", what);
+  if (!aligned(conv_state, esize(dtype)) || !aligned(conv_weight, 4) ||
+      (conv_bias && !aligned(conv_bias, 4)))
+    return fail(SSM_ERR_INVALID_ARG, "%s: misaligned conv pointer", what);
+  if (y == conv_state || conv_state == x || conv_state == ssm_state)
+    return fail(SSM_ERR_INVALID_ARG, "%s: conv_state must not alias another argument", what);
+  ssm::StepParams p{ssm_state, x, dt, A, B, C, D, z, dt_bias, y, b, d_in, dt_softplus,
+                    conv_state, conv_weight, conv_bias, (int)d_conv};
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == SSM_BF16) return dispatch_step_n<__nv_bfloat16, true>(p, d_state, st, what);
+  return dispatch_step_n<float, true>(p, d_state, st, what);
 }
 
 ssm_status ss2d_cross_scan(const void *u, void *xs, int64_t b, int64_t H, int64_t W,

@@ -27,10 +27,73 @@ struct StepParams {
   void *y;
   int64_t b, d_in;
   int dt_softplus;
+  // fused causal-conv1d step in front of the SSM step (conv_state == nullptr: none)
+  void *conv_state;             // (b, d_in, d_conv), activation dtype, in place
+  const float *conv_w, *conv_b; // (d_in, d_conv), (d_in) nullable
+  int d_conv;
 };
 
+// The conv step of Mamba.step() ("代码连连看——mamba"): the window is rolled
+// left with x appended, dotted with the depthwise weight, plus the bias.
+// The G lanes of a channel split the taps (lane g owns taps g, g + G, ...),
+// so a warp reads and writes its channels' windows and weights as contiguous
+// runs; conv_partial returns this lane's share of the sum and fills the new
+// window entries it owns into nw.  Every value in the window is an input of
+// the activation dtype, so storing it back is exact.
+constexpr int kMaxConv = 8;
+template <int G> constexpr int conv_taps_per_lane() { return (kMaxConv + G - 1) / G; }
+
+// This lane's taps of the old window (the tap that takes x is left for
+// conv_partial) and of the weight; loaded ahead of the arithmetic.
+template <int G>
+struct ConvTaps {
+  float v[conv_taps_per_lane<G>()], w[conv_taps_per_lane<G>()], bias;
+};
+
+template <typename T, int G>
+__device__ __forceinline__ void conv_load(const StepParams &p, int64_t bd, int64_t d, int g,
+                                          ConvTaps<G> &c) {
+  const T *cs = static_cast<const T *>(p.conv_state) + bd * p.d_conv;
+  const float *w = p.conv_w + d * p.d_conv;
+  const int K = p.d_conv;
+  c.bias = (g == 0 && p.conv_b) ? p.conv_b[d] : 0.0f;
+#pragma unroll
+  for (int i = 0; i < conv_taps_per_lane<G>(); ++i) {
+    const int j = g + i * G;
+    c.v[i] = (j + 1 < K) ? Elem<T>::load(cs, j + 1) : 0.0f;
+    c.w[i] = (j < K) ? w[j] : 0.0f;
+  }
+}
+
+// This lane's share of the conv sum; fills the new window entries it owns
+// into nw (x goes into the last tap).
+template <int G>
+__device__ __forceinline__ float conv_partial(const ConvTaps<G> &c, int K, int g, float xraw,
+                                              float (&nw)[conv_taps_per_lane<G>()]) {
+  float acc = c.bias;
+#pragma unroll
+  for (int i = 0; i < conv_taps_per_lane<G>(); ++i) {
+    const int j = g + i * G;
+    const float v = (j + 1 < K) ? c.v[i] : xraw;
+    nw[i] = v;
+    if (j < K) acc = fmaf(v, c.w[i], acc);
+  }
+  return acc;
+}
+
+template <typename T, int G>
+__device__ __forceinline__ void conv_store(const StepParams &p, int64_t bd, int g,
+                                           const float (&nw)[conv_taps_per_lane<G>()]) {
+  T *cs = static_cast<T *>(p.conv_state) + bd * p.d_conv;
+#pragma unroll
+  for (int i = 0; i < conv_taps_per_lane<G>(); ++i) {
+    const int j = g + i * G;
+    if (j < p.d_conv) Elem<T>::store(cs, j, nw[i]);
+  }
+}
+
 // NPT states per thread (4, or N when N < 4); G = N / NPT threads per channel.
-template <typename T, int N, int NPT>
+template <typename T, int N, int NPT, bool CONV>
 __global__ void __launch_bounds__(256) state_update_kernel(StepParams p) {
   constexpr int G = N / NPT;
   static_assert(G >= 1 && G <= 32 && (32 % G) == 0, "bad N");
@@ -47,10 +110,19 @@ __global__ void __launch_bounds__(256) state_update_kernel(StepParams p) {
   const T *zs = static_cast<const T *>(p.z);
 
   float acc = 0.0f, xv = 0.0f;
+  float nw[conv_taps_per_lane<G>()];
+  if (active) xv = Elem<T>::load(xs, bd);
+  if constexpr (CONV) {
+    ConvTaps<G> taps;
+    if (active) conv_load<T, G>(p, bd, d, g, taps);
+    float c = active ? conv_partial<G>(taps, p.d_conv, g, xv, nw) : 0.0f;
+#pragma unroll
+    for (int m = 1; m < G; m <<= 1) c += __shfl_xor_sync(0xffffffffu, c, m);
+    xv = silu_f32(c);
+  }
   if (active) {
     float delta = Elem<T>::load(dts, bd) + (p.dt_bias ? p.dt_bias[d] : 0.0f);
     if (p.dt_softplus) delta = softplus_f32(delta);
-    xv = Elem<T>::load(xs, bd);
     const float dx = delta * xv;
     float *sp = p.state + bd * N + g * NPT;
     float s[NPT];
@@ -77,6 +149,10 @@ __global__ void __launch_bounds__(256) state_update_kernel(StepParams p) {
   }
 #pragma unroll
   for (int m = 1; m < G; m <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+  if constexpr (CONV) {
+    __syncwarp();  // every lane of the channel has read the old window
+    if (active) conv_store<T, G>(p, bd, g, nw);
+  }
   if (active && g == 0) {
     float yv = fmaf(p.D ? p.D[d] : 0.0f, xv, acc);
     if (zs) yv *= silu_f32(Elem<T>::load(zs, bd));
@@ -89,7 +165,7 @@ __global__ void __launch_bounds__(256) state_update_kernel(StepParams p) {
 // thread handles CPT channels spaced total / CPT apart, so CPT independent
 // 16-byte state loads are in flight per thread and every warp instruction
 // still touches one contiguous 512-byte span of the state.
-template <typename T, int N, int CPT>
+template <typename T, int N, int CPT, bool CONV>
 __global__ void __launch_bounds__(256) state_update_vec_kernel(StepParams p) {
   constexpr int G = N / 4;
   static_assert(N % 4 == 0 && G <= 32 && 32 % G == 0, "bad N");
@@ -103,24 +179,39 @@ __global__ void __launch_bounds__(256) state_update_vec_kernel(StepParams p) {
   const T *zs = static_cast<const T *>(p.z);
 
   float4 st[CPT];
-  int64_t bd[CPT];
+  int64_t bd[CPT], ibs[CPT], ds[CPT];
   bool on[CPT];
+  ConvTaps<G> taps[CPT];
+  const bool narrow = total <= 0xffffffffll;  // 32-bit division suffices
 #pragma unroll
-  for (int i = 0; i < CPT; ++i) {  // issue every state load first
+  for (int i = 0; i < CPT; ++i) {  // issue every state (and conv window) load first
     bd[i] = base + i * per;
     on[i] = base < per && bd[i] < total;
     st[i] = on[i] ? __ldcs(reinterpret_cast<const float4 *>(p.state + bd[i] * N + 4 * g))
                   : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    const int64_t c = on[i] ? bd[i] : 0;
+    ibs[i] = narrow ? (int64_t)((uint32_t)c / (uint32_t)p.d_in) : c / p.d_in;
+    ds[i] = c - ibs[i] * p.d_in;
+    if constexpr (CONV) {
+      if (on[i]) conv_load<T, G>(p, bd[i], ds[i], g, taps[i]);
+    }
   }
 #pragma unroll
   for (int i = 0; i < CPT; ++i) {
-    const int64_t ib = on[i] ? bd[i] / p.d_in : 0;
-    const int64_t d = on[i] ? bd[i] - ib * p.d_in : 0;
+    const int64_t ib = ibs[i];
+    const int64_t d = ds[i];
     float acc = 0.0f, xv = 0.0f;
+    float nw[conv_taps_per_lane<G>()];
+    if (on[i]) xv = Elem<T>::load(xs, bd[i]);
+    if constexpr (CONV) {  // the G lanes of a channel are all on or all off
+      float c = on[i] ? conv_partial<G>(taps[i], p.d_conv, g, xv, nw) : 0.0f;
+#pragma unroll
+      for (int m = 1; m < G; m <<= 1) c += __shfl_xor_sync(0xffffffffu, c, m);
+      xv = silu_f32(c);
+    }
     if (on[i]) {
       float delta = Elem<T>::load(dts, bd[i]) + (p.dt_bias ? p.dt_bias[d] : 0.0f);
       if (p.dt_softplus) delta = softplus_f32(delta);
-      xv = Elem<T>::load(xs, bd[i]);
       const float4 a4 = *reinterpret_cast<const float4 *>(p.A + d * N + 4 * g);
       float4 b4, c4;
       if constexpr (sizeof(T) == 2) {
@@ -144,6 +235,10 @@ __global__ void __launch_bounds__(256) state_update_vec_kernel(StepParams p) {
     }
 #pragma unroll
     for (int m = 1; m < G; m <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    if constexpr (CONV) {
+      __syncwarp();  // every lane of the channel has read the old window
+      if (on[i]) conv_store<T, G>(p, bd[i], g, nw);
+    }
     if (on[i] && g == 0) {
       float yv = fmaf(p.D ? p.D[d] : 0.0f, xv, acc);
       if (zs) yv *= silu_for<T>(Elem<T>::load(zs, bd[i]));

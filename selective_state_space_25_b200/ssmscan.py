@@ -43,12 +43,18 @@ _lib.ssm_scan_fwd_workspace_bytes.argtypes = [_I64] * 4
 _lib.ssm_scan_fwd_workspace_bytes.restype = _SZ
 _lib.ssm_scan_fwd.argtypes = [_P] * 8 + [_INT, _P, _P, _P] + [_I64] * 4 + [_INT, _P, _SZ, _P]
 _lib.ssm_scan_fwd.restype = _INT
+_lib.ssm_scan_bwd_workspace_bytes.argtypes = [_I64] * 4
+_lib.ssm_scan_bwd_workspace_bytes.restype = _SZ
+_lib.ssm_scan_bwd.argtypes = [_P] * 8 + [_INT] + [_P] * 12 + [_I64] * 4 + [_INT, _P, _SZ, _P]
+_lib.ssm_scan_bwd.restype = _INT
 _lib.ss2d_scan_fwd_workspace_bytes.argtypes = [_I64] * 5
 _lib.ss2d_scan_fwd_workspace_bytes.restype = _SZ
 _lib.ss2d_scan_fwd.argtypes = [_P] * 7 + [_INT, _P] + [_I64] * 5 + [_INT, _P, _SZ, _P]
 _lib.ss2d_scan_fwd.restype = _INT
 _lib.ssm_state_update.argtypes = [_P] * 9 + [_INT, _P] + [_I64] * 3 + [_INT, _P]
 _lib.ssm_state_update.restype = _INT
+_lib.ssm_conv_state_update.argtypes = [_P, _P, _P, _I64] + [_P] * 9 + [_INT, _P] + [_I64] * 3 + [_INT, _P]
+_lib.ssm_conv_state_update.restype = _INT
 _lib.ss2d_cross_scan.argtypes = [_P, _P] + [_I64] * 4 + [_INT, _P]
 _lib.ss2d_cross_scan.restype = _INT
 _lib.ss2d_cross_merge.argtypes = [_P, _P] + [_I64] * 4 + [_INT, _P]
@@ -168,6 +174,62 @@ def ssm_scan_fwd(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus
     return y
 
 
+def ssm_scan_bwd_workspace_bytes(b: int, L: int, d_in: int, d_state: int) -> int:
+    return int(_lib.ssm_scan_bwd_workspace_bytes(b, L, d_in, d_state))
+
+
+def ssm_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_softplus=True,
+                 h0=None, dh_last=None, want_dh0=False, workspace=None, stream=None, out=None):
+    """Gradients of sum(dout * y) [+ sum(dh_last * h_last)] for ssm_scan_fwd
+    with the same inputs.  Returns a dict: du, ddelta, dz (activation dtype,
+    (b, L, d_in); dz only with z); dA (d_in, N), dB, dC (b, L, N), dD,
+    ddt_bias (d_in) in fp32; dh0 (b, d_in, N) fp32 when want_dh0.  ``out``
+    (a dict returned by an earlier call with the same shapes) is refilled
+    in place instead of allocating."""
+    b, L, d_in = u.shape
+    N = A.shape[1]
+    dev, act, f32 = u.device, u.dtype, torch.float32
+    _need(u, "u", (b, L, d_in), act, dev)
+    _need(delta, "delta", (b, L, d_in), act, dev)
+    _need(A, "A", (d_in, N), f32, dev)
+    _need(B, "B", (b, L, N), act, dev)
+    _need(C, "C", (b, L, N), act, dev)
+    _need(dout, "dout", (b, L, d_in), act, dev)
+    _need(D, "D", (d_in,), f32, dev)
+    _need(z, "z", (b, L, d_in), act, dev)
+    _need(dt_bias, "dt_bias", (d_in,), f32, dev)
+    _need(h0, "h0", (b, d_in, N), f32, dev)
+    _need(dh_last, "dh_last", (b, d_in, N), f32, dev)
+    if out is not None:
+        g = {k: out.get(k) for k in ("du", "ddelta", "dz", "dA", "dB", "dC", "dD", "ddt_bias", "dh0")}
+        for k, shp, dt in (("du", (b, L, d_in), act), ("ddelta", (b, L, d_in), act),
+                           ("dz", (b, L, d_in), act), ("dA", (d_in, N), f32),
+                           ("dB", (b, L, N), f32), ("dC", (b, L, N), f32), ("dD", (d_in,), f32),
+                           ("ddt_bias", (d_in,), f32), ("dh0", (b, d_in, N), f32)):
+            _need(g[k], k, shp, dt, dev)
+    else:
+        g = dict(du=torch.empty_like(u), ddelta=torch.empty_like(u),
+                 dz=torch.empty_like(u) if z is not None else None,
+                 dA=torch.empty((d_in, N), dtype=f32, device=dev),
+                 dB=torch.empty((b, L, N), dtype=f32, device=dev),
+                 dC=torch.empty((b, L, N), dtype=f32, device=dev),
+                 dD=torch.empty(d_in, dtype=f32, device=dev),
+                 ddt_bias=torch.empty(d_in, dtype=f32, device=dev),
+                 dh0=torch.empty((b, d_in, N), dtype=f32, device=dev) if want_dh0 else None)
+    need = ssm_scan_bwd_workspace_bytes(b, L, d_in, N)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = _lib.ssm_scan_bwd(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                           _ptr(dt_bias), int(bool(delta_softplus)), _ptr(h0), _ptr(dout),
+                           _ptr(dh_last), _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]),
+                           _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dD"]), _ptr(g["dz"]),
+                           _ptr(g["ddt_bias"]), _ptr(g["dh0"]), b, L, d_in, N, _dtype_code(u),
+                           _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "ssm_scan_bwd")
+    return {k: v for k, v in g.items() if v is not None}
+
+
 def ss2d_scan_fwd_workspace_bytes(b: int, H: int, W: int, d_in: int, d_state: int) -> int:
     return int(_lib.ss2d_scan_fwd_workspace_bytes(b, H, W, d_in, d_state))
 
@@ -226,6 +288,37 @@ def ssm_state_update(ssm_state, x, dt, A, B, C, D=None, z=None, dt_bias=None, dt
                                _ptr(D), _ptr(z), _ptr(dt_bias), int(bool(dt_softplus)), _ptr(y),
                                b, d_in, N, _dtype_code(x), _stream(stream))
     _check(st, "ssm_state_update")
+    return y
+
+
+def ssm_conv_state_update(conv_state, conv_weight, ssm_state, x, dt, A, B, C, conv_bias=None,
+                          D=None, z=None, dt_bias=None, dt_softplus=True, y=None, stream=None):
+    """One decode step with the causal-conv1d step in front; conv_state
+    (b, d_in, d_conv) in the activation dtype and ssm_state (b, d_in, N) fp32
+    are updated in place.  conv_weight (d_in, d_conv) fp32.  Returns y (b, d_in)."""
+    b, d_in, N = ssm_state.shape
+    d_conv = conv_state.shape[-1]
+    dev, act, f32 = x.device, x.dtype, torch.float32
+    _need(conv_state, "conv_state", (b, d_in, d_conv), act, dev)
+    _need(conv_weight, "conv_weight", (d_in, d_conv), f32, dev)
+    _need(conv_bias, "conv_bias", (d_in,), f32, dev)
+    _need(ssm_state, "ssm_state", (b, d_in, N), f32, dev)
+    _need(x, "x", (b, d_in), act, dev)
+    _need(dt, "dt", (b, d_in), act, dev)
+    _need(A, "A", (d_in, N), f32, dev)
+    _need(B, "B", (b, N), act, dev)
+    _need(C, "C", (b, N), act, dev)
+    _need(D, "D", (d_in,), f32, dev)
+    _need(z, "z", (b, d_in), act, dev)
+    _need(dt_bias, "dt_bias", (d_in,), f32, dev)
+    if y is None:
+        y = torch.empty_like(x)
+    _need(y, "y", (b, d_in), act, dev)
+    st = _lib.ssm_conv_state_update(_ptr(conv_state), _ptr(conv_weight), _ptr(conv_bias), d_conv,
+                                    _ptr(ssm_state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
+                                    _ptr(D), _ptr(z), _ptr(dt_bias), int(bool(dt_softplus)),
+                                    _ptr(y), b, d_in, N, _dtype_code(x), _stream(stream))
+    _check(st, "ssm_conv_state_update")
     return y
 
 

@@ -26,7 +26,7 @@ from dataclasses import dataclass, field
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "scan_inputs", "ss2d_inputs", "step_inputs",
+__all__ = ["Workload", "WORKLOADS", "scan_inputs", "ss2d_inputs", "step_inputs", "conv_inputs",
            "s4d_real_A", "dt_bias_init"]
 
 
@@ -34,7 +34,7 @@ __all__ = ["Workload", "WORKLOADS", "scan_inputs", "ss2d_inputs", "step_inputs",
 class Workload:
     """A named synthetic workload (sizes, dtype, seed)."""
     name: str
-    kind: str                 # "scan" | "ss2d" | "step"
+    kind: str                 # "scan" | "scan_bwd" | "ss2d" | "step"
     dims: dict = field(default_factory=dict)
     dtype: str = "bf16"
     seed: int = 0
@@ -43,7 +43,7 @@ class Workload:
     def elements(self) -> int:
         """b * L * d_in * N (times the 4 directions for SS2D), per step."""
         d = self.dims
-        if self.kind == "scan":
+        if self.kind in ("scan", "scan_bwd"):
             return d["b"] * d["L"] * d["d_in"] * d["N"]
         if self.kind == "ss2d":
             return d["b"] * 4 * d["H"] * d["W"] * d["d_in"] * d["N"]
@@ -57,6 +57,9 @@ WORKLOADS = {
     "mamba130m-scan": Workload(
         "mamba130m-scan", "scan", dict(b=8, L=2048, d_in=1536, N=16), "bf16", 1,
         "Mamba-130M-shaped prefill scan"),
+    "mamba130m-scan-bwd": Workload(
+        "mamba130m-scan-bwd", "scan_bwd", dict(b=8, L=2048, d_in=1536, N=16), "bf16", 1,
+        "backward of the Mamba-130M-shaped prefill scan (all input gradients)"),
     "mamba1.4b-long-scan": Workload(
         "mamba1.4b-long-scan", "scan", dict(b=2, L=16384, d_in=4096, N=16), "bf16", 2,
         "Mamba-1.4B-shaped long-sequence prefill scan"),
@@ -66,6 +69,9 @@ WORKLOADS = {
     "mamba-decode-step": Workload(
         "mamba-decode-step", "step", dict(b=256, d_in=5120, N=16, steps=1000), "bf16", 4,
         "Mamba.step() state update, fp32 state resident in HBM"),
+    "mamba-decode-conv-step": Workload(
+        "mamba-decode-conv-step", "step", dict(b=256, d_in=5120, N=16, d_conv=4, steps=1000),
+        "bf16", 6, "Mamba.step(): causal-conv1d step fused with the state update"),
 }
 
 
@@ -151,6 +157,24 @@ def step_inputs(b: int, d_in: int, N: int, dtype: str = "bf16", seed: int = 4,
                 z=z if with_z else None, dt_bias=dt_bias)
 
 
+def conv_inputs(b: int, d_in: int, d_conv: int = 4, dtype: str = "bf16", seed: int = 5,
+                with_bias: bool = True) -> dict:
+    """Inputs of the causal-conv1d decode step, on the CPU.
+
+    Draw order: conv_state, conv_weight, conv_bias.  conv_state (b, d_in,
+    d_conv) holds past inputs (activation dtype); the depthwise weight
+    (d_in, d_conv) and bias (d_in) are fp32, uniform in +-1/sqrt(d_conv) like
+    a freshly initialised depthwise Conv1d."""
+    g = torch.Generator().manual_seed(seed)
+    td = _torch_dtype(dtype)
+    conv_state = torch.randn(b, d_in, d_conv, generator=g).to(td)
+    bound = 1.0 / math.sqrt(d_conv)
+    conv_weight = (torch.rand(d_in, d_conv, generator=g) * 2 - 1) * bound
+    conv_bias = (torch.rand(d_in, generator=g) * 2 - 1) * bound
+    return dict(conv_state=conv_state, conv_weight=conv_weight,
+                conv_bias=conv_bias if with_bias else None)
+
+
 def workload_inputs(name: str, **overrides) -> dict:
     """Full-size inputs of a named workload (CPU tensors)."""
     w = WORKLOADS[name]
@@ -158,6 +182,14 @@ def workload_inputs(name: str, **overrides) -> dict:
     d.update(overrides)
     if w.kind == "scan":
         return scan_inputs(d["b"], d["L"], d["d_in"], d["N"], w.dtype, w.seed)
+    if w.kind == "scan_bwd":
+        inp = scan_inputs(d["b"], d["L"], d["d_in"], d["N"], w.dtype, w.seed)
+        g = torch.Generator().manual_seed(w.seed + 1000)
+        inp["dout"] = torch.randn(d["b"], d["L"], d["d_in"], generator=g).to(_torch_dtype(w.dtype))
+        return inp
     if w.kind == "ss2d":
         return ss2d_inputs(d["b"], d["H"], d["W"], d["d_in"], d["N"], w.dtype, w.seed)
-    return step_inputs(d["b"], d["d_in"], d["N"], w.dtype, w.seed)
+    inp = step_inputs(d["b"], d["d_in"], d["N"], w.dtype, w.seed)
+    if "d_conv" in d:
+        inp.update(conv_inputs(d["b"], d["d_in"], d["d_conv"], w.dtype, w.seed + 1000))
+    return inp

@@ -25,6 +25,10 @@ def test_algorithmic_bytes():
     assert bench.alg_bytes(WORKLOADS["mamba130m-scan"]) == exp == 202485760
     # decode: fp32 state read + write dominates
     assert bench.alg_bytes(WORKLOADS["mamba-decode-step"]) > 2 * 256 * 5120 * 16 * 4
+    # the conv decode step adds the bf16 window read + write, weight and bias
+    b, d, K = 256, 5120, 4
+    assert (bench.alg_bytes(WORKLOADS["mamba-decode-conv-step"])
+            - bench.alg_bytes(WORKLOADS["mamba-decode-step"])) == 2 * b * d * K * 2 + d * K * 4 + d * 4
 
 
 def test_alu_roofline_bounds():

@@ -1,0 +1,160 @@
+"""GPU parity of ssm_scan_bwd (the reverse-time adjoint of the selective
+scan) against the fp64 oracle's backward, through the C ABI.
+
+Activation-dtype gradients (du, ddelta, dz) are held to the forward's
+tolerances (1e-4 fp32, 2e-2 bf16: one rounding to bf16 at the store).  The
+fp32 gradients (dA, dB, dC, dD, ddt_bias, dh0) come from fp32 arithmetic in
+both modes; they are sums of up to b*L or d_in terms, so they are held to
+1e-4 (fp32 inputs) / 2e-4 (bf16 inputs) in the same metric (fp32's 6e-8 unit
+roundoff times the few hundred roundings of the longest accumulation chain,
+with margin)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from _helpers import TOL, rel_err, to_cuda
+from selective_state_space_25_b200.synthetic import WORKLOADS, scan_inputs
+
+pytestmark = pytest.mark.gpu
+
+ACT = ("du", "ddelta", "dz")
+F32 = ("dA", "dB", "dC", "dD", "ddt_bias", "dh0")
+
+
+def _tol(name, dtype):
+    if name in ACT:
+        return TOL[dtype]
+    return 1e-4 if dtype == torch.float32 else 2e-4
+
+
+def _dout(b, L, d_in, dtype, seed):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn(b, L, d_in, generator=g).to(dtype)
+
+
+def _run(S, inp, dout, h0=None, dh_last=None, softplus=True):
+    g = to_cuda(inp)
+    return S.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], dout.cuda(), D=g["D"],
+                          z=g["z"], dt_bias=g["dt_bias"], delta_softplus=softplus,
+                          h0=None if h0 is None else h0.cuda(),
+                          dh_last=None if dh_last is None else dh_last.cuda(), want_dh0=True)
+
+
+def _ref(inp, dout, h0=None, dh_last=None, softplus=True):
+    return oracle.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dout,
+                                     D=inp["D"], z=inp["z"], dt_bias=inp["dt_bias"],
+                                     delta_softplus=softplus, h0=h0, dh_last=dh_last)
+
+
+def _compare(got, ref, dtype, names=None):
+    for k in names or ref:
+        e = rel_err(got[k], ref[k])
+        assert e <= _tol(k, dtype), (k, e)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("b,L,d_in,N", [
+    (2, 64, 32, 16), (1, 97, 40, 16), (2, 33, 8, 4), (1, 50, 130, 1), (2, 17, 64, 2),
+    (1, 70, 20, 8), (1, 45, 24, 32), (1, 31, 12, 64), (3, 1, 16, 16), (1, 300, 48, 16),
+])
+def test_bwd_shapes(ssm, dtype, b, L, d_in, N):
+    dt = "bf16" if dtype == torch.bfloat16 else "fp32"
+    inp = scan_inputs(b, L, d_in, N, dt, seed=b * 7 + L + d_in + N)
+    dout = _dout(b, L, d_in, dtype, seed=L)
+    g = torch.Generator().manual_seed(d_in)
+    h0 = torch.randn(b, d_in, N, generator=g)
+    dhl = torch.randn(b, d_in, N, generator=g)
+    got = _run(ssm, inp, dout, h0, dhl)
+    _compare(got, _ref(inp, dout, h0, dhl), dtype)
+
+
+def test_bwd_no_softplus_no_gate_no_D(ssm):
+    inp = scan_inputs(2, 77, 24, 16, "fp32", seed=3, with_z=False, with_D=False)
+    inp["delta"] = inp["delta"].abs() * 0.2
+    inp["dt_bias"] = None
+    dout = _dout(2, 77, 24, torch.float32, seed=4)
+    got = _run(ssm, inp, dout, softplus=False)
+    ref = _ref(inp, dout, softplus=False)
+    assert "dz" not in got
+    _compare(got, ref, torch.float32)
+
+
+def test_bwd_L0(ssm):
+    """No steps: every summed gradient is zero and dh0 is dh_last."""
+    b, d_in, N = 2, 16, 16
+    A = -torch.rand(d_in, N, device="cuda") - 0.5
+    e = torch.empty(b, 0, d_in, device="cuda")
+    eB = torch.empty(b, 0, N, device="cuda")
+    dhl = torch.randn(b, d_in, N, device="cuda")
+    got = ssm.ssm_scan_bwd(e, e, A, eB, eB, e, D=torch.ones(d_in, device="cuda"),
+                           dt_bias=torch.zeros(d_in, device="cuda"), dh_last=dhl, want_dh0=True)
+    assert torch.equal(got["dh0"], dhl)
+    assert not got["dA"].any() and not got["dD"].any() and not got["ddt_bias"].any()
+
+
+def test_bwd_rejects_small_workspace(ssm):
+    inp = to_cuda(scan_inputs(1, 40, 16, 16, "fp32", seed=5))
+    dout = torch.randn(1, 40, 16, device="cuda")
+    ws = torch.empty(ssm.ssm_scan_bwd_workspace_bytes(1, 40, 16, 16) - 4, dtype=torch.uint8,
+                     device="cuda")
+    with pytest.raises(ssm.SsmError, match="workspace"):
+        ssm.ssm_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dout, workspace=ws)
+
+
+def test_bwd_split_sequence_chains_through_dh(ssm):
+    """Backward over [0, L) equals the backward of the second half (from the
+    first half's last state) followed by the first half's backward with
+    dh_last = the second half's dh0: the gradient of a resumed scan."""
+    b, L, d_in, N, L1 = 2, 150, 32, 16, 61
+    inp = to_cuda(scan_inputs(b, L, d_in, N, "fp32", seed=9))
+    dout = torch.randn(b, L, d_in, device="cuda")
+    full = ssm.ssm_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dout, D=inp["D"],
+                            z=inp["z"], dt_bias=inp["dt_bias"], want_dh0=True)
+    part = lambda t, s: t[:, s].contiguous()
+    first, second = slice(0, L1), slice(L1, L)
+    h_mid = torch.empty(b, d_in, N, device="cuda")
+    ssm.ssm_scan_fwd(part(inp["u"], first), part(inp["delta"], first), inp["A"],
+                     part(inp["B"], first), part(inp["C"], first), D=inp["D"],
+                     z=part(inp["z"], first), dt_bias=inp["dt_bias"], h_last=h_mid)
+    g2 = ssm.ssm_scan_bwd(part(inp["u"], second), part(inp["delta"], second), inp["A"],
+                          part(inp["B"], second), part(inp["C"], second), part(dout, second),
+                          D=inp["D"], z=part(inp["z"], second), dt_bias=inp["dt_bias"],
+                          h0=h_mid, want_dh0=True)
+    g1 = ssm.ssm_scan_bwd(part(inp["u"], first), part(inp["delta"], first), inp["A"],
+                          part(inp["B"], first), part(inp["C"], first), part(dout, first),
+                          D=inp["D"], z=part(inp["z"], first), dt_bias=inp["dt_bias"],
+                          dh_last=g2["dh0"], want_dh0=True)
+    for k in ("du", "ddelta", "dz", "dB", "dC"):
+        assert rel_err(torch.cat([g1[k], g2[k]], 1), full[k].cpu().double().numpy()) <= 1e-4, k
+    for k in ("dA", "dD", "ddt_bias"):
+        assert rel_err(g1[k] + g2[k], full[k].cpu().double().numpy()) <= 1e-4, k
+    assert rel_err(g1["dh0"], full["dh0"].cpu().double().numpy()) <= 1e-4
+
+
+def test_bwd_mamba130m_workload_sampled(ssm):
+    """The Mamba-130M-shaped prefill (b=8, L=2048, d_in=1536, N=16, bf16) at
+    full size: per-channel gradients on sampled channels of every batch, and
+    the channel sums dB, dC on one whole batch."""
+    w = WORKLOADS["mamba130m-scan"]
+    d = w.dims
+    b, L, d_in, N = d["b"], d["L"], d["d_in"], d["N"]
+    inp = scan_inputs(b, L, d_in, N, w.dtype, w.seed)
+    dout = _dout(b, L, d_in, torch.bfloat16, seed=11)
+    got = _run(ssm, inp, dout)
+    torch.cuda.synchronize()
+    chans = [0, 1, 31, 32, 767, 1000, 1535]
+    sl = lambda t: t[..., chans].contiguous()
+    sub = dict(u=sl(inp["u"]), delta=sl(inp["delta"]), A=inp["A"][chans], B=inp["B"],
+               C=inp["C"], D=inp["D"][chans], z=sl(inp["z"]), dt_bias=inp["dt_bias"][chans])
+    ref = _ref(sub, sl(dout))
+    for k in ("du", "ddelta", "dz"):
+        assert rel_err(got[k][..., chans], ref[k]) <= TOL[torch.bfloat16], k
+    for k in ("dA", "dD", "ddt_bias"):
+        assert rel_err(got[k][chans], ref[k]) <= 2e-4, k
+    one = lambda t: t[:1].contiguous()
+    ref1 = _ref(dict(u=one(inp["u"]), delta=one(inp["delta"]), A=inp["A"], B=one(inp["B"]),
+                     C=one(inp["C"]), D=inp["D"], z=one(inp["z"]), dt_bias=inp["dt_bias"]),
+                one(dout))
+    for k in ("dB", "dC"):
+        assert rel_err(got[k][:1], ref1[k]) <= 2e-4, k

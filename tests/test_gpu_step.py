@@ -9,7 +9,7 @@ import torch
 
 import oracle
 from _helpers import TOL, rel_err, to_cuda, to64
-from selective_state_space_25_b200.synthetic import WORKLOADS, scan_inputs, step_inputs
+from selective_state_space_25_b200.synthetic import WORKLOADS, conv_inputs, scan_inputs, step_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -106,3 +106,85 @@ def test_prefill_then_decode_handoff(ssm, dtype):
     assert rel_err(y_pre, y_ref[:, :L]) <= tol
     assert rel_err(y_tok, y_ref[:, L]) <= tol
     assert rel_err(state, h_ref) <= max(tol, 1e-4)
+
+
+# ------------------------------------------------ fused causal-conv1d decode step
+def gpu_conv_step(S, g, c, conv_state, state, y=None):
+    return S.ssm_conv_state_update(conv_state, c["conv_weight"], state, g["x"], g["dt"], g["A"],
+                                   g["B"], g["C"], conv_bias=c["conv_bias"], D=g["D"], z=g["z"],
+                                   dt_bias=g["dt_bias"], y=y)
+
+
+def oracle_conv_then_step(inp, c, conv_state, state):
+    """Mamba.step() order: the conv step on x, then the SSM step on its output."""
+    xc, cs = oracle.conv_step(conv_state, inp["x"], c["conv_weight"], c["conv_bias"])
+    y, st = oracle.state_update(state, xc, inp["dt"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                                z=inp["z"], dt_bias=inp["dt_bias"])
+    return y, st, cs
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("b,d_in,N,d_conv", [(1, 1, 16, 4), (3, 37, 16, 4), (2, 64, 1, 2),
+                                             (4, 33, 4, 3), (2, 40, 8, 1), (2, 24, 32, 4),
+                                             (1, 16, 64, 8), (2, 50, 2, 5)])
+def test_conv_step_shapes(ssm, dtype, b, d_in, N, d_conv):
+    dt = "bf16" if dtype == torch.bfloat16 else "fp32"
+    inp = step_inputs(b, d_in, N, dt, seed=7 * b + d_in + N)
+    c = conv_inputs(b, d_in, d_conv, dt, seed=d_conv + d_in)
+    g, gc = to_cuda(inp), to_cuda(c)
+    st, cs = g["state"].clone(), gc["conv_state"].clone()
+    y = gpu_conv_step(ssm, g, gc, cs, st)
+    y_ref, st_ref, cs_ref = oracle_conv_then_step(inp, c, c["conv_state"], inp["state"])
+    assert rel_err(y, y_ref) <= TOL[dtype]
+    assert rel_err(st, st_ref) <= 1e-5
+    np.testing.assert_array_equal(to64(cs), cs_ref)      # the window only moves stored values
+
+
+def test_conv_step_no_bias_no_gate_misaligned(ssm):
+    """Optional conv bias, z and D absent; a 4-byte-aligned state takes the
+    scalar kernel."""
+    inp = step_inputs(2, 20, 16, "fp32", seed=9, with_z=False)
+    inp["D"] = None
+    c = conv_inputs(2, 20, 4, "fp32", seed=10, with_bias=False)
+    g, gc = to_cuda(inp), to_cuda(c)
+    buf = torch.empty(inp["state"].numel() + 4, device="cuda")
+    st = buf[1:1 + inp["state"].numel()].view(inp["state"].shape)
+    st.copy_(g["state"])
+    cs = gc["conv_state"].clone()
+    y = gpu_conv_step(ssm, g, gc, cs, st)
+    y_ref, st_ref, cs_ref = oracle_conv_then_step(inp, c, c["conv_state"], inp["state"])
+    assert rel_err(y, y_ref) <= 1e-4 and rel_err(st, st_ref) <= 1e-5
+    np.testing.assert_array_equal(to64(cs), cs_ref)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_conv_step_decode_sequence(ssm, dtype):
+    """Twelve decode steps with fresh tokens each step: the window carries
+    tokens across steps exactly as the oracle's does."""
+    dt = "bf16" if dtype == torch.bfloat16 else "fp32"
+    b, d_in, N, d_conv = 3, 48, 16, 4
+    c = conv_inputs(b, d_in, d_conv, dt, seed=21)
+    gc = to_cuda(c)
+    cs, o_cs = gc["conv_state"].clone(), c["conv_state"]
+    first = step_inputs(b, d_in, N, dt, seed=22)
+    st, o_st = to_cuda(first)["state"].clone(), first["state"]
+    for k in range(12):
+        inp = step_inputs(b, d_in, N, dt, seed=100 + k)
+        g = to_cuda(inp)
+        y = gpu_conv_step(ssm, g, gc, cs, st)
+        o_y, o_st, o_cs = oracle_conv_then_step(inp, c, o_cs, o_st)
+        assert rel_err(y, o_y) <= TOL[dtype], k
+        np.testing.assert_array_equal(to64(cs), o_cs)
+    assert rel_err(st, o_st) <= 1e-5
+
+
+def test_conv_step_rejects_bad_d_conv(ssm):
+    inp = to_cuda(step_inputs(1, 8, 16, "fp32", seed=1))
+    for d_conv in (0, 9):
+        cs = torch.zeros(1, 8, max(d_conv, 1), device="cuda")
+        w = torch.zeros(8, max(d_conv, 1), device="cuda")
+        st = ssm.lib().ssm_conv_state_update(
+            ssm._ptr(cs), ssm._ptr(w), None, d_conv, ssm._ptr(inp["state"]), ssm._ptr(inp["x"]),
+            ssm._ptr(inp["dt"]), ssm._ptr(inp["A"]), ssm._ptr(inp["B"]), ssm._ptr(inp["C"]), None,
+            None, None, 1, ssm._ptr(torch.empty(1, 8, device="cuda")), 1, 8, 16, 0, None)
+        assert st != 0 and "d_conv" in ssm.last_error()
