@@ -59,6 +59,9 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--override", action="append", default=[], metavar="KEY=INT",
+                    help="change one size of the workload (a smaller case for profiling); "
+                         "the line's config shows the sizes used and traffic is null")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -208,7 +211,7 @@ class ClockSampler:
 # ----------------------------------------------------------------- workloads
 def make_inputs(w):
     from selective_state_space_25_b200.synthetic import workload_inputs
-    return workload_inputs(w.name)
+    return workload_inputs(w.name, **w.dims)
 
 
 def build_step(S, w, dev_in):
@@ -426,7 +429,7 @@ def run_ours(args, w):
     alu_ach = w.elements() / avg_launch_s / 1e9
     alu_time = w.elements() / (alu_peak * 1e9)
     hbm_time = abytes / (hbm_peak * 1e9)
-    traffic = traffic_for(w.name)
+    traffic = None if args.override else traffic_for(w.name)
     if alu_time > hbm_time:
         roof = {"bound": "alu", "achieved": alu_ach, "peak": alu_peak, "unit": "Gelem/s",
                 "frac": alu_ach / alu_peak, "traffic": traffic,
@@ -456,6 +459,7 @@ def run_ours(args, w):
             "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": w.name, **w.dims, "io_dtype": w.dtype,
+                       **({"sizes_overridden": args.override} if args.override else {}),
                        "parallelism": f"replicas{world}", "l2": "flushed between steps (256 MB write, then read, outside the timed events)"},
             "gpu_launches": K,
             "roofline": roof,
@@ -517,6 +521,15 @@ def main():
     if args.workload not in WORKLOADS:
         raise SystemExit(f"unknown workload {args.workload}; choose from {sorted(WORKLOADS)}")
     w = WORKLOADS[args.workload]
+    if args.override:
+        import dataclasses
+        dims = dict(w.dims)
+        for kv in args.override:
+            k, _, v = kv.partition("=")
+            if k not in dims:
+                raise SystemExit(f"--override: {w.name} has no size {k!r}; sizes: {sorted(dims)}")
+            dims[k] = int(v)
+        w = dataclasses.replace(w, dims=dims, note=w.note + " (sizes overridden)")
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

@@ -53,28 +53,46 @@ struct BwdParams {
   int vec_atomics;  // dB and dC 16-byte aligned: float4 atomics
 };
 
-template <int N>
+template <typename T, int N, int NPT_>
 struct BwdCfg {
-  static constexpr int NPT = N < 4 ? N : 4;  // states per thread
+  static constexpr int NPT = NPT_;           // states per thread
   static constexpr int G = N / NPT;          // threads per channel
   static constexpr int THREADS = 128;
   static constexpr int DT = THREADS / G;     // channels per CTA
   static constexpr int TT = 16;              // steps per chunk
   static constexpr int PROW = DT + 1;        // plane row (padded: column reads hit distinct banks)
   static constexpr int PL = TT * PROW;       // one (step, channel) plane
-  static constexpr int HROW = THREADS * NPT + (NPT == 4 ? 16 : 0);  // state row, padded
-  // planes: delta, u, g, dz factor, softplus'
-  static constexpr int OFF_B = 5 * PL;
-  static constexpr int OFF_C = OFF_B + TT * N;
-  static constexpr int OFF_P1 = OFF_C + TT * N;      // partial sum_n lam B       [t][thread]
-  static constexpr int OFF_P2 = OFF_P1 + TT * THREADS;  // partial sum_n A lam a h  [t][thread]
-  static constexpr int OFF_PY = OFF_P2 + TT * THREADS;  // partial C.h              [t][thread]
-  static constexpr int OFF_H = OFF_PY + TT * THREADS;   // states, then adjoints     [t][thread][NPT]
+  // state row, padded so the column passes' vector reads of 4 (NPT 2) or 2
+  // (NPT 4) step rows per wavefront fall in distinct banks
+  static constexpr int HROW = THREADS * NPT + (NPT == 1 ? 1 : 16);
+  // raw input tiles of one chunk (cp.async targets): u, delta, z, dout
+  // [TT][DT] and B, C [TT][N] in the activation dtype; two of them
+  static constexpr int RAW_ACT = TT * DT, RAW_BC = TT * N;
+  static constexpr int RAW_BYTES = ((4 * RAW_ACT + 2 * RAW_BC) * (int)sizeof(T) + 15) / 16 * 16;
+  static constexpr int OFF_F = 2 * RAW_BYTES / 4;  // first float after the raw tiles
+  // planes: {delta, delta u, g, -} as one 16-byte entry, then u, the dz
+  // factor and softplus' (one float each)
+  static constexpr int OFF_Q = OFF_F;
+  static constexpr int OFF_U = OFF_Q + 4 * PL;
+  static constexpr int OFF_DZF = OFF_U + PL;
+  static constexpr int OFF_SPG = OFF_DZF + PL;
+  static constexpr int OFF_BC = (OFF_SPG + PL + 3) / 4 * 4;  // {B, C} pairs [t][n]
+  static constexpr int OFF_P1 = OFF_BC + 2 * TT * N;     // partial sum_n lam B      [t][thread]
+  static constexpr int OFF_P2 = OFF_P1 + TT * THREADS;  // partial sum_n A lam a h [t][thread]
+  static constexpr int OFF_PY = OFF_P2 + TT * THREADS;  // partial C.h             [t][thread]
+  static constexpr int OFF_H = (OFF_PY + TT * THREADS + 3) / 4 * 4;  // states, then adjoints
   static constexpr int FLOATS = OFF_H + TT * HROW;
   static constexpr size_t SMEM = FLOATS * sizeof(float);
-  static_assert(OFF_H % 4 == 0 && HROW % 4 == 0, "state rows must be 16-byte aligned");
-  static_assert(G >= 1 && G <= 32 && 32 % G == 0 && THREADS % DT == 0, "bad N");
+  static_assert(N % NPT == 0 && (NPT == 1 || NPT == 2 || NPT == 4), "bad NPT");
+  static_assert(G >= 1 && G <= 32 && 32 % G == 0 && THREADS % DT == 0, "bad N / NPT");
 };
+
+// The cp.async staging copies whole 16-byte groups of a CTA's channel run
+// and of a B / C row.
+template <typename T, int N, int NPT>
+__host__ __device__ constexpr bool bwd_async_ok() {
+  return BwdCfg<T, N, NPT>::DT % (16 / (int)sizeof(T)) == 0 && N % (16 / (int)sizeof(T)) == 0;
+}
 
 template <int NPT>
 __device__ __forceinline__ void load_vec(const float *s, float (&v)[NPT]) {
@@ -102,6 +120,21 @@ __device__ __forceinline__ void store_vec(float *s, const float (&v)[NPT]) {
   }
 }
 
+// B and C of NPT consecutive states from {B, C} pairs.
+template <int NPT>
+__device__ __forceinline__ void load_bc(const float *s, float (&b)[NPT], float (&c)[NPT]) {
+  if constexpr (NPT == 1) {
+    const float2 w = *reinterpret_cast<const float2 *>(s);
+    b[0] = w.x; c[0] = w.y;
+  } else {
+#pragma unroll
+    for (int k = 0; k < NPT; k += 2) {
+      const float4 w = *reinterpret_cast<const float4 *>(s + 2 * k);
+      b[k] = w.x; c[k] = w.y; b[k + 1] = w.z; c[k + 1] = w.w;
+    }
+  }
+}
+
 // Sum of the G consecutive partials starting at s.
 template <int G>
 __device__ __forceinline__ float sum_partials(const float *s) {
@@ -121,15 +154,17 @@ __device__ __forceinline__ float sum_partials(const float *s) {
   return acc;
 }
 
-template <typename T, int N>
-__global__ void __launch_bounds__(128) scan_bwd_kernel(BwdParams p) {
-  using Cfg = BwdCfg<N>;
+template <typename T, int N, int NPT_, bool ASYNC>
+__global__ void __launch_bounds__(128, 4) scan_bwd_kernel(BwdParams p) {
+  using Cfg = BwdCfg<T, N, NPT_>;
   constexpr int NPT = Cfg::NPT, G = Cfg::G, DT = Cfg::DT, TT = Cfg::TT, NT = Cfg::THREADS;
-  constexpr int PROW = Cfg::PROW, PL = Cfg::PL, HROW = Cfg::HROW;
+  constexpr int PROW = Cfg::PROW, HROW = Cfg::HROW;
+  static_assert(!ASYNC || bwd_async_ok<T, N, NPT_>(), "raw tiles need whole 16-byte groups");
   extern __shared__ float4 bwd_smem4[];
   float *sm = reinterpret_cast<float *>(bwd_smem4);
-  float *sDelta = sm, *sU = sm + PL, *sG = sm + 2 * PL, *sDzf = sm + 3 * PL, *sSpg = sm + 4 * PL;
-  float *sB = sm + Cfg::OFF_B, *sC = sm + Cfg::OFF_C;
+  float4 *sQ = reinterpret_cast<float4 *>(sm + Cfg::OFF_Q);
+  float *sU = sm + Cfg::OFF_U, *sDzf = sm + Cfg::OFF_DZF, *sSpg = sm + Cfg::OFF_SPG;
+  float *sBC = sm + Cfg::OFF_BC;
   float *sP1 = sm + Cfg::OFF_P1, *sP2 = sm + Cfg::OFF_P2, *sPy = sm + Cfg::OFF_PY;
   float *sH = sm + Cfg::OFF_H;
 
@@ -155,19 +190,60 @@ __global__ void __launch_bounds__(128) scan_bwd_kernel(BwdParams p) {
     A2[j] = Av[j] * kLog2e;
   }
 
+  // staging keeps one channel per thread (NT is a multiple of DT)
+  const float sbias = (p.dt_bias && d0 + tid % DT < d_in) ? p.dt_bias[d0 + tid % DT] : 0.0f;
+
+  auto rows_of = [&](int c) { return (int)(L - (int64_t)c * TT < TT ? L - (int64_t)c * TT : TT); };
+
+  // --- raw tiles (ASYNC): chunk c's inputs copied as they are, 16 bytes at
+  // a time; rows past the sequence and channels past d_in are zero-filled.
+  auto raw_base = [&](int buf) {
+    return reinterpret_cast<T *>(reinterpret_cast<char *>(bwd_smem4) + buf * Cfg::RAW_BYTES);
+  };
+  auto issue = [&](int c, bool full, int buf) {
+    constexpr int EPG = 16 / (int)sizeof(T);  // elements per 16-byte group
+    // groups per activation row and per B / C row (>= 1 so instantiations
+    // that never stage asynchronously still compile cleanly)
+    constexpr int GA = DT / EPG > 0 ? DT / EPG : 1;
+    constexpr int GB = N / EPG > 0 ? N / EPG : 1;
+    T *raw = raw_base(buf);
+    const int64_t t0 = (int64_t)c * TT;
+    const int nT = rows_of(c);
+    const int ntens = full ? 4 : 2;  // u, delta [, z, dout]
+    for (int i = tid; i < ntens * TT * GA; i += NT) {
+      const int k = i / (TT * GA), r = (i / GA) % TT, q = i % GA;
+      const T *src = k == 0 ? gu : k == 1 ? gdelta : k == 2 ? (gz ? gz : gdout) : gdout;
+      const int64_t col = d0 + q * EPG;
+      const bool ok = r < nT && col < d_in && (k != 2 || gz);
+      const T *gp = ok ? src + (ib * L + t0 + r) * d_in + col : src;
+      cp_async16(raw + k * Cfg::RAW_ACT + r * DT + q * EPG, gp, ok ? 16 : 0);
+    }
+    for (int i = tid; i < (full ? 2 : 1) * TT * GB; i += NT) {
+      const int k = i / (TT * GB), r = (i / GB) % TT, q = i % GB;
+      const T *src = k == 0 ? gB : gC;
+      const bool ok = r < nT;
+      const T *gp = ok ? src + (ib * L + t0 + r) * N + q * EPG : src;
+      cp_async16(raw + 4 * Cfg::RAW_ACT + k * Cfg::RAW_BC + r * N + q * EPG, gp, ok ? 16 : 0);
+    }
+  };
+
   // Chunk c's (step, channel) inputs into the planes; with `full` also the
   // gate terms and C.  Rows past the sequence and channels past d_in are 0.
-  auto stage = [&](int c, bool full) {
+  // ASYNC reads the raw tile in smem buffer `buf`, else global memory.
+  auto stage = [&](int c, bool full, int buf) {
     const int64_t t0 = (int64_t)c * TT;
-    const int nT = (int)(L - t0 < TT ? L - t0 : TT);
+    const int nT = rows_of(c);
+    const T *raw = raw_base(buf);
     for (int i = tid; i < TT * DT; i += NT) {
       const int t = i / DT, cc = i - t * DT;
       const int64_t dd = d0 + cc;
       float dl = 0.0f, uu = 0.0f, gg = 0.0f, dzf = 0.0f, spg = 0.0f;
       if (t < nT && dd < d_in) {
         const int64_t at = (ib * L + t0 + t) * d_in + dd;
-        const float pre = Elem<T>::load(gdelta, at) + (p.dt_bias ? p.dt_bias[dd] : 0.0f);
-        uu = Elem<T>::load(gu, at);
+        const int ra = t * DT + cc;
+        const float pre =
+            (ASYNC ? Elem<T>::load(raw + Cfg::RAW_ACT, ra) : Elem<T>::load(gdelta, at)) + sbias;
+        uu = ASYNC ? Elem<T>::load(raw, ra) : Elem<T>::load(gu, at);
         if (p.softplus) {
           dl = softplus_f32(pre);
           if (full) spg = pre > 20.0f ? 1.0f : rcp_approx(1.0f + ex2_approx(-pre * kLog2e));
@@ -176,9 +252,11 @@ __global__ void __launch_bounds__(128) scan_bwd_kernel(BwdParams p) {
           spg = 1.0f;
         }
         if (full) {
-          const float go = Elem<T>::load(gdout, at);
+          const float go =
+              ASYNC ? Elem<T>::load(raw + 3 * Cfg::RAW_ACT, ra) : Elem<T>::load(gdout, at);
           if (gz) {
-            const float zz = Elem<T>::load(gz, at);
+            const float zz =
+                ASYNC ? Elem<T>::load(raw + 2 * Cfg::RAW_ACT, ra) : Elem<T>::load(gz, at);
             const float sg = rcp_approx(1.0f + ex2_approx(-zz * kLog2e));
             gg = go * zz * sg;
             dzf = go * sg * fmaf(zz, 1.0f - sg, 1.0f);
@@ -188,10 +266,9 @@ __global__ void __launch_bounds__(128) scan_bwd_kernel(BwdParams p) {
         }
       }
       const int s = t * PROW + cc;
-      sDelta[s] = dl;
+      sQ[s] = make_float4(dl, dl * uu, gg, 0.0f);
       sU[s] = uu;
       if (full) {
-        sG[s] = gg;
         sDzf[s] = dzf;
         sSpg[s] = spg;
       }
@@ -199,8 +276,15 @@ __global__ void __launch_bounds__(128) scan_bwd_kernel(BwdParams p) {
     for (int i = tid; i < TT * N; i += NT) {
       const int t = i / N;
       const int64_t row = (ib * L + t0 + t) * N + (i - t * N);
-      sB[i] = t < nT ? Elem<T>::load(gB, row) : 0.0f;
-      if (full) sC[i] = t < nT ? Elem<T>::load(gC, row) : 0.0f;
+      float bb, cc = 0.0f;
+      if constexpr (ASYNC) {  // zero-filled past the sequence already
+        bb = Elem<T>::load(raw + 4 * Cfg::RAW_ACT, i);
+        if (full) cc = Elem<T>::load(raw + 4 * Cfg::RAW_ACT + Cfg::RAW_BC, i);
+      } else {
+        bb = t < nT ? Elem<T>::load(gB, row) : 0.0f;
+        if (full) cc = t < nT ? Elem<T>::load(gC, row) : 0.0f;
+      }
+      *reinterpret_cast<float2 *>(sBC + 2 * i) = make_float2(bb, cc);
     }
     return nT;
   };
@@ -210,11 +294,10 @@ __global__ void __launch_bounds__(128) scan_bwd_kernel(BwdParams p) {
 
   // one forward step of this thread's states (pass 1 and the recompute)
   auto fwd_step = [&](int t) -> float {
-    const float dl = sDelta[t * PROW + ch];
-    const float du = dl * sU[t * PROW + ch];
+    const float4 q = sQ[t * PROW + ch];
+    const float dl = q.x, du = q.y;
     float bv[NPT], cv[NPT];
-    load_vec<NPT>(sB + t * N + g * NPT, bv);
-    load_vec<NPT>(sC + t * N + g * NPT, cv);
+    load_bc<NPT>(sBC + 2 * (t * N + g * NPT), bv, cv);
     float yp = 0.0f;
 #pragma unroll
     for (int j = 0; j < NPT; ++j) {
@@ -228,11 +311,22 @@ __global__ void __launch_bounds__(128) scan_bwd_kernel(BwdParams p) {
 #pragma unroll
   for (int j = 0; j < NPT; ++j)
     h[j] = (active && p.h0) ? p.h0[(ib * d_in + d) * N + g * NPT + j] : 0.0f;
+  if constexpr (ASYNC) {
+    // chunks 0 .. nC-2 (partial input), then the first chunk of pass 2 (full)
+    if (nC >= 2) issue(0, false, 0); else issue(nC - 1, true, (nC - 1) & 1);
+    cp_async_commit();
+  }
   for (int c = 0; c < nC; ++c) {
     if (active) store_vec<NPT>(my_chunk_h + (int64_t)c * d_in * N, h);
     if (c == nC - 1) break;  // the last chunk's end state is not needed
+    if constexpr (ASYNC) {
+      if (c + 1 <= nC - 2) issue(c + 1, false, (c + 1) & 1);
+      else issue(nC - 1, true, (nC - 1) & 1);
+      cp_async_commit();
+      cp_async_wait<1>();
+    }
     __syncthreads();
-    stage(c, false);  // a chunk before the last is full
+    stage(c, false, c & 1);  // a chunk before the last is full
     __syncthreads();
 #pragma unroll
     for (int t = 0; t < TT; ++t) (void)fwd_step(t);
@@ -251,8 +345,8 @@ __global__ void __launch_bounds__(128) scan_bwd_kernel(BwdParams p) {
   float Dacc = 0.0f, bias_acc = 0.0f;
 
   auto adj_step = [&](int t, const float (&hs)[NPT]) {
-    const float gt = sG[t * PROW + ch];
-    const float dl = sDelta[t * PROW + ch];
+    const float4 qv = sQ[t * PROW + ch];
+    const float gt = qv.z, dl = qv.x;
     float hp[NPT], bv[NPT], cv[NPT], lt[NPT];
     if (t > 0) {
       load_vec<NPT>(sH + (t - 1) * HROW + tid * NPT, hp);
@@ -260,8 +354,7 @@ __global__ void __launch_bounds__(128) scan_bwd_kernel(BwdParams p) {
 #pragma unroll
       for (int j = 0; j < NPT; ++j) hp[j] = hs[j];
     }
-    load_vec<NPT>(sB + t * N + g * NPT, bv);
-    load_vec<NPT>(sC + t * N + g * NPT, cv);
+    load_bc<NPT>(sBC + 2 * (t * N + g * NPT), bv, cv);
     float S1 = 0.0f, S2 = 0.0f;
 #pragma unroll
     for (int j = 0; j < NPT; ++j) {
@@ -290,7 +383,8 @@ __global__ void __launch_bounds__(128) scan_bwd_kernel(BwdParams p) {
       const float *xs = sH + t * HROW + gi * NPT;
 #pragma unroll 4
       for (int cc = 0; cc < DT; ++cc) {
-        const float w = use_g ? sG[t * PROW + cc] : sDelta[t * PROW + cc] * sU[t * PROW + cc];
+        const float *qw = reinterpret_cast<const float *>(sQ + t * PROW + cc);
+        const float w = use_g ? qw[2] : qw[1];
         float x[NPT];
         load_vec<NPT>(xs + cc * G * NPT, x);
 #pragma unroll
@@ -298,9 +392,12 @@ __global__ void __launch_bounds__(128) scan_bwd_kernel(BwdParams p) {
       }
       if (t < nT) {
         float *dst = out + (ib * L + t0 + t) * N + gi * NPT;
-        if constexpr (NPT == 4) {
-          if (p.vec_atomics) {
+        if (p.vec_atomics) {
+          if constexpr (NPT == 4) {
             atomicAdd(reinterpret_cast<float4 *>(dst), make_float4(acc[0], acc[1], acc[2], acc[3]));
+            continue;
+          } else if constexpr (NPT == 2) {
+            atomicAdd(reinterpret_cast<float2 *>(dst), make_float2(acc[0], acc[1]));
             continue;
           }
         }
@@ -310,17 +407,21 @@ __global__ void __launch_bounds__(128) scan_bwd_kernel(BwdParams p) {
     }
   };
 
+  float hs_next[NPT];
+  if (active) load_vec<NPT>(my_chunk_h + (int64_t)(nC - 1) * d_in * N, hs_next);
   for (int c = nC - 1; c >= 0; --c) {
-    __syncthreads();  // the previous chunk's planes have been read
-    const int nT = stage(c, true);
-    const int64_t t0 = (int64_t)c * TT;
     float hs[NPT];
-    if (active) {
-      load_vec<NPT>(my_chunk_h + (int64_t)c * d_in * N, hs);
-    } else {
 #pragma unroll
-      for (int j = 0; j < NPT; ++j) hs[j] = 0.0f;
+    for (int j = 0; j < NPT; ++j) hs[j] = active ? hs_next[j] : 0.0f;
+    if (c > 0 && active) load_vec<NPT>(my_chunk_h + (int64_t)(c - 1) * d_in * N, hs_next);
+    if constexpr (ASYNC) {
+      if (c > 0) issue(c - 1, true, (c - 1) & 1);
+      cp_async_commit();
+      cp_async_wait<1>();
     }
+    __syncthreads();  // the previous chunk's planes have been read; this chunk's tile landed
+    const int nT = stage(c, true, c & 1);
+    const int64_t t0 = (int64_t)c * TT;
     __syncthreads();
 
     // recompute the chunk's states and the partial pre-gate outputs
@@ -360,7 +461,8 @@ __global__ void __launch_bounds__(128) scan_bwd_kernel(BwdParams p) {
       const float S1 = sum_partials<G>(sP1 + t * NT + pch * G);
       const float S2 = sum_partials<G>(sP2 + t * NT + pch * G);
       const float yp = sum_partials<G>(sPy + t * NT + pch * G);
-      const float gt = sG[s], dl = sDelta[s], uu = sU[s];
+      const float4 qv = sQ[s];
+      const float gt = qv.z, dl = qv.x, uu = sU[s];
       const float ddt = fmaf(uu, S1, S2) * sSpg[s];
       if (t < nT && dd < d_in) {
         const int64_t at = (ib * L + t0 + t) * d_in + dd;
@@ -372,6 +474,7 @@ __global__ void __launch_bounds__(128) scan_bwd_kernel(BwdParams p) {
       }
     }
   }
+  if constexpr (ASYNC) cp_async_wait<0>();  // nothing may be in flight at exit
 
   if (active) {
 #pragma unroll

@@ -69,8 +69,9 @@ struct Ss2dParams {
 // of LC = 8 WARPS TS steps:
 //   1. the chunk's delta rows and the u rows of the pixels it visits (16
 //      bytes = 8 bf16 channels each) are copied global -> shared with
-//      cp.async, one chunk ahead; B / C values likewise when they are 16-byte
-//      aligned, else read directly;
+//      cp.async, one chunk ahead, and the accumulator row each step lands on
+//      is worked out once per step for all channels; B / C values likewise
+//      when they are 16-byte aligned, else read directly;
 //   2. thread (segment s, channel pair cp) takes TS consecutive steps of its
 //      two channels: delta = softplus(dt + bias), dA = exp2(delta A log2 e)
 //      (FMA-pipe polynomial or SFU), delta u B, C and D u go to registers,
@@ -102,7 +103,8 @@ struct Ss2dCfg {
   static constexpr int OFF_C = OFF_B + (LC + BC_PAD) * ESZ;
   static constexpr int OFF_AGG = (OFF_C + (LC + BC_PAD) * ESZ + 15) / 16 * 16;  // float4 [WARPS][PAIRS]
   static constexpr int OFF_CARRY = OFF_AGG + WARPS * PAIRS * 16;              // float [8]
-  static constexpr int OFF_ACC = OFF_CARRY + 32;                               // float [L][8]
+  static constexpr int OFF_ROW = OFF_CARRY + 32;   // int [LC]: accumulator row of each step
+  static constexpr int OFF_ACC = (OFF_ROW + LC * 4 + 15) / 16 * 16;           // float [L][8]
   static constexpr int AUX_BYTES = OFF_ACC;
   static_assert(TS % 2 == 1, "TS odd keeps the warp's segments on distinct bank groups");
   static_assert(ROWB % 16 == 0 && (LC * ESZ) % 16 == 0, "16-byte staging");
@@ -133,79 +135,6 @@ __device__ __forceinline__ int add_mod(int x, int dx, int m) {
   x += (x < 0) ? m : 0;
   return x;
 }
-
-// Walks the pixels direction k visits at consecutive steps without
-// divisions: (h, w) and sk = (kappa h) mod W for the skewed accumulator row.
-template <int ORDER>
-struct PixWalk {
-  int h, w, sk;
-  int H, W, kappa, skH1;  // skH1 = (kappa (H - 1)) mod W
-  __device__ __forceinline__ void init(int k, int l, int H_, int W_, float invH, float invW,
-                                       int skH1_) {
-    H = H_;
-    W = W_;
-    kappa = (W & 1) ? 2 : 1;
-    skH1 = skH1_;
-    const int ll = k >= 2 ? H * W - 1 - l : l;
-    if ((k & 1) == 0) {
-      h = div_small(ll, W, invW);
-      w = ll - h * W;
-      if (ORDER == kOrderSnake && (h & 1)) w = W - 1 - w;
-    } else {
-      w = div_small(ll, H, invH);
-      h = ll - w * H;
-      if (ORDER == kOrderSnake && (w & 1)) h = H - 1 - h;
-    }
-    const int kh = kappa * h;
-    sk = kh - div_small(kh, W, invW) * W;
-  }
-  template <int k>
-  __device__ __forceinline__ void step() {
-    if constexpr (ORDER == kOrderCross) {
-      if constexpr ((k & 1) == 0) {  // row-major: w moves, h on wrap
-        if constexpr (k == 0) {
-          if (++w == W) { w = 0; ++h; sk = add_mod(sk, kappa, W); }
-        } else {
-          if (--w < 0) { w = W - 1; --h; sk = add_mod(sk, -kappa, W); }
-        }
-      } else {                       // column-major: h moves, w on wrap
-        if constexpr (k == 1) {
-          if (++h == H) { h = 0; ++w; sk = 0; } else { sk = add_mod(sk, kappa, W); }
-        } else {
-          if (--h < 0) { h = H - 1; --w; sk = skH1; } else { sk = add_mod(sk, -kappa, W); }
-        }
-      }
-    } else {  // snake: at a row (column) end the walk turns into the next one
-      if constexpr ((k & 1) == 0) {
-        // forward: even rows left to right, odd rows right to left
-        const bool right = ((h & 1) == 0) == (k == 0);
-        const bool turn = right ? w == W - 1 : w == 0;
-        if (turn) {
-          h += k == 0 ? 1 : -1;
-          sk = add_mod(sk, k == 0 ? kappa : -kappa, W);
-        } else {
-          w += right ? 1 : -1;
-        }
-      } else {
-        // forward: even columns top to bottom, odd columns bottom to top
-        const bool down = ((w & 1) == 0) == (k == 1);
-        const bool turn = down ? h == H - 1 : h == 0;
-        if (turn) {
-          w += k == 1 ? 1 : -1;
-        } else {
-          h += down ? 1 : -1;
-          sk = add_mod(sk, down ? kappa : -kappa, W);
-        }
-      }
-    }
-  }
-  __device__ __forceinline__ int pix() const { return h * W + w; }
-  __device__ __forceinline__ int acc_row() const {
-    int s = w + sk;
-    if (s >= W) s -= W;
-    return h * W + s;
-  }
-};
 
 // Pixel -> accumulator row (see the skew above), for one-off lookups.
 __device__ __forceinline__ int ss2d_acc_row(int pix, int W, float invW) {
@@ -248,6 +177,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
   T *tC = reinterpret_cast<T *>(smem + Cfg::OFF_C);
   float4 *agg = reinterpret_cast<float4 *>(smem + Cfg::OFF_AGG);
   float *carry = reinterpret_cast<float *>(smem + Cfg::OFF_CARRY);
+  int *tR = reinterpret_cast<int *>(smem + Cfg::OFF_ROW);
   float *acc_s = reinterpret_cast<float *>(smem + Cfg::OFF_ACC);
 
   const int tid = threadIdx.x;
@@ -263,7 +193,6 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
   const int Hi = (int)H, Wi = (int)W, Li = (int)L, di = (int)d_in;
   const float invH = 1.0f / (float)Hi, invW = 1.0f / (float)Wi;
   const int kappa = (Wi & 1) ? 2 : 1;
-  const int skH1 = (kappa * (Hi - 1)) % Wi;
   const int64_t dA = d0 + 2 * cp;    // first channel of the pair
   const bool ok0 = dA < d_in, ok1 = dA + 1 < d_in;
 
@@ -275,13 +204,11 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
 
   float *acc_g = p.acc_global + ib * L * d_in + d0;  // this image, channel d0
 
-  const int64_t nchunks = (L + LC - 1) / LC;
-  const int64_t nsteps = 4 * nchunks;  // (direction, chunk) pairs, walked in order
+  const int nchunks = (Li + LC - 1) / LC;
 
-  // stage the delta / u rows (and B / C) of step block q = k * nchunks + c
-  auto prefetch = [&](int64_t q) {
-    const int k = (int)(q / nchunks);
-    const int l0 = (int)(q - (int64_t)k * nchunks) * LC;
+  // stage the delta / u rows (and B / C) of chunk c of direction k
+  auto prefetch = [&](int k, int c) {
+    const int l0 = c * LC;
     const T *dk = gdt + (int64_t)k * L * d_in;  // delta rows of direction k
     if constexpr (ROW_ASYNC) {
       for (int r = tid; r < LC * Cfg::GRAN_PER_ROW; r += THREADS) {
@@ -289,6 +216,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
         const int l = l0 + row;
         const bool ok = l < Li;
         const int pix = ok ? ss2d_pixel32<ORDER>(k, l, Hi, Wi, invH, invW) : 0;
+        if (part == 0) tR[row] = ACC_SMEM ? ss2d_acc_row(pix, Wi, invW) : pix;
         const int so = row * DT + part * (16 / Cfg::ESZ);
         const int po = part * (16 / Cfg::ESZ);
         cp_async16(tD + so, dk + (ok ? l * di : 0) + po, ok ? 16 : 0);
@@ -300,6 +228,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
         const int l = l0 + row;
         const bool ok = l < Li && d0 + ch < d_in;
         const int pix = ok ? ss2d_pixel32<ORDER>(k, l, Hi, Wi, invH, invW) : 0;
+        if (ch == 0) tR[row] = ACC_SMEM ? ss2d_acc_row(pix, Wi, invW) : pix;
         tD[r] = ok ? dk[l * di + ch] : T(0.0f);
         tU[r] = ok ? gu[pix * di + ch] : T(0.0f);
       }
@@ -318,13 +247,13 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
   };
 
   if (tid < DT) carry[tid] = 0.0f;  // the first direction starts from h = 0
-  prefetch(0);
+  prefetch(0, 0);
   float2 A2 = make_float2(0.0f, 0.0f), bias = A2, Dd = A2;
 
   // one chunk of direction K (index arithmetic specialised per direction)
-  auto chunk = [&](auto kc, int64_t q, int64_t c) {
+  auto chunk = [&](auto kc, int c) {
     constexpr int K = decltype(kc)::value;
-    const int l0 = (int)c * LC;
+    const int l0 = c * LC;
     [[maybe_unused]] const T *Bk = gB + (int64_t)K * L;
     [[maybe_unused]] const T *Ck = gC + (int64_t)K * L;
     cp_async_wait<0>();
@@ -334,11 +263,13 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     const int lb = l0 + seg * TS;
     float2 a[TS], bu[TS], du[TS];
     float cc[TS];
+    int rows[TS];  // accumulator row (or pixel) each step lands on
     Aff2 mine{make_float2(1.0f, 1.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
     for (int j = 0; j < TS; ++j) {
       const int row = seg * TS + j;
       const bool valid = lb + j < Li;
+      rows[j] = tR[row];
       float2 dv, uv, bc;
       if constexpr (sizeof(T) == 2) {
         const uint32_t wd = *reinterpret_cast<const uint32_t *>(tD + row * DT + 2 * cp);
@@ -366,7 +297,8 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
       mine = aff2_then(mine, Aff2{a[j], bu[j]});
     }
     __syncthreads();  // staged rows consumed
-    if (q + 1 < nsteps) prefetch(q + 1);
+    if (c + 1 < nchunks) prefetch(K, c + 1);
+    else if (K < 3) prefetch(K + 1, 0);
 
     // ---- 2. inclusive scan over the warp's segments (lanes cp, cp + 4, ...)
     Aff2 inc = mine;
@@ -397,15 +329,12 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     h = __ffma2_rn(exc.a, h, exc.b);
 
     // ---- 4. replay, accumulate y at the visited pixels
-    PixWalk<ORDER> pw;
-    pw.init(K, lb < Li ? lb : 0, Hi, Wi, invH, invW, skH1);
 #pragma unroll
     for (int j = 0; j < TS; ++j) {
       h = __ffma2_rn(a[j], h, bu[j]);
       if (lb + j < Li) {
         const float2 yv = __ffma2_rn(make_float2(cc[j], cc[j]), h, du[j]);
-        float *dst = ACC_SMEM ? acc_s + pw.acc_row() * DT + 2 * cp
-                              : acc_g + pw.pix() * di + 2 * cp;
+        float *dst = ACC_SMEM ? acc_s + rows[j] * DT + 2 * cp : acc_g + rows[j] * di + 2 * cp;
         if (ok1) {
           float2 *d2 = reinterpret_cast<float2 *>(dst);
           if constexpr (K == 0)
@@ -415,7 +344,6 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
         } else if (ok0) {
           dst[0] = K == 0 ? yv.x : dst[0] + yv.x;
         }
-        if (j + 1 < TS) pw.template step<K>();
       }
     }
     __syncthreads();  // chunk's accumulator updates and carry reads done
@@ -432,13 +360,12 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     bias = make_float2((ok0 && p.dt_bias) ? p.dt_bias[pk0] : 0.0f,
                        (ok1 && p.dt_bias) ? p.dt_bias[pk0 + 1] : 0.0f);
     Dd = make_float2((ok0 && p.D) ? p.D[pk0] : 0.0f, (ok1 && p.D) ? p.D[pk0 + 1] : 0.0f);
-    for (int64_t c = 0; c < nchunks; ++c) {
-      const int64_t q = (int64_t)k * nchunks + c;
+    for (int c = 0; c < nchunks; ++c) {
       switch (k) {
-        case 0: chunk(std::integral_constant<int, 0>{}, q, c); break;
-        case 1: chunk(std::integral_constant<int, 1>{}, q, c); break;
-        case 2: chunk(std::integral_constant<int, 2>{}, q, c); break;
-        default: chunk(std::integral_constant<int, 3>{}, q, c); break;
+        case 0: chunk(std::integral_constant<int, 0>{}, c); break;
+        case 1: chunk(std::integral_constant<int, 1>{}, c); break;
+        case 2: chunk(std::integral_constant<int, 2>{}, c); break;
+        default: chunk(std::integral_constant<int, 3>{}, c); break;
       }
     }
   }

@@ -299,32 +299,43 @@ unsigned grid_for(int64_t n) {
 }
 
 // ------------------------------------------------------------ backward scan
-constexpr int64_t bwd_chunk(int64_t) { return ssm::BwdCfg<16>::TT; }
-static_assert(ssm::BwdCfg<1>::TT == ssm::BwdCfg<16>::TT && ssm::BwdCfg<2>::TT == ssm::BwdCfg<16>::TT &&
-                  ssm::BwdCfg<4>::TT == ssm::BwdCfg<16>::TT && ssm::BwdCfg<8>::TT == ssm::BwdCfg<16>::TT &&
-                  ssm::BwdCfg<32>::TT == ssm::BwdCfg<16>::TT && ssm::BwdCfg<64>::TT == ssm::BwdCfg<16>::TT,
-              "bwd_chunk must match BwdCfg");
+// States per thread of the backward kernel for d_state >= 4.
+#ifndef SSM_BWD_NPT
+#define SSM_BWD_NPT 2
+#endif
 
-template <typename T, int N>
-ssm_status launch_bwd(const ssm::BwdParams &p, cudaStream_t st) {
-  using Cfg = ssm::BwdCfg<N>;
-  constexpr auto k = ssm::scan_bwd_kernel<T, N>;
+constexpr int64_t bwd_chunk(int64_t) { return ssm::BwdCfg<float, 16, 4>::TT; }
+
+template <typename T, int N, int NPT, bool ASYNC>
+ssm_status launch_bwd_cfg(const ssm::BwdParams &p, cudaStream_t st) {
+  using Cfg = ssm::BwdCfg<T, N, NPT>;
+  static_assert(Cfg::TT == bwd_chunk(N), "bwd_chunk must match BwdCfg");
+  constexpr auto k = ssm::scan_bwd_kernel<T, N, NPT, ASYNC>;
   if (ssm_status s = ensure_smem<k>((int)Cfg::SMEM, "ssm_scan_bwd")) return s;
   const dim3 grid((unsigned)((p.d_in + Cfg::DT - 1) / Cfg::DT), (unsigned)p.b);
   k<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(p);
   return check_launch("ssm_scan_bwd");
 }
 
+template <typename T, int N>
+ssm_status launch_bwd(const ssm::BwdParams &p, bool async, cudaStream_t st) {
+  constexpr int NPT = N < 4 ? N : SSM_BWD_NPT;
+  if constexpr (ssm::bwd_async_ok<T, N, NPT>()) {
+    if (async) return launch_bwd_cfg<T, N, NPT, true>(p, st);
+  }
+  return launch_bwd_cfg<T, N, NPT, false>(p, st);
+}
+
 template <typename T>
-ssm_status dispatch_bwd_n(const ssm::BwdParams &p, int64_t N, cudaStream_t st) {
+ssm_status dispatch_bwd_n(const ssm::BwdParams &p, int64_t N, bool async, cudaStream_t st) {
   switch (N) {
-    case 1: return launch_bwd<T, 1>(p, st);
-    case 2: return launch_bwd<T, 2>(p, st);
-    case 4: return launch_bwd<T, 4>(p, st);
-    case 8: return launch_bwd<T, 8>(p, st);
-    case 16: return launch_bwd<T, 16>(p, st);
-    case 32: return launch_bwd<T, 32>(p, st);
-    case 64: return launch_bwd<T, 64>(p, st);
+    case 1: return launch_bwd<T, 1>(p, async, st);
+    case 2: return launch_bwd<T, 2>(p, async, st);
+    case 4: return launch_bwd<T, 4>(p, async, st);
+    case 8: return launch_bwd<T, 8>(p, async, st);
+    case 16: return launch_bwd<T, 16>(p, async, st);
+    case 32: return launch_bwd<T, 32>(p, async, st);
+    case 64: return launch_bwd<T, 64>(p, async, st);
   }
   return fail(SSM_ERR_UNSUPPORTED, "ssm_scan_bwd: d_state %lld not compiled", (long long)N);
 }
@@ -484,8 +495,11 @@ ssm_status ssm_scan_bwd(const void *u, const void *delta, const float *A, const 
   ssm::BwdParams p{u, delta, A, B, C, D, z, dt_bias, h0, dout, dh_last, du, ddelta, dz,
                    dA, dB, dC, dD, ddt_bias, dh0, static_cast<float *>(workspace),
                    b, L, d_in, delta_softplus, aligned(dB, 16) && aligned(dC, 16)};
-  if (dtype == SSM_BF16) return dispatch_bwd_n<__nv_bfloat16>(p, d_state, st);
-  return dispatch_bwd_n<float>(p, d_state, st);
+  // the raw-tile prefetch copies 16-byte groups straight from the inputs
+  const bool async = (d_in * (int64_t)es) % 16 == 0 && aligned(u, 16) && aligned(delta, 16) &&
+                     aligned(dout, 16) && aligned(B, 16) && aligned(C, 16) && (!z || aligned(z, 16));
+  if (dtype == SSM_BF16) return dispatch_bwd_n<__nv_bfloat16>(p, d_state, async, st);
+  return dispatch_bwd_n<float>(p, d_state, async, st);
 }
 
 size_t ss2d_scan_fwd_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_in,
