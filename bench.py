@@ -10,8 +10,8 @@ prefill scan (b=8, L=2048, d_in=1536, N=16, bf16 activations, fp32 state):
 the configuration the headline metric (Gelem/s = b L d_in N per second, and
 HBM GB/s as a fraction of the measured peak) is quoted on.  Other workloads
 (--workload mamba1.4b-long-scan | vmamba-ss2d | mamba-decode-step |
-mamba-decode-conv-step | mamba130m-scan-bwd | tiny-fp32-scan) measure the
-companion kernels.
+mamba-decode-conv-step | mamba130m-scan-bwd | mamba130m-scan-bwd-saved |
+tiny-fp32-scan) measure the companion kernels.
 
 Timing: W untimed warm-up steps, then exactly K timed steps bracketed by a
 barrier and torch.cuda.synchronize() on both sides; each step's kernel is
@@ -78,7 +78,7 @@ def alg_bytes(w) -> int:
     if w.kind == "scan":
         b, L, di, N = d["b"], d["L"], d["d_in"], d["N"]
         return 4 * b * L * di * es + 2 * b * L * N * es + di * N * 4 + 2 * di * 4
-    if w.kind == "scan_bwd":
+    if w.kind in ("scan_bwd", "scan_bwd_saved"):
         # read u, delta, z, dout, B, C, A, D, dt_bias; write du, ddelta, dz,
         # dB, dC (fp32), dA, dD, ddt_bias (fp32)
         b, L, di, N = d["b"], d["L"], d["d_in"], d["N"]
@@ -107,6 +107,12 @@ def alu_peak_elems_per_s(w) -> float:
     N = w.dims["N"]
     if w.kind == "ss2d":
         X, F = 3.0, 12.0
+    elif w.kind == "scan_bwd_saved":
+        # the chunk states come from the forward: two passes over each
+        # element (recompute, adjoint), 2 exps and ~14 FMA-pipe ops; per
+        # (t, d) softplus once, its derivative and the gate's SiLU and
+        # derivative (7 / N)
+        X, F = 2.0 + 7.0 / N, 14.0
     elif w.kind == "scan_bwd":
         # three passes over each element (chunk states, recompute, adjoint):
         # 3 exps and ~18 FMA-pipe ops; per (t, d) softplus twice, its
@@ -230,6 +236,18 @@ def build_step(S, w, dev_in):
         fn = lambda: S.ss2d_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], d["H"], d["W"],
                                      D=g["D"], dt_bias=g["dt_bias"], y=y)
         return fn, y
+    if w.kind == "scan_bwd_saved":
+        # the training split: the forward (run once here, before any timing)
+        # saves the chunk-start states; the timed step is the backward from them
+        states = torch.empty(S.ssm_scan_bwd_workspace_bytes(d["b"], d["L"], d["d_in"], d["N"]) // 4,
+                             dtype=torch.float32, device=g["u"].device)
+        S.ssm_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], D=g["D"], z=g["z"],
+                       dt_bias=g["dt_bias"], chunk_states=states)
+        out = S.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["dout"], D=g["D"],
+                             z=g["z"], dt_bias=g["dt_bias"], states=states)
+        fn = lambda: S.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["dout"], D=g["D"],
+                                    z=g["z"], dt_bias=g["dt_bias"], states=states, out=out)
+        return fn, list(out.values())
     if w.kind == "scan_bwd":
         out = S.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["dout"], D=g["D"],
                              z=g["z"], dt_bias=g["dt_bias"])
@@ -253,7 +271,7 @@ def build_step(S, w, dev_in):
 def default_steps(w) -> int:
     if w.name == "mamba1.4b-long-scan":
         return 60
-    return {"scan": 200, "scan_bwd": 60, "ss2d": 300, "step": 1000}[w.kind]
+    return {"scan": 200, "scan_bwd": 60, "scan_bwd_saved": 60, "ss2d": 300, "step": 1000}[w.kind]
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -268,7 +286,7 @@ def oracle_sample(w, inp, target_s: float):
 
     def run(nch):
         t0 = time.perf_counter()
-        if w.kind == "scan_bwd":
+        if w.kind in ("scan_bwd", "scan_bwd_saved"):
             sl = lambda t: t[:, :, :nch].contiguous()
             oracle.selective_scan_bwd(sl(inp["u"]), sl(inp["delta"]), inp["A"][:nch], inp["B"],
                                       inp["C"], sl(inp["dout"]), D=inp["D"][:nch], z=sl(inp["z"]),

@@ -20,7 +20,9 @@
  *                     dB = dt B, state = state dA + x dB (in place),
  *                     y = state.C + D x, y * act(z)).
  *   ssm_scan_bwd      the gradients of ssm_scan_fwd by the reverse-time
- *                     adjoint of its recurrence (same passages).
+ *                     adjoint of its recurrence (same passages);
+ *                     ssm_scan_fwd_save / ssm_scan_bwd_saved split it as a
+ *                     training step does (the forward keeps chunk states).
  *   ssm_conv_state_update  the same step with the depthwise causal-conv1d
  *                     step of Mamba.step() in front of it (roll conv_state
  *                     left, append x, sum conv_state * weight + bias, SiLU).
@@ -117,6 +119,25 @@ ssm_status ssm_scan_fwd(const void *u, const void *delta, const float *A,
                         ssm_stream_t stream);
 
 /*
+ * ssm_scan_fwd that also saves the state at the start of every 16-step
+ * chunk (h before step 16 c, c = 0 .. ceil(L / 16) - 1) into chunk_states:
+ * device fp32 (b, ceil(L / 16), d_in, d_state), chunk_states_bytes >=
+ * ssm_scan_bwd_workspace_bytes(b, L, d_in, d_state), 16-byte aligned, not
+ * aliasing another argument.  This is the backward's workspace layout: a
+ * following ssm_scan_bwd_saved with the same inputs starts from these
+ * states instead of walking the sequence forwards again (the saved chunk
+ * states the backward of a training step keeps from its forward).  Every
+ * other argument as for ssm_scan_fwd.
+ */
+ssm_status ssm_scan_fwd_save(const void *u, const void *delta, const float *A,
+                             const void *B, const void *C, const float *D,
+                             const void *z, const float *dt_bias, int delta_softplus,
+                             const float *h0, float *h_last, void *y,
+                             float *chunk_states, size_t chunk_states_bytes,
+                             int64_t b, int64_t L, int64_t d_in, int64_t d_state,
+                             ssm_dtype dtype, ssm_stream_t stream);
+
+/*
  * Workspace of ssm_scan_bwd: the state at the start of every 16-step chunk
  * of the sequence, fp32: b * ceil(L / 16) * d_in * d_state * 4 bytes.
  * Returns (size_t)-1 for invalid sizes.
@@ -169,6 +190,21 @@ ssm_status ssm_scan_bwd(const void *u, const void *delta, const float *A,
                         int64_t b, int64_t L, int64_t d_in, int64_t d_state,
                         ssm_dtype dtype, void *workspace, size_t workspace_bytes,
                         ssm_stream_t stream);
+
+/*
+ * ssm_scan_bwd from the chunk-start states ssm_scan_fwd_save wrote for the
+ * same inputs (chunk_states, read only; h0 is not needed, it is chunk 0's
+ * state).  Same outputs and rules as ssm_scan_bwd.
+ */
+ssm_status ssm_scan_bwd_saved(const void *u, const void *delta, const float *A,
+                              const void *B, const void *C, const float *D,
+                              const void *z, const float *dt_bias, int delta_softplus,
+                              const void *dout, const float *dh_last,
+                              void *du, void *ddelta, float *dA, float *dB, float *dC,
+                              float *dD, void *dz, float *ddt_bias, float *dh0,
+                              int64_t b, int64_t L, int64_t d_in, int64_t d_state,
+                              ssm_dtype dtype, const float *chunk_states,
+                              size_t chunk_states_bytes, ssm_stream_t stream);
 
 /*
  * SS2D forward on an H x W grid (pixels row-major, p = h W + w, L = H W).

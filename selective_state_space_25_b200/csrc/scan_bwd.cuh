@@ -50,7 +50,8 @@ struct BwdParams {
   float *chunk_h;  // workspace (b, n_chunks, d_in, N) fp32
   int64_t b, L, d_in;
   int softplus;
-  int vec_atomics;  // dB and dC 16-byte aligned: float4 atomics
+  int vec_atomics;   // dB and dC 16-byte aligned: float4 atomics
+  int states_saved;  // chunk_h already holds the chunk-start states (saved by the forward)
 };
 
 template <typename T, int N, int NPT_>
@@ -59,7 +60,7 @@ struct BwdCfg {
   static constexpr int G = N / NPT;          // threads per channel
   static constexpr int THREADS = 128;
   static constexpr int DT = THREADS / G;     // channels per CTA
-  static constexpr int TT = 16;              // steps per chunk
+  static constexpr int TT = kStateChunk;     // steps per chunk
   static constexpr int PROW = DT + 1;        // plane row (padded: column reads hit distinct banks)
   static constexpr int PL = TT * PROW;       // one (step, channel) plane
   // state row, padded so the column passes' vector reads of 4 (NPT 2) or 2
@@ -307,16 +308,17 @@ __global__ void __launch_bounds__(128, 4) scan_bwd_kernel(BwdParams p) {
     return yp;
   };
 
-  // ---------------- pass 1: chunk-start states, forwards
+  // ---------------- pass 1: chunk-start states, forwards (unless saved)
+  const int n_pass1 = p.states_saved ? 0 : nC;
 #pragma unroll
   for (int j = 0; j < NPT; ++j)
     h[j] = (active && p.h0) ? p.h0[(ib * d_in + d) * N + g * NPT + j] : 0.0f;
   if constexpr (ASYNC) {
     // chunks 0 .. nC-2 (partial input), then the first chunk of pass 2 (full)
-    if (nC >= 2) issue(0, false, 0); else issue(nC - 1, true, (nC - 1) & 1);
+    if (n_pass1 >= 2) issue(0, false, 0); else issue(nC - 1, true, (nC - 1) & 1);
     cp_async_commit();
   }
-  for (int c = 0; c < nC; ++c) {
+  for (int c = 0; c < n_pass1; ++c) {
     if (active) store_vec<NPT>(my_chunk_h + (int64_t)c * d_in * N, h);
     if (c == nC - 1) break;  // the last chunk's end state is not needed
     if constexpr (ASYNC) {

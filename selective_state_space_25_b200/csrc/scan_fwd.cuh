@@ -26,6 +26,9 @@ struct ScanParams {
   void *y;
   int64_t b, L, d_in;
   int delta_softplus;
+  // optional: the state at the start of every kStateChunk-step chunk,
+  // (b, ceil(L / kStateChunk), d_in, N) fp32 (the backward scan's workspace)
+  float *chunk_h = nullptr;
 };
 
 // ---------------------------------------------------------------------------
@@ -55,7 +58,13 @@ __global__ void __launch_bounds__(128) scan_generic_kernel(ScanParams p) {
   const float bias = p.dt_bias ? p.dt_bias[d] : 0.0f;
   const float Dd = p.D ? p.D[d] : 0.0f;
 
+  const int64_t n_chunks = (p.L + kStateChunk - 1) / kStateChunk;
   for (int64_t t = 0; t < p.L; ++t) {
+    if (p.chunk_h && t % kStateChunk == 0) {
+      float *dst = p.chunk_h + ((ib * n_chunks + t / kStateChunk) * p.d_in + d) * N;
+#pragma unroll
+      for (int n = 0; n < N; ++n) dst[n] = h[n];
+    }
     const int64_t row = ib * p.L + t;
     const int64_t i = row * p.d_in + d;
     float delta = Elem<T>::load(dt, i) + bias;
@@ -211,7 +220,8 @@ template <typename T, int NPT> struct PassBuf {
   StateWords<T, NPT> B[4], C[4];    // B, C entries of this thread's states
 };
 
-template <typename T, int N, int NPT, int DT, int TC, bool HAS_Z, int NPOLY, bool BCF>
+// SAVE: also store the state at every kStateChunk-step chunk start (p.chunk_h).
+template <typename T, int N, int NPT, int DT, int TC, bool HAS_Z, int NPOLY, bool BCF, bool SAVE>
 __global__ void __launch_bounds__(FastScan<T, N, NPT, DT, TC, BCF>::THREADS)
     scan_fast_kernel(ScanParams p) {
   using S = FastScan<T, N, NPT, DT, TC, BCF>;
@@ -328,6 +338,8 @@ __global__ void __launch_bounds__(FastScan<T, N, NPT, DT, TC, BCF>::THREADS)
   };
 
   const int64_t nchunks = (L + TC - 1) / TC;
+  const int64_t n_saved = (L + kStateChunk - 1) / kStateChunk;
+  static_assert(TC % kStateChunk == 0, "saved chunk starts fall on pass boundaries");
   prefetch(0, 0);
   for (int64_t ch = 0; ch < nchunks; ++ch) {
     const int stage = S::STAGES == 2 ? (int)(ch & 1) : 0;
@@ -382,6 +394,12 @@ __global__ void __launch_bounds__(FastScan<T, N, NPT, DT, TC, BCF>::THREADS)
     // ---- scan over the chunk, 4 steps per pass
     const int tcr = (tc + 3) / 4 * 4;
     for (int t = 0; t < tcr; t += 4) {
+      if (SAVE && (t % kStateChunk) == 0 && t < tc && d_ok) {  // a saved chunk start
+        float2 *dst = reinterpret_cast<float2 *>(
+            p.chunk_h + ((ib * n_saved + (t0 + t) / kStateChunk) * d_in + d) * N + g * NPT);
+#pragma unroll
+        for (int k = 0; k < NP2; ++k) dst[k] = h[k];
+      }
       PassBuf<TB, NPT> pb;
       stage1(t, cB, cC, pb);
       stage2(t, pb);

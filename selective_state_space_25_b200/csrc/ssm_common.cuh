@@ -12,6 +12,8 @@
 namespace ssm {
 
 constexpr float kLog2e = 1.4426950408889634f;
+// Steps between the saved chunk-start states the backward scan works from.
+constexpr int kStateChunk = 16;
 constexpr float kLn2 = 0.6931471805599453f;
 
 // ---------------------------------------------------------------- SFU calls

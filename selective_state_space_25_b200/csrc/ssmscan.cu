@@ -98,6 +98,14 @@ constexpr int fast_npt(int n, int want, int dt) {
 #define SSM_SCAN_BCF 0
 #endif
 
+template <auto Kernel>
+ssm_status launch_fast_kernel(const ssm::ScanParams &p, dim3 grid, int threads, int smem,
+                              cudaStream_t st) {
+  if (ssm_status s = ensure_smem<Kernel>(smem, "ssm_scan_fwd")) return s;
+  Kernel<<<grid, threads, smem, st>>>(p);
+  return check_launch("ssm_scan_fwd");
+}
+
 template <typename T, int N, bool HAS_Z, int WANT_NPT>
 ssm_status launch_scan_fast_npt(const ssm::ScanParams &p, cudaStream_t st) {
   constexpr int NPT = fast_npt(N, WANT_NPT, SSM_SCAN_DT);
@@ -105,11 +113,12 @@ ssm_status launch_scan_fast_npt(const ssm::ScanParams &p, cudaStream_t st) {
   constexpr int NPOLY = SSM_SCAN_NPOLY < NPT / 2 ? SSM_SCAN_NPOLY : NPT / 2;
   constexpr bool BCF = SSM_SCAN_BCF != 0 && sizeof(T) == 2;  // widen bf16 B / C once per CTA
   using Cfg = ssm::FastScan<T, N, NPT, DT, TC, BCF>;
-  constexpr auto k = ssm::scan_fast_kernel<T, N, NPT, DT, TC, HAS_Z, NPOLY, BCF>;
-  if (ssm_status s = ensure_smem<k>(Cfg::SMEM, "ssm_scan_fwd")) return s;
   const dim3 grid((unsigned)((p.d_in + DT - 1) / DT), (unsigned)p.b);
-  k<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(p);
-  return check_launch("ssm_scan_fwd");
+  if (p.chunk_h)  // the forward that also saves chunk-start states
+    return launch_fast_kernel<ssm::scan_fast_kernel<T, N, NPT, DT, TC, HAS_Z, NPOLY, BCF, true>>(
+        p, grid, Cfg::THREADS, Cfg::SMEM, st);
+  return launch_fast_kernel<ssm::scan_fast_kernel<T, N, NPT, DT, TC, HAS_Z, NPOLY, BCF, false>>(
+      p, grid, Cfg::THREADS, Cfg::SMEM, st);
 }
 
 // Fewer channels leave fewer warps per SM: split each channel's states over
@@ -357,12 +366,15 @@ size_t ssm_scan_fwd_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t 
   return 0;
 }
 
-ssm_status ssm_scan_fwd(const void *u, const void *delta, const float *A, const void *B,
-                        const void *C, const float *D, const void *z, const float *dt_bias,
-                        int delta_softplus, const float *h0, float *h_last, void *y, int64_t b,
-                        int64_t L, int64_t d_in, int64_t d_state, ssm_dtype dtype,
-                        void *workspace, size_t workspace_bytes, ssm_stream_t stream) {
-  (void)workspace;
+}  // extern "C"
+
+namespace {
+
+ssm_status scan_fwd_impl(const void *u, const void *delta, const float *A, const void *B,
+                         const void *C, const float *D, const void *z, const float *dt_bias,
+                         int delta_softplus, const float *h0, float *h_last, void *y, int64_t b,
+                         int64_t L, int64_t d_in, int64_t d_state, ssm_dtype dtype,
+                         size_t workspace_bytes, float *chunk_h, ssm_stream_t stream) {
   g_last_error.clear();
   if (b < 0 || L < 0 || d_in < 0)
     return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd: negative size (b=%lld L=%lld d_in=%lld)",
@@ -405,12 +417,50 @@ ssm_status ssm_scan_fwd(const void *u, const void *delta, const float *A, const 
   if (y == u || y == delta || y == z || y == B || y == C)
     return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd: y must not alias an input");
 
-  ssm::ScanParams p{u, delta, A, B, C, D, z, dt_bias, h0, h_last, y, b, L, d_in, delta_softplus};
+  ssm::ScanParams p{u, delta, A, B, C, D, z, dt_bias, h0, h_last, y, b, L, d_in, delta_softplus,
+                    chunk_h};
   const bool fast = d_state >= 8 && (d_in * (int64_t)es) % 16 == 0 && aligned(u, 16) &&
                     aligned(delta, 16) && aligned(B, 16) && aligned(C, 16) && aligned(y, 16) &&
                     (!z || aligned(z, 16)) && b <= 65535;
   if (dtype == SSM_BF16) return dispatch_scan_n<__nv_bfloat16>(p, d_state, fast, st);
   return dispatch_scan_n<float>(p, d_state, fast, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+ssm_status ssm_scan_fwd(const void *u, const void *delta, const float *A, const void *B,
+                        const void *C, const float *D, const void *z, const float *dt_bias,
+                        int delta_softplus, const float *h0, float *h_last, void *y, int64_t b,
+                        int64_t L, int64_t d_in, int64_t d_state, ssm_dtype dtype,
+                        void *workspace, size_t workspace_bytes, ssm_stream_t stream) {
+  (void)workspace;
+  return scan_fwd_impl(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, h_last, y, b, L,
+                       d_in, d_state, dtype, workspace_bytes, nullptr, stream);
+}
+
+ssm_status ssm_scan_fwd_save(const void *u, const void *delta, const float *A, const void *B,
+                             const void *C, const float *D, const void *z, const float *dt_bias,
+                             int delta_softplus, const float *h0, float *h_last, void *y,
+                             float *chunk_states, size_t chunk_states_bytes, int64_t b,
+                             int64_t L, int64_t d_in, int64_t d_state, ssm_dtype dtype,
+                             ssm_stream_t stream) {
+  g_last_error.clear();
+  const size_t need = ssm_scan_bwd_workspace_bytes(b, L, d_in, d_state);
+  if (need == (size_t)-1)
+    return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd_save: invalid sizes");
+  if (chunk_states_bytes < need || (need > 0 && !chunk_states))
+    return fail(SSM_ERR_WORKSPACE, "ssm_scan_fwd_save: chunk_states %zu bytes < %zu needed",
+                chunk_states_bytes, need);
+  if (chunk_states && !aligned(chunk_states, 16))
+    return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd_save: chunk_states not 16-byte aligned");
+  const void *ins[] = {u, delta, A, B, C, D, z, dt_bias, h0, h_last, y};
+  for (const void *q : ins)
+    if (q && q == chunk_states)
+      return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd_save: chunk_states aliases an argument");
+  return scan_fwd_impl(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, h_last, y, b, L,
+                       d_in, d_state, dtype, 0, need > 0 ? chunk_states : nullptr, stream);
 }
 
 size_t ssm_scan_bwd_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t d_state) {
@@ -423,15 +473,19 @@ size_t ssm_scan_bwd_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t 
   return (size_t)t * sizeof(float);
 }
 
-ssm_status ssm_scan_bwd(const void *u, const void *delta, const float *A, const void *B,
-                        const void *C, const float *D, const void *z, const float *dt_bias,
-                        int delta_softplus, const float *h0, const void *dout,
-                        const float *dh_last, void *du, void *ddelta, float *dA, float *dB,
-                        float *dC, float *dD, void *dz, float *ddt_bias, float *dh0, int64_t b,
-                        int64_t L, int64_t d_in, int64_t d_state, ssm_dtype dtype,
-                        void *workspace, size_t workspace_bytes, ssm_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+ssm_status scan_bwd_impl(const char *what, const void *u, const void *delta, const float *A,
+                         const void *B, const void *C, const float *D, const void *z,
+                         const float *dt_bias, int delta_softplus, const float *h0,
+                         const void *dout, const float *dh_last, void *du, void *ddelta,
+                         float *dA, float *dB, float *dC, float *dD, void *dz, float *ddt_bias,
+                         float *dh0, int64_t b, int64_t L, int64_t d_in, int64_t d_state,
+                         ssm_dtype dtype, void *workspace, size_t workspace_bytes,
+                         int states_saved, ssm_stream_t stream) {
   g_last_error.clear();
-  const char *what = "ssm_scan_bwd";
   if (b < 0 || L < 0 || d_in < 0)
     return fail(SSM_ERR_INVALID_ARG, "%s: negative size (b=%lld L=%lld d_in=%lld)", what,
                 (long long)b, (long long)L, (long long)d_in);
@@ -494,12 +548,43 @@ ssm_status ssm_scan_bwd(const void *u, const void *delta, const float *A, const 
   }
   ssm::BwdParams p{u, delta, A, B, C, D, z, dt_bias, h0, dout, dh_last, du, ddelta, dz,
                    dA, dB, dC, dD, ddt_bias, dh0, static_cast<float *>(workspace),
-                   b, L, d_in, delta_softplus, aligned(dB, 16) && aligned(dC, 16)};
+                   b, L, d_in, delta_softplus, aligned(dB, 16) && aligned(dC, 16), states_saved};
   // the raw-tile prefetch copies 16-byte groups straight from the inputs
   const bool async = (d_in * (int64_t)es) % 16 == 0 && aligned(u, 16) && aligned(delta, 16) &&
                      aligned(dout, 16) && aligned(B, 16) && aligned(C, 16) && (!z || aligned(z, 16));
   if (dtype == SSM_BF16) return dispatch_bwd_n<__nv_bfloat16>(p, d_state, async, st);
   return dispatch_bwd_n<float>(p, d_state, async, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+ssm_status ssm_scan_bwd(const void *u, const void *delta, const float *A, const void *B,
+                        const void *C, const float *D, const void *z, const float *dt_bias,
+                        int delta_softplus, const float *h0, const void *dout,
+                        const float *dh_last, void *du, void *ddelta, float *dA, float *dB,
+                        float *dC, float *dD, void *dz, float *ddt_bias, float *dh0, int64_t b,
+                        int64_t L, int64_t d_in, int64_t d_state, ssm_dtype dtype,
+                        void *workspace, size_t workspace_bytes, ssm_stream_t stream) {
+  return scan_bwd_impl("ssm_scan_bwd", u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0,
+                       dout, dh_last, du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, b, L, d_in,
+                       d_state, dtype, workspace, workspace_bytes, 0, stream);
+}
+
+ssm_status ssm_scan_bwd_saved(const void *u, const void *delta, const float *A, const void *B,
+                              const void *C, const float *D, const void *z, const float *dt_bias,
+                              int delta_softplus, const void *dout, const float *dh_last,
+                              void *du, void *ddelta, float *dA, float *dB, float *dC, float *dD,
+                              void *dz, float *ddt_bias, float *dh0, int64_t b, int64_t L,
+                              int64_t d_in, int64_t d_state, ssm_dtype dtype,
+                              const float *chunk_states, size_t chunk_states_bytes,
+                              ssm_stream_t stream) {
+  // the kernel only reads the saved states in this mode
+  return scan_bwd_impl("ssm_scan_bwd_saved", u, delta, A, B, C, D, z, dt_bias, delta_softplus,
+                       nullptr, dout, dh_last, du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, b, L,
+                       d_in, d_state, dtype, const_cast<float *>(chunk_states),
+                       chunk_states_bytes, 1, stream);
 }
 
 size_t ss2d_scan_fwd_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_in,

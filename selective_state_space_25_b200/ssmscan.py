@@ -47,6 +47,11 @@ _lib.ssm_scan_bwd_workspace_bytes.argtypes = [_I64] * 4
 _lib.ssm_scan_bwd_workspace_bytes.restype = _SZ
 _lib.ssm_scan_bwd.argtypes = [_P] * 8 + [_INT] + [_P] * 12 + [_I64] * 4 + [_INT, _P, _SZ, _P]
 _lib.ssm_scan_bwd.restype = _INT
+_lib.ssm_scan_fwd_save.argtypes = [_P] * 8 + [_INT, _P, _P, _P, _P, _SZ] + [_I64] * 4 + [_INT, _P]
+_lib.ssm_scan_fwd_save.restype = _INT
+_lib.ssm_scan_bwd_saved.argtypes = ([_P] * 8 + [_INT] + [_P] * 11 + [_I64] * 4
+                                    + [_INT, _P, _SZ, _P])
+_lib.ssm_scan_bwd_saved.restype = _INT
 _lib.ss2d_scan_fwd_workspace_bytes.argtypes = [_I64] * 5
 _lib.ss2d_scan_fwd_workspace_bytes.restype = _SZ
 _lib.ss2d_scan_fwd.argtypes = [_P] * 7 + [_INT, _P] + [_I64] * 5 + [_INT, _P, _SZ, _P]
@@ -139,10 +144,12 @@ def ssm_scan_fwd_workspace_bytes(b: int, L: int, d_in: int, d_state: int) -> int
 
 
 def ssm_scan_fwd(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True,
-                 h0=None, h_last=None, y=None, workspace=None, stream=None):
+                 h0=None, h_last=None, y=None, workspace=None, stream=None, chunk_states=None):
     """Selective scan forward (see include/ssmscan.h).  u, delta, z: (b, L, d_in);
     A: (d_in, N) fp32; B, C: (b, L, N); D, dt_bias: (d_in,) fp32; h0, h_last:
-    (b, d_in, N) fp32.  Returns y (b, L, d_in)."""
+    (b, d_in, N) fp32.  Returns y (b, L, d_in).  With ``chunk_states`` (a
+    device buffer of ssm_scan_bwd_workspace_bytes(...) bytes) the forward
+    also saves the chunk-start states for ssm_scan_bwd(..., states=...)."""
     if u.dim() != 3:
         raise ValueError("u must be (b, L, d_in)")
     b, L, d_in = u.shape
@@ -162,6 +169,14 @@ def ssm_scan_fwd(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus
     if y is None:
         y = torch.empty_like(u)
     _need(y, "y", (b, L, d_in), act, dev)
+    if chunk_states is not None:
+        st = _lib.ssm_scan_fwd_save(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                    _ptr(z), _ptr(dt_bias), int(bool(delta_softplus)), _ptr(h0),
+                                    _ptr(h_last), _ptr(y), _ptr(chunk_states),
+                                    chunk_states.numel() * chunk_states.element_size(),
+                                    b, L, d_in, N, _dtype_code(u), _stream(stream))
+        _check(st, "ssm_scan_fwd_save")
+        return y
     ws_bytes = ssm_scan_fwd_workspace_bytes(b, L, d_in, N)
     if workspace is None and ws_bytes > 0:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
@@ -179,13 +194,16 @@ def ssm_scan_bwd_workspace_bytes(b: int, L: int, d_in: int, d_state: int) -> int
 
 
 def ssm_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_softplus=True,
-                 h0=None, dh_last=None, want_dh0=False, workspace=None, stream=None, out=None):
+                 h0=None, dh_last=None, want_dh0=False, workspace=None, stream=None, out=None,
+                 states=None):
     """Gradients of sum(dout * y) [+ sum(dh_last * h_last)] for ssm_scan_fwd
     with the same inputs.  Returns a dict: du, ddelta, dz (activation dtype,
     (b, L, d_in); dz only with z); dA (d_in, N), dB, dC (b, L, N), dD,
     ddt_bias (d_in) in fp32; dh0 (b, d_in, N) fp32 when want_dh0.  ``out``
     (a dict returned by an earlier call with the same shapes) is refilled
-    in place instead of allocating."""
+    in place instead of allocating.  ``states``: the chunk_states buffer a
+    forward with the same inputs filled (ssm_scan_fwd(..., chunk_states=));
+    the backward then starts from it (ssm_scan_bwd_saved) and h0 is unused."""
     b, L, d_in = u.shape
     N = A.shape[1]
     dev, act, f32 = u.device, u.dtype, torch.float32
@@ -216,6 +234,15 @@ def ssm_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_so
                  dD=torch.empty(d_in, dtype=f32, device=dev),
                  ddt_bias=torch.empty(d_in, dtype=f32, device=dev),
                  dh0=torch.empty((b, d_in, N), dtype=f32, device=dev) if want_dh0 else None)
+    if states is not None:
+        st = _lib.ssm_scan_bwd_saved(
+            _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
+            int(bool(delta_softplus)), _ptr(dout), _ptr(dh_last), _ptr(g["du"]),
+            _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dD"]),
+            _ptr(g["dz"]), _ptr(g["ddt_bias"]), _ptr(g["dh0"]), b, L, d_in, N, _dtype_code(u),
+            _ptr(states), states.numel() * states.element_size(), _stream(stream))
+        _check(st, "ssm_scan_bwd_saved")
+        return {k: v for k, v in g.items() if v is not None}
     need = ssm_scan_bwd_workspace_bytes(b, L, d_in, N)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)

@@ -34,7 +34,7 @@ __all__ = ["Workload", "WORKLOADS", "scan_inputs", "ss2d_inputs", "step_inputs",
 class Workload:
     """A named synthetic workload (sizes, dtype, seed)."""
     name: str
-    kind: str                 # "scan" | "scan_bwd" | "ss2d" | "step"
+    kind: str                 # "scan" | "scan_bwd" | "scan_bwd_saved" | "ss2d" | "step"
     dims: dict = field(default_factory=dict)
     dtype: str = "bf16"
     seed: int = 0
@@ -43,7 +43,7 @@ class Workload:
     def elements(self) -> int:
         """b * L * d_in * N (times the 4 directions for SS2D), per step."""
         d = self.dims
-        if self.kind in ("scan", "scan_bwd"):
+        if self.kind in ("scan", "scan_bwd", "scan_bwd_saved"):
             return d["b"] * d["L"] * d["d_in"] * d["N"]
         if self.kind == "ss2d":
             return d["b"] * 4 * d["H"] * d["W"] * d["d_in"] * d["N"]
@@ -60,6 +60,9 @@ WORKLOADS = {
     "mamba130m-scan-bwd": Workload(
         "mamba130m-scan-bwd", "scan_bwd", dict(b=8, L=2048, d_in=1536, N=16), "bf16", 1,
         "backward of the Mamba-130M-shaped prefill scan (all input gradients)"),
+    "mamba130m-scan-bwd-saved": Workload(
+        "mamba130m-scan-bwd-saved", "scan_bwd_saved", dict(b=8, L=2048, d_in=1536, N=16), "bf16",
+        1, "the same backward from the chunk states its forward saved (training split)"),
     "mamba1.4b-long-scan": Workload(
         "mamba1.4b-long-scan", "scan", dict(b=2, L=16384, d_in=4096, N=16), "bf16", 2,
         "Mamba-1.4B-shaped long-sequence prefill scan"),
@@ -182,7 +185,7 @@ def workload_inputs(name: str, **overrides) -> dict:
     d.update(overrides)
     if w.kind == "scan":
         return scan_inputs(d["b"], d["L"], d["d_in"], d["N"], w.dtype, w.seed)
-    if w.kind == "scan_bwd":
+    if w.kind in ("scan_bwd", "scan_bwd_saved"):
         inp = scan_inputs(d["b"], d["L"], d["d_in"], d["N"], w.dtype, w.seed)
         g = torch.Generator().manual_seed(w.seed + 1000)
         inp["dout"] = torch.randn(d["b"], d["L"], d["d_in"], generator=g).to(_torch_dtype(w.dtype))

@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import oracle
-from _helpers import TOL, rel_err, to_cuda
+from _helpers import TOL, rel_err, to64, to_cuda
 from selective_state_space_25_b200.synthetic import WORKLOADS, scan_inputs
 
 pytestmark = pytest.mark.gpu
@@ -158,3 +158,63 @@ def test_bwd_mamba130m_workload_sampled(ssm):
                 one(dout))
     for k in ("dB", "dC"):
         assert rel_err(got[k][:1], ref1[k]) <= 2e-4, k
+
+
+# ------------------------------------ forward-saved chunk states (training split)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("b,L,d_in,N", [(2, 100, 32, 16), (1, 33, 20, 4), (2, 48, 16, 1),
+                                        (1, 70, 24, 8), (1, 16, 8, 64)])
+def test_fwd_save_states_match_oracle_prefix_scans(ssm, dtype, b, L, d_in, N):
+    """Saved state c is the state after the first 16 c steps: the oracle's
+    h_last of the scan over that prefix (chunk 0 is h0)."""
+    dt = "bf16" if dtype == torch.bfloat16 else "fp32"
+    inp = scan_inputs(b, L, d_in, N, dt, seed=L + N, with_h0=True)
+    g = to_cuda(inp)
+    nbytes = ssm.ssm_scan_bwd_workspace_bytes(b, L, d_in, N)
+    states = torch.empty(nbytes // 4, device="cuda")
+    y = ssm.ssm_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], D=g["D"], z=g["z"],
+                         dt_bias=g["dt_bias"], h0=g["h0"], chunk_states=states)
+    y_ref = oracle.selective_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                                  z=inp["z"], dt_bias=inp["dt_bias"], h0=inp["h0"])
+    assert rel_err(y, y_ref) <= TOL[dtype]
+    nC = (L + 15) // 16
+    got = states.view(b, nC, d_in, N)
+    for c in range(nC):
+        if c == 0:
+            ref = to64(inp["h0"])
+        else:
+            pre = lambda t: t[:, :16 * c].contiguous()
+            _, ref = oracle.selective_scan(pre(inp["u"]), pre(inp["delta"]), inp["A"], pre(inp["B"]),
+                                           pre(inp["C"]), dt_bias=inp["dt_bias"], h0=inp["h0"],
+                                           return_last_state=True)
+        assert rel_err(got[:, c], ref) <= 1e-4, c
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_bwd_saved_equals_self_contained(ssm, dtype):
+    """The backward from the forward's saved states gives the gradients of
+    the self-contained backward (the same states, the same arithmetic; only
+    the order of the atomic channel sums may differ)."""
+    dt = "bf16" if dtype == torch.bfloat16 else "fp32"
+    b, L, d_in, N = 2, 203, 48, 16
+    inp = scan_inputs(b, L, d_in, N, dt, seed=17, with_h0=True)
+    g = to_cuda(inp)
+    dout = _dout(b, L, d_in, dtype, seed=18).cuda()
+    dhl = torch.randn(b, d_in, N, device="cuda")
+    states = torch.empty(ssm.ssm_scan_bwd_workspace_bytes(b, L, d_in, N) // 4, device="cuda")
+    ssm.ssm_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], D=g["D"], z=g["z"],
+                     dt_bias=g["dt_bias"], h0=g["h0"], chunk_states=states)
+    kw = dict(D=g["D"], z=g["z"], dt_bias=g["dt_bias"], dh_last=dhl, want_dh0=True)
+    full = ssm.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], dout, h0=g["h0"], **kw)
+    saved = ssm.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], dout, states=states, **kw)
+    for k in full:
+        assert rel_err(saved[k], to64(full[k])) <= 1e-5, k
+    ref = _ref(inp, dout.cpu(), inp["h0"], dhl.cpu())
+    _compare(saved, ref, dtype)
+
+
+def test_fwd_save_rejects_small_buffer(ssm):
+    inp = to_cuda(scan_inputs(1, 40, 16, 16, "fp32", seed=5))
+    states = torch.empty(ssm.ssm_scan_bwd_workspace_bytes(1, 40, 16, 16) // 4 - 1, device="cuda")
+    with pytest.raises(ssm.SsmError, match="chunk_states"):
+        ssm.ssm_scan_fwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], chunk_states=states)
