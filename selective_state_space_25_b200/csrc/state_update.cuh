@@ -160,68 +160,6 @@ __global__ void __launch_bounds__(256) state_update_kernel(StepParams p) {
   }
 }
 
-// One channel of the vector kernels: thread g of the channel owns states
-// 4g .. 4g + 3, given already loaded (st) with the channel's conv taps.  Every
-// lane of the warp calls this (the G lanes of a channel are all on or all
-// off), since the channel's partial sums meet in shuffles.
-template <typename T, int N, bool CONV>
-__device__ __forceinline__ void step_channel(const StepParams &p, float4 s4, int64_t bd,
-                                             int64_t ib, int64_t d, int g, bool on,
-                                             const ConvTaps<N / 4> &taps) {
-  constexpr int G = N / 4;
-  const T *zs = static_cast<const T *>(p.z);
-  float acc = 0.0f, xv = 0.0f;
-  float nw[conv_taps_per_lane<G>()];
-  if (on) xv = Elem<T>::load(static_cast<const T *>(p.x), bd);
-  if constexpr (CONV) {
-    float c = on ? conv_partial<G>(taps, p.d_conv, g, xv, nw) : 0.0f;
-#pragma unroll
-    for (int m = 1; m < G; m <<= 1) c += __shfl_xor_sync(0xffffffffu, c, m);
-    xv = silu_f32(c);
-  }
-  if (on) {
-    float delta = Elem<T>::load(static_cast<const T *>(p.dt), bd) + (p.dt_bias ? p.dt_bias[d] : 0.0f);
-    if (p.dt_softplus) delta = softplus_f32(delta);
-    const float4 a4 = *reinterpret_cast<const float4 *>(p.A + d * N + 4 * g);
-    float4 b4, c4;
-    if constexpr (sizeof(T) == 2) {
-      const uint2 wb = *reinterpret_cast<const uint2 *>(static_cast<const T *>(p.B) + ib * N + 4 * g);
-      const uint2 wc = *reinterpret_cast<const uint2 *>(static_cast<const T *>(p.C) + ib * N + 4 * g);
-      b4 = make_float4(bf16lo(wb.x), bf16hi(wb.x), bf16lo(wb.y), bf16hi(wb.y));
-      c4 = make_float4(bf16lo(wc.x), bf16hi(wc.x), bf16lo(wc.y), bf16hi(wc.y));
-    } else {
-      b4 = *reinterpret_cast<const float4 *>(static_cast<const T *>(p.B) + ib * N + 4 * g);
-      c4 = *reinterpret_cast<const float4 *>(static_cast<const T *>(p.C) + ib * N + 4 * g);
-    }
-    const float dx = delta * xv;
-    const float dl = delta * kLog2e;
-    s4.x = fmaf(s4.x, ex2_approx(dl * a4.x), dx * b4.x);
-    s4.y = fmaf(s4.y, ex2_approx(dl * a4.y), dx * b4.y);
-    s4.z = fmaf(s4.z, ex2_approx(dl * a4.z), dx * b4.z);
-    s4.w = fmaf(s4.w, ex2_approx(dl * a4.w), dx * b4.w);
-    __stcs(reinterpret_cast<float4 *>(p.state + bd * N + 4 * g), s4);
-    acc = fmaf(s4.x, c4.x, fmaf(s4.y, c4.y, fmaf(s4.z, c4.z, s4.w * c4.w)));
-  }
-#pragma unroll
-  for (int m = 1; m < G; m <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
-  if constexpr (CONV) {
-    __syncwarp();  // every lane of the channel has read the old window
-    if (on) conv_store<T, G>(p, bd, g, nw);
-  }
-  if (on && g == 0) {
-    float yv = fmaf(p.D ? p.D[d] : 0.0f, xv, acc);
-    if (zs) yv *= silu_for<T>(Elem<T>::load(zs, bd));
-    Elem<T>::store(static_cast<T *>(p.y), bd, yv);
-  }
-}
-
-// Channel c's batch and channel index (32-bit division when it suffices).
-__device__ __forceinline__ void split_channel(int64_t c, int64_t d_in, bool narrow, int64_t &ib,
-                                              int64_t &d) {
-  ib = narrow ? (int64_t)((uint32_t)c / (uint32_t)d_in) : c / d_in;
-  d = c - ib * d_in;
-}
-
 // Vector kernel (N a multiple of 4, state and A 16-byte aligned, B and C
 // 8-byte aligned): thread g of a channel owns states 4g .. 4g + 3 and each
 // thread handles CPT channels spaced total / CPT apart, so CPT independent
@@ -236,6 +174,9 @@ __global__ void __launch_bounds__(256) state_update_vec_kernel(StepParams p) {
   const int64_t gid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   const int64_t base = gid / G;
   const int g = (int)(gid - base * G);
+  const T *xs = static_cast<const T *>(p.x);
+  const T *dts = static_cast<const T *>(p.dt);
+  const T *zs = static_cast<const T *>(p.z);
 
   float4 st[CPT];
   int64_t bd[CPT], ibs[CPT], ds[CPT];
@@ -248,13 +189,62 @@ __global__ void __launch_bounds__(256) state_update_vec_kernel(StepParams p) {
     on[i] = base < per && bd[i] < total;
     st[i] = on[i] ? __ldcs(reinterpret_cast<const float4 *>(p.state + bd[i] * N + 4 * g))
                   : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    split_channel(on[i] ? bd[i] : 0, p.d_in, narrow, ibs[i], ds[i]);
+    const int64_t c = on[i] ? bd[i] : 0;
+    ibs[i] = narrow ? (int64_t)((uint32_t)c / (uint32_t)p.d_in) : c / p.d_in;
+    ds[i] = c - ibs[i] * p.d_in;
     if constexpr (CONV) {
       if (on[i]) conv_load<T, G>(p, bd[i], ds[i], g, taps[i]);
     }
   }
 #pragma unroll
-  for (int i = 0; i < CPT; ++i) step_channel<T, N, CONV>(p, st[i], bd[i], ibs[i], ds[i], g, on[i], taps[i]);
+  for (int i = 0; i < CPT; ++i) {
+    const int64_t ib = ibs[i];
+    const int64_t d = ds[i];
+    float acc = 0.0f, xv = 0.0f;
+    float nw[conv_taps_per_lane<G>()];
+    if (on[i]) xv = Elem<T>::load(xs, bd[i]);
+    if constexpr (CONV) {  // the G lanes of a channel are all on or all off
+      float c = on[i] ? conv_partial<G>(taps[i], p.d_conv, g, xv, nw) : 0.0f;
+#pragma unroll
+      for (int m = 1; m < G; m <<= 1) c += __shfl_xor_sync(0xffffffffu, c, m);
+      xv = silu_f32(c);
+    }
+    if (on[i]) {
+      float delta = Elem<T>::load(dts, bd[i]) + (p.dt_bias ? p.dt_bias[d] : 0.0f);
+      if (p.dt_softplus) delta = softplus_f32(delta);
+      const float4 a4 = *reinterpret_cast<const float4 *>(p.A + d * N + 4 * g);
+      float4 b4, c4;
+      if constexpr (sizeof(T) == 2) {
+        const uint2 wb = *reinterpret_cast<const uint2 *>(static_cast<const T *>(p.B) + ib * N + 4 * g);
+        const uint2 wc = *reinterpret_cast<const uint2 *>(static_cast<const T *>(p.C) + ib * N + 4 * g);
+        b4 = make_float4(bf16lo(wb.x), bf16hi(wb.x), bf16lo(wb.y), bf16hi(wb.y));
+        c4 = make_float4(bf16lo(wc.x), bf16hi(wc.x), bf16lo(wc.y), bf16hi(wc.y));
+      } else {
+        b4 = *reinterpret_cast<const float4 *>(static_cast<const T *>(p.B) + ib * N + 4 * g);
+        c4 = *reinterpret_cast<const float4 *>(static_cast<const T *>(p.C) + ib * N + 4 * g);
+      }
+      const float dx = delta * xv;
+      const float dl = delta * kLog2e;
+      float4 s4 = st[i];
+      s4.x = fmaf(s4.x, ex2_approx(dl * a4.x), dx * b4.x);
+      s4.y = fmaf(s4.y, ex2_approx(dl * a4.y), dx * b4.y);
+      s4.z = fmaf(s4.z, ex2_approx(dl * a4.z), dx * b4.z);
+      s4.w = fmaf(s4.w, ex2_approx(dl * a4.w), dx * b4.w);
+      __stcs(reinterpret_cast<float4 *>(p.state + bd[i] * N + 4 * g), s4);
+      acc = fmaf(s4.x, c4.x, fmaf(s4.y, c4.y, fmaf(s4.z, c4.z, s4.w * c4.w)));
+    }
+#pragma unroll
+    for (int m = 1; m < G; m <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    if constexpr (CONV) {
+      __syncwarp();  // every lane of the channel has read the old window
+      if (on[i]) conv_store<T, G>(p, bd[i], g, nw);
+    }
+    if (on[i] && g == 0) {
+      float yv = fmaf(p.D ? p.D[d] : 0.0f, xv, acc);
+      if (zs) yv *= silu_for<T>(Elem<T>::load(zs, bd[i]));
+      Elem<T>::store(static_cast<T *>(p.y), bd[i], yv);
+    }
+  }
 }
 
 }  // namespace ssm
