@@ -102,8 +102,8 @@ struct Ss2dCfg {
   static constexpr int OFF_B = OFF_U + LC * ROWB;
   static constexpr int OFF_C = OFF_B + (LC + BC_PAD) * ESZ;
   static constexpr int OFF_AGG = (OFF_C + (LC + BC_PAD) * ESZ + 15) / 16 * 16;  // float4 [WARPS][PAIRS]
-  static constexpr int OFF_CARRY = OFF_AGG + WARPS * PAIRS * 16;              // float [8]
-  static constexpr int OFF_ROW = OFF_CARRY + 32;   // int [LC]: accumulator row of each step
+  static constexpr int OFF_CARRY = OFF_AGG + WARPS * PAIRS * 16;              // float [2][8]
+  static constexpr int OFF_ROW = OFF_CARRY + 64;   // int [LC]: accumulator row of each step
   static constexpr int OFF_ACC = (OFF_ROW + LC * 4 + 15) / 16 * 16;           // float [L][8]
   static constexpr int AUX_BYTES = OFF_ACC;
   static_assert(TS % 2 == 1, "TS odd keeps the warp's segments on distinct bank groups");
@@ -246,14 +246,19 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     cp_async_commit();
   };
 
-  if (tid < DT) carry[tid] = 0.0f;  // the first direction starts from h = 0
+  if (tid < DT) carry[tid] = 0.0f;  // the first direction starts from h = 0 (buffer 0)
   prefetch(0, 0);
   float2 A2 = make_float2(0.0f, 0.0f), bias = A2, Dd = A2;
 
   // one chunk of direction K (index arithmetic specialised per direction)
+  // chunk q = k nchunks + c reads the carry in buffer q & 1 and leaves the
+  // next one in the other buffer, so consecutive chunks need no barrier
+  // between them (their pixels differ); a direction's last chunk ends with
+  // one, since the next direction revisits every pixel.
   auto chunk = [&](auto kc, int c) {
     constexpr int K = decltype(kc)::value;
     const int l0 = c * LC;
+    const int cq = (K * nchunks + c) & 1;
     [[maybe_unused]] const T *Bk = gB + (int64_t)K * L;
     [[maybe_unused]] const T *Ck = gC + (int64_t)K * L;
     cp_async_wait<0>();
@@ -321,7 +326,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     __syncthreads();
 
     // ---- 3. incoming state: previous chunk's carry, earlier warps, earlier segments
-    float2 h = make_float2(carry[2 * cp], carry[2 * cp + 1]);
+    float2 h = make_float2(carry[cq * DT + 2 * cp], carry[cq * DT + 2 * cp + 1]);
     for (int w = 0; w < warp; ++w) {
       const float4 g4 = agg[w * Cfg::PAIRS + cp];
       h = __ffma2_rn(make_float2(g4.x, g4.y), h, make_float2(g4.z, g4.w));
@@ -346,11 +351,11 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
         }
       }
     }
-    __syncthreads();  // chunk's accumulator updates and carry reads done
-    if (warp == WARPS - 1 && sl == Cfg::SPW - 1) {
-      const bool last = c == nchunks - 1;  // the next direction starts from h = 0
-      carry[2 * cp] = last ? 0.0f : h.x;
-      carry[2 * cp + 1] = last ? 0.0f : h.y;
+    const bool last = c == nchunks - 1;
+    if (last) __syncthreads();  // the next direction's updates touch the same pixels
+    if (warp == WARPS - 1 && sl == Cfg::SPW - 1) {  // the next direction starts from h = 0
+      carry[(cq ^ 1) * DT + 2 * cp] = last ? 0.0f : h.x;
+      carry[(cq ^ 1) * DT + 2 * cp + 1] = last ? 0.0f : h.y;
     }
   };
 
