@@ -136,14 +136,19 @@ __device__ __forceinline__ void load_bc(const float *s, float (&b)[NPT], float (
   }
 }
 
-// Sum of the G consecutive partials starting at s.
+// Sum of the G consecutive partials starting at s, read by the lane of
+// channel pch.  With more than one 16-byte group per lane the lanes start at
+// rotated groups, so the eight lanes of a quarter warp (G floats apart) hit
+// eight different bank groups.
 template <int G>
-__device__ __forceinline__ float sum_partials(const float *s) {
+__device__ __forceinline__ float sum_partials(const float *s, int pch) {
   float acc = 0.0f;
   if constexpr (G % 4 == 0) {
+    constexpr int M = G / 4;  // 16-byte groups per lane
+    const int rot = M > 1 ? (pch >> (M >= 8 ? 0 : (M == 4 ? 1 : 2))) & (M - 1) : 0;
 #pragma unroll
-    for (int k = 0; k < G; k += 4) {
-      const float4 w = *reinterpret_cast<const float4 *>(s + k);
+    for (int k = 0; k < M; ++k) {
+      const float4 w = *reinterpret_cast<const float4 *>(s + 4 * ((k + rot) & (M - 1)));
       acc += (w.x + w.y) + (w.z + w.w);
     }
   } else if constexpr (G == 2) {
@@ -383,7 +388,7 @@ __global__ void __launch_bounds__(128, 4) scan_bwd_kernel(BwdParams p) {
 #pragma unroll
       for (int j = 0; j < NPT; ++j) acc[j] = 0.0f;
       const float *xs = sH + t * HROW + gi * NPT;
-#pragma unroll 4
+#pragma unroll 8
       for (int cc = 0; cc < DT; ++cc) {
         const float *qw = reinterpret_cast<const float *>(sQ + t * PROW + cc);
         const float w = use_g ? qw[2] : qw[1];
@@ -460,9 +465,9 @@ __global__ void __launch_bounds__(128, 4) scan_bwd_kernel(BwdParams p) {
       const int t = i / DT;  // i % DT == pch
       const int64_t dd = d0 + pch;
       const int s = t * PROW + pch;
-      const float S1 = sum_partials<G>(sP1 + t * NT + pch * G);
-      const float S2 = sum_partials<G>(sP2 + t * NT + pch * G);
-      const float yp = sum_partials<G>(sPy + t * NT + pch * G);
+      const float S1 = sum_partials<G>(sP1 + t * NT + pch * G, pch);
+      const float S2 = sum_partials<G>(sP2 + t * NT + pch * G, pch);
+      const float yp = sum_partials<G>(sPy + t * NT + pch * G, pch);
       const float4 qv = sQ[s];
       const float gt = qv.z, dl = qv.x, uu = sU[s];
       const float ddt = fmaf(uu, S1, S2) * sSpg[s];
