@@ -41,8 +41,9 @@
  *   - Outputs must not alias inputs unless stated.
  *   - dtype: SSM_F32 or SSM_BF16 applies to every activation-sized tensor of
  *     the call (u, delta, z, B, C, y / x, dt); A, D, dt_bias and every
- *     recurrent state are always fp32.  Arithmetic is fp32 throughout; the
- *     output is rounded once to `dtype`.
+ *     recurrent state are always fp32, and so are the backward's sums over
+ *     channels or batch (dA, dB, dC, dD, ddt_bias, dh0).  Arithmetic is fp32
+ *     throughout; each output is rounded once to its type.
  *   - d_state (N) must be one of 1, 2, 4, 8, 16, 32, 64; other values return
  *     SSM_ERR_UNSUPPORTED.  Any b, L, d_in >= 0 is accepted; b, L or d_in of
  *     0 is a valid empty problem.  Sizes whose element counts overflow int64

@@ -327,9 +327,13 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
 
     // ---- 3. incoming state: previous chunk's carry, earlier warps, earlier segments
     float2 h = make_float2(carry[cq * DT + 2 * cp], carry[cq * DT + 2 * cp + 1]);
-    for (int w = 0; w < warp; ++w) {
-      const float4 g4 = agg[w * Cfg::PAIRS + cp];
-      h = __ffma2_rn(make_float2(g4.x, g4.y), h, make_float2(g4.z, g4.w));
+    {  // all warp totals are loaded at once; earlier warps' maps applied in order
+      float4 g4[WARPS - 1];
+#pragma unroll
+      for (int w = 0; w < WARPS - 1; ++w) g4[w] = agg[w * Cfg::PAIRS + cp];
+#pragma unroll
+      for (int w = 0; w < WARPS - 1; ++w)
+        if (w < warp) h = __ffma2_rn(make_float2(g4[w].x, g4[w].y), h, make_float2(g4[w].z, g4[w].w));
     }
     h = __ffma2_rn(exc.a, h, exc.b);
 
