@@ -1,9 +1,12 @@
-"""Writes tests/golden/tiny_fp32_scan.json from the fp64 oracle ONLY.
+"""Writes tests/golden/tiny_fp32_scan.json (and tiny_fp32_scan_bwd.json) from
+the fp64 oracle ONLY.
 
 The tiny fp32 workload (b=2, L=64, d_in=32, N=16, seed 0: the Mamba block of
 "代码连连看——mamba"'s usage example, d_model=16, expand=2, d_state=16) is run
 through ``oracle.selective_scan``; 64 sampled outputs, the last state's
-per-batch sums and the whole-output sum are stored.  The test
+per-batch sums and the whole-output sum are stored; for the backward
+(``oracle.selective_scan_bwd`` with dout ~ N(0, 1) from torch seed 1) the
+sum and a sample of every gradient.  The test
 ``tests/test_golden.py`` checks the oracle still reproduces them, so an
 accidental change to the oracle's arithmetic is visible in review.
 
@@ -44,6 +47,20 @@ def main():
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "tiny_fp32_scan.json")
     with open(path, "w") as f:
         json.dump(out, f, indent=1)
+    print("wrote", path)
+
+    import torch
+    dout = torch.randn(y.shape, generator=torch.Generator().manual_seed(1))
+    g = oracle.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dout,
+                                  D=inp["D"], z=inp["z"], dt_bias=inp["dt_bias"])
+    bwd = {"workload": w.name, "dims": d, "seed": w.seed, "dout_seed": 1,
+           "source": "oracle.selective_scan_bwd (fp64), tests/golden/make_golden.py",
+           "sums": {k: float(v.sum()) for k, v in g.items()},
+           "samples": {k: [float(x) for x in v.ravel()[:: max(1, v.size // 16)][:16]]
+                       for k, v in g.items()}}
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "tiny_fp32_scan_bwd.json")
+    with open(path, "w") as f:
+        json.dump(bwd, f, indent=1)
     print("wrote", path)
 
 
