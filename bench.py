@@ -141,6 +141,8 @@ def measured_peaks():
 # device helpers, and the launch-shape knobs of the dispatcher.
 KERNEL_SOURCES = {"scan": "scan_fwd.cuh", "ss2d": "ss2d_fwd.cuh", "step": "state_update.cuh",
                   "scan_bwd": "scan_bwd.cuh", "scan_bwd_saved": "scan_bwd.cuh"}
+KERNEL_KNOBS = {"scan": ("SSM_SCAN_",), "ss2d": ("SSM_SS2D_",), "step": ("SSM_STEP_", "SSM_CONV_"),
+                "scan_bwd": ("SSM_BWD_",), "scan_bwd_saved": ("SSM_BWD_",)}
 
 
 def source_hash(kind: str = "") -> str:
@@ -153,8 +155,9 @@ def source_hash(kind: str = "") -> str:
         files = [KERNEL_SOURCES[kind], "ssm_common.cuh"]
     for fn in files:
         h.update(open(os.path.join(csrc, fn), "rb").read())
+    knobs = KERNEL_KNOBS.get(kind, ("SSM_",))
     for line in open(os.path.join(csrc, "ssmscan.cu"), encoding="utf-8"):
-        if line.startswith("#define SSM_"):
+        if line.startswith("#define ") and line[8:].startswith(knobs):
             h.update(line.encode())
     return h.hexdigest()[:16]
 

@@ -124,7 +124,10 @@ ssm_status launch_scan_fast_npt(const ssm::ScanParams &p, cudaStream_t st) {
 // Fewer channels leave fewer warps per SM: split each channel's states over
 // more threads (2 per thread instead of 4) when b * d_in is below the size
 // where the measured crossover lies.
-constexpr int64_t kScanSplitChannels = 12288;
+#ifndef SSM_SCAN_SPLIT_CHANNELS
+#define SSM_SCAN_SPLIT_CHANNELS 12288
+#endif
+constexpr int64_t kScanSplitChannels = SSM_SCAN_SPLIT_CHANNELS;
 
 template <typename T, int N, bool HAS_Z>
 ssm_status launch_scan_fast(const ssm::ScanParams &p, cudaStream_t st) {

@@ -41,6 +41,11 @@ struct StepParams {
 // window entries it owns into nw.  Every value in the window is an input of
 // the activation dtype, so storing it back is exact.
 constexpr int kMaxConv = 8;
+
+// CTAs of 256 threads the decode kernels are compiled to fit per SM.
+#ifndef SSM_STEP_MIN_CTAS
+#define SSM_STEP_MIN_CTAS 8
+#endif
 template <int G> constexpr int conv_taps_per_lane() { return (kMaxConv + G - 1) / G; }
 
 // This lane's taps of the old window (the tap that takes x is left for
@@ -166,7 +171,7 @@ __global__ void __launch_bounds__(256) state_update_kernel(StepParams p) {
 // 16-byte state loads are in flight per thread and every warp instruction
 // still touches one contiguous 512-byte span of the state.
 template <typename T, int N, int CPT, bool CONV>
-__global__ void __launch_bounds__(256) state_update_vec_kernel(StepParams p) {
+__global__ void __launch_bounds__(256, SSM_STEP_MIN_CTAS) state_update_vec_kernel(StepParams p) {
   constexpr int G = N / 4;
   static_assert(N % 4 == 0 && G <= 32 && 32 % G == 0, "bad N");
   const int64_t total = p.b * p.d_in;                 // channels
