@@ -188,3 +188,23 @@ def test_conv_step_rejects_bad_d_conv(ssm):
             ssm._ptr(inp["dt"]), ssm._ptr(inp["A"]), ssm._ptr(inp["B"]), ssm._ptr(inp["C"]), None,
             None, None, 1, ssm._ptr(torch.empty(1, 8, device="cuda")), 1, 8, 16, 0, None)
         assert st != 0 and "d_conv" in ssm.last_error()
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("b,d_in,N", [(3, 1000, 16), (8, 8192, 16), (5, 40, 4), (2, 616, 64)])
+def test_step_large_and_ragged(ssm, dtype, b, d_in, N):
+    """Channel counts that are not multiples of a CTA's channels, more
+    channels than one wave of CTAs covers, N = 4 and N = 64; three steps in a
+    row from the updated state."""
+    dt = "bf16" if dtype == torch.bfloat16 else "fp32"
+    inp = step_inputs(b, d_in, N, dt, seed=b + d_in + N)
+    g = to_cuda(inp)
+    st = g["state"].clone()
+    o_st = inp["state"]
+    for _ in range(3):
+        y = gpu_step(ssm, g, st)
+        y_ref, o_st = oracle.state_update(o_st, inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"],
+                                          D=inp["D"], z=inp["z"], dt_bias=inp["dt_bias"])
+        assert rel_err(y, y_ref) <= TOL[dtype]
+    assert rel_err(st, o_st) <= 1e-5
+    ssm.check_device_errors()
