@@ -47,6 +47,12 @@ def test_traffic_is_null_when_kernels_changed(tmp_path, monkeypatch):
     f.write_text(json.dumps({"w": {"dram_bytes_per_launch": 123,
                                    "source_hash": bench.source_hash()}}))
     assert bench.traffic_for("w") == 123
+    # per kernel: a workload's figure is tied to its own kernel's sources
+    f.write_text(json.dumps({"w": {"dram_bytes_per_launch": 7,
+                                   "source_hash": bench.source_hash("ss2d")}}))
+    assert bench.traffic_for("w", "ss2d") == 7
+    assert bench.traffic_for("w", "scan") is None
+    assert bench.source_hash("scan") != bench.source_hash("ss2d")
 
 
 def test_reference_arm_non_zero_rank_exits_without_work():
