@@ -131,3 +131,84 @@ def test_binding_rejects_wrong_tensors():
     u = torch.zeros(1, 4, 8)
     with pytest.raises((ValueError, TypeError)):
         S.ssm_scan_fwd(u, u, torch.zeros(8, 16), torch.zeros(1, 4, 16), torch.zeros(1, 4, 15))
+
+
+def bwd(saved=False, **kw):
+    a = dict(u=FAKE, delta=FAKE, A=FAKE, B=FAKE, C=FAKE, D=None, z=None, dt_bias=None, sp=1,
+             h0=None, dout=FAKE + 1024, dh_last=None, du=FAKE + 4096, ddelta=FAKE + 8192,
+             dA=FAKE + 12288, dB=FAKE + 16384, dC=FAKE + 20480, dD=None, dz=None, ddt_bias=None,
+             dh0=None, b=2, L=40, d_in=16, N=16, dtype=S.SSM_BF16, ws=FAKE + 65536,
+             ws_bytes=1 << 20, stream=None)
+    a.update(kw)
+    if saved:
+        return L.ssm_scan_bwd_saved(a["u"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"],
+                                    a["dt_bias"], a["sp"], a["dout"], a["dh_last"], a["du"],
+                                    a["ddelta"], a["dA"], a["dB"], a["dC"], a["dD"], a["dz"],
+                                    a["ddt_bias"], a["dh0"], a["b"], a["L"], a["d_in"], a["N"],
+                                    a["dtype"], a["ws"], a["ws_bytes"], a["stream"])
+    return L.ssm_scan_bwd(a["u"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"], a["dt_bias"],
+                          a["sp"], a["h0"], a["dout"], a["dh_last"], a["du"], a["ddelta"], a["dA"],
+                          a["dB"], a["dC"], a["dD"], a["dz"], a["ddt_bias"], a["dh0"], a["b"], a["L"],
+                          a["d_in"], a["N"], a["dtype"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("saved", [False, True])
+@pytest.mark.parametrize("kw,status", [
+    (dict(b=-1), S.SSM_ERR_INVALID_ARG),
+    (dict(N=12), S.SSM_ERR_UNSUPPORTED),
+    (dict(dtype=3), S.SSM_ERR_UNSUPPORTED),
+    (dict(ws_bytes=16), S.SSM_ERR_WORKSPACE),
+    (dict(ws=None), S.SSM_ERR_WORKSPACE),
+    (dict(b=70000, L=1, d_in=8, ws_bytes=1 << 30), S.SSM_ERR_UNSUPPORTED),  # grid.y limit
+    (dict(dA=None), S.SSM_ERR_INVALID_ARG),
+    (dict(dout=None), S.SSM_ERR_INVALID_ARG),
+    (dict(du=FAKE), S.SSM_ERR_INVALID_ARG),           # an output aliases an input
+    (dict(dB=FAKE + 12288), S.SSM_ERR_INVALID_ARG),   # two outputs share a buffer
+    (dict(dout=ODD), S.SSM_ERR_INVALID_ARG),
+    (dict(b=0), S.SSM_OK),
+])
+def test_bwd_validation(saved, kw, status):
+    assert bwd(saved=saved, **kw) == status
+    if status != S.SSM_OK:
+        assert S.last_error() != ""
+
+
+def test_bwd_workspace_query():
+    assert S.ssm_scan_bwd_workspace_bytes(8, 2048, 1536, 16) == 8 * 128 * 1536 * 16 * 4
+    assert S.ssm_scan_bwd_workspace_bytes(1, 17, 3, 4) == 1 * 2 * 3 * 4 * 4   # ceil(17 / 16) chunks
+    assert L.ssm_scan_bwd_workspace_bytes(1, 1, 1, 3) == ctypes.c_size_t(-1).value
+
+
+def test_fwd_save_validation():
+    args = lambda cs, nbytes, b=2: (FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 1, None, None,
+                                    FAKE + 4096, cs, nbytes, b, 40, 16, 16, S.SSM_BF16, None)
+    need = S.ssm_scan_bwd_workspace_bytes(2, 40, 16, 16)
+    assert L.ssm_scan_fwd_save(*args(FAKE + 65536, need - 16)) == S.SSM_ERR_WORKSPACE
+    assert L.ssm_scan_fwd_save(*args(None, need)) == S.SSM_ERR_WORKSPACE
+    assert L.ssm_scan_fwd_save(*args(FAKE + 65540, need)) == S.SSM_ERR_INVALID_ARG  # misaligned
+    assert L.ssm_scan_fwd_save(*args(FAKE, need)) == S.SSM_ERR_INVALID_ARG         # aliases u
+    assert L.ssm_scan_fwd_save(*args(None, 0, b=0)) == S.SSM_OK
+
+
+def conv_step(**kw):
+    a = dict(cs=FAKE + 32768, w=FAKE + 40960, cb=None, K=4, state=FAKE, x=FAKE + 1024,
+             dt=FAKE + 2048, A=FAKE + 3072, B=FAKE + 5120, C=FAKE + 6144, D=None, z=None,
+             dt_bias=None, sp=1, y=FAKE + 8192, b=2, d_in=16, N=16, dtype=S.SSM_BF16, stream=None)
+    a.update(kw)
+    return L.ssm_conv_state_update(a["cs"], a["w"], a["cb"], a["K"], a["state"], a["x"], a["dt"],
+                                   a["A"], a["B"], a["C"], a["D"], a["z"], a["dt_bias"], a["sp"],
+                                   a["y"], a["b"], a["d_in"], a["N"], a["dtype"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(K=0), S.SSM_ERR_UNSUPPORTED),
+    (dict(K=9), S.SSM_ERR_UNSUPPORTED),
+    (dict(cs=None), S.SSM_ERR_INVALID_ARG),
+    (dict(w=None), S.SSM_ERR_INVALID_ARG),
+    (dict(cs=FAKE + 1024), S.SSM_ERR_INVALID_ARG),    # conv_state aliases x
+    (dict(w=FAKE + 2), S.SSM_ERR_INVALID_ARG),        # misaligned fp32 weight
+    (dict(N=7), S.SSM_ERR_UNSUPPORTED),
+    (dict(b=0), S.SSM_OK),
+])
+def test_conv_step_validation(kw, status):
+    assert conv_step(**kw) == status
