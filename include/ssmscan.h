@@ -37,6 +37,10 @@
  *     reported by the call that launched.  Errors found by a kernel at run
  *     time (a bounded wait that ran out) are reported by
  *     ssm_check_device_errors().
+ *   - Calls allocate nothing and never synchronise, so they can be captured
+ *     in a CUDA graph; make the first call of each kind and d_state outside
+ *     any capture (it sets the kernel's shared-memory attribute once per
+ *     device).
  *   - A non-OK status leaves a message in ssm_last_error() (per thread).
  *   - Outputs must not alias inputs unless stated.
  *   - dtype: SSM_F32 or SSM_BF16 applies to every activation-sized tensor of
