@@ -15,7 +15,8 @@
 // One CTA owns DT channels of one batch for the whole sequence; G = N / NPT
 // threads share a channel, NPT states each.
 //   pass 1  walks the sequence forwards and saves the state at the start of
-//           every TT-step chunk in the caller's workspace;
+//           every TT-step chunk in the caller's workspace (skipped when the
+//           forward already saved them there: states_saved);
 //   pass 2  walks the chunks backwards.  Per chunk: recompute the states
 //           from the saved start into shared memory (with each thread's
 //           partial C.h); dC_t = sum over channels of g_t h_t as a column
@@ -25,7 +26,9 @@
 //           lam_t delta_t u_t as a second column pass; and a pass per
 //           (step, channel) that adds the G partials and writes du, ddelta
 //           and dz.
-// Nothing in the per-step loops crosses lanes, so each step's critical
+// A chunk's inputs are copied into shared memory one chunk ahead (cp.async)
+// when they are 16-byte aligned.  Nothing in the per-step loops crosses
+// lanes, so each step's critical
 // path is the adjoint's own FMA chain.  dB and dC rows of the chunk go to
 // the fp32 outputs with (vector) global atomics, one per CTA and row;
 // dA, dD and ddt_bias are added once per CTA at the end.
