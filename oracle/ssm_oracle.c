@@ -22,7 +22,7 @@
  *   [VMamba-206]    "关于代码SS2D中的d_state设置" (VMamba issue 206):
  *                   CrossScan / CrossMerge only arrange the sequence.
  *
- * Readings where the pages are silent (each also listed in the design doc):
+ * Readings where the pages are silent:
  *   - softplus is torch's F.softplus: x for x > 20, log1p(exp(x)) otherwise.
  *   - dt_bias is added before the softplus, whether or not softplus is on.
  *   - y uses the state AFTER the update of the same step ([Minimal-scan] §4:
