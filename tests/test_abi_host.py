@@ -56,6 +56,10 @@ def scan(**kw):
     (dict(A=FAKE + 2), S.SSM_ERR_INVALID_ARG),
     (dict(h0=FAKE + 1), S.SSM_ERR_INVALID_ARG),
     (dict(y=FAKE), S.SSM_ERR_INVALID_ARG),            # y aliases u
+    (dict(y=FAKE + 2), S.SSM_ERR_INVALID_ARG),        # y overlaps u, shifted by one element
+    (dict(y=FAKE + 510), S.SSM_ERR_INVALID_ARG),      # y starts on u's last element
+    (dict(y=FAKE + 512), S.SSM_ERR_INVALID_ARG),      # y overlaps A (d_in * N * 4 bytes at FAKE)
+    (dict(y=FAKE + 4096, h_last=FAKE + 4096 + 256), S.SSM_ERR_INVALID_ARG),  # h_last overlaps y
     (dict(b=0), S.SSM_OK),                            # empty problem, no CUDA call
     (dict(d_in=0), S.SSM_OK),
 ])
@@ -89,6 +93,7 @@ def ss2d(**kw):
     (dict(dtype=5), S.SSM_ERR_UNSUPPORTED),
     (dict(delta=None), S.SSM_ERR_INVALID_ARG),
     (dict(y=FAKE), S.SSM_ERR_INVALID_ARG),
+    (dict(y=FAKE + 2558), S.SSM_ERR_INVALID_ARG),     # y overlaps delta's last element
     (dict(B=ODD), S.SSM_ERR_INVALID_ARG),
     (dict(H=100, W=100), S.SSM_ERR_WORKSPACE),        # accumulator needs the workspace
     (dict(b=0), S.SSM_OK),
@@ -99,8 +104,8 @@ def test_ss2d_validation(kw, status):
 
 
 def step(**kw):
-    a = dict(state=FAKE, x=FAKE, dt=FAKE, A=FAKE, B=FAKE, C=FAKE, D=None, z=None, dt_bias=None,
-             sp=1, y=FAKE + 4096, b=2, d_in=16, N=16, dtype=S.SSM_BF16, stream=None)
+    a = dict(state=FAKE + 65536, x=FAKE, dt=FAKE, A=FAKE, B=FAKE, C=FAKE, D=None, z=None,
+             dt_bias=None, sp=1, y=FAKE + 4096, b=2, d_in=16, N=16, dtype=S.SSM_BF16, stream=None)
     a.update(kw)
     return L.ssm_state_update(a["state"], a["x"], a["dt"], a["A"], a["B"], a["C"], a["D"], a["z"],
                               a["dt_bias"], a["sp"], a["y"], a["b"], a["d_in"], a["N"], a["dtype"],
@@ -112,7 +117,9 @@ def step(**kw):
     (dict(N=5), S.SSM_ERR_UNSUPPORTED),
     (dict(state=None), S.SSM_ERR_INVALID_ARG),
     (dict(state=FAKE + 2), S.SSM_ERR_INVALID_ARG),
-    (dict(y=FAKE), S.SSM_ERR_INVALID_ARG),            # y aliases the state
+    (dict(y=FAKE + 65536), S.SSM_ERR_INVALID_ARG),    # y aliases the state
+    (dict(y=FAKE + 65536 + 2046), S.SSM_ERR_INVALID_ARG),  # y overlaps the state's last bytes
+    (dict(state=FAKE + 32), S.SSM_ERR_INVALID_ARG),   # the state overlaps x
     (dict(x=ODD), S.SSM_ERR_INVALID_ARG),
     (dict(b=0), S.SSM_OK),
 ])
@@ -122,6 +129,9 @@ def test_step_validation(kw, status):
 
 def test_cross_permutation_validation():
     assert L.ss2d_cross_scan(None, FAKE, 1, 2, 2, 4, S.SSM_BF16, None) == S.SSM_ERR_INVALID_ARG
+    # xs (1 x 4 x 4 x 4 bf16, 128 bytes) must not overlap u (32 bytes)
+    assert L.ss2d_cross_scan(FAKE, FAKE + 16, 1, 2, 2, 4, S.SSM_BF16, None) == S.SSM_ERR_INVALID_ARG
+    assert L.ss2d_cross_merge(FAKE, FAKE + 96, 1, 2, 2, 4, S.SSM_BF16, None) == S.SSM_ERR_INVALID_ARG
     assert L.ss2d_cross_merge(FAKE, FAKE + 64, -1, 2, 2, 4, S.SSM_BF16, None) == S.SSM_ERR_INVALID_ARG
     assert L.ss2d_cross_scan(FAKE, FAKE + 64, 0, 2, 2, 4, S.SSM_BF16, None) == S.SSM_OK
 
@@ -136,7 +146,7 @@ def test_binding_rejects_wrong_tensors():
 def bwd(saved=False, **kw):
     a = dict(u=FAKE, delta=FAKE, A=FAKE, B=FAKE, C=FAKE, D=None, z=None, dt_bias=None, sp=1,
              h0=None, dout=FAKE + 1024, dh_last=None, du=FAKE + 4096, ddelta=FAKE + 8192,
-             dA=FAKE + 12288, dB=FAKE + 16384, dC=FAKE + 20480, dD=None, dz=None, ddt_bias=None,
+             dA=FAKE + 12288, dB=FAKE + 16384, dC=FAKE + 24576, dD=None, dz=None, ddt_bias=None,
              dh0=None, b=2, L=40, d_in=16, N=16, dtype=S.SSM_BF16, ws=FAKE + 65536,
              ws_bytes=1 << 20, stream=None)
     a.update(kw)
@@ -164,6 +174,8 @@ def bwd(saved=False, **kw):
     (dict(dout=None), S.SSM_ERR_INVALID_ARG),
     (dict(du=FAKE), S.SSM_ERR_INVALID_ARG),           # an output aliases an input
     (dict(dB=FAKE + 12288), S.SSM_ERR_INVALID_ARG),   # two outputs share a buffer
+    (dict(dC=FAKE + 20480), S.SSM_ERR_INVALID_ARG),   # dC overlaps the end of dB
+    (dict(ddelta=FAKE + 2048), S.SSM_ERR_INVALID_ARG),  # ddelta overlaps u and dout
     (dict(dout=ODD), S.SSM_ERR_INVALID_ARG),
     (dict(b=0), S.SSM_OK),
 ])
@@ -187,13 +199,22 @@ def test_fwd_save_validation():
     assert L.ssm_scan_fwd_save(*args(None, need)) == S.SSM_ERR_WORKSPACE
     assert L.ssm_scan_fwd_save(*args(FAKE + 65540, need)) == S.SSM_ERR_INVALID_ARG  # misaligned
     assert L.ssm_scan_fwd_save(*args(FAKE, need)) == S.SSM_ERR_INVALID_ARG         # aliases u
+    assert L.ssm_scan_fwd_save(*args(FAKE + 6144, need)) == S.SSM_ERR_INVALID_ARG  # overlaps y
     assert L.ssm_scan_fwd_save(*args(None, 0, b=0)) == S.SSM_OK
 
 
+def test_h_last_may_equal_h0_but_not_overlap_it():
+    # L = 0 returns before any launch when h_last is h0 itself
+    H0 = FAKE + 16384
+    assert scan(L=0, h0=H0, h_last=H0) == S.SSM_OK
+    assert scan(L=0, h0=H0, h_last=H0 + 4) == S.SSM_ERR_INVALID_ARG
+    assert scan(L=0, h0=H0, h_last=H0 - 2044) == S.SSM_ERR_INVALID_ARG
+
+
 def conv_step(**kw):
-    a = dict(cs=FAKE + 32768, w=FAKE + 40960, cb=None, K=4, state=FAKE, x=FAKE + 1024,
-             dt=FAKE + 2048, A=FAKE + 3072, B=FAKE + 5120, C=FAKE + 6144, D=None, z=None,
-             dt_bias=None, sp=1, y=FAKE + 8192, b=2, d_in=16, N=16, dtype=S.SSM_BF16, stream=None)
+    a = dict(cs=FAKE + 32768, w=FAKE + 40960, cb=None, K=4, state=FAKE, x=FAKE + 4096,
+             dt=FAKE + 5120, A=FAKE + 6144, B=FAKE + 8192, C=FAKE + 9216, D=None, z=None,
+             dt_bias=None, sp=1, y=FAKE + 12288, b=2, d_in=16, N=16, dtype=S.SSM_BF16, stream=None)
     a.update(kw)
     return L.ssm_conv_state_update(a["cs"], a["w"], a["cb"], a["K"], a["state"], a["x"], a["dt"],
                                    a["A"], a["B"], a["C"], a["D"], a["z"], a["dt_bias"], a["sp"],
@@ -205,7 +226,8 @@ def conv_step(**kw):
     (dict(K=9), S.SSM_ERR_UNSUPPORTED),
     (dict(cs=None), S.SSM_ERR_INVALID_ARG),
     (dict(w=None), S.SSM_ERR_INVALID_ARG),
-    (dict(cs=FAKE + 1024), S.SSM_ERR_INVALID_ARG),    # conv_state aliases x
+    (dict(cs=FAKE + 4096), S.SSM_ERR_INVALID_ARG),    # conv_state aliases x
+    (dict(cs=FAKE + 2000), S.SSM_ERR_INVALID_ARG),    # conv_state overlaps the ssm state
     (dict(w=FAKE + 2), S.SSM_ERR_INVALID_ARG),        # misaligned fp32 weight
     (dict(N=7), S.SSM_ERR_UNSUPPORTED),
     (dict(b=0), S.SSM_OK),
