@@ -5,13 +5,13 @@
                     [--workload NAME] [--no-e2e] [--no-cpu-baseline]
 
 A step is one pass of the hot path over one batch of synthetic input that is
-already resident in HBM.  The default workload is the Mamba-130M-shaped
-prefill scan (b=8, L=2048, d_in=1536, N=16, bf16 activations, fp32 state):
-the configuration the headline metric (Gelem/s = b L d_in N per second, and
-HBM GB/s as a fraction of the measured peak) is quoted on.  Other workloads
-(--workload mamba1.4b-long-scan | vmamba-ss2d | mamba-decode-step |
-mamba-decode-conv-step | mamba130m-scan-bwd | mamba130m-scan-bwd-saved |
-tiny-fp32-scan) measure the companion kernels.
+already resident in HBM.  The default workload is the long-sequence
+Mamba-1.4B-shaped scan (b=2, L=16384, d_in=4096, N=16, bf16 activations,
+fp32 state), the largest single-GPU configuration of the headline metric
+(Gelem/s = b L d_in N per second, and algorithmic HBM GB/s as a fraction of
+the measured peak).  Other workloads (--workload mamba130m-scan |
+vmamba-ss2d | mamba-decode-step | mamba-decode-conv-step | mamba130m-scan-bwd
+| mamba130m-scan-bwd-saved | tiny-fp32-scan) measure the companion kernels.
 
 Timing: W untimed warm-up steps, then exactly K timed steps bracketed by a
 barrier and torch.cuda.synchronize() on both sides; each step's kernel is
@@ -40,17 +40,16 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-DEFAULT_WORKLOAD = "mamba130m-scan"
+DEFAULT_WORKLOAD = "mamba1.4b-long-scan"
 METRIC = "selective-scan Gelem/s (b*L*d_in*N per second)"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK_HBM_GBS = 6650.0
 
-# Unit counts of one B200 SM used for the ALU roofline (measured on this
-# part with a throughput probe: 16 SFU ex2/lg2 lanes and 128 FP32 FMA lanes
-# per clock per SM), 148 SMs, 1965 MHz maximum SM clock.
-SMS, SFU_PER_CLK, FMA_PER_CLK, SM_MAX_HZ = 148, 16, 128, 1.965e9
-
+# SFU (MUFU) rate of one B200 SM, measured on this part with a throughput
+# probe (independent ex2.approx chains: 0.496 warp instructions per clock per
+# SM, i.e. 15.9 lanes), 148 SMs, 1965 MHz maximum SM clock.
+SMS, SFU_PER_CLK, SM_MAX_HZ = 148, 16, 1.965e9
 
 def parse_args():
     ap = argparse.ArgumentParser()
@@ -93,39 +92,30 @@ def alg_bytes(w) -> int:
     return step + (2 * b * di * K * es + di * K * 4 + di * 4 if K else 0)
 
 
-def alu_peak_elems_per_s(w) -> float:
-    """Element rate the SFU + FMA pipes allow for this workload's arithmetic.
+def sfu_ops_per_element(w) -> float:
+    """Transcendentals (SFU ops) the kernel issues per element.
 
-    Per element (b, t, d, n) the path needs one exp and F FMA-pipe ops;
-    per (b, t, d) it adds the softplus of delta (2 transcendentals) and, with
-    the gate, SiLU (2), so X = 1 + 4/N transcendentals per element (3 for
-    SS2D with N = 1: softplus + exp, no gate).  A transcendental costs one SFU
-    op or P = 8 FMA-pipe ops on the FMA pipe (range reduction + a degree-5
-    polynomial).  With a fraction f moved to the FMA pipe:
-        E X (1 - f) <= SFU,   E (F + X f P) <= FMA
-    whose best f gives  E = (FMA + P SFU) / (F + X P)  per SM per clock."""
+    Per element (b, t, d, n) one exp2 of delta A; per (b, t, d) the softplus
+    of delta (one exp2; its log1p is an FMA-pipe polynomial) and, with the
+    gate, SiLU (one tanh or exp2 + reciprocal, counted as one).  SS2D (N = 1)
+    has no gate: softplus + exp2 per (b, k, t, d).  The backward recomputes
+    the forward exponentials (pass 1 unless the states are saved, the chunk
+    recompute, the adjoint's decay) and takes the softplus, its derivative
+    and the gate's SiLU and derivative per (t, d)."""
     N = w.dims["N"]
     if w.kind == "ss2d":
-        X, F = 3.0, 12.0
-    elif w.kind == "scan_bwd_saved":
-        # the chunk states come from the forward: two passes over each
-        # element (recompute, adjoint), 2 exps and ~14 FMA-pipe ops; per
-        # (t, d) softplus once, its derivative and the gate's SiLU and
-        # derivative (7 / N)
-        X, F = 2.0 + 7.0 / N, 14.0
-    elif w.kind == "scan_bwd":
-        # three passes over each element (chunk states, recompute, adjoint):
-        # 3 exps and ~18 FMA-pipe ops; per (t, d) softplus twice, its
-        # derivative once and the gate's SiLU and derivative (8 / N)
-        X, F = 3.0 + 8.0 / N, 18.0
-    else:
-        X, F = 1.0 + 4.0 / N, 4.0
-    P = 8.0
-    e_clk = (FMA_PER_CLK + P * SFU_PER_CLK) / (F + X * P)      # both pipes saturated
-    f = 1.0 - SFU_PER_CLK / (e_clk * X)
-    if f < 0.0:                                                 # SFU alone suffices
-        e_clk = min(SFU_PER_CLK / X, FMA_PER_CLK / F)
-    return e_clk * SMS * SM_MAX_HZ
+        return 2.0
+    if w.kind == "scan_bwd":
+        return 3.0 + 6.0 / N
+    if w.kind == "scan_bwd_saved":
+        return 2.0 + 6.0 / N
+    return 1.0 + 2.0 / N
+
+
+def sfu_peak_elems_per_s(w) -> float:
+    """Element rate the SFU allows: the bound of a kernel that issues every
+    transcendental on it (all of this repository's kernels do)."""
+    return SFU_PER_CLK * SMS * SM_MAX_HZ / sfu_ops_per_element(w)
 
 
 def measured_peaks():
@@ -139,10 +129,12 @@ def measured_peaks():
 
 # The sources each workload's kernel is built from: its header, the shared
 # device helpers, and the launch-shape knobs of the dispatcher.
-KERNEL_SOURCES = {"scan": "scan_fwd.cuh", "ss2d": "ss2d_fwd.cuh", "step": "state_update.cuh",
-                  "scan_bwd": "scan_bwd.cuh", "scan_bwd_saved": "scan_bwd.cuh"}
-KERNEL_KNOBS = {"scan": ("SSM_SCAN_",), "ss2d": ("SSM_SS2D_",), "step": ("SSM_STEP_", "SSM_CONV_"),
-                "scan_bwd": ("SSM_BWD_",), "scan_bwd_saved": ("SSM_BWD_",)}
+KERNEL_SOURCES = {"scan": ("scan_ws.cuh", "scan_fwd.cuh"), "ss2d": ("ss2d_fwd.cuh",),
+                  "step": ("state_update.cuh",), "scan_bwd": ("scan_bwd.cuh",),
+                  "scan_bwd_saved": ("scan_bwd.cuh",)}
+KERNEL_KNOBS = {"scan": ("SSM_SCAN_", "SSM_WS_"), "ss2d": ("SSM_SS2D_",),
+                "step": ("SSM_STEP_", "SSM_CONV_"), "scan_bwd": ("SSM_BWD_",),
+                "scan_bwd_saved": ("SSM_BWD_",)}
 
 
 def source_hash(kind: str = "") -> str:
@@ -152,7 +144,7 @@ def source_hash(kind: str = "") -> str:
     csrc = os.path.join(ROOT, "selective_state_space_25_b200", "csrc")
     files = sorted(fn for fn in os.listdir(csrc) if fn.endswith((".cu", ".cuh")))
     if kind in KERNEL_SOURCES:
-        files = [KERNEL_SOURCES[kind], "ssm_common.cuh"]
+        files = [*KERNEL_SOURCES[kind], "ssm_common.cuh"]
     for fn in files:
         h.update(open(os.path.join(csrc, fn), "rb").read())
     knobs = KERNEL_KNOBS.get(kind, ("SSM_",))
@@ -353,9 +345,20 @@ def oracle_cores(w) -> int:
 
 
 def cpu_baseline(w, inp, target_s):
+    """The oracle on all of the host's cores (the reported value) and on one
+    core, each on a bounded sample of the workload."""
+    import oracle
     el, dt, desc = oracle_sample(w, inp, target_s)
+    n = oracle.num_threads()
+    oracle.set_num_threads(1)
+    try:
+        el1, dt1, desc1 = oracle_sample(w, inp, max(1.0, target_s / 4))
+    finally:
+        oracle.set_num_threads(n)
     return {"value": el / dt / 1e9, "unit": "Gelem/s", "cores": oracle_cores(w),
-            "kind": "oracle", "sample": desc + f" ({dt:.1f} s, fp64 C oracle, OpenMP)"}
+            "kind": "oracle", "sample": desc + f" ({dt:.1f} s, fp64 C oracle, OpenMP)",
+            "one_core": {"value": el1 / dt1 / 1e9, "unit": "Gelem/s", "cores": 1,
+                         "sample": desc1 + f" ({dt1:.1f} s)"}}
 
 
 # ------------------------------------------------------------------- drivers
@@ -462,28 +465,24 @@ def run_ours(args, w):
     ms_step = max_ms / K
     avg_launch_s = statistics.mean(per) * 1e-3
 
-    # ---- roofline of the (only) kernel of the step
+    # ---- roofline of the (only) kernel of the step: the algorithmic HBM
+    # bytes over its time against the measured copy bandwidth (the headline
+    # metric's fraction), with the SFU ceiling beside it
     hbm_peak, hbm_src = measured_peaks()
     abytes = alg_bytes(w)
     hbm_ach = abytes / avg_launch_s / 1e9
-    alu_peak = alu_peak_elems_per_s(w) / 1e9
-    alu_ach = w.elements() / avg_launch_s / 1e9
-    alu_time = w.elements() / (alu_peak * 1e9)
-    hbm_time = abytes / (hbm_peak * 1e9)
+    sfu_peak = sfu_peak_elems_per_s(w) / 1e9
+    el_ach = w.elements() / avg_launch_s / 1e9
     traffic = None if args.override else traffic_for(w.name, w.kind)
-    if alu_time > hbm_time:
-        roof = {"bound": "alu", "achieved": alu_ach, "peak": alu_peak, "unit": "Gelem/s",
-                "frac": alu_ach / alu_peak, "traffic": traffic,
-                "peak_source": "derived: SFU 16 + FMA 128 lanes/clk/SM x 148 SMs x 1965 MHz",
-                "hbm": {"achieved": hbm_ach, "peak": hbm_peak, "unit": "GB/s",
-                        "frac": hbm_ach / hbm_peak, "peak_source": hbm_src}}
-    else:
-        roof = {"bound": "hbm", "achieved": hbm_ach, "peak": hbm_peak, "unit": "GB/s",
-                "frac": hbm_ach / hbm_peak, "traffic": traffic,
-                "peak_source": f"{hbm_src} (MEASURED_PEAKS hbm_gbs)" if hbm_src == "measured" else hbm_src,
-                "alu": {"achieved": alu_ach, "peak": alu_peak, "unit": "Gelem/s",
-                        "frac": alu_ach / alu_peak}}
-    roof["algorithmic_bytes_per_launch"] = abytes
+    roof = {"bound": "hbm", "achieved": hbm_ach, "peak": hbm_peak, "unit": "GB/s",
+            "frac": hbm_ach / hbm_peak, "traffic": traffic,
+            "peak_source": (f"{hbm_src} (MEASURED_PEAKS hbm_gbs)" if hbm_src == "measured"
+                            else f"{hbm_src} ({FALLBACK_HBM_GBS:.0f} GB/s)"),
+            "algorithmic_bytes_per_launch": abytes,
+            "sfu": {"achieved": el_ach, "peak": sfu_peak, "unit": "Gelem/s",
+                    "frac": el_ach / sfu_peak, "sfu_ops_per_element": sfu_ops_per_element(w),
+                    "peak_source": "derived: 16 SFU lanes/clk/SM (measured 15.9) x 148 SMs "
+                                   "x 1965 MHz / SFU ops per element"}}
 
     # ---- end to end: host (pinned) buffers, copies inside the timed region
     e2e = None

@@ -87,11 +87,11 @@ typedef enum {
 } ssm_ss2d_order;
 
 /*
- * Bytes of device workspace ssm_scan_fwd needs for this problem (0 when the
- * launch it picks needs none).  The chunked path, which splits L across
- * thread blocks when b * d_in is too small to fill the GPU, keeps one fp32
- * (decay, state) pair per (batch, channel, state, chunk) there.  Returns
- * (size_t)-1 for invalid sizes.
+ * Bytes of device workspace ssm_scan_fwd needs for this problem.  Every
+ * kernel of this build keeps the recurrent state and its chunk carries on
+ * chip, so this is 0 for every valid size; callers that pass what it returns
+ * stay correct if a later build needs scratch.  Returns (size_t)-1 for
+ * invalid sizes.
  */
 size_t ssm_scan_fwd_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t d_state);
 
@@ -113,7 +113,7 @@ size_t ssm_scan_fwd_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t 
  *   h_last        device fp32 (b, d_in, d_state), nullable; may equal h0
  *   y             device, (b, L, d_in), dtype; must not alias an input
  *   workspace     device, >= ssm_scan_fwd_workspace_bytes(...) bytes; may be
- *                 NULL when that is 0.  Contents on entry are ignored.
+ *                 NULL when that is 0 (always, in this build).  Not read.
  */
 ssm_status ssm_scan_fwd(const void *u, const void *delta, const float *A,
                         const void *B, const void *C, const float *D,

@@ -89,34 +89,8 @@ __global__ void __launch_bounds__(128) scan_generic_kernel(ScanParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// Fast kernel.  A CTA owns (batch i, a tile of DT channels) for the whole
-// sequence and walks it in chunks of TC steps:
-//   1. the chunk's u / delta / z tile [TC x DT] and B / C rows [TC x N] are
-//      copied global -> shared with 16-byte cp.async, issued as soon as the
-//      previous chunk's u / delta / z tile has been consumed (B / C rows,
-//      which the scan reads, are double-buffered), so the copy overlaps that
-//      chunk's scan;
-//   2. pre-pass, one thread per (channel, 4 steps): delta = softplus(dt +
-//      bias), delta u, u and silu(z) are formed once per (t, d) (not once per
-//      state) and stored channel-major ([d][t], rows padded against bank
-//      conflicts) so the scan reads 4 steps of a channel in one 16-byte
-//      load; B, C rows are widened to fp32 once for all channels, laid out
-//      so each thread's states are one contiguous run.  Steps past the end
-//      of the sequence get delta = 0, which makes them identity steps;
-//   3. scan: G = N / NPT threads share a channel, each owning NPT states in
-//      registers, and take U = G steps per pass (4 when G = 1).  Per step and
-//      state pair: a packed multiply for delta A log2 e, two SFU exp2 (the
-//      last NPOLY pairs use the FMA-pipe polynomial instead), packed
-//      delta u * B, the packed recurrence FMA and the packed C.h FMA.  The U
-//      partial C.h sums of a pass meet in a reduce-scatter over the G lanes
-//      (log2 G shuffle rounds), leaving lane g with step g's sum;
-//   4. post-pass, one thread per (channel, 4 steps): y = (C.h + D u) silu(z),
-//      rounded once and stored (a warp writes whole channel rows).
-// Requires N % NPT == 0, TC % 4 == 0, d_in * sizeof(T) a multiple of 16 and
-// u, delta, z, B, C, y 16-byte aligned (checked by the launcher).
-// ---------------------------------------------------------------------------
-// ---------------------------------------------------------------------------
-// Fast kernel.  A CTA owns (batch i, a tile of DT channels) for the whole
+// Fast kernel (d_state 64; d_state 8 to 32 take the warp-specialised kernel of
+// scan_ws.cuh).  A CTA owns (batch i, a tile of DT channels) for the whole
 // sequence and walks it in chunks of TC steps:
 //   1. the chunk's u / delta / z tile [TC x DT] and B / C rows [TC x N] are
 //      copied global -> shared with 16-byte cp.async, issued as soon as the

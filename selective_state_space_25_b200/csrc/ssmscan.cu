@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 #include <string>
 #include <type_traits>
@@ -13,6 +14,7 @@
 #include "ssmscan.h"
 #include "scan_bwd.cuh"
 #include "scan_fwd.cuh"
+#include "scan_ws.cuh"
 #include "ss2d_fwd.cuh"
 #include "state_update.cuh"
 
@@ -44,6 +46,38 @@ bool supported_state(int64_t n) {
 size_t esize(ssm_dtype t) { return t == SSM_BF16 ? 2 : 4; }
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// A named byte range of one argument; NULL or empty ranges overlap nothing.
+struct Span {
+  const char *name;
+  const void *p;
+  int64_t bytes;
+};
+
+bool overlap(const Span &a, const Span &b) {
+  if (!a.p || !b.p || a.bytes <= 0 || b.bytes <= 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a.p), b0 = reinterpret_cast<uintptr_t>(b.p);
+  return a0 < b0 + (uintptr_t)b.bytes && b0 < a0 + (uintptr_t)a.bytes;
+}
+
+// Outputs (and in-place buffers) must not overlap an input or each other.
+// same_out / same_in name one output allowed to be exactly the given input
+// (the same address: h_last == h0); any other overlap is an error.
+ssm_status check_disjoint(const char *what, std::initializer_list<Span> outs,
+                          std::initializer_list<Span> ins, const void *same_out = nullptr,
+                          const void *same_in = nullptr) {
+  for (const Span &o : outs) {
+    for (const Span &i : ins) {
+      if (same_out && o.p == same_out && i.p == same_in && o.p == i.p && o.bytes == i.bytes) continue;
+      if (overlap(o, i))
+        return fail(SSM_ERR_INVALID_ARG, "%s: %s overlaps the input %s", what, o.name, i.name);
+    }
+    for (const Span &o2 : outs)
+      if (&o2 != &o && overlap(o, o2))
+        return fail(SSM_ERR_INVALID_ARG, "%s: outputs %s and %s overlap", what, o.name, o2.name);
+  }
+  return SSM_OK;
+}
 
 ssm_status check_launch(const char *what) {
   const cudaError_t e = cudaGetLastError();
@@ -136,9 +170,41 @@ ssm_status launch_scan_fast(const ssm::ScanParams &p, cudaStream_t st) {
   return launch_scan_fast_npt<T, N, HAS_Z, SSM_SCAN_NPT>(p, st);
 }
 
+// Warp-specialised scan (scan_ws.cuh): steps per chunk, helper warps, and
+// chunks copied ahead of the pre-pass.
+#ifndef SSM_WS_TC
+#define SSM_WS_TC 32
+#endif
+#ifndef SSM_WS_HELPERS
+#define SSM_WS_HELPERS 4
+#endif
+#ifndef SSM_WS_AHEAD
+#define SSM_WS_AHEAD 1
+#endif
+
+// States per scan thread of the warp-specialised kernel: 4 up to d_state 16,
+// 8 for 32 (four scan warps either way); 0 = not compiled for this d_state.
+constexpr int ws_states(int n) { return n == 8 || n == 16 ? 4 : (n == 32 ? 8 : 0); }
+
+template <typename T, int N, bool HAS_Z, bool SAVE>
+ssm_status launch_scan_ws(const ssm::ScanParams &p, cudaStream_t st) {
+  constexpr int NS = ws_states(N);
+  using Cfg = ssm::WsScan<T, N, NS, SSM_WS_TC, SSM_WS_HELPERS, SSM_WS_AHEAD>;
+  constexpr auto k =
+      ssm::scan_ws_kernel<T, N, NS, SSM_WS_TC, SSM_WS_HELPERS, SSM_WS_AHEAD, HAS_Z, SAVE>;
+  const dim3 grid((unsigned)((p.d_in + Cfg::DT - 1) / Cfg::DT), (unsigned)p.b);
+  return launch_fast_kernel<k>(p, grid, Cfg::THREADS, Cfg::SMEM, st);
+}
+
 template <typename T, int N>
 ssm_status launch_scan(const ssm::ScanParams &p, bool fast, cudaStream_t st) {
-  if constexpr (N >= 8) {
+  if constexpr (ws_states(N) > 0) {
+    if (fast) {
+      if (p.chunk_h)
+        return p.z ? launch_scan_ws<T, N, true, true>(p, st) : launch_scan_ws<T, N, false, true>(p, st);
+      return p.z ? launch_scan_ws<T, N, true, false>(p, st) : launch_scan_ws<T, N, false, false>(p, st);
+    }
+  } else if constexpr (N >= 8) {
     if (fast)
       return p.z ? launch_scan_fast<T, N, true>(p, st) : launch_scan_fast<T, N, false>(p, st);
   }
@@ -245,9 +311,11 @@ ssm_status check_step_args(const char *what, float *ssm_state, const void *x, co
   const void *f32[] = {ssm_state, A, D, dt_bias};
   for (const void *q : f32)
     if (q && !aligned(q, 4)) return fail(SSM_ERR_INVALID_ARG, "%s: fp32 pointer not 4-byte aligned", what);
-  if (y == x || y == dt || y == z || y == B || y == C || y == ssm_state)
-    return fail(SSM_ERR_INVALID_ARG, "%s: y must not alias an input", what);
-  return ok();
+  const int64_t na = b * d_in * (int64_t)es, ns = b * d_in * d_state * 4;
+  const int64_t nbc = b * d_state * (int64_t)es, np = d_in * 4;
+  return check_disjoint(what, {{"ssm_state", ssm_state, ns}, {"y", y, na}},
+                        {{"x", x, na}, {"dt", dt, na}, {"z", z, na}, {"B", B, nbc}, {"C", C, nbc},
+                         {"A", A, np * d_state}, {"D", D, np}, {"dt_bias", dt_bias, np}});
 }
 
 // ------------------------------------------------------------ SS2D launch
@@ -409,6 +477,17 @@ ssm_status scan_fwd_impl(const void *u, const void *delta, const float *A, const
   for (const void *q : f32)
     if (q && !aligned(q, 4))
       return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd: fp32 pointer not 4-byte aligned");
+  {
+    const int64_t ba = n_act * (int64_t)es, bbc = n_bc * (int64_t)es, bs = n_state * 4;
+    const int64_t nc = chunk_h ? (int64_t)ssm_scan_bwd_workspace_bytes(b, L, d_in, d_state) : 0;
+    if (ssm_status s = check_disjoint(
+            "ssm_scan_fwd", {{"y", y, ba}, {"h_last", h_last, bs}, {"chunk_states", chunk_h, nc}},
+            {{"u", u, ba}, {"delta", delta, ba}, {"z", z, ba}, {"B", B, bbc}, {"C", C, bbc},
+             {"A", A, d_in * d_state * 4}, {"D", D, d_in * 4}, {"dt_bias", dt_bias, d_in * 4},
+             {"h0", h0, bs}},
+            h_last, h0))
+      return s;
+  }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (L == 0) {  // no steps: the last state is the start state (or zeros)
     if (h_last && h_last != h0) {
@@ -417,8 +496,6 @@ ssm_status scan_fwd_impl(const void *u, const void *delta, const float *A, const
     }
     return ok();
   }
-  if (y == u || y == delta || y == z || y == B || y == C)
-    return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd: y must not alias an input");
 
   ssm::ScanParams p{u, delta, A, B, C, D, z, dt_bias, h0, h_last, y, b, L, d_in, delta_softplus,
                     chunk_h};
@@ -458,10 +535,6 @@ ssm_status ssm_scan_fwd_save(const void *u, const void *delta, const float *A, c
                 chunk_states_bytes, need);
   if (chunk_states && !aligned(chunk_states, 16))
     return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd_save: chunk_states not 16-byte aligned");
-  const void *ins[] = {u, delta, A, B, C, D, z, dt_bias, h0, h_last, y};
-  for (const void *q : ins)
-    if (q && q == chunk_states)
-      return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd_save: chunk_states aliases an argument");
   return scan_fwd_impl(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, h_last, y, b, L,
                        d_in, d_state, dtype, 0, need > 0 ? chunk_states : nullptr, stream);
 }
@@ -522,15 +595,21 @@ ssm_status scan_bwd_impl(const char *what, const void *u, const void *delta, con
   for (const void *q : f32)
     if (q && !aligned(q, 4))
       return fail(SSM_ERR_INVALID_ARG, "%s: fp32 pointer not 4-byte aligned", what);
-  const void *outs[] = {du, ddelta, dz, dA, dB, dC, dD, ddt_bias, dh0, workspace};
-  const void *ins[] = {u, delta, A, B, C, D, z, dt_bias, h0, dout, dh_last};
-  for (const void *o : outs) {
-    if (!o) continue;
-    for (const void *i : ins)
-      if (o == i) return fail(SSM_ERR_INVALID_ARG, "%s: an output aliases an input", what);
-    int same = 0;
-    for (const void *o2 : outs) same += (o2 == o);
-    if (same > 1) return fail(SSM_ERR_INVALID_ARG, "%s: two outputs share a buffer", what);
+  {
+    const int64_t ba = n_act * (int64_t)es, bbc = n_bc * (int64_t)es, bs = n_state * 4;
+    const int64_t bp = d_in * 4, bA = d_in * d_state * 4, bw = (int64_t)need;
+    // the saved states are read, not written, in the split mode
+    const Span ws{"workspace", states_saved ? nullptr : workspace, bw};
+    const Span ws_in{"chunk_states", states_saved ? workspace : nullptr, bw};
+    if (ssm_status s = check_disjoint(
+            what,
+            {{"du", du, ba}, {"ddelta", ddelta, ba}, {"dz", z ? dz : nullptr, ba}, {"dA", dA, bA},
+             {"dB", dB, n_bc * 4}, {"dC", dC, n_bc * 4}, {"dD", dD, bp},
+             {"ddt_bias", ddt_bias, bp}, {"dh0", dh0, bs}, ws},
+            {{"u", u, ba}, {"delta", delta, ba}, {"z", z, ba}, {"dout", dout, ba}, {"B", B, bbc},
+             {"C", C, bbc}, {"A", A, bA}, {"D", D, bp}, {"dt_bias", dt_bias, bp}, {"h0", h0, bs},
+             {"dh_last", dh_last, bs}, ws_in}))
+      return s;
   }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // the sums over channels and over the batch accumulate into zeroed outputs
@@ -647,8 +726,15 @@ ssm_status ss2d_scan_fwd_ex(const void *u, const void *delta, const float *A, co
   for (const void *q : f32)
     if (q && !aligned(q, 4))
       return fail(SSM_ERR_INVALID_ARG, "ss2d_scan_fwd: fp32 pointer not 4-byte aligned");
-  if (y == u || y == delta || y == B || y == C)
-    return fail(SSM_ERR_INVALID_ARG, "ss2d_scan_fwd: y must not alias an input");
+  {
+    const int64_t by = b * L * d_in * (int64_t)es, bk = 4 * by, bbc = b * 4 * L * d_state * (int64_t)es;
+    if (ssm_status s = check_disjoint(
+            "ss2d_scan_fwd", {{"y", y, by}, {"workspace", workspace, (int64_t)need}},
+            {{"u", u, by}, {"delta", delta, bk}, {"B", B, bbc}, {"C", C, bbc},
+             {"A", A, 4 * d_in * d_state * 4}, {"D", D, 4 * d_in * 4},
+             {"dt_bias", dt_bias, 4 * d_in * 4}}))
+      return s;
+  }
 
   ssm::Ss2dParams p{u, delta, A, B, C, D, dt_bias, y, static_cast<float *>(workspace),
                     b, H, W, d_in, delta_softplus};
@@ -696,8 +782,18 @@ ssm_status ssm_conv_state_update(void *conv_state, const float *conv_weight, con
   if (!aligned(conv_state, esize(dtype)) || !aligned(conv_weight, 4) ||
       (conv_bias && !aligned(conv_bias, 4)))
     return fail(SSM_ERR_INVALID_ARG, "%s: misaligned conv pointer", what);
-  if (y == conv_state || conv_state == x || conv_state == ssm_state)
-    return fail(SSM_ERR_INVALID_ARG, "%s: conv_state must not alias another argument", what);
+  {
+    const int64_t es = (int64_t)esize(dtype), bw = b * d_in * d_conv * es;
+    if (ssm_status s = check_disjoint(
+            what, {{"conv_state", conv_state, bw}},
+            {{"ssm_state", ssm_state, b * d_in * d_state * 4}, {"y", y, b * d_in * es},
+             {"x", x, b * d_in * es}, {"dt", dt, b * d_in * es}, {"z", z, b * d_in * es},
+             {"B", B, b * d_state * es}, {"C", C, b * d_state * es},
+             {"A", A, d_in * d_state * 4}, {"D", D, d_in * 4}, {"dt_bias", dt_bias, d_in * 4},
+             {"conv_weight", conv_weight, d_in * d_conv * 4},
+             {"conv_bias", conv_bias, d_in * 4}}))
+      return s;
+  }
   ssm::StepParams p{ssm_state, x, dt, A, B, C, D, z, dt_bias, y, b, d_in, dt_softplus,
                     conv_state, conv_weight, conv_bias, (int)d_conv};
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -726,6 +822,9 @@ ssm_status ss2d_cross_scan_ex(const void *u, void *xs, int64_t b, int64_t H, int
   if (!u || !xs) return fail(SSM_ERR_INVALID_ARG, "ss2d_cross_scan: NULL pointer");
   if (!aligned(u, esize(dtype)) || !aligned(xs, esize(dtype)))
     return fail(SSM_ERR_INVALID_ARG, "ss2d_cross_scan: misaligned pointer");
+  if (ssm_status s = check_disjoint("ss2d_cross_scan", {{"xs", xs, n * (int64_t)esize(dtype)}},
+                                    {{"u", u, n / 4 * (int64_t)esize(dtype)}}))
+    return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   auto run = [&](auto tag, auto ord) {
     using T = decltype(tag);
@@ -763,6 +862,9 @@ ssm_status ss2d_cross_merge_ex(const void *ys, void *y, int64_t b, int64_t H, in
   if (!ys || !y) return fail(SSM_ERR_INVALID_ARG, "ss2d_cross_merge: NULL pointer");
   if (!aligned(ys, esize(dtype)) || !aligned(y, esize(dtype)))
     return fail(SSM_ERR_INVALID_ARG, "ss2d_cross_merge: misaligned pointer");
+  if (ssm_status s = check_disjoint("ss2d_cross_merge", {{"y", y, n / 4 * (int64_t)esize(dtype)}},
+                                    {{"ys", ys, n * (int64_t)esize(dtype)}}))
+    return s;
   const int64_t m = b * L * d_in;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   auto run = [&](auto tag, auto ord) {

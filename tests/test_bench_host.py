@@ -1,5 +1,5 @@
-"""Host logic of bench.py, on the CPU: algorithmic bytes, the derived ALU
-roofline, the traffic-figure staleness rule, the reference arm's rank rule,
+"""Host logic of bench.py, on the CPU: algorithmic bytes, the derived SFU
+ceiling, the traffic-figure staleness rule, the reference arm's rank rule,
 and the cross-rank aggregation (world size 2 over gloo)."""
 import json
 import os
@@ -31,12 +31,19 @@ def test_algorithmic_bytes():
             - bench.alg_bytes(WORKLOADS["mamba-decode-step"])) == 2 * b * d * K * 2 + d * K * 4 + d * 4
 
 
-def test_alu_roofline_bounds():
-    w = WORKLOADS["mamba130m-scan"]
-    e = bench.alu_peak_elems_per_s(w)
-    sfu_only = bench.SMS * bench.SFU_PER_CLK * bench.SM_MAX_HZ / (1 + 4 / 16)
-    fma_only = bench.SMS * bench.FMA_PER_CLK * bench.SM_MAX_HZ / 4
-    assert sfu_only < e < fma_only
+def test_sfu_ceiling():
+    # N = 16 with the gate: one exp2 per element, softplus and SiLU per (t, d)
+    w = WORKLOADS["mamba1.4b-long-scan"]
+    assert bench.sfu_ops_per_element(w) == 1 + 2 / 16
+    e = bench.sfu_peak_elems_per_s(w)
+    assert e == pytest.approx(16 * 148 * 1.965e9 / 1.125)
+    # SS2D (N = 1, no gate): softplus and exp2 per (k, t, d)
+    assert bench.sfu_ops_per_element(WORKLOADS["vmamba-ss2d"]) == 2.0
+    # the long scan's SFU ceiling is below its HBM roofline: the bound the
+    # kernel can reach is about a third of the measured copy bandwidth
+    t_sfu = w.elements() / e
+    t_hbm = bench.alg_bytes(w) / (bench.FALLBACK_HBM_GBS * 1e9)
+    assert 0.25 < t_hbm / t_sfu < 0.4
 
 
 def test_traffic_is_null_when_kernels_changed(tmp_path, monkeypatch):
