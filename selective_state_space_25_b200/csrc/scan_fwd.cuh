@@ -29,6 +29,14 @@ struct ScanParams {
   // optional: the state at the start of every kStateChunk-step chunk,
   // (b, ceil(L / kStateChunk), d_in, N) fp32 (the backward scan's workspace)
   float *chunk_h = nullptr;
+  // Sequence blocks of the split scan (scan_ws.cuh): grid z-index k covers
+  // steps [k Lb, min(L, (k + 1) Lb)); Lb = 0 means one block.  blk_decay and
+  // blk_state are (b, nblk, d_in, N) fp32: the summary pass leaves each
+  // block's decay product and its end state from zero there, the carry pass
+  // turns blk_state[k] (k >= 1) into the state block k starts from.
+  int64_t Lb = 0;
+  float *blk_decay = nullptr;
+  float *blk_state = nullptr;
 };
 
 // ---------------------------------------------------------------------------

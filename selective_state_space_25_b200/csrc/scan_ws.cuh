@@ -76,9 +76,10 @@ __device__ __forceinline__ void helper_barrier(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
 
-template <typename T, int N, int NS, int TC, int H, int P, bool HAS_Z, bool SAVE>
+template <typename T, int N, int NS, int TC, int H, int P, bool HAS_Z, bool SAVE, bool SUMMARY>
 __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
     scan_ws_kernel(ScanParams p) {
+  static_assert(!(SUMMARY && SAVE), "the summary pass saves no states");
   using K = WsScan<T, N, NS, TC, H, P>;
   constexpr int DT = K::DT, G = K::G, NP2 = K::NP2, R = K::R, TCP = K::TCP;
   extern __shared__ __align__(16) unsigned char smem[];
@@ -87,7 +88,13 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
   const int64_t ib = blockIdx.y;
   const int64_t d0 = (int64_t)blockIdx.x * DT;
   const int64_t L = p.L, d_in = p.d_in;
-  const int64_t nchunks = (L + TC - 1) / TC;
+  // this CTA's block of the sequence: [t_begin, t_end)
+  // (the summary pass runs the first nblk - 1 blocks only: nblk comes from Lb)
+  const int64_t blk = blockIdx.z, nblk = p.Lb > 0 ? (L + p.Lb - 1) / p.Lb : 1;
+  const int64_t t_begin = blk * p.Lb;
+  const int64_t t_end = p.Lb > 0 && t_begin + p.Lb < L ? t_begin + p.Lb : L;
+  const int64_t nchunks = (t_end - t_begin + TC - 1) / TC;
+  const int64_t blk_row = (ib * nblk + blk) * d_in;  // row of (batch, block) in blk_decay / blk_state
   auto arr = [&](int off, int buf) {
     return reinterpret_cast<float *>(smem + off + buf * K::ARR);
   };
@@ -110,15 +117,20 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
       const int n = g * NS + 2 * k;
       A2[k] = d_ok ? make_float2(p.A[d * N + n] * kLog2e, p.A[d * N + n + 1] * kLog2e)
                    : make_float2(0.0f, 0.0f);
-      const float *h0 = p.h0 + (ib * d_in + d) * N + n;
-      h[k] = (d_ok && p.h0) ? make_float2(h0[0], h0[1]) : make_float2(0.0f, 0.0f);
+      // the summary starts every block from zero; the scan starts block 0
+      // from h0 and block k > 0 from the carry the carry pass left
+      const float *h0 = blk == 0 ? p.h0 + (ib * d_in + d) * N + n
+                                 : p.blk_state + (blk_row + d) * N + n;
+      const bool from = d_ok && !SUMMARY && (blk > 0 || p.h0);
+      h[k] = from ? make_float2(h0[0], h0[1]) : make_float2(0.0f, 0.0f);
     }
+    float dsum = 0.0f;  // sum of delta over the block (summary pass)
     const int64_t n_saved = (L + kStateChunk - 1) / kStateChunk;
     __syncthreads();  // the first chunk's pre-pass is done
     int slot = 0;     // ch % R
     for (int64_t ch = 0; ch < nchunks; ++ch) {
       const int buf = (int)(ch & 1);
-      const int64_t t0 = ch * TC;
+      const int64_t t0 = t_begin + ch * TC;
       const float *rdl = arr(K::OFF_DL, buf) + c * TCP;
       const float *rdu = arr(K::OFF_DU, buf) + c * TCP;
       float *pl_own = s_planes + ((buf * G + g) * DT + c) * TCP;
@@ -139,7 +151,8 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
           const int t = 4 * j4 + jj;
           StateWords<T, NS> Bw;
           Bw.load(rB + t * N + g * NS);
-          q.C[jj].load(rC + t * N + g * NS);
+          if constexpr (SUMMARY) dsum += dls[jj];
+          else q.C[jj].load(rC + t * N + g * NS);
           const float2 d2 = make_float2(dls[jj], dls[jj]);
           const float2 u2 = make_float2(dus[jj], dus[jj]);
 #pragma unroll
@@ -168,17 +181,31 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
 #pragma unroll
           for (int k = 0; k < NP2; ++k) {
             h[k] = __ffma2_rn(cur.a[jj][k], h[k], cur.b[jj][k]);
-            acc = __ffma2_rn(h[k], cur.C[jj].pair(k), acc);
+            if constexpr (!SUMMARY) acc = __ffma2_rn(h[k], cur.C[jj].pair(k), acc);
           }
           ys[jj] = acc.x + acc.y;
         }
-        *reinterpret_cast<float4 *>(pl_own + 4 * j4) = make_float4(ys[0], ys[1], ys[2], ys[3]);
+        if constexpr (!SUMMARY)
+          *reinterpret_cast<float4 *>(pl_own + 4 * j4) = make_float4(ys[0], ys[1], ys[2], ys[3]);
         if (j4 + 1 < TC / 4) cur = nxt;
       }
       slot = slot == R - 1 ? 0 : slot + 1;
       __syncthreads();  // partials of this chunk written; next chunk's pre-pass done
     }
-    if (p.h_last && d_ok) {
+    if constexpr (SUMMARY) {  // the block's map h -> P h + Q
+      if (d_ok) {
+        float *q = p.blk_state + (blk_row + d) * N + g * NS;
+        float *pd = p.blk_decay + (blk_row + d) * N + g * NS;
+#pragma unroll
+        for (int k = 0; k < NP2; ++k) {
+          q[2 * k] = h[k].x;
+          q[2 * k + 1] = h[k].y;
+          const float2 e = exp2_sfu2(__fmul2_rn(make_float2(dsum, dsum), A2[k]));
+          pd[2 * k] = e.x;
+          pd[2 * k + 1] = e.y;
+        }
+      }
+    } else if (p.h_last && d_ok && blk == nblk - 1) {
       float *hl = p.h_last + (ib * d_in + d) * N + g * NS;
 #pragma unroll
       for (int k = 0; k < NP2; ++k) {
@@ -200,24 +227,24 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
 
   // copy chunk ch into ring slot `slot` (one cp.async group per call)
   auto prefetch = [&](int64_t ch, int slot) {
-    const int64_t t0 = ch * TC;
+    const int64_t t0 = t_begin + ch * TC;
     for (int q = hid; q < TC * K::ROW_GRAN; q += K::HELP_THREADS) {
       const int t = q / K::ROW_GRAN, gq = q - t * K::ROW_GRAN;
       const int64_t dd = d0 + gq * K::VEC;
-      const bool ok = (t0 + t < L) && (dd < d_in);
+      const bool ok = (t0 + t < t_end) && (dd < d_in);
       const int64_t off = ok ? ((ib * L + t0 + t) * d_in + dd) : 0;
       const int so = t * K::RAWROW + gq * 16;
       cp_async16(raw(slot, 0) + so, gu + off, ok ? 16 : 0);
       cp_async16(raw(slot, 1) + so, gdt + off, ok ? 16 : 0);
-      if (HAS_Z) cp_async16(raw(slot, 2) + so, gz + off, ok ? 16 : 0);
+      if (HAS_Z && !SUMMARY) cp_async16(raw(slot, 2) + so, gz + off, ok ? 16 : 0);
     }
     for (int q = hid; q < TC * K::BC_GRAN; q += K::HELP_THREADS) {
       const int t = q / K::BC_GRAN, gq = q - t * K::BC_GRAN;
-      const bool ok = t0 + t < L;
+      const bool ok = t0 + t < t_end;
       const int64_t off = ok ? ((ib * L + t0 + t) * N + gq * K::VEC) : 0;
       const int so = t * N + gq * K::VEC;
       cp_async16(rawbc(slot, 0) + so, gB + off, ok ? 16 : 0);
-      cp_async16(rawbc(slot, 1) + so, gC + off, ok ? 16 : 0);
+      if (!SUMMARY) cp_async16(rawbc(slot, 1) + so, gC + off, ok ? 16 : 0);
     }
     cp_async_commit();
   };
@@ -242,8 +269,8 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
   // the D u / gate entries of exactly the items its own pre-pass writes, so
   // the pre-pass of chunk ch + 2 may reuse the buffer right after.
   auto post = [&](int64_t ch, int tc, int buf) {
-    if (!p_ok) return;
-    const int64_t t0 = ch * TC;
+    if (SUMMARY || !p_ok) return;
+    const int64_t t0 = t_begin + ch * TC;
     const float *pdz = arr(K::OFF_DZ, buf), *pgt = arr(K::OFF_GT, buf);
     const float *ppl = s_planes + buf * G * DT * TCP;
     for (int sg = sg0; sg * 4 < tc; sg += SG_STRIDE) {
@@ -298,14 +325,14 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
           const uint32_t wd = *reinterpret_cast<const uint32_t *>(rd + t * K::RAWROW);
           u2 = make_float2(bf16lo(wu), bf16hi(wu));
           e2 = make_float2(bf16lo(wd), bf16hi(wd));
-          if (HAS_Z) {
+          if (HAS_Z && !SUMMARY) {
             const uint32_t wz = *reinterpret_cast<const uint32_t *>(rz + t * K::RAWROW);
             z2 = make_float2(bf16lo(wz), bf16hi(wz));
           }
         } else {
           u2 = *reinterpret_cast<const float2 *>(ru + t * K::RAWROW);
           e2 = *reinterpret_cast<const float2 *>(rd + t * K::RAWROW);
-          if (HAS_Z) z2 = *reinterpret_cast<const float2 *>(rz + t * K::RAWROW);
+          if (HAS_Z && !SUMMARY) z2 = *reinterpret_cast<const float2 *>(rz + t * K::RAWROW);
         }
         e2 = __fadd2_rn(e2, bias2);
         if (p.delta_softplus) e2 = softplus2_f32(e2);
@@ -315,7 +342,7 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
         dl[0][jj] = e2.x; dl[1][jj] = e2.y;
         dlu[0][jj] = eu.x; dlu[1][jj] = eu.y;
         dd[0][jj] = du2.x; dd[1][jj] = du2.y;
-        if (HAS_Z) {
+        if (HAS_Z && !SUMMARY) {
           gg[0][jj] = silu_for<T>(z2.x);
           gg[1][jj] = silu_for<T>(z2.y);
         }
@@ -331,6 +358,7 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
       *reinterpret_cast<float4 *>(pdl + ibb) = swp ? l0 : l1;
       *reinterpret_cast<float4 *>(pdu + ia) = swp ? u1 : u0;
       *reinterpret_cast<float4 *>(pdu + ibb) = swp ? u0 : u1;
+      if (SUMMARY) continue;  // the summary needs delta and delta u only
       *reinterpret_cast<float4 *>(pdz + ia) = swp ? z1 : z0;
       *reinterpret_cast<float4 *>(pdz + ibb) = swp ? z0 : z1;
       if (HAS_Z) {
@@ -343,7 +371,7 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
   };
 
   auto tc_of = [&](int64_t ch) {
-    const int64_t rem = L - ch * TC;
+    const int64_t rem = t_end - t_begin - ch * TC;
     return (int)(rem < (int64_t)TC ? rem : (int64_t)TC);
   };
 
@@ -378,6 +406,26 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
   }
   if (nchunks > 0) post(nchunks - 1, tc_of(nchunks - 1), (int)((nchunks - 1) & 1));
   cp_async_wait<0>();  // only empty groups can remain
+}
+
+// Carry pass of the split scan: per chain (batch, channel, state), the block
+// maps composed in order from h0, blk_state[k] (k >= 1) overwritten with the
+// state block k starts from (block k's own end state is read before that).
+__global__ void scan_carry_kernel(const float *h0, const float *blk_decay, float *blk_state,
+                                  int64_t b, int64_t nblk, int64_t d_in, int N) {
+  const int64_t q = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;  // (batch, channel, state)
+  const int64_t per = d_in * N;
+  if (q >= b * per) return;
+  const int64_t ib = q / per, r = q - ib * per;
+  float h = h0 ? h0[q] : 0.0f;
+  float qn = blk_state[(ib * nblk) * per + r];
+  for (int64_t k = 0; k + 1 < nblk; ++k) {
+    const int64_t i = (ib * nblk + k) * per + r;
+    const float qk = qn;
+    qn = blk_state[i + per];
+    h = fmaf(blk_decay[i], h, qk);
+    blk_state[i + per] = h;
+  }
 }
 
 }  // namespace ssm

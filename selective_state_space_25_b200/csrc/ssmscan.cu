@@ -186,14 +186,76 @@ ssm_status launch_scan_fast(const ssm::ScanParams &p, cudaStream_t st) {
 // 8 for 32 (four scan warps either way); 0 = not compiled for this d_state.
 constexpr int ws_states(int n) { return n == 8 || n == 16 ? 4 : (n == 32 ? 8 : 0); }
 
-template <typename T, int N, bool HAS_Z, bool SAVE>
-ssm_status launch_scan_ws(const ssm::ScanParams &p, cudaStream_t st) {
+// SMs of the current device (148 on B200; also the answer when no device is
+// visible, so the workspace query works on a host without a GPU).
+int device_sms() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return 148;
+  }
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = 148;
+    }
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+// Split of the sequence into blocks (scan_ws.cuh, split scan) for problems
+// whose b * ceil(d_in / 32) CTAs would leave more than half of the SMs idle:
+// about four CTAs per SM, each block a whole number of chunks and at least
+// four chunks long.  nblk = 1: one pass.  Depends on the sizes only, so
+// ssm_scan_fwd_workspace_bytes and the launch agree.  Measured on B200
+// (b = 1, L = 16384, N = 16, bf16): d_in = 256 575 -> 94 us, d_in = 1536
+// 575 -> 321 us; at d_in = 4096 (128 CTAs) one pass is faster (577 against
+// 754 us), hence the half-the-SMs threshold.
+struct SplitPlan {
+  int64_t nblk = 1, Lb = 0;
+};
+SplitPlan split_plan(int64_t b, int64_t L, int64_t d_in, int64_t N) {
+  SplitPlan sp;
+  if (b <= 0 || L <= 0 || d_in <= 0 || d_in % 8 != 0 || !(N == 8 || N == 16 || N == 32)) return sp;
+  const int64_t sms = device_sms();
+  const int64_t ctas = b * ((d_in + 31) / 32);
+  if (2 * ctas > sms) return sp;
+  int64_t nblk = (4 * sms + ctas - 1) / ctas;
+  const int64_t by_len = L / (4 * SSM_WS_TC);
+  if (nblk > by_len) nblk = by_len;
+  if (nblk > 4096) nblk = 4096;
+  if (nblk < 2) return sp;
+  const int64_t per = (L + nblk - 1) / nblk;
+  sp.Lb = (per + SSM_WS_TC - 1) / SSM_WS_TC * SSM_WS_TC;
+  sp.nblk = (L + sp.Lb - 1) / sp.Lb;
+  if (sp.nblk < 2) sp = SplitPlan{};
+  return sp;
+}
+
+template <typename T, int N, bool HAS_Z, bool SAVE, bool SUMMARY>
+ssm_status launch_scan_ws_pass(const ssm::ScanParams &p, unsigned nz, cudaStream_t st) {
   constexpr int NS = ws_states(N);
   using Cfg = ssm::WsScan<T, N, NS, SSM_WS_TC, SSM_WS_HELPERS, SSM_WS_AHEAD>;
-  constexpr auto k =
-      ssm::scan_ws_kernel<T, N, NS, SSM_WS_TC, SSM_WS_HELPERS, SSM_WS_AHEAD, HAS_Z, SAVE>;
-  const dim3 grid((unsigned)((p.d_in + Cfg::DT - 1) / Cfg::DT), (unsigned)p.b);
+  constexpr auto k = ssm::scan_ws_kernel<T, N, NS, SSM_WS_TC, SSM_WS_HELPERS, SSM_WS_AHEAD,
+                                         HAS_Z, SAVE, SUMMARY>;
+  const dim3 grid((unsigned)((p.d_in + Cfg::DT - 1) / Cfg::DT), (unsigned)p.b, nz);
   return launch_fast_kernel<k>(p, grid, Cfg::THREADS, Cfg::SMEM, st);
+}
+
+template <typename T, int N, bool HAS_Z, bool SAVE>
+ssm_status launch_scan_ws(const ssm::ScanParams &p, cudaStream_t st) {
+  if (p.Lb <= 0) return launch_scan_ws_pass<T, N, HAS_Z, SAVE, false>(p, 1, st);
+  // split scan: block summaries, the carry pass, then every block at once
+  const unsigned nblk = (unsigned)((p.L + p.Lb - 1) / p.Lb);
+  if (ssm_status s = launch_scan_ws_pass<T, N, false, false, true>(p, nblk - 1, st)) return s;
+  const int64_t chains = p.b * p.d_in * N;
+  ssm::scan_carry_kernel<<<(unsigned)((chains + 255) / 256), 256, 0, st>>>(
+      p.h0, p.blk_decay, p.blk_state, p.b, nblk, p.d_in, N);
+  if (ssm_status s = check_launch("ssm_scan_fwd")) return s;
+  return launch_scan_ws_pass<T, N, HAS_Z, SAVE, false>(p, nblk, st);
 }
 
 template <typename T, int N>
@@ -434,7 +496,10 @@ size_t ssm_scan_fwd_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t 
   if (b < 0 || L < 0 || d_in < 0 || d_state < 1 || !mul_ok(b, L, &t) || !mul_ok(t, d_in, &t) ||
       !mul_ok(t, d_state, &t))
     return (size_t)-1;
-  return 0;
+  const SplitPlan sp = split_plan(b, L, d_in, d_state);
+  if (sp.nblk <= 1) return 0;
+  // block decays and block states, (b, nblk, d_in, d_state) fp32 each
+  return (size_t)(2 * b * sp.nblk * d_in * d_state) * sizeof(float);
 }
 
 }  // extern "C"
@@ -445,7 +510,8 @@ ssm_status scan_fwd_impl(const void *u, const void *delta, const float *A, const
                          const void *C, const float *D, const void *z, const float *dt_bias,
                          int delta_softplus, const float *h0, float *h_last, void *y, int64_t b,
                          int64_t L, int64_t d_in, int64_t d_state, ssm_dtype dtype,
-                         size_t workspace_bytes, float *chunk_h, ssm_stream_t stream) {
+                         void *workspace, size_t workspace_bytes, float *chunk_h,
+                         ssm_stream_t stream) {
   g_last_error.clear();
   if (b < 0 || L < 0 || d_in < 0)
     return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd: negative size (b=%lld L=%lld d_in=%lld)",
@@ -460,10 +526,13 @@ ssm_status scan_fwd_impl(const void *u, const void *delta, const float *A, const
       !mul_ok(n_bc, d_state, &n_bc) || !mul_ok(b, d_in, &n_state) ||
       !mul_ok(n_state, d_state, &n_state) || n_act > INT64_MAX / 4)
     return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd: sizes overflow int64");
-  const size_t need = ssm_scan_fwd_workspace_bytes(b, L, d_in, d_state);
-  if (workspace_bytes < need)
+  // the forward that saves chunk states always runs in one pass (no workspace)
+  const size_t need = chunk_h ? 0 : ssm_scan_fwd_workspace_bytes(b, L, d_in, d_state);
+  if (workspace_bytes < need || (need > 0 && !workspace))
     return fail(SSM_ERR_WORKSPACE, "ssm_scan_fwd: workspace %zu bytes < %zu needed",
                 workspace_bytes, need);
+  if (need > 0 && !aligned(workspace, 16))
+    return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd: workspace not 16-byte aligned");
   if (b == 0 || d_in == 0) return ok();
   if (!A) return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd: A is NULL");
   if (L > 0 && (!u || !delta || !B || !C || !y))
@@ -481,7 +550,9 @@ ssm_status scan_fwd_impl(const void *u, const void *delta, const float *A, const
     const int64_t ba = n_act * (int64_t)es, bbc = n_bc * (int64_t)es, bs = n_state * 4;
     const int64_t nc = chunk_h ? (int64_t)ssm_scan_bwd_workspace_bytes(b, L, d_in, d_state) : 0;
     if (ssm_status s = check_disjoint(
-            "ssm_scan_fwd", {{"y", y, ba}, {"h_last", h_last, bs}, {"chunk_states", chunk_h, nc}},
+            "ssm_scan_fwd",
+            {{"y", y, ba}, {"h_last", h_last, bs}, {"chunk_states", chunk_h, nc},
+             {"workspace", need > 0 ? workspace : nullptr, (int64_t)need}},
             {{"u", u, ba}, {"delta", delta, ba}, {"z", z, ba}, {"B", B, bbc}, {"C", C, bbc},
              {"A", A, d_in * d_state * 4}, {"D", D, d_in * 4}, {"dt_bias", dt_bias, d_in * 4},
              {"h0", h0, bs}},
@@ -499,6 +570,12 @@ ssm_status scan_fwd_impl(const void *u, const void *delta, const float *A, const
 
   ssm::ScanParams p{u, delta, A, B, C, D, z, dt_bias, h0, h_last, y, b, L, d_in, delta_softplus,
                     chunk_h};
+  if (!chunk_h && need > 0) {  // the split scan (its plan is the one need was sized for)
+    const SplitPlan sp = split_plan(b, L, d_in, d_state);
+    p.Lb = sp.Lb;
+    p.blk_decay = static_cast<float *>(workspace);
+    p.blk_state = p.blk_decay + b * sp.nblk * d_in * d_state;
+  }
   const bool fast = d_state >= 8 && (d_in * (int64_t)es) % 16 == 0 && aligned(u, 16) &&
                     aligned(delta, 16) && aligned(B, 16) && aligned(C, 16) && aligned(y, 16) &&
                     (!z || aligned(z, 16)) && b <= 65535;
@@ -515,9 +592,8 @@ ssm_status ssm_scan_fwd(const void *u, const void *delta, const float *A, const 
                         int delta_softplus, const float *h0, float *h_last, void *y, int64_t b,
                         int64_t L, int64_t d_in, int64_t d_state, ssm_dtype dtype,
                         void *workspace, size_t workspace_bytes, ssm_stream_t stream) {
-  (void)workspace;
   return scan_fwd_impl(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, h_last, y, b, L,
-                       d_in, d_state, dtype, workspace_bytes, nullptr, stream);
+                       d_in, d_state, dtype, workspace, workspace_bytes, nullptr, stream);
 }
 
 ssm_status ssm_scan_fwd_save(const void *u, const void *delta, const float *A, const void *B,
@@ -536,7 +612,8 @@ ssm_status ssm_scan_fwd_save(const void *u, const void *delta, const float *A, c
   if (chunk_states && !aligned(chunk_states, 16))
     return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd_save: chunk_states not 16-byte aligned");
   return scan_fwd_impl(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, h_last, y, b, L,
-                       d_in, d_state, dtype, 0, need > 0 ? chunk_states : nullptr, stream);
+                       d_in, d_state, dtype, nullptr, 0, need > 0 ? chunk_states : nullptr,
+                       stream);
 }
 
 size_t ssm_scan_bwd_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t d_state) {

@@ -70,7 +70,16 @@ def test_scan_validation(kw, status):
 
 
 def test_workspace_query():
-    assert S.ssm_scan_fwd_workspace_bytes(8, 2048, 1536, 16) >= 0
+    # channels enough to fill the GPU: one pass, no workspace
+    assert S.ssm_scan_fwd_workspace_bytes(8, 2048, 1536, 16) == 0
+    assert S.ssm_scan_fwd_workspace_bytes(2, 16384, 4096, 16) == 0
+    # few channels and a long sequence: the split scan keeps two fp32
+    # (b, blocks, d_in, N) arrays (block decays and block states)
+    ws = S.ssm_scan_fwd_workspace_bytes(1, 16384, 64, 16)
+    assert ws > 0 and ws % (2 * 64 * 16 * 4) == 0
+    assert S.ssm_scan_fwd_workspace_bytes(1, 200, 64, 16) == 0       # too short to split
+    assert S.ssm_scan_fwd_workspace_bytes(1, 16384, 64, 64) == 0     # d_state 64: one pass
+    assert S.ssm_scan_fwd_workspace_bytes(1, 16384, 60, 16) == 0     # d_in not a multiple of 8
     assert L.ssm_scan_fwd_workspace_bytes(-1, 1, 1, 16) == ctypes.c_size_t(-1).value
     assert S.ss2d_scan_fwd_workspace_bytes(32, 56, 56, 192, 1) == 0
     big = S.ss2d_scan_fwd_workspace_bytes(2, 100, 100, 16, 1)
@@ -201,6 +210,17 @@ def test_fwd_save_validation():
     assert L.ssm_scan_fwd_save(*args(FAKE, need)) == S.SSM_ERR_INVALID_ARG         # aliases u
     assert L.ssm_scan_fwd_save(*args(FAKE + 6144, need)) == S.SSM_ERR_INVALID_ARG  # overlaps y
     assert L.ssm_scan_fwd_save(*args(None, 0, b=0)) == S.SSM_OK
+
+
+def test_split_scan_needs_its_workspace():
+    need = S.ssm_scan_fwd_workspace_bytes(1, 4096, 64, 16)
+    assert need > 0
+    kw = dict(b=1, L=4096, d_in=64, N=16, y=FAKE + (1 << 22))
+    assert scan(**kw) == S.SSM_ERR_WORKSPACE
+    assert scan(ws=FAKE + (1 << 23), ws_bytes=need - 4, **kw) == S.SSM_ERR_WORKSPACE
+    assert scan(ws=None, ws_bytes=need, **kw) == S.SSM_ERR_WORKSPACE
+    assert scan(ws=FAKE + (1 << 23) + 4, ws_bytes=need, **kw) == S.SSM_ERR_INVALID_ARG  # misaligned
+    assert scan(ws=FAKE, ws_bytes=need, **kw) == S.SSM_ERR_INVALID_ARG  # overlaps the inputs
 
 
 def test_h_last_may_equal_h0_but_not_overlap_it():

@@ -176,3 +176,54 @@ def test_mamba130m_workload_sampled(ssm):
 def test_mamba14b_long_workload_sampled(ssm):
     ey, eh = _sampled_parity(ssm, "mamba1.4b-long-scan", 12)
     assert ey <= 2e-2 and eh <= 2e-2, (ey, eh)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("b,L,d_in,N", [
+    (1, 3000, 64, 16), (2, 777, 32, 8), (1, 1000, 32, 32), (1, 257, 32, 16), (3, 4100, 40, 16),
+])
+def test_split_scan(ssm, dtype, b, L, d_in, N):
+    """Few channels and a long sequence: the sequence is cut into blocks whose
+    maps are summarised, composed from h0 block after block and replayed in
+    parallel (the chunked associative scan with a carry).  The blocks' last
+    one is ragged in every case."""
+    dt = "bf16" if dtype == torch.bfloat16 else "fp32"
+    need = ssm.ssm_scan_fwd_workspace_bytes(b, L, d_in, N)
+    if d_in % 8 == 0:
+        assert need > 0, "this shape should take the split scan"
+    inp = scan_inputs(b, L, d_in, N, dt, seed=L + d_in + N, with_h0=True)
+    hl = torch.empty(b, d_in, N, device="cuda")
+    y, _ = run_gpu(ssm, inp, h_last=hl)
+    y_ref, h_ref = run_oracle(inp, last=True)
+    assert rel_err(y, y_ref) <= TOL[dtype]
+    assert rel_err(hl, h_ref) <= TOL[dtype]
+
+
+def test_split_scan_resume_and_zero_start(ssm):
+    """The split scan from a carried state equals one scan over both parts,
+    and without h0 its first block starts from zero."""
+    inp = scan_inputs(1, 2048, 64, 16, "fp32", seed=21)
+    g = to_cuda(inp)
+    assert ssm.ssm_scan_fwd_workspace_bytes(1, 1024, 64, 16) > 0
+    y_full = ssm.ssm_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], D=g["D"], z=g["z"],
+                               dt_bias=g["dt_bias"])
+    h = torch.empty(1, 64, 16, device="cuda")
+    part = lambda t, s: t[:, s].contiguous()
+    s1, s2 = slice(0, 1024), slice(1024, None)
+    y1 = ssm.ssm_scan_fwd(part(g["u"], s1), part(g["delta"], s1), g["A"], part(g["B"], s1),
+                           part(g["C"], s1), D=g["D"], z=part(g["z"], s1), dt_bias=g["dt_bias"],
+                           h_last=h)
+    y2 = ssm.ssm_scan_fwd(part(g["u"], s2), part(g["delta"], s2), g["A"], part(g["B"], s2),
+                           part(g["C"], s2), D=g["D"], z=part(g["z"], s2), dt_bias=g["dt_bias"],
+                           h0=h)
+    assert rel_err(torch.cat([y1, y2], 1), y_full) <= 1e-5
+    assert rel_err(y_full, run_oracle(inp)) <= 1e-4
+
+
+def test_split_scan_rejects_a_short_workspace(ssm):
+    inp = scan_inputs(1, 3000, 64, 16, "bf16", seed=2)
+    g = to_cuda(inp)
+    need = ssm.ssm_scan_fwd_workspace_bytes(1, 3000, 64, 16)
+    ws = torch.empty(need - 16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(Exception):
+        ssm.ssm_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], workspace=ws)
