@@ -34,9 +34,9 @@
  *   - Every call enqueues its kernels on `stream` (NULL = the legacy default
  *     stream) and returns without synchronising.  Argument errors are
  *     reported synchronously, before anything is enqueued; launch errors are
- *     reported by the call that launched.  Errors found by a kernel at run
- *     time (a bounded wait that ran out) are reported by
- *     ssm_check_device_errors().
+ *     reported by the call that launched.  A fault while a kernel runs is a
+ *     CUDA error of the stream, reported by the next call that synchronises
+ *     it (ssm_check_device_errors() does).
  *   - Calls allocate nothing and never synchronise, so they can be captured
  *     in a CUDA graph; make the first call of each kind and d_state outside
  *     any capture (it sets the kernel's shared-memory attribute once per
@@ -72,7 +72,9 @@ typedef enum {
     SSM_ERR_UNSUPPORTED = 2,    /* valid but not compiled: d_state not in {1,2,4,...,64}, unknown dtype */
     SSM_ERR_WORKSPACE = 3,      /* workspace smaller than ssm_scan_fwd_workspace_bytes() */
     SSM_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed (message has the CUDA error) */
-    SSM_ERR_DEVICE_TIMEOUT = 5  /* a kernel's bounded wait ran out (ssm_check_device_errors) */
+    SSM_ERR_DEVICE_TIMEOUT = 5  /* reserved for a kernel's bounded wait running out; no kernel of
+                                   this build waits on another thread block or device, so no call
+                                   returns it */
 } ssm_status;
 
 typedef enum {
@@ -282,11 +284,14 @@ size_t ss2d_scan_fwd_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_
  * the process exits.  Limit: b * H * W * d_in * 4 bytes (the value
  * ss2d_scan_fwd_workspace_bytes returns) must not exceed 16 MiB, else
  * SSM_ERR_WORKSPACE; images whose accumulator fits in shared memory need
- * none of it.  The first call on a device looks the array's device address
- * up (cudaGetSymbolAddress) and caches it; make that first call before any
- * stream capture.  All calls on a device share the one array, which keeps
- * the last call's contents (nothing needs clearing: every call overwrites
- * the part it reads); calls whose kernels overlap on the GPU race on it.
+ * none of it.  A call made outside a stream capture looks the array's
+ * device address up (cudaGetSymbolAddress, the device current) and caches
+ * it per device, so a device reset leaves no stale address behind; a call
+ * made while the stream is being captured uses the cached address, so make
+ * one call on each device before capturing (else SSM_ERR_CUDA).  All calls
+ * on a device share the one array, which keeps the last call's contents
+ * (nothing needs clearing: every call overwrites the part it reads); calls
+ * whose kernels overlap on the GPU race on it.
  */
 ssm_status ss2d_scan_fwd_noalloc(const void *u, const void *delta, const float *A,
                                  const void *B, const void *C, const float *D,
@@ -367,9 +372,8 @@ ssm_status ss2d_cross_merge(const void *ys, void *y, int64_t b, int64_t H,
                             ssm_stream_t stream);
 
 /*
- * Synchronises `stream`, then reads and clears the library's device error
- * word on the current device.  Returns SSM_OK, SSM_ERR_DEVICE_TIMEOUT when a
- * kernel gave up a bounded wait since the last check, or SSM_ERR_CUDA.
+ * Synchronises `stream` and returns SSM_OK, or SSM_ERR_CUDA with the CUDA
+ * error of the stream (a kernel fault) in ssm_last_error().
  */
 ssm_status ssm_check_device_errors(ssm_stream_t stream);
 

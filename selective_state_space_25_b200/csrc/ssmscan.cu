@@ -18,9 +18,6 @@
 #include "ss2d_fwd.cuh"
 #include "state_update.cuh"
 
-// Set by a kernel whose bounded wait ran out; read by ssm_check_device_errors.
-__device__ unsigned int g_ssm_device_error = 0;
-
 namespace {
 
 thread_local std::string g_last_error;
@@ -972,22 +969,35 @@ namespace {
 
 // Device address of the scratch array on the current device.  In host code
 // the array's name is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
-ssm_status noalloc_scratch(float **out) {
+// with cudaGetSymbolAddress (that device current).  Calls outside a stream
+// capture look it up every time (cheap next to the launch; a device reset,
+// which reloads the module, cannot leave a stale address behind) and cache
+// it per device; a call made while `st` is being captured uses the cached
+// address, so the first call on a device must come before any capture.
+ssm_status noalloc_scratch(cudaStream_t st, float **out) {
   static std::mutex mu;
   static float *ptr[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess || dev < 0 || dev >= 64)
     return fail(SSM_ERR_CUDA, "ss2d_scan_fwd_noalloc: cudaGetDevice failed");
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(st, &cap);
+  if (e != cudaSuccess)
+    return fail(SSM_ERR_CUDA, "ss2d_scan_fwd_noalloc: cudaStreamIsCapturing: %s",
+                cudaGetErrorString(e));
   std::lock_guard<std::mutex> lock(mu);
-  if (!ptr[dev]) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void *addr = nullptr;
     e = cudaGetSymbolAddress(&addr, g_ss2d_noalloc_scratch);
     if (e != cudaSuccess || !addr)
       return fail(SSM_ERR_CUDA, "ss2d_scan_fwd_noalloc: cudaGetSymbolAddress: %s",
                   cudaGetErrorString(e));
     ptr[dev] = static_cast<float *>(addr);
+  } else if (!ptr[dev]) {
+    return fail(SSM_ERR_CUDA,
+                "ss2d_scan_fwd_noalloc: first call on this device made during a stream "
+                "capture; make one call before capturing");
   }
   *out = ptr[dev];
   return ok();
@@ -1013,7 +1023,7 @@ ssm_status ss2d_scan_fwd_noalloc(const void *u, const void *delta, const float *
                 need, kNoAllocScratchBytes);
   float *scratch = nullptr;
   if (need > 0) {
-    if (ssm_status s = noalloc_scratch(&scratch)) return s;
+    if (ssm_status s = noalloc_scratch(reinterpret_cast<cudaStream_t>(stream), &scratch)) return s;
   }
   // The accumulator needs no clearing: the first direction stores every
   // pixel before the others add to it.
@@ -1023,17 +1033,9 @@ ssm_status ss2d_scan_fwd_noalloc(const void *u, const void *delta, const float *
 
 ssm_status ssm_check_device_errors(ssm_stream_t stream) {
   g_last_error.clear();
-  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  const cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess)
     return fail(SSM_ERR_CUDA, "ssm_check_device_errors: %s", cudaGetErrorString(e));
-  unsigned int v = 0, zero = 0;
-  e = cudaMemcpyFromSymbol(&v, g_ssm_device_error, sizeof v);
-  if (e != cudaSuccess)
-    return fail(SSM_ERR_CUDA, "ssm_check_device_errors: %s", cudaGetErrorString(e));
-  if (v) {
-    cudaMemcpyToSymbol(g_ssm_device_error, &zero, sizeof zero);
-    return fail(SSM_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait ran out (code %u)", v);
-  }
   return ok();
 }
 
