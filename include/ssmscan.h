@@ -72,9 +72,11 @@ typedef enum {
     SSM_ERR_UNSUPPORTED = 2,    /* valid but not compiled: d_state not in {1,2,4,...,64}, unknown dtype */
     SSM_ERR_WORKSPACE = 3,      /* workspace smaller than ssm_scan_fwd_workspace_bytes() */
     SSM_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed (message has the CUDA error) */
-    SSM_ERR_DEVICE_TIMEOUT = 5  /* reserved for a kernel's bounded wait running out; no kernel of
+    SSM_ERR_DEVICE_TIMEOUT = 5, /* reserved for a kernel's bounded wait running out; no kernel of
                                    this build waits on another thread block or device, so no call
                                    returns it */
+    SSM_ERR_DEVICE_BOUNDS = 6   /* debug-bounds build only: a kernel computed a global index outside
+                                   its buffer and skipped that access (ssm_check_device_errors) */
 } ssm_status;
 
 typedef enum {
@@ -373,9 +375,28 @@ ssm_status ss2d_cross_merge(const void *ys, void *y, int64_t b, int64_t H,
 
 /*
  * Synchronises `stream` and returns SSM_OK, or SSM_ERR_CUDA with the CUDA
- * error of the stream (a kernel fault) in ssm_last_error().
+ * error of the stream (a kernel fault) in ssm_last_error().  In the
+ * debug-bounds build (libssmscan_debug.so, compiled with SSM_DEBUG_BOUNDS)
+ * it then reads and clears the device's bounds word: SSM_ERR_DEVICE_BOUNDS
+ * when a kernel computed a global index outside its buffer since the last
+ * check (the access was skipped; the message names the buffer kinds).
  */
 ssm_status ssm_check_device_errors(ssm_stream_t stream);
+
+/*
+ * Debug-bounds build: every kernel checks the global index of each load,
+ * store and atomic against the size of its buffer, records a miss in a
+ * device word and skips the access (no fault).  ssm_debug_bounds_enabled()
+ * returns 1 in libssmscan_debug.so and 0 in libssmscan.so.
+ * ssm_debug_bounds_self_test() enqueues one kernel whose single check is
+ * given an index one past its one-element range: the check records it and
+ * the access is skipped, so the next ssm_check_device_errors() on `stream`
+ * returns SSM_ERR_DEVICE_BOUNDS.  It returns SSM_ERR_UNSUPPORTED in the
+ * release library.  The pages have no counterpart; this is test
+ * infrastructure for the kernels' index arithmetic.
+ */
+int ssm_debug_bounds_enabled(void);
+ssm_status ssm_debug_bounds_self_test(ssm_stream_t stream);
 
 /* Message of the last non-OK status returned on this thread ("" if none). */
 const char *ssm_last_error(void);

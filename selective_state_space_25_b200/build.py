@@ -14,6 +14,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libssmscan.so")
+# the debug-bounds build: every kernel checks its global indices (SSM_DEBUG_BOUNDS)
+LIB_DEBUG = os.path.join(PKG, "libssmscan_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-shared",
@@ -36,18 +38,23 @@ def deps():
         sorted(glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(f) <= t for f in deps())
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *ARCH, *FLAGS, f"-I{INCLUDE}", f"-I{CSRC}", *sources(), "-o", tmp]
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False,
+          debug_bounds: bool = False) -> str:
+    """Builds libssmscan.so, or with debug_bounds libssmscan_debug.so (the
+    same sources compiled with SSM_DEBUG_BOUNDS)."""
+    lib = LIB_DEBUG if debug_bounds else LIB
+    if not force and up_to_date(lib):
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
+    defs = ["-DSSM_DEBUG_BOUNDS"] if debug_bounds else []
+    cmd = [nvcc(), *ARCH, *FLAGS, *defs, f"-I{INCLUDE}", f"-I{CSRC}", *sources(), "-o", tmp]
     if ptxas_info:
         cmd.insert(1, "-Xptxas=-v")
     if verbose:
@@ -57,10 +64,11 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
         raise RuntimeError(f"nvcc failed ({r.returncode}):\n{r.stdout}\n{r.stderr}")
     if verbose or ptxas_info:
         sys.stdout.write(r.stdout + r.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True, ptxas_info="--ptxas-info" in sys.argv)
-    print("built", LIB)
+    for dbg in (False, True):
+        print("built", build(force="--force" in sys.argv, verbose=True,
+                             ptxas_info="--ptxas-info" in sys.argv, debug_bounds=dbg))

@@ -223,14 +223,16 @@ __global__ void __launch_bounds__(128, 4) scan_bwd_kernel(BwdParams p) {
       const int k = i / (TT * GA), r = (i / GA) % TT, q = i % GA;
       const T *src = k == 0 ? gu : k == 1 ? gdelta : k == 2 ? (gz ? gz : gdout) : gdout;
       const int64_t col = d0 + q * EPG;
-      const bool ok = r < nT && col < d_in && (k != 2 || gz);
+      const bool ok = r < nT && col < d_in && (k != 2 || gz) &&
+                      in_bounds((ib * L + t0 + r) * d_in + col + EPG - 1, p.b * L * d_in, kBndAct);
       const T *gp = ok ? src + (ib * L + t0 + r) * d_in + col : src;
       cp_async16(raw + k * Cfg::RAW_ACT + r * DT + q * EPG, gp, ok ? 16 : 0);
     }
     for (int i = tid; i < (full ? 2 : 1) * TT * GB; i += NT) {
       const int k = i / (TT * GB), r = (i / GB) % TT, q = i % GB;
       const T *src = k == 0 ? gB : gC;
-      const bool ok = r < nT;
+      const bool ok =
+          r < nT && in_bounds((ib * L + t0 + r) * N + q * EPG + EPG - 1, p.b * L * N, kBndBC);
       const T *gp = ok ? src + (ib * L + t0 + r) * N + q * EPG : src;
       cp_async16(raw + 4 * Cfg::RAW_ACT + k * Cfg::RAW_BC + r * N + q * EPG, gp, ok ? 16 : 0);
     }
@@ -247,7 +249,7 @@ __global__ void __launch_bounds__(128, 4) scan_bwd_kernel(BwdParams p) {
       const int t = i / DT, cc = i - t * DT;
       const int64_t dd = d0 + cc;
       float dl = 0.0f, uu = 0.0f, gg = 0.0f, dzf = 0.0f, spg = 0.0f;
-      if (t < nT && dd < d_in) {
+      if (t < nT && dd < d_in && in_bounds((ib * L + t0 + t) * d_in + dd, p.b * L * d_in, kBndAct)) {
         const int64_t at = (ib * L + t0 + t) * d_in + dd;
         const int ra = t * DT + cc;
         const float pre =
@@ -299,6 +301,11 @@ __global__ void __launch_bounds__(128, 4) scan_bwd_kernel(BwdParams p) {
   };
 
   float *my_chunk_h = p.chunk_h + ((ib * nC) * d_in + d) * N + g * NPT;  // + c * d_in * N
+  // chunk c's saved state of this thread lies inside the workspace
+  auto chunk_ok = [&](int64_t c) {
+    return in_bounds(((ib * nC + c) * d_in + d) * N + g * NPT + NPT - 1, p.b * nC * d_in * N,
+                     kBndChunk);
+  };
   float h[NPT];
 
   // one forward step of this thread's states (pass 1 and the recompute)
@@ -327,7 +334,7 @@ __global__ void __launch_bounds__(128, 4) scan_bwd_kernel(BwdParams p) {
     cp_async_commit();
   }
   for (int c = 0; c < n_pass1; ++c) {
-    if (active) store_vec<NPT>(my_chunk_h + (int64_t)c * d_in * N, h);
+    if (active && chunk_ok(c)) store_vec<NPT>(my_chunk_h + (int64_t)c * d_in * N, h);
     if (c == nC - 1) break;  // the last chunk's end state is not needed
     if constexpr (ASYNC) {
       if (c + 1 <= nC - 2) issue(c + 1, false, (c + 1) & 1);
@@ -400,7 +407,7 @@ __global__ void __launch_bounds__(128, 4) scan_bwd_kernel(BwdParams p) {
 #pragma unroll
         for (int j = 0; j < NPT; ++j) acc[j] = fmaf(w, x[j], acc[j]);
       }
-      if (t < nT) {
+      if (t < nT && in_bounds((ib * L + t0 + t) * N + gi * NPT + NPT - 1, p.b * L * N, kBndBC)) {
         float *dst = out + (ib * L + t0 + t) * N + gi * NPT;
         if (p.vec_atomics) {
           if constexpr (NPT == 4) {
@@ -418,12 +425,13 @@ __global__ void __launch_bounds__(128, 4) scan_bwd_kernel(BwdParams p) {
   };
 
   float hs_next[NPT];
-  if (active) load_vec<NPT>(my_chunk_h + (int64_t)(nC - 1) * d_in * N, hs_next);
+  if (active && chunk_ok(nC - 1)) load_vec<NPT>(my_chunk_h + (int64_t)(nC - 1) * d_in * N, hs_next);
   for (int c = nC - 1; c >= 0; --c) {
     float hs[NPT];
 #pragma unroll
     for (int j = 0; j < NPT; ++j) hs[j] = active ? hs_next[j] : 0.0f;
-    if (c > 0 && active) load_vec<NPT>(my_chunk_h + (int64_t)(c - 1) * d_in * N, hs_next);
+    if (c > 0 && active && chunk_ok(c - 1))
+      load_vec<NPT>(my_chunk_h + (int64_t)(c - 1) * d_in * N, hs_next);
     if constexpr (ASYNC) {
       if (c > 0) issue(c - 1, true, (c - 1) & 1);
       cp_async_commit();
@@ -474,7 +482,7 @@ __global__ void __launch_bounds__(128, 4) scan_bwd_kernel(BwdParams p) {
       const float4 qv = sQ[s];
       const float gt = qv.z, dl = qv.x, uu = sU[s];
       const float ddt = fmaf(uu, S1, S2) * sSpg[s];
-      if (t < nT && dd < d_in) {
+      if (t < nT && dd < d_in && in_bounds((ib * L + t0 + t) * d_in + dd, p.b * L * d_in, kBndAct)) {
         const int64_t at = (ib * L + t0 + t) * d_in + dd;
         Elem<T>::store(static_cast<T *>(p.du), at, fmaf(gt, pD, dl * S1));
         Elem<T>::store(static_cast<T *>(p.ddelta), at, ddt);
@@ -486,7 +494,8 @@ __global__ void __launch_bounds__(128, 4) scan_bwd_kernel(BwdParams p) {
   }
   if constexpr (ASYNC) cp_async_wait<0>();  // nothing may be in flight at exit
 
-  if (active) {
+  if (active && in_bounds(d * N + g * NPT + NPT - 1, d_in * N, kBndParam) &&
+      in_bounds((ib * d_in + d) * N + g * NPT + NPT - 1, p.b * d_in * N, kBndState)) {
 #pragma unroll
     for (int j = 0; j < NPT; ++j) {
       atomicAdd(p.dA + d * N + g * NPT + j, dAacc[j]);

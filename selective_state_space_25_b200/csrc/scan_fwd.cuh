@@ -47,7 +47,7 @@ struct ScanParams {
 template <typename T, int N>
 __global__ void __launch_bounds__(128) scan_generic_kernel(ScanParams p) {
   const int64_t bd = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  if (bd >= p.b * p.d_in) return;
+  if (bd >= p.b * p.d_in || !in_bounds(bd * N + N - 1, p.b * p.d_in * N, kBndState)) return;
   const int64_t ib = bd / p.d_in;
   const int64_t d = bd - ib * p.d_in;
   const T *u = static_cast<const T *>(p.u);
@@ -68,13 +68,17 @@ __global__ void __launch_bounds__(128) scan_generic_kernel(ScanParams p) {
 
   const int64_t n_chunks = (p.L + kStateChunk - 1) / kStateChunk;
   for (int64_t t = 0; t < p.L; ++t) {
-    if (p.chunk_h && t % kStateChunk == 0) {
+    if (p.chunk_h && t % kStateChunk == 0 &&
+        in_bounds(((ib * n_chunks + t / kStateChunk) * p.d_in + d) * N + N - 1,
+                  p.b * n_chunks * p.d_in * N, kBndChunk)) {
       float *dst = p.chunk_h + ((ib * n_chunks + t / kStateChunk) * p.d_in + d) * N;
 #pragma unroll
       for (int n = 0; n < N; ++n) dst[n] = h[n];
     }
     const int64_t row = ib * p.L + t;
     const int64_t i = row * p.d_in + d;
+    if (!in_bounds(i, p.b * p.L * p.d_in, kBndAct) || !in_bounds(row * N + N - 1, p.b * p.L * N, kBndBC))
+      break;
     float delta = Elem<T>::load(dt, i) + bias;
     if (p.delta_softplus) delta = softplus_f32(delta);
     const float ut = Elem<T>::load(u, i);
@@ -239,7 +243,8 @@ __global__ void __launch_bounds__(FastScan<T, N, NPT, DT, TC, BCF>::THREADS)
     for (int q = tid; q < TC * S::ROW_GRAN; q += THREADS) {
       const int t = q / S::ROW_GRAN, gq = q - t * S::ROW_GRAN;
       const int64_t dd = d0 + gq * S::VEC;
-      const bool ok = (t0 + t < L) && (dd < d_in);
+      const bool ok = (t0 + t < L) && (dd < d_in) &&
+                      in_bounds((ib * L + t0 + t) * d_in + dd + S::VEC - 1, p.b * L * d_in, kBndAct);
       const int64_t off = ok ? ((ib * L + t0 + t) * d_in + dd) : 0;
       const int so = t * DT + gq * S::VEC;
       cp_async16(su + so, gu + off, ok ? 16 : 0);
@@ -248,7 +253,8 @@ __global__ void __launch_bounds__(FastScan<T, N, NPT, DT, TC, BCF>::THREADS)
     }
     for (int q = tid; q < TC * S::BC_GRAN; q += THREADS) {
       const int t = q / S::BC_GRAN, gq = q - t * S::BC_GRAN;
-      const bool ok = (t0 + t < L);
+      const bool ok =
+          (t0 + t < L) && in_bounds((ib * L + t0 + t) * N + gq * S::VEC + S::VEC - 1, p.b * L * N, kBndBC);
       const int64_t off = ok ? ((ib * L + t0 + t) * N + gq * S::VEC) : 0;
       const int so = stage * TC * N + t * N + gq * S::VEC;
       cp_async16(sB + so, gB + off, ok ? 16 : 0);
@@ -376,7 +382,9 @@ __global__ void __launch_bounds__(FastScan<T, N, NPT, DT, TC, BCF>::THREADS)
     // ---- scan over the chunk, 4 steps per pass
     const int tcr = (tc + 3) / 4 * 4;
     for (int t = 0; t < tcr; t += 4) {
-      if (SAVE && (t % kStateChunk) == 0 && t < tc && d_ok) {  // a saved chunk start
+      if (SAVE && (t % kStateChunk) == 0 && t < tc && d_ok &&
+          in_bounds(((ib * n_saved + (t0 + t) / kStateChunk) * d_in + d) * N + g * NPT + NPT - 1,
+                    p.b * n_saved * d_in * N, kBndChunk)) {  // a saved chunk start
         float2 *dst = reinterpret_cast<float2 *>(
             p.chunk_h + ((ib * n_saved + (t0 + t) / kStateChunk) * d_in + d) * N + g * NPT);
 #pragma unroll
@@ -405,14 +413,14 @@ __global__ void __launch_bounds__(FastScan<T, N, NPT, DT, TC, BCF>::THREADS)
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
           const int t = sg * 4 + s;
-          if (t < tc)
+          if (t < tc && in_bounds((ib * L + t0 + t) * d_in + dc, p.b * L * d_in, kBndAct))
             Elem<T>::store(gy, (ib * L + t0 + t) * d_in + dc, fmaf(Dc, uu[s], yy[s]) * gg[s]);
         }
       }
     }
   }
 
-  if (p.h_last && d_ok) {
+  if (p.h_last && d_ok && in_bounds((ib * d_in + d) * N + g * NPT + NPT - 1, p.b * d_in * N, kBndState)) {
     float *hl = p.h_last + (ib * d_in + d) * N + g * NPT;
 #pragma unroll
     for (int k = 0; k < NP2; ++k) {

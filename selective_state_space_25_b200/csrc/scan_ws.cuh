@@ -95,6 +95,9 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
   const int64_t t_end = p.Lb > 0 && t_begin + p.Lb < L ? t_begin + p.Lb : L;
   const int64_t nchunks = (t_end - t_begin + TC - 1) / TC;
   const int64_t blk_row = (ib * nblk + blk) * d_in;  // row of (batch, block) in blk_decay / blk_state
+  // buffer sizes (elements) for the debug-bounds checks
+  const int64_t n_act = p.b * L * d_in, n_bc = p.b * L * N, n_state = p.b * d_in * N;
+  const int64_t n_blk = p.b * nblk * d_in * N, n_par = d_in * N;
   auto arr = [&](int off, int buf) {
     return reinterpret_cast<float *>(smem + off + buf * K::ARR);
   };
@@ -115,13 +118,16 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
 #pragma unroll
     for (int k = 0; k < NP2; ++k) {
       const int n = g * NS + 2 * k;
-      A2[k] = d_ok ? make_float2(p.A[d * N + n] * kLog2e, p.A[d * N + n + 1] * kLog2e)
-                   : make_float2(0.0f, 0.0f);
+      A2[k] = d_ok && in_bounds(d * N + n + 1, n_par, kBndParam)
+                  ? make_float2(p.A[d * N + n] * kLog2e, p.A[d * N + n + 1] * kLog2e)
+                  : make_float2(0.0f, 0.0f);
       // the summary starts every block from zero; the scan starts block 0
       // from h0 and block k > 0 from the carry the carry pass left
       const float *h0 = blk == 0 ? p.h0 + (ib * d_in + d) * N + n
                                  : p.blk_state + (blk_row + d) * N + n;
-      const bool from = d_ok && !SUMMARY && (blk > 0 || p.h0);
+      const bool from = d_ok && !SUMMARY && (blk > 0 || p.h0) &&
+                        (blk == 0 ? in_bounds((ib * d_in + d) * N + n + 1, n_state, kBndState)
+                                  : in_bounds((blk_row + d) * N + n + 1, n_blk, kBndChunk));
       h[k] = from ? make_float2(h0[0], h0[1]) : make_float2(0.0f, 0.0f);
     }
     float dsum = 0.0f;  // sum of delta over the block (summary pass)
@@ -171,7 +177,9 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
           const int t = 4 * j4 + jj;
-          if (SAVE && t % kStateChunk == 0 && d_ok && t0 + t < L) {  // the state before step t
+          if (SAVE && t % kStateChunk == 0 && d_ok && t0 + t < L &&
+              in_bounds(((ib * n_saved + (t0 + t) / kStateChunk) * d_in + d) * N + g * NS + NS - 1,
+                        p.b * n_saved * d_in * N, kBndChunk)) {  // the state before step t
             float2 *dst = reinterpret_cast<float2 *>(
                 p.chunk_h + ((ib * n_saved + (t0 + t) / kStateChunk) * d_in + d) * N + g * NS);
 #pragma unroll
@@ -193,7 +201,7 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
       __syncthreads();  // partials of this chunk written; next chunk's pre-pass done
     }
     if constexpr (SUMMARY) {  // the block's map h -> P h + Q
-      if (d_ok) {
+      if (d_ok && in_bounds((blk_row + d) * N + g * NS + NS - 1, n_blk, kBndChunk)) {
         float *q = p.blk_state + (blk_row + d) * N + g * NS;
         float *pd = p.blk_decay + (blk_row + d) * N + g * NS;
 #pragma unroll
@@ -205,7 +213,8 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
           pd[2 * k + 1] = e.y;
         }
       }
-    } else if (p.h_last && d_ok && blk == nblk - 1) {
+    } else if (p.h_last && d_ok && blk == nblk - 1 &&
+               in_bounds((ib * d_in + d) * N + g * NS + NS - 1, n_state, kBndState)) {
       float *hl = p.h_last + (ib * d_in + d) * N + g * NS;
 #pragma unroll
       for (int k = 0; k < NP2; ++k) {
@@ -231,7 +240,8 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
     for (int q = hid; q < TC * K::ROW_GRAN; q += K::HELP_THREADS) {
       const int t = q / K::ROW_GRAN, gq = q - t * K::ROW_GRAN;
       const int64_t dd = d0 + gq * K::VEC;
-      const bool ok = (t0 + t < t_end) && (dd < d_in);
+      const bool ok = (t0 + t < t_end) && (dd < d_in) &&
+                      in_bounds((ib * L + t0 + t) * d_in + dd + K::VEC - 1, n_act, kBndAct);
       const int64_t off = ok ? ((ib * L + t0 + t) * d_in + dd) : 0;
       const int so = t * K::RAWROW + gq * 16;
       cp_async16(raw(slot, 0) + so, gu + off, ok ? 16 : 0);
@@ -240,7 +250,8 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
     }
     for (int q = hid; q < TC * K::BC_GRAN; q += K::HELP_THREADS) {
       const int t = q / K::BC_GRAN, gq = q - t * K::BC_GRAN;
-      const bool ok = t0 + t < t_end;
+      const bool ok = t0 + t < t_end &&
+                      in_bounds((ib * L + t0 + t) * N + gq * K::VEC + K::VEC - 1, n_bc, kBndBC);
       const int64_t off = ok ? ((ib * L + t0 + t) * N + gq * K::VEC) : 0;
       const int so = t * N + gq * K::VEC;
       cp_async16(rawbc(slot, 0) + so, gB + off, ok ? 16 : 0);
@@ -255,9 +266,10 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
   const int sg0 = hid / K::CPS;
   const int64_t dp = d0 + 2 * cp;
   const bool p_ok = dp < d_in;  // d_in is a multiple of VEC >= 4, so dp + 1 < d_in too
-  const float2 bias2 = (p_ok && p.dt_bias) ? make_float2(p.dt_bias[dp], p.dt_bias[dp + 1])
-                                           : make_float2(0.0f, 0.0f);
-  const float2 D2 = (p_ok && p.D) ? make_float2(p.D[dp], p.D[dp + 1]) : make_float2(0.0f, 0.0f);
+  const bool par_ok = p_ok && in_bounds(dp + 1, d_in, kBndParam);
+  const float2 bias2 = (par_ok && p.dt_bias) ? make_float2(p.dt_bias[dp], p.dt_bias[dp + 1])
+                                             : make_float2(0.0f, 0.0f);
+  const float2 D2 = (par_ok && p.D) ? make_float2(p.D[dp], p.D[dp + 1]) : make_float2(0.0f, 0.0f);
   // Every other group of four pairs visits its two channel rows in swapped
   // order, so a quarter-warp's 16-byte accesses hit distinct banks.  Rows are
   // chosen by register selects: a runtime index into the per-thread arrays
@@ -296,8 +308,8 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
         const int t = sg * 4 + jj;
-        if (t < tc) {
-          const int64_t o = (ib * L + t0 + t) * d_in + dp;
+        const int64_t o = (ib * L + t0 + t) * d_in + dp;
+        if (t < tc && in_bounds(o + 1, n_act, kBndAct)) {
           if constexpr (sizeof(T) == 2)
             *reinterpret_cast<uint32_t *>(gy + o) = pack_bf16x2(y0[jj], y1[jj]);
           else
@@ -416,6 +428,7 @@ __global__ void scan_carry_kernel(const float *h0, const float *blk_decay, float
   const int64_t q = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;  // (batch, channel, state)
   const int64_t per = d_in * N;
   if (q >= b * per) return;
+  if (!in_bounds((q / per * nblk + nblk - 1) * per + q % per, b * nblk * per, kBndChunk)) return;
   const int64_t ib = q / per, r = q - ib * per;
   float h = h0 ? h0[q] : 0.0f;
   float qn = blk_state[(ib * nblk) * per + r];

@@ -214,8 +214,14 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
       for (int r = tid; r < LC * Cfg::GRAN_PER_ROW; r += THREADS) {
         const int row = r / Cfg::GRAN_PER_ROW, part = r - row * Cfg::GRAN_PER_ROW;
         const int l = l0 + row;
-        const bool ok = l < Li;
-        const int pix = ok ? ss2d_pixel32<ORDER>(k, l, Hi, Wi, invH, invW) : 0;
+        const int pix0 = l < Li ? ss2d_pixel32<ORDER>(k, l, Hi, Wi, invH, invW) : 0;
+        const int po0 = part * (16 / Cfg::ESZ);
+        const bool ok =
+            l < Li &&
+            in_bounds((ib * L + pix0) * d_in + d0 + po0 + 16 / Cfg::ESZ - 1, p.b * L * d_in, kBndAct) &&
+            in_bounds(((ib * 4 + k) * L + l) * d_in + d0 + po0 + 16 / Cfg::ESZ - 1,
+                      p.b * 4 * L * d_in, kBndAct);
+        const int pix = ok ? pix0 : 0;
         if (part == 0) tR[row] = ACC_SMEM ? ss2d_acc_row(pix, Wi, invW) : pix;
         const int so = row * DT + part * (16 / Cfg::ESZ);
         const int po = part * (16 / Cfg::ESZ);
@@ -226,8 +232,11 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
       for (int r = tid; r < LC * DT; r += THREADS) {
         const int row = r / DT, ch = r - row * DT;
         const int l = l0 + row;
-        const bool ok = l < Li && d0 + ch < d_in;
-        const int pix = ok ? ss2d_pixel32<ORDER>(k, l, Hi, Wi, invH, invW) : 0;
+        const int pix0 = l < Li ? ss2d_pixel32<ORDER>(k, l, Hi, Wi, invH, invW) : 0;
+        const bool ok = l < Li && d0 + ch < d_in &&
+                        in_bounds((ib * L + pix0) * d_in + d0 + ch, p.b * L * d_in, kBndAct) &&
+                        in_bounds(((ib * 4 + k) * L + l) * d_in + d0 + ch, p.b * 4 * L * d_in, kBndAct);
+        const int pix = ok ? pix0 : 0;
         if (ch == 0) tR[row] = ACC_SMEM ? ss2d_acc_row(pix, Wi, invW) : pix;
         tD[r] = ok ? dk[l * di + ch] : T(0.0f);
         tU[r] = ok ? gu[pix * di + ch] : T(0.0f);
@@ -237,7 +246,9 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
       for (int r = tid; r < LC / Cfg::BC_VEC; r += THREADS) {
         const int l = l0 + r * Cfg::BC_VEC;
         const int rem = Li - l;
-        const int bytes = rem <= 0 ? 0 : (rem >= Cfg::BC_VEC ? 16 : rem * Cfg::ESZ);
+        int bytes = rem <= 0 ? 0 : (rem >= Cfg::BC_VEC ? 16 : rem * Cfg::ESZ);
+        if (bytes && !in_bounds((ib * 4 + k) * L + l + bytes / Cfg::ESZ - 1, p.b * 4 * L, kBndBC))
+          bytes = 0;
         const int64_t off = bytes ? (int64_t)k * L + l : 0;
         cp_async16(tB + r * Cfg::BC_VEC, gB + off, bytes);
         cp_async16(tC + r * Cfg::BC_VEC, gC + off, bytes);
@@ -341,7 +352,10 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
 #pragma unroll
     for (int j = 0; j < TS; ++j) {
       h = __ffma2_rn(a[j], h, bu[j]);
-      if (lb + j < Li) {
+      if (lb + j < Li &&
+          (ACC_SMEM ? in_bounds(rows[j] * DT + 2 * cp + 1, (int64_t)Li * DT, kBndWork)
+                    : in_bounds((ib * L + rows[j]) * d_in + d0 + 2 * cp + (ok1 ? 1 : 0),
+                                p.b * L * d_in, kBndWork))) {
         const float2 yv = __ffma2_rn(make_float2(cc[j], cc[j]), h, du[j]);
         float *dst = ACC_SMEM ? acc_s + rows[j] * DT + 2 * cp : acc_g + rows[j] * di + 2 * cp;
         if (ok1) {
@@ -390,6 +404,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
         int sc = w + sk;
         if (sc >= Wi) sc -= Wi;
         const int pix = hh * Wi + w;
+        if (!in_bounds((ib * L + pix) * d_in + d0 + ch, p.b * L * d_in, kBndAct)) continue;
         const float v = ACC_SMEM ? acc_s[(hh * Wi + sc) * DT + ch] : acc_g[pix * di + ch];
         Elem<T>::store(gy, pix * di + ch, v);
       }
@@ -413,7 +428,8 @@ __global__ void cross_scan_kernel(const T *u, T *xs, int64_t b, int64_t H, int64
     const int64_t l = (i / d_in) % L;
     const int k = (int)((i / (d_in * L)) % 4);
     const int64_t ib = i / (d_in * L * 4);
-    xs[i] = u[(ib * L + ss2d_pixel<ORDER>(k, l, H, W)) * d_in + d];
+    const int64_t src = (ib * L + ss2d_pixel<ORDER>(k, l, H, W)) * d_in + d;
+    if (in_bounds(src, b * L * d_in, kBndAct)) xs[i] = u[src];
   }
 }
 
@@ -430,8 +446,10 @@ __global__ void cross_merge_kernel(const T *ys, T *y, int64_t b, int64_t H, int6
     const int64_t hh = pix / W, ww = pix - hh * W;
     float s = 0.0f;
 #pragma unroll
-    for (int k = 0; k < 4; ++k)  // summed k0 + k1 + k2 + k3, rounded once
-      s += Elem<T>::load(ys, ((ib * 4 + k) * L + ss2d_step_of<ORDER>(k, hh, ww, H, W)) * d_in + d);
+    for (int k = 0; k < 4; ++k) {  // summed k0 + k1 + k2 + k3, rounded once
+      const int64_t src = ((ib * 4 + k) * L + ss2d_step_of<ORDER>(k, hh, ww, H, W)) * d_in + d;
+      if (in_bounds(src, b * 4 * L * d_in, kBndAct)) s += Elem<T>::load(ys, src);
+    }
     Elem<T>::store(y, i, s);
   }
 }

@@ -9,7 +9,38 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#ifdef SSM_DEBUG_BOUNDS
+// Error word of the debug-bounds build: every checked global access whose
+// index falls outside its buffer ORs its buffer-kind bit in here (and is
+// skipped); read and cleared by ssm_check_device_errors.
+__device__ unsigned int g_ssm_bounds_word = 0;
+#endif
+
 namespace ssm {
+
+// Buffer kinds of the debug-bounds checks (bits of the error word).
+enum BoundsKind : unsigned {
+  kBndAct = 1u << 0,      // (b, L, d_in) / (b, d_in) activations and their gradients
+  kBndBC = 1u << 1,       // B, C and their gradients
+  kBndParam = 1u << 2,    // A, D, dt_bias (and dA, dD, ddt_bias)
+  kBndState = 1u << 3,    // h0, h_last, the decode state, dh_last, dh0
+  kBndChunk = 1u << 4,    // saved chunk states, split-scan block maps
+  kBndWork = 1u << 5,     // SS2D accumulator workspace, conv window
+  kBndSelfTest = 1u << 31 // the library's own check of the mechanism
+};
+
+// True when 0 <= i < n.  The debug-bounds build (SSM_DEBUG_BOUNDS) checks
+// and records a miss in the error word; other builds compile this to true.
+__device__ __forceinline__ bool in_bounds(int64_t i, int64_t n, unsigned kind) {
+#ifdef SSM_DEBUG_BOUNDS
+  if (i >= 0 && i < n) return true;
+  atomicOr(&g_ssm_bounds_word, kind);
+  return false;
+#else
+  (void)i; (void)n; (void)kind;
+  return true;
+#endif
+}
 
 constexpr float kLog2e = 1.4426950408889634f;
 // Steps between the saved chunk-start states the backward scan works from.

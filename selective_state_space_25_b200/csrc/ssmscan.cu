@@ -1033,10 +1033,58 @@ ssm_status ss2d_scan_fwd_noalloc(const void *u, const void *delta, const float *
 
 ssm_status ssm_check_device_errors(ssm_stream_t stream) {
   g_last_error.clear();
-  const cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess)
     return fail(SSM_ERR_CUDA, "ssm_check_device_errors: %s", cudaGetErrorString(e));
+#ifdef SSM_DEBUG_BOUNDS
+  unsigned int w = 0;
+  e = cudaMemcpyFromSymbol(&w, g_ssm_bounds_word, sizeof w);
+  if (e != cudaSuccess)
+    return fail(SSM_ERR_CUDA, "ssm_check_device_errors: %s", cudaGetErrorString(e));
+  if (w) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(g_ssm_bounds_word, &zero, sizeof zero);
+    if (e != cudaSuccess)
+      return fail(SSM_ERR_CUDA, "ssm_check_device_errors: %s", cudaGetErrorString(e));
+    return fail(SSM_ERR_DEVICE_BOUNDS,
+                "a kernel computed an index outside its buffer (kinds 0x%08x: 1 activations, "
+                "2 B / C, 4 parameters, 8 states, 16 chunk states / block maps, 32 workspace, "
+                "0x80000000 self-test); the access was skipped",
+                w);
+  }
+#endif
   return ok();
+}
+
+int ssm_debug_bounds_enabled(void) {
+#ifdef SSM_DEBUG_BOUNDS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+}  // extern "C"
+
+namespace {
+// One check whose index is one past its one-element range: recorded and
+// skipped in the debug-bounds build (nothing is read or written).
+__global__ void bounds_self_test_kernel(float *never_written) {
+  if (ssm::in_bounds(1, 1, ssm::kBndSelfTest)) never_written[0] = 0.0f;
+}
+}  // namespace
+
+extern "C" {
+
+ssm_status ssm_debug_bounds_self_test(ssm_stream_t stream) {
+  g_last_error.clear();
+#ifdef SSM_DEBUG_BOUNDS
+  bounds_self_test_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(nullptr);
+  return check_launch("ssm_debug_bounds_self_test");
+#else
+  (void)stream;
+  return fail(SSM_ERR_UNSUPPORTED, "ssm_debug_bounds_self_test: not a debug-bounds build");
+#endif
 }
 
 }  // extern "C"

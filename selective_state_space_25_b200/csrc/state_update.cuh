@@ -105,7 +105,9 @@ __global__ void __launch_bounds__(256) state_update_kernel(StepParams p) {
   const int64_t gid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   const int64_t bd = gid / G;
   const int g = (int)(gid - bd * G);
-  const bool active = bd < p.b * p.d_in;
+  const bool active =
+      bd < p.b * p.d_in && in_bounds(bd * N + g * NPT + NPT - 1, p.b * p.d_in * N, kBndState) &&
+      (!CONV || in_bounds(bd * p.d_conv + p.d_conv - 1, p.b * p.d_in * p.d_conv, kBndWork));
   const int64_t ib = active ? bd / p.d_in : 0;
   const int64_t d = active ? bd - ib * p.d_in : 0;
   const T *xs = static_cast<const T *>(p.x);
@@ -191,7 +193,9 @@ __global__ void __launch_bounds__(256, SSM_STEP_MIN_CTAS) state_update_vec_kerne
 #pragma unroll
   for (int i = 0; i < CPT; ++i) {  // issue every state (and conv window) load first
     bd[i] = base + i * per;
-    on[i] = base < per && bd[i] < total;
+    on[i] = base < per && bd[i] < total &&
+            in_bounds(bd[i] * N + 4 * g + 3, total * N, kBndState) &&
+            (!CONV || in_bounds(bd[i] * p.d_conv + p.d_conv - 1, total * p.d_conv, kBndWork));
     st[i] = on[i] ? __ldcs(reinterpret_cast<const float4 *>(p.state + bd[i] * N + 4 * g))
                   : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     const int64_t c = on[i] ? bd[i] : 0;

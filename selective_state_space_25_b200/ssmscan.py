@@ -16,7 +16,10 @@ import re
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libssmscan.so")
+# SSM_DEBUG_BOUNDS=1 selects the debug-bounds build (every kernel checks its
+# global indices and records misses for check_device_errors)
+DEBUG_BOUNDS = os.environ.get("SSM_DEBUG_BOUNDS", "") == "1"
+LIB_PATH = os.path.join(_PKG, "libssmscan_debug.so" if DEBUG_BOUNDS else "libssmscan.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "ssmscan.h")
 
 if not os.path.exists(LIB_PATH):
@@ -27,10 +30,10 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 SSM_OK, SSM_ERR_INVALID_ARG, SSM_ERR_UNSUPPORTED, SSM_ERR_WORKSPACE, SSM_ERR_CUDA, \
-    SSM_ERR_DEVICE_TIMEOUT = range(6)
+    SSM_ERR_DEVICE_TIMEOUT, SSM_ERR_DEVICE_BOUNDS = range(7)
 SSM_F32, SSM_BF16 = 0, 1
 _STATUS = {0: "SSM_OK", 1: "SSM_ERR_INVALID_ARG", 2: "SSM_ERR_UNSUPPORTED", 3: "SSM_ERR_WORKSPACE",
-           4: "SSM_ERR_CUDA", 5: "SSM_ERR_DEVICE_TIMEOUT"}
+           4: "SSM_ERR_CUDA", 5: "SSM_ERR_DEVICE_TIMEOUT", 6: "SSM_ERR_DEVICE_BOUNDS"}
 
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
@@ -73,6 +76,10 @@ _lib.ss2d_cross_merge_ex.restype = _INT
 SS2D_ORDERS = {"cross": 0, "snake": 1}
 _lib.ssm_check_device_errors.argtypes = [_P]
 _lib.ssm_check_device_errors.restype = _INT
+_lib.ssm_debug_bounds_enabled.argtypes = []
+_lib.ssm_debug_bounds_enabled.restype = _INT
+_lib.ssm_debug_bounds_self_test.argtypes = [_P]
+_lib.ssm_debug_bounds_self_test.restype = _INT
 
 
 class SsmError(RuntimeError):
@@ -376,3 +383,14 @@ def ss2d_cross_merge(ys, H, W, y=None, stream=None, order="cross"):
 def check_device_errors(stream=None) -> None:
     """Synchronise and raise if a kernel reported a device-side error."""
     _check(_lib.ssm_check_device_errors(_stream(stream)), "ssm_check_device_errors")
+
+
+def debug_bounds_enabled() -> bool:
+    """True when the loaded library is the debug-bounds build."""
+    return bool(_lib.ssm_debug_bounds_enabled())
+
+
+def debug_bounds_self_test(stream=None) -> int:
+    """Enqueue the debug-bounds build's self-test (one index one past its
+    range: recorded, access skipped); returns the status of the call."""
+    return int(_lib.ssm_debug_bounds_self_test(_stream(stream)))

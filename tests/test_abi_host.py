@@ -254,3 +254,19 @@ def conv_step(**kw):
 ])
 def test_conv_step_validation(kw, status):
     assert conv_step(**kw) == status
+
+
+def test_debug_bounds_library_loads_and_exports_every_function():
+    """libssmscan_debug.so (the kernels with every global index checked) has
+    the release library's ABI and says which build it is; the release
+    library's self-test is rejected before any CUDA call."""
+    from selective_state_space_25_b200 import build as libbuild
+    path = libbuild.build(debug_bounds=True)
+    dbg = ctypes.CDLL(path)
+    for n in S.header_functions():
+        assert hasattr(dbg, n), f"libssmscan_debug.so does not export {n}"
+    dbg.ssm_debug_bounds_enabled.restype = ctypes.c_int
+    L.ssm_debug_bounds_enabled.restype = ctypes.c_int
+    assert dbg.ssm_debug_bounds_enabled() == 1
+    assert L.ssm_debug_bounds_enabled() == 0
+    assert L.ssm_debug_bounds_self_test(None) == S.SSM_ERR_UNSUPPORTED
