@@ -91,11 +91,16 @@ typedef enum {
 } ssm_ss2d_order;
 
 /*
- * Bytes of device workspace ssm_scan_fwd needs for this problem.  Every
- * kernel of this build keeps the recurrent state and its chunk carries on
- * chip, so this is 0 for every valid size; callers that pass what it returns
- * stay correct if a later build needs scratch.  Returns (size_t)-1 for
- * invalid sizes.
+ * Bytes of device workspace ssm_scan_fwd needs for this problem.  It is 0
+ * unless the problem has too few (batch, channel) pairs to fill the device,
+ * i.e. b * ceil(d_in / 32) CTAs fewer than half the SMs (d_state 8, 16 or 32,
+ * d_in a multiple of 8, L long enough to cut).  Such a scan is split along L
+ * into blocks scanned in parallel: every block's map h -> P h + Q is stored
+ * in the workspace, a carry pass turns the maps into each block's start
+ * state, and a replay writes y.  The workspace then holds two fp32 arrays
+ * (b, nblk, d_in, d_state) (the block decays P, then the block states Q and
+ * carries); nblk depends on the device's SM count, so query it on the device
+ * that runs the scan.  Returns (size_t)-1 for invalid sizes.
  */
 size_t ssm_scan_fwd_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t d_state);
 
@@ -116,8 +121,11 @@ size_t ssm_scan_fwd_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t 
  *   h0            device fp32 (b, d_in, d_state), nullable (zero start)
  *   h_last        device fp32 (b, d_in, d_state), nullable; may equal h0
  *   y             device, (b, L, d_in), dtype; must not alias an input
- *   workspace     device, >= ssm_scan_fwd_workspace_bytes(...) bytes; may be
- *                 NULL when that is 0 (always, in this build).  Not read.
+ *   workspace     device, >= ssm_scan_fwd_workspace_bytes(...) bytes, 16-byte
+ *                 aligned, not overlapping any other argument; may be NULL when
+ *                 that is 0.  Scratch: its contents on entry are not read and
+ *                 on return are unspecified.  Too small (or NULL when needed):
+ *                 SSM_ERR_WORKSPACE and nothing is launched.
  */
 ssm_status ssm_scan_fwd(const void *u, const void *delta, const float *A,
                         const void *B, const void *C, const float *D,

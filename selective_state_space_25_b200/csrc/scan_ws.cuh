@@ -32,13 +32,15 @@
 
 namespace ssm {
 
-template <typename T, int N, int NS, int TC, int H, int P>
+template <typename T, int N, int NS, int TC, int H, int P, int DT_ = 32>
 struct WsScan {
-  static constexpr int DT = 32;                 // channels per CTA: one per lane
+  // channels per CTA: one per lane; with DT < 32 a warp holds 32 / DT state
+  // groups of DT channels (each quarter- or half-warp reads one B / C address)
+  static constexpr int DT = DT_;
   static constexpr int G = N / NS;              // state groups = scan warps
   static constexpr int NP2 = NS / 2;            // state pairs per scan thread
   static constexpr int R = P + 2;               // ring slots
-  static constexpr int SCAN_THREADS = 32 * G;
+  static constexpr int SCAN_THREADS = DT * G;
   static constexpr int HELP_THREADS = 32 * H;
   static constexpr int THREADS = SCAN_THREADS + HELP_THREADS;
   static constexpr int TCP = TC + 4;            // padded channel-major row (floats)
@@ -66,6 +68,7 @@ struct WsScan {
   static_assert(TC % 4 == 0 && TC % kStateChunk == 0, "chunk length");
   static_assert(DT % VEC == 0 && N % VEC == 0, "whole granules");
   static_assert(HELP_THREADS % CPS == 0 && P >= 1, "helper layout");
+  static_assert((DT == 8 || DT == 16 || DT == 32) && SCAN_THREADS % 32 == 0, "channel tile");
   static_assert(RAWROW % 16 == 0 && OFF_BC % 16 == 0 && OFF_DL % 16 == 0, "alignment");
   static_assert(PL_FLOATS * 4 <= 48 * 1024, "static shared memory");
   static_assert(SMEM + PL_FLOATS * 4 <= 227 * 1024, "shared memory");
@@ -76,11 +79,12 @@ __device__ __forceinline__ void helper_barrier(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
 
-template <typename T, int N, int NS, int TC, int H, int P, bool HAS_Z, bool SAVE, bool SUMMARY>
-__global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
+template <typename T, int N, int NS, int TC, int H, int P, bool HAS_Z, bool SAVE, bool SUMMARY,
+          int DT_ = 32>
+__global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P, DT_>::THREADS)
     scan_ws_kernel(ScanParams p) {
   static_assert(!(SUMMARY && SAVE), "the summary pass saves no states");
-  using K = WsScan<T, N, NS, TC, H, P>;
+  using K = WsScan<T, N, NS, TC, H, P, DT_>;
   constexpr int DT = K::DT, G = K::G, NP2 = K::NP2, R = K::R, TCP = K::TCP;
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ __align__(16) float s_planes[K::PL_FLOATS];
@@ -110,8 +114,8 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
 
   if (tid < K::SCAN_THREADS) {
     // =================================================== scan warps
-    const int c = tid % DT;  // lane = channel
-    const int g = tid / DT;  // warp = state group
+    const int c = tid % DT;  // channel
+    const int g = tid / DT;  // state group
     const int64_t d = d0 + c;
     const bool d_ok = d < d_in;
     float2 A2[NP2], h[NP2];
@@ -142,41 +146,49 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
       float *pl_own = s_planes + ((buf * G + g) * DT + c) * TCP;
       const T *rB = rawbc(slot, 0), *rC = rawbc(slot, 1);
       // the exponentials and delta u B of the next 4-step group are formed
-      // while this group's recurrence runs, keeping the SFU busy
+      // one step at a time between this group's recurrence steps, so the SFU
+      // sees a steady stream instead of bursts of 4 * NP2 requests
       struct Grp {
         float2 a[4][NP2], b[4][NP2];
         StateWords<T, NS> C[4];
       };
-      auto stage1 = [&](int j4, Grp &q) {
-        const float4 dv = *reinterpret_cast<const float4 *>(rdl + 4 * j4);
-        const float4 uv = *reinterpret_cast<const float4 *>(rdu + 4 * j4);
-        const float dls[4] = {dv.x, dv.y, dv.z, dv.w};
-        const float dus[4] = {uv.x, uv.y, uv.z, uv.w};
+      auto stage1_step = [&](int t, int jj, float dl, float du, Grp &q) {
+        StateWords<T, NS> Bw;
+        Bw.load(rB + t * N + g * NS);
+        if constexpr (SUMMARY) dsum += dl;
+        else q.C[jj].load(rC + t * N + g * NS);
+        const float2 d2 = make_float2(dl, dl);
+        const float2 u2 = make_float2(du, du);
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const int t = 4 * j4 + jj;
-          StateWords<T, NS> Bw;
-          Bw.load(rB + t * N + g * NS);
-          if constexpr (SUMMARY) dsum += dls[jj];
-          else q.C[jj].load(rC + t * N + g * NS);
-          const float2 d2 = make_float2(dls[jj], dls[jj]);
-          const float2 u2 = make_float2(dus[jj], dus[jj]);
-#pragma unroll
-          for (int k = 0; k < NP2; ++k) {
-            q.a[jj][k] = exp2_sfu2(__fmul2_rn(d2, A2[k]));
-            q.b[jj][k] = __fmul2_rn(u2, Bw.pair(k));
-          }
+        for (int k = 0; k < NP2; ++k) {
+          q.a[jj][k] = exp2_sfu2(__fmul2_rn(d2, A2[k]));
+          q.b[jj][k] = __fmul2_rn(u2, Bw.pair(k));
         }
       };
       Grp cur, nxt;
-      stage1(0, cur);
+      {
+        const float4 dv = *reinterpret_cast<const float4 *>(rdl);
+        const float4 uv = *reinterpret_cast<const float4 *>(rdu);
+        stage1_step(0, 0, dv.x, uv.x, cur);
+        stage1_step(1, 1, dv.y, uv.y, cur);
+        stage1_step(2, 2, dv.z, uv.z, cur);
+        stage1_step(3, 3, dv.w, uv.w, cur);
+      }
 #pragma unroll
       for (int j4 = 0; j4 < TC / 4; ++j4) {
-        if (j4 + 1 < TC / 4) stage1(j4 + 1, nxt);
+        const bool ahead = j4 + 1 < TC / 4;
+        float4 ndv = make_float4(0.0f, 0.0f, 0.0f, 0.0f), nuv = ndv;
+        if (ahead) {
+          ndv = *reinterpret_cast<const float4 *>(rdl + 4 * (j4 + 1));
+          nuv = *reinterpret_cast<const float4 *>(rdu + 4 * (j4 + 1));
+        }
+        const float nds[4] = {ndv.x, ndv.y, ndv.z, ndv.w};
+        const float nus[4] = {nuv.x, nuv.y, nuv.z, nuv.w};
         float ys[4];
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
           const int t = 4 * j4 + jj;
+          if (ahead) stage1_step(t + 4, jj, nds[jj], nus[jj], nxt);
           if (SAVE && t % kStateChunk == 0 && d_ok && t0 + t < L &&
               in_bounds(((ib * n_saved + (t0 + t) / kStateChunk) * d_in + d) * N + g * NS + NS - 1,
                         p.b * n_saved * d_in * N, kBndChunk)) {  // the state before step t
@@ -195,7 +207,7 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P>::THREADS)
         }
         if constexpr (!SUMMARY)
           *reinterpret_cast<float4 *>(pl_own + 4 * j4) = make_float4(ys[0], ys[1], ys[2], ys[3]);
-        if (j4 + 1 < TC / 4) cur = nxt;
+        if (ahead) cur = nxt;
       }
       slot = slot == R - 1 ? 0 : slot + 1;
       __syncthreads();  // partials of this chunk written; next chunk's pre-pass done
