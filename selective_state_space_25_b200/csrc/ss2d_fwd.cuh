@@ -203,6 +203,10 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
   T *gy = static_cast<T *>(p.y) + ib * L * d_in + d0;
 
   float *acc_g = p.acc_global + ib * L * d_in + d0;  // this image, channel d0
+  // a channel pair is one 8-byte access: always in shared memory; in the
+  // caller's workspace only for even d_in and an 8-byte aligned workspace
+  const bool acc_pairs =
+      ACC_SMEM || ((d_in & 1) == 0 && (reinterpret_cast<uintptr_t>(p.acc_global) & 7) == 0);
 
   const int nchunks = (Li + LC - 1) / LC;
 
@@ -358,7 +362,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
                                 p.b * L * d_in, kBndWork))) {
         const float2 yv = __ffma2_rn(make_float2(cc[j], cc[j]), h, du[j]);
         float *dst = ACC_SMEM ? acc_s + rows[j] * DT + 2 * cp : acc_g + rows[j] * di + 2 * cp;
-        if (ok1) {
+        if (ok1 && acc_pairs) {
           float2 *d2 = reinterpret_cast<float2 *>(dst);
           if constexpr (K == 0)
             *d2 = yv;
@@ -366,6 +370,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
             *d2 = __fadd2_rn(*d2, yv);
         } else if (ok0) {
           dst[0] = K == 0 ? yv.x : dst[0] + yv.x;
+          if (ok1) dst[1] = K == 0 ? yv.y : dst[1] + yv.y;
         }
       }
     }

@@ -78,6 +78,30 @@ def test_ss2d_large_image_uses_workspace(ssm):
     assert rel_err(y, oracle_ss2d(inp, H, W)) <= 2e-2
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("order", ["cross", "snake"])
+@pytest.mark.parametrize("d_in,offset", [(13, 0), (16, 4), (13, 4)])
+def test_ss2d_workspace_odd_channels_or_4_byte_aligned(ssm, dtype, order, d_in, offset):
+    """The workspace accumulator when channel pairs cannot be 8-byte accesses:
+    odd d_in puts every other pair on an odd float, and a workspace that is
+    4- but not 8-byte aligned (the entry point asks for 4) shifts all of them."""
+    H, W = 80, 81
+    dt = "bf16" if dtype == torch.bfloat16 else "fp32"
+    need = ssm.ss2d_scan_fwd_workspace_bytes(1, H, W, d_in, 1)
+    assert need > 0
+    raw = torch.empty(need + 16, dtype=torch.uint8, device="cuda")
+    base = raw.data_ptr() % 8
+    ws = raw[(offset - base) % 8:][:need]
+    assert ws.data_ptr() % 8 == offset
+    inp = ss2d_inputs(1, H, W, d_in, 1, dt, seed=d_in * 7 + offset, with_dt_bias=True)
+    g = to_cuda(inp)
+    y = ssm.ss2d_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], H, W, D=g["D"],
+                          dt_bias=g["dt_bias"], workspace=ws, order=order)
+    ref = oracle.ss2d_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], H, W,
+                           D=inp["D"], dt_bias=inp["dt_bias"], order=order)
+    assert rel_err(y, ref) <= TOL[dtype]
+
+
 def test_ss2d_equals_composition_of_gpu_scans(ssm):
     """Fused SS2D == CrossScan, four 1-D scans, CrossMerge, all on the GPU."""
     b, H, W, d_in = 2, 12, 10, 16
