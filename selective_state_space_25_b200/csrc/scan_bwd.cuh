@@ -164,7 +164,7 @@ __device__ __forceinline__ float sum_partials(const float *s, int pch) {
 }
 
 template <typename T, int N, int NPT_, bool ASYNC>
-__global__ void __launch_bounds__(128, 4) scan_bwd_kernel(BwdParams p) {
+__global__ void __launch_bounds__(128, 3) scan_bwd_kernel(BwdParams p) {
   using Cfg = BwdCfg<T, N, NPT_>;
   constexpr int NPT = Cfg::NPT, G = Cfg::G, DT = Cfg::DT, TT = Cfg::TT, NT = Cfg::THREADS;
   constexpr int PROW = Cfg::PROW, HROW = Cfg::HROW;
@@ -361,16 +361,11 @@ __global__ void __launch_bounds__(128, 4) scan_bwd_kernel(BwdParams p) {
   const float pD = (d0 + pch < d_in && p.D) ? p.D[d0 + pch] : 0.0f;
   float Dacc = 0.0f, bias_acc = 0.0f;
 
-  auto adj_step = [&](int t, const float (&hs)[NPT]) {
+  // one adjoint step; hp = h_{t-1} (this thread's states before step t)
+  auto adj_step_h = [&](int t, const float (&hp)[NPT]) {
     const float4 qv = sQ[t * PROW + ch];
     const float gt = qv.z, dl = qv.x;
-    float hp[NPT], bv[NPT], cv[NPT], lt[NPT];
-    if (t > 0) {
-      load_vec<NPT>(sH + (t - 1) * HROW + tid * NPT, hp);
-    } else {
-#pragma unroll
-      for (int j = 0; j < NPT; ++j) hp[j] = hs[j];
-    }
+    float bv[NPT], cv[NPT], lt[NPT];
     load_bc<NPT>(sBC + 2 * (t * N + g * NPT), bv, cv);
     float S1 = 0.0f, S2 = 0.0f;
 #pragma unroll
@@ -387,6 +382,17 @@ __global__ void __launch_bounds__(128, 4) scan_bwd_kernel(BwdParams p) {
     store_vec<NPT>(sH + t * HROW + tid * NPT, lt);
     sP1[t * NT + tid] = S1;
     sP2[t * NT + tid] = S2;
+  };
+  // the same with h_{t-1} read back from the chunk's state rows
+  auto adj_step = [&](int t, const float (&hs)[NPT]) {
+    float hp[NPT];
+    if (t > 0) {
+      load_vec<NPT>(sH + (t - 1) * HROW + tid * NPT, hp);
+    } else {
+#pragma unroll
+      for (int j = 0; j < NPT; ++j) hp[j] = hs[j];
+    }
+    adj_step_h(t, hp);
   };
 
   // sum over the CTA's channels of w[t][ch] X[t][ch][n] for every (t, n) of
@@ -442,7 +448,9 @@ __global__ void __launch_bounds__(128, 4) scan_bwd_kernel(BwdParams p) {
     const int64_t t0 = (int64_t)c * TT;
     __syncthreads();
 
-    // recompute the chunk's states and the partial pre-gate outputs
+    // recompute the chunk's states and the partial pre-gate outputs; a full
+    // chunk also keeps them in registers for the adjoint
+    float hreg[TT][NPT];
 #pragma unroll
     for (int j = 0; j < NPT; ++j) h[j] = hs[j];
     if (nT == TT) {
@@ -450,6 +458,8 @@ __global__ void __launch_bounds__(128, 4) scan_bwd_kernel(BwdParams p) {
       for (int t = 0; t < TT; ++t) {
         sPy[t * NT + tid] = fwd_step(t);
         store_vec<NPT>(sH + t * HROW + tid * NPT, h);
+#pragma unroll
+        for (int j = 0; j < NPT; ++j) hreg[t][j] = h[j];
       }
     } else {
       for (int t = 0; t < nT; ++t) {
@@ -464,7 +474,8 @@ __global__ void __launch_bounds__(128, 4) scan_bwd_kernel(BwdParams p) {
     // the adjoint through the chunk (state rows become adjoint rows)
     if (nT == TT) {
 #pragma unroll
-      for (int t = TT - 1; t >= 0; --t) adj_step(t, hs);
+      for (int t = TT - 1; t >= 1; --t) adj_step_h(t, hreg[t - 1]);
+      adj_step_h(0, hs);
     } else {
       for (int t = nT - 1; t >= 0; --t) adj_step(t, hs);
     }
