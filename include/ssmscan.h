@@ -272,10 +272,10 @@ ssm_status ss2d_scan_fwd_ex(const void *u, const void *delta, const float *A,
 
 /*
  * Bytes of device workspace ss2d_scan_fwd needs (0 for d_state = 1 when
- * the fp32 accumulator of one (batch, 8-channel) tile, 32 * H * W bytes, fits
- * in shared memory, i.e. H * W <= 6272).  Larger images keep that
- * accumulator in the workspace: b * H * W * d_in fp32.  Returns (size_t)-1
- * for invalid sizes.
+ * the fp32 accumulator of one (batch, 8-channel) tile, 32 * H * W' bytes with
+ * W' = W rounded up to odd, fits in shared memory, i.e. H * W' <= 6272).
+ * Larger images keep that accumulator in the workspace: b * H * W * d_in
+ * fp32.  Returns (size_t)-1 for invalid sizes.
  */
 size_t ss2d_scan_fwd_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_in,
                                      int64_t d_state);

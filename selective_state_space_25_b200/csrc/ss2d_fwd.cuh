@@ -82,9 +82,9 @@ struct Ss2dParams {
 //   4. the segment replays its steps, h = dA h + delta u B, and adds
 //      y = C h + D u into the accumulator at the pixel each step visits.
 // TS is odd so the 8 segments of a warp hit distinct bank groups in the
-// staged rows; the accumulator rows are skewed (pixel (h, w) lives in row
-// h W + (w + kappa h) mod W, W + kappa odd) so both row- and column-major
-// runs spread over the banks.
+// staged rows; the accumulator row of pixel (h, w) is h RS + w with the
+// row stride RS = W rounded up to odd, so both row- and column-major runs
+// spread over the banks.
 // ---------------------------------------------------------------------------
 template <typename T, int TS, int WARPS>
 struct Ss2dCfg {
@@ -126,38 +126,26 @@ __device__ __forceinline__ int div_small(int a, int b, float inv_b) {
   return q;
 }
 
-// (x + dx) mod m for 0 <= x < m and |dx| <= 2 (m = 1 gives 0), branch-free.
-__device__ __forceinline__ int add_mod(int x, int dx, int m) {
-  x += dx;
-  x -= (x >= m) ? m : 0;
-  x -= (x >= m) ? m : 0;
-  x += (x < 0) ? m : 0;
-  x += (x < 0) ? m : 0;
-  return x;
-}
+// Row stride (pixels) of the shared accumulator: W rounded up to odd, so
+// runs TS (odd) steps apart in row- or column-major order fall on distinct
+// 32-byte bank groups.
+__host__ __device__ __forceinline__ int ss2d_acc_stride(int W) { return W | 1; }
 
-// Pixel -> accumulator row (see the skew above), for one-off lookups.
-__device__ __forceinline__ int ss2d_acc_row(int pix, int W, float invW) {
-  const int h = div_small(pix, W, invW), w = pix - h * W;
-  const int kh = ((W & 1) ? 2 : 1) * h;
-  int s = w + kh - div_small(kh, W, invW) * W;
-  if (s >= W) s -= W;
-  return h * W + s;
-}
-
-// Pixel direction k visits at step l (32-bit, for one-off lookups).
+// Image position (h, w) that direction k visits at step l (32-bit, one
+// division).
 template <int ORDER>
-__device__ __forceinline__ int ss2d_pixel32(int k, int l, int H, int W, float invH, float invW) {
+__device__ __forceinline__ void ss2d_pos(int k, int l, int H, int W, float invH, float invW,
+                                         int &h, int &w) {
   const int ll = k >= 2 ? H * W - 1 - l : l;
   if ((k & 1) == 0) {
-    if constexpr (ORDER == kOrderCross) return ll;
-    const int h = div_small(ll, W, invW), r = ll - h * W;
-    return h * W + ((h & 1) ? W - 1 - r : r);
+    h = div_small(ll, W, invW);
+    const int r = ll - h * W;
+    w = (ORDER == kOrderSnake && (h & 1)) ? W - 1 - r : r;
+  } else {
+    w = div_small(ll, H, invH);
+    const int r = ll - w * H;
+    h = (ORDER == kOrderSnake && (w & 1)) ? H - 1 - r : r;
   }
-  const int w = div_small(ll, H, invH);
-  const int r = ll - w * H;
-  const int h = (ORDER == kOrderSnake && (w & 1)) ? H - 1 - r : r;
-  return h * W + w;
 }
 
 // ROW_ASYNC: delta / u rows staged with cp.async (needs d_in a multiple of 8
@@ -192,7 +180,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
   // offsets fit 32-bit integers; only the per-(batch, direction) bases are 64-bit
   const int Hi = (int)H, Wi = (int)W, Li = (int)L, di = (int)d_in;
   const float invH = 1.0f / (float)Hi, invW = 1.0f / (float)Wi;
-  const int kappa = (Wi & 1) ? 2 : 1;
+  const int RS = ss2d_acc_stride(Wi);
   const int64_t dA = d0 + 2 * cp;    // first channel of the pair
   const bool ok0 = dA < d_in, ok1 = dA + 1 < d_in;
 
@@ -218,7 +206,9 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
       for (int r = tid; r < LC * Cfg::GRAN_PER_ROW; r += THREADS) {
         const int row = r / Cfg::GRAN_PER_ROW, part = r - row * Cfg::GRAN_PER_ROW;
         const int l = l0 + row;
-        const int pix0 = l < Li ? ss2d_pixel32<ORDER>(k, l, Hi, Wi, invH, invW) : 0;
+        int hh = 0, ww = 0;
+        if (l < Li) ss2d_pos<ORDER>(k, l, Hi, Wi, invH, invW, hh, ww);
+        const int pix0 = hh * Wi + ww;
         const int po0 = part * (16 / Cfg::ESZ);
         const bool ok =
             l < Li &&
@@ -226,7 +216,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
             in_bounds(((ib * 4 + k) * L + l) * d_in + d0 + po0 + 16 / Cfg::ESZ - 1,
                       p.b * 4 * L * d_in, kBndAct);
         const int pix = ok ? pix0 : 0;
-        if (part == 0) tR[row] = ACC_SMEM ? ss2d_acc_row(pix, Wi, invW) : pix;
+        if (part == 0) tR[row] = ACC_SMEM ? (ok ? hh * RS + ww : 0) : pix;
         const int so = row * DT + part * (16 / Cfg::ESZ);
         const int po = part * (16 / Cfg::ESZ);
         cp_async16(tD + so, dk + (ok ? l * di : 0) + po, ok ? 16 : 0);
@@ -236,12 +226,14 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
       for (int r = tid; r < LC * DT; r += THREADS) {
         const int row = r / DT, ch = r - row * DT;
         const int l = l0 + row;
-        const int pix0 = l < Li ? ss2d_pixel32<ORDER>(k, l, Hi, Wi, invH, invW) : 0;
+        int hh = 0, ww = 0;
+        if (l < Li) ss2d_pos<ORDER>(k, l, Hi, Wi, invH, invW, hh, ww);
+        const int pix0 = hh * Wi + ww;
         const bool ok = l < Li && d0 + ch < d_in &&
                         in_bounds((ib * L + pix0) * d_in + d0 + ch, p.b * L * d_in, kBndAct) &&
                         in_bounds(((ib * 4 + k) * L + l) * d_in + d0 + ch, p.b * 4 * L * d_in, kBndAct);
         const int pix = ok ? pix0 : 0;
-        if (ch == 0) tR[row] = ACC_SMEM ? ss2d_acc_row(pix, Wi, invW) : pix;
+        if (ch == 0) tR[row] = ACC_SMEM ? (ok ? hh * RS + ww : 0) : pix;
         tD[r] = ok ? dk[l * di + ch] : T(0.0f);
         tU[r] = ok ? gu[pix * di + ch] : T(0.0f);
       }
@@ -263,7 +255,17 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
 
   if (tid < DT) carry[tid] = 0.0f;  // the first direction starts from h = 0 (buffer 0)
   prefetch(0, 0);
-  float2 A2 = make_float2(0.0f, 0.0f), bias = A2, Dd = A2;
+  float2 A2 = make_float2(0.0f, 0.0f), bias = A2;
+  // the skip term of all four directions, (sum_k D_k) u, is added once, with
+  // direction 0's outputs
+  float2 Dsum = A2;
+  if (p.D) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (ok0) Dsum.x += p.D[k * d_in + dA];
+      if (ok1) Dsum.y += p.D[k * d_in + dA + 1];
+    }
+  }
 
   // one chunk of direction K (index arithmetic specialised per direction)
   // chunk q = k nchunks + c reads the carry in buffer q & 1 and leaves the
@@ -281,10 +283,11 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
 
     // ---- 1. this segment's steps into registers
     const int lb = l0 + seg * TS;
-    float2 a[TS], bu[TS], du[TS];
-    float cc[TS];
+    // the segment run from h = 0: Q its state, P the product of its decays,
+    // so step j's true output is C_j (P_j h_in + Q_j) = gg_j h_in + yl_j
+    float2 yl[TS], gg[TS];
     int rows[TS];  // accumulator row (or pixel) each step lands on
-    Aff2 mine{make_float2(1.0f, 1.0f), make_float2(0.0f, 0.0f)};
+    float2 P = make_float2(1.0f, 1.0f), Q = make_float2(0.0f, 0.0f);
 #pragma unroll
     for (int j = 0; j < TS; ++j) {
       const int row = seg * TS + j;
@@ -310,12 +313,14 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
       if (p.delta_softplus) e = softplus2_f32(e);
       if (!valid) e = make_float2(0.0f, 0.0f);  // identity step past the end
       const float2 x = __fmul2_rn(e, A2);
-      a[j] = A_POLY ? exp2_poly2(x) : exp2_sfu2(x);
-      bu[j] = __fmul2_rn(__fmul2_rn(e, uv), make_float2(bc.x, bc.x));
-      du[j] = __fmul2_rn(Dd, uv);
-      cc[j] = bc.y;
-      mine = aff2_then(mine, Aff2{a[j], bu[j]});
+      const float2 a = A_POLY ? exp2_poly2(x) : exp2_sfu2(x);
+      Q = __ffma2_rn(a, Q, __fmul2_rn(__fmul2_rn(e, uv), make_float2(bc.x, bc.x)));
+      P = __fmul2_rn(a, P);
+      const float2 c2 = make_float2(bc.y, bc.y);
+      yl[j] = K == 0 ? __ffma2_rn(c2, Q, __fmul2_rn(Dsum, uv)) : __fmul2_rn(c2, Q);
+      gg[j] = __fmul2_rn(c2, P);
     }
+    const Aff2 mine{P, Q};
     __syncthreads();  // staged rows consumed
     if (c + 1 < nchunks) prefetch(K, c + 1);
     else if (K < 3) prefetch(K + 1, 0);
@@ -355,12 +360,11 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     // ---- 4. replay, accumulate y at the visited pixels
 #pragma unroll
     for (int j = 0; j < TS; ++j) {
-      h = __ffma2_rn(a[j], h, bu[j]);
       if (lb + j < Li &&
-          (ACC_SMEM ? in_bounds(rows[j] * DT + 2 * cp + 1, (int64_t)Li * DT, kBndWork)
+          (ACC_SMEM ? in_bounds(rows[j] * DT + 2 * cp + 1, (int64_t)Hi * RS * DT, kBndWork)
                     : in_bounds((ib * L + rows[j]) * d_in + d0 + 2 * cp + (ok1 ? 1 : 0),
                                 p.b * L * d_in, kBndWork))) {
-        const float2 yv = __ffma2_rn(make_float2(cc[j], cc[j]), h, du[j]);
+        const float2 yv = __ffma2_rn(gg[j], h, yl[j]);
         float *dst = ACC_SMEM ? acc_s + rows[j] * DT + 2 * cp : acc_g + rows[j] * di + 2 * cp;
         if (ok1 && acc_pairs) {
           float2 *d2 = reinterpret_cast<float2 *>(dst);
@@ -377,8 +381,9 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     const bool last = c == nchunks - 1;
     if (last) __syncthreads();  // the next direction's updates touch the same pixels
     if (warp == WARPS - 1 && sl == Cfg::SPW - 1) {  // the next direction starts from h = 0
-      carry[(cq ^ 1) * DT + 2 * cp] = last ? 0.0f : h.x;
-      carry[(cq ^ 1) * DT + 2 * cp + 1] = last ? 0.0f : h.y;
+      const float2 hend = __ffma2_rn(P, h, Q);  // the state after the chunk
+      carry[(cq ^ 1) * DT + 2 * cp] = last ? 0.0f : hend.x;
+      carry[(cq ^ 1) * DT + 2 * cp + 1] = last ? 0.0f : hend.y;
     }
   };
 
@@ -387,7 +392,6 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     A2 = make_float2(ok0 ? p.A[pk0] * kLog2e : 0.0f, ok1 ? p.A[pk0 + 1] * kLog2e : 0.0f);
     bias = make_float2((ok0 && p.dt_bias) ? p.dt_bias[pk0] : 0.0f,
                        (ok1 && p.dt_bias) ? p.dt_bias[pk0 + 1] : 0.0f);
-    Dd = make_float2((ok0 && p.D) ? p.D[pk0] : 0.0f, (ok1 && p.D) ? p.D[pk0 + 1] : 0.0f);
     for (int c = 0; c < nchunks; ++c) {
       switch (k) {
         case 0: chunk(std::integral_constant<int, 0>{}, c); break;
@@ -400,20 +404,16 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
   __syncthreads();
 
   // ---- round once and store: image row by image row (a warp writes 4
-  // pixels x 8 channels per instruction), the skew undone per row
+  // pixels x 8 channels per instruction)
   const int ch = tid & (DT - 1);
   if (d0 + ch < d_in) {
-    int sk = 0;  // (kappa h) mod W
     for (int hh = 0; hh < Hi; ++hh) {
       for (int w = tid / DT; w < Wi; w += THREADS / DT) {
-        int sc = w + sk;
-        if (sc >= Wi) sc -= Wi;
         const int pix = hh * Wi + w;
         if (!in_bounds((ib * L + pix) * d_in + d0 + ch, p.b * L * d_in, kBndAct)) continue;
-        const float v = ACC_SMEM ? acc_s[(hh * Wi + sc) * DT + ch] : acc_g[pix * di + ch];
+        const float v = ACC_SMEM ? acc_s[(hh * RS + w) * DT + ch] : acc_g[pix * di + ch];
         Elem<T>::store(gy, pix * di + ch, v);
       }
-      sk = add_mod(sk, kappa, Wi);
     }
   }
 }

@@ -389,15 +389,17 @@ ssm_status check_step_args(const char *what, float *ssm_state, const void *x, co
 #define SSM_SS2D_APOLY 0
 #endif
 constexpr int kSs2dDT = 8;
-constexpr int64_t kSs2dSmemPixels = 6272;  // H W of the shared-memory fp32 accumulator, 32 B each
+// H RS (RS = W rounded up to odd) of the shared-memory fp32 accumulator, 32 B each
+constexpr int64_t kSs2dSmemPixels = 6272;
+int64_t ss2d_acc_pixels(int64_t H, int64_t W) { return H * (W | 1); }
 
 template <typename T, bool ACC_SMEM, bool ROW_ASYNC, bool BC_ASYNC, int ORDER>
 ssm_status launch_ss2d_cfg(const ssm::Ss2dParams &p, cudaStream_t st) {
   using Cfg = ssm::Ss2dCfg<T, SSM_SS2D_TS, SSM_SS2D_WARPS>;
   constexpr auto k = ssm::ss2d_n1_kernel<T, SSM_SS2D_TS, SSM_SS2D_WARPS, ACC_SMEM,
                                          SSM_SS2D_APOLY != 0, ROW_ASYNC, BC_ASYNC, ORDER>;
-  const int64_t L = p.H * p.W;
-  const int smem = Cfg::AUX_BYTES + (ACC_SMEM ? (int)(L * kSs2dDT * sizeof(float)) : 0);
+  const int smem =
+      Cfg::AUX_BYTES + (ACC_SMEM ? (int)(ss2d_acc_pixels(p.H, p.W) * kSs2dDT * sizeof(float)) : 0);
   if (ssm_status s = ensure_smem<k>(Cfg::AUX_BYTES + (int)(kSs2dSmemPixels * kSs2dDT * 4),
                                     "ss2d_scan_fwd"))
     return s;
@@ -422,7 +424,8 @@ ssm_status launch_ss2d_order(const ssm::Ss2dParams &p, cudaStream_t st) {
   const size_t es = sizeof(T);
   const bool row_async = (p.d_in % kSs2dDT) == 0 && aligned(p.u, 16) && aligned(p.delta, 16);
   const bool bc_async = (L * (int64_t)es) % 16 == 0 && aligned(p.B, 16) && aligned(p.C, 16);
-  if (L <= kSs2dSmemPixels) return launch_ss2d_acc<T, true, ORDER>(p, row_async, bc_async, st);
+  if (ss2d_acc_pixels(p.H, p.W) <= kSs2dSmemPixels)
+    return launch_ss2d_acc<T, true, ORDER>(p, row_async, bc_async, st);
   return launch_ss2d_acc<T, false, ORDER>(p, row_async, bc_async, st);
 }
 
@@ -750,7 +753,7 @@ size_t ss2d_scan_fwd_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_
       !mul_ok(b, L, &t) || !mul_ok(t, d_in, &t) || !mul_ok(t, 4 * d_state, &t) ||
       t > INT64_MAX / 8)
     return (size_t)-1;
-  if (L <= kSs2dSmemPixels) return 0;
+  if (ss2d_acc_pixels(H, W) <= kSs2dSmemPixels) return 0;
   return (size_t)(b * L * d_in) * sizeof(float);
 }
 
