@@ -166,6 +166,28 @@ __device__ __forceinline__ float2 exp2_sfu2(float2 x) {
   return make_float2(ex2_approx(x.x), ex2_approx(x.y));
 }
 
+// 32-byte vector accesses (sm_100 and later); the address must be 32-byte
+// aligned.  The streaming load is volatile so it stays ordered before the
+// (volatile) store that writes the same state back.
+__device__ __forceinline__ void ld8_stream(const float *q, float *v) {
+  asm volatile("ld.global.cs.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]),
+                 "=f"(v[6]), "=f"(v[7])
+               : "l"(q));
+}
+__device__ __forceinline__ void st8_stream(float *q, const float *v) {
+  asm volatile("st.global.cs.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(q), "f"(v[0]),
+               "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
+               : "memory");
+}
+// read-only data (not written while the kernel runs)
+__device__ __forceinline__ void ld8_ro(const void *q, uint32_t *w) {
+  asm("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+      : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]),
+        "=r"(w[7])
+      : "l"(q));
+}
+
 // ------------------------------------------------------- element access
 template <typename T> struct Elem;
 template <> struct Elem<float> {

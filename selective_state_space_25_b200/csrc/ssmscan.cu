@@ -305,6 +305,15 @@ __global__ void copy_or_zero_kernel(const float *src, float *dst, int64_t n) {
 template <typename T, int N, bool CONV>
 ssm_status launch_step(const ssm::StepParams &p, cudaStream_t st, const char *what) {
   const int block = 256;
+  if constexpr (N == 4 || N == 8 || N == 16) {  // one thread per channel, 32-byte vectors
+    constexpr size_t al = N == 4 ? 16 : 32;
+    if (aligned(p.state, al) && aligned(p.A, al) && aligned(p.B, al) && aligned(p.C, al)) {
+      const int64_t threads = p.b * p.d_in;
+      ssm::state_update_lane_kernel<T, N, CONV>
+          <<<(unsigned)((threads + block - 1) / block), block, 0, st>>>(p);
+      return check_launch(what);
+    }
+  }
   if constexpr (N >= 4) {
     if (aligned(p.state, 16) && aligned(p.A, 16) && aligned(p.B, 16) && aligned(p.C, 16)) {
       constexpr int CPT = CONV ? SSM_CONV_STEP_CPT : SSM_STEP_CPT;

@@ -7,9 +7,11 @@
 // + D x, y = y * act(z).
 //
 // The step is a streaming read-modify-write of the fp32 state: 8 bytes per
-// (batch, channel, state) plus a few bytes per channel.  G = N / 4 threads
-// share a channel, each moving 4 states as one 16-byte vector; the partial
-// C.state sums meet in a G-lane shuffle.
+// (batch, channel, state) plus a few bytes per channel.  For N = 4, 8, 16 one
+// thread owns a channel and moves its states as 32-byte vectors
+// (state_update_lane_kernel); for N = 32, 64 G = N / 4 threads share a
+// channel, each moving 4 states as one 16-byte vector, and the partial
+// C.state sums meet in a G-lane shuffle (state_update_vec_kernel).
 #pragma once
 
 #include "ssm_common.cuh"
@@ -254,6 +256,152 @@ __global__ void __launch_bounds__(256, SSM_STEP_MIN_CTAS) state_update_vec_kerne
       Elem<T>::store(static_cast<T *>(p.y), bd[i], yv);
     }
   }
+}
+
+// A whole B or C row (N entries of the activation dtype) as packed words.
+template <typename T, int N> struct RowWords {
+  static constexpr int W = N * (int)sizeof(T) / 4;  // 32-bit words
+  uint32_t w[W];
+  __device__ __forceinline__ void load(const T *row) {
+    if constexpr (W % 8 == 0) {  // 32-byte rows: one 32-byte load each
+#pragma unroll
+      for (int i = 0; i < W; i += 8) ld8_ro(reinterpret_cast<const uint32_t *>(row) + i, w + i);
+    } else if constexpr (W % 4 == 0) {
+#pragma unroll
+      for (int i = 0; i < W; i += 4) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4 *>(row) + i / 4);
+        w[i] = q.x; w[i + 1] = q.y; w[i + 2] = q.z; w[i + 3] = q.w;
+      }
+    } else {
+      static_assert(W == 2, "row of 8 bytes");
+      const uint2 q = __ldg(reinterpret_cast<const uint2 *>(row));
+      w[0] = q.x; w[1] = q.y;
+    }
+  }
+  // entries 2k, 2k + 1 as an fp32 pair
+  __device__ __forceinline__ float2 pair(int k) const {
+    if constexpr (sizeof(T) == 2)
+      return make_float2(bf16lo(w[k]), bf16hi(w[k]));
+    else
+      return make_float2(__uint_as_float(w[2 * k]), __uint_as_float(w[2 * k + 1]));
+  }
+};
+
+#ifndef SSM_LANE_MIN_CTAS
+#define SSM_LANE_MIN_CTAS 3
+#endif
+
+// One thread per (batch, channel) (N = 4, 8 or 16; state, A, B and C 32-byte
+// aligned, 16 for N = 4): the channel's N states are 32-byte vectors (one
+// 16-byte vector for N = 4), issued with its A row and the batch's B / C
+// rows before any arithmetic, so every per-channel term (the division that
+// splits the channel index, softplus, the conv step, the gate, y) is formed
+// once per channel rather than on each of G lanes of a channel.  Each lane
+// moves whole 32-byte sectors: a warp's state loads cover one contiguous
+// 32 N-float span in N / 8 instructions.
+template <typename T, int N, bool CONV>
+__global__ void __launch_bounds__(256, SSM_LANE_MIN_CTAS) state_update_lane_kernel(StepParams p) {
+  static_assert(N == 4 || N == 8 || N == 16, "one thread per channel for N = 4, 8, 16");
+  const int64_t total = p.b * p.d_in;
+  const int64_t bd = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (bd >= total || !in_bounds(bd * N + N - 1, total * N, kBndState) ||
+      (CONV && !in_bounds(bd * p.d_conv + p.d_conv - 1, total * p.d_conv, kBndWork)))
+    return;  // nothing below synchronises, so idle threads may leave
+  const int64_t ib = total <= 0xffffffffll ? (int64_t)((uint32_t)bd / (uint32_t)p.d_in)
+                                           : bd / p.d_in;
+  const int64_t d = bd - ib * p.d_in;
+  if (!in_bounds(d * N + N - 1, p.d_in * N, kBndParam)) return;
+
+  float sv[N], av[N];
+  float *sp = p.state + bd * N;
+  if constexpr (N % 8 == 0) {
+#pragma unroll
+    for (int v = 0; v < N; v += 8) ld8_stream(sp + v, sv + v);
+#pragma unroll
+    for (int v = 0; v < N; v += 8) ld8_ro(p.A + d * N + v, reinterpret_cast<uint32_t *>(av + v));
+  } else {
+    const float4 s4 = __ldcs(reinterpret_cast<const float4 *>(sp));
+    const float4 a4 = __ldg(reinterpret_cast<const float4 *>(p.A + d * N));
+    sv[0] = s4.x; sv[1] = s4.y; sv[2] = s4.z; sv[3] = s4.w;
+    av[0] = a4.x; av[1] = a4.y; av[2] = a4.z; av[3] = a4.w;
+  }
+  RowWords<T, N> brow, crow;
+  brow.load(static_cast<const T *>(p.B) + ib * N);
+  crow.load(static_cast<const T *>(p.C) + ib * N);
+  float xv = Elem<T>::load(static_cast<const T *>(p.x), bd);
+  const float dtv = Elem<T>::load(static_cast<const T *>(p.dt), bd);
+  const T *zs = static_cast<const T *>(p.z);
+  const float zv = zs ? Elem<T>::load(zs, bd) : 0.0f;
+  const float bias = p.dt_bias ? p.dt_bias[d] : 0.0f;
+  const float Dv = p.D ? p.D[d] : 0.0f;
+
+  if constexpr (CONV) {  // the window rolled left with x appended, dotted with the weight
+    T *cs = static_cast<T *>(p.conv_state) + bd * p.d_conv;
+    const float *w = p.conv_w + d * p.d_conv;
+    const int K = p.d_conv;
+    float acc = p.conv_b ? p.conv_b[d] : 0.0f;
+    if (K == 4 && (reinterpret_cast<uintptr_t>(cs) & (4 * sizeof(T) - 1)) == 0 &&
+        (reinterpret_cast<uintptr_t>(w) & 15) == 0) {
+      // the common width: window and weight as one vector each
+      const float4 w4 = __ldg(reinterpret_cast<const float4 *>(w));
+      if constexpr (sizeof(T) == 2) {
+        const uint2 q = *reinterpret_cast<const uint2 *>(cs);  // taps 0, 1 | 2, 3
+        acc = fmaf(bf16hi(q.x), w4.x, acc);
+        acc = fmaf(bf16lo(q.y), w4.y, acc);
+        acc = fmaf(bf16hi(q.y), w4.z, acc);
+        acc = fmaf(xv, w4.w, acc);
+        // rolled window: taps 1, 2 | 3, x (x is a widened bf16, so its top
+        // half is its exact bit pattern)
+        const uint32_t xb = __float_as_uint(xv) >> 16;
+        *reinterpret_cast<uint2 *>(cs) =
+            make_uint2(__byte_perm(q.x, q.y, 0x5432), __byte_perm(q.y, xb, 0x5432));
+      } else {
+        const float4 q = *reinterpret_cast<const float4 *>(cs);
+        acc = fmaf(q.y, w4.x, acc);
+        acc = fmaf(q.z, w4.y, acc);
+        acc = fmaf(q.w, w4.z, acc);
+        acc = fmaf(xv, w4.w, acc);
+        *reinterpret_cast<float4 *>(cs) = make_float4(q.y, q.z, q.w, xv);
+      }
+    } else {
+      float win[kMaxConv];
+#pragma unroll
+      for (int j = 0; j < kMaxConv; ++j) {
+        if (j < K) {
+          win[j] = j + 1 < K ? Elem<T>::load(cs, j + 1) : xv;
+          acc = fmaf(win[j], w[j], acc);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kMaxConv; ++j)
+        if (j < K) Elem<T>::store(cs, j, win[j]);
+    }
+    xv = silu_f32(acc);
+  }
+
+  float delta = dtv + bias;
+  if (p.dt_softplus) delta = softplus_f32(delta);
+  const float2 dl2 = make_float2(delta * kLog2e, delta * kLog2e);
+  const float2 dx2 = make_float2(delta * xv, delta * xv);
+  float2 yacc = make_float2(0.0f, 0.0f);
+#pragma unroll
+  for (int k = 0; k < N / 2; ++k) {
+    float2 s2 = make_float2(sv[2 * k], sv[2 * k + 1]);
+    const float2 a2 = exp2_sfu2(__fmul2_rn(dl2, make_float2(av[2 * k], av[2 * k + 1])));
+    s2 = __ffma2_rn(s2, a2, __fmul2_rn(dx2, brow.pair(k)));
+    sv[2 * k] = s2.x;
+    sv[2 * k + 1] = s2.y;
+    yacc = __ffma2_rn(s2, crow.pair(k), yacc);
+  }
+  if constexpr (N % 8 == 0) {
+#pragma unroll
+    for (int v = 0; v < N; v += 8) st8_stream(sp + v, sv + v);
+  } else {
+    __stcs(reinterpret_cast<float4 *>(sp), make_float4(sv[0], sv[1], sv[2], sv[3]));
+  }
+  float yv = fmaf(Dv, xv, yacc.x + yacc.y);
+  if (zs) yv *= silu_for<T>(zv);
+  Elem<T>::store(static_cast<T *>(p.y), bd, yv);
 }
 
 }  // namespace ssm
