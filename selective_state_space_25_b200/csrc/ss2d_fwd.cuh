@@ -403,16 +403,38 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
   }
   __syncthreads();
 
-  // ---- round once and store: image row by image row (a warp writes 4
-  // pixels x 8 channels per instruction)
-  const int ch = tid & (DT - 1);
-  if (d0 + ch < d_in) {
-    for (int hh = 0; hh < Hi; ++hh) {
-      for (int w = tid / DT; w < Wi; w += THREADS / DT) {
-        const int pix = hh * Wi + w;
-        if (!in_bounds((ib * L + pix) * d_in + d0 + ch, p.b * L * d_in, kBndAct)) continue;
-        const float v = ACC_SMEM ? acc_s[(hh * RS + w) * DT + ch] : acc_g[pix * di + ch];
-        Elem<T>::store(gy, pix * di + ch, v);
+  // ---- round once and store.  Shared accumulator, whole 8-channel tile and
+  // 16-byte aligned rows: one pixel per thread, its 8 channels as one vector;
+  // otherwise image row by image row, a channel per thread.
+  if (ACC_SMEM && d0 + DT <= d_in && (d_in * Cfg::ESZ) % 16 == 0 &&
+      (reinterpret_cast<uintptr_t>(p.y) & 15) == 0) {
+    for (int pix = tid; pix < Li; pix += THREADS) {
+      const int hh = div_small(pix, Wi, invW), w = pix - hh * Wi;
+      if (!in_bounds((ib * L + pix) * d_in + d0 + DT - 1, p.b * L * d_in, kBndAct) ||
+          !in_bounds((int64_t)(hh * RS + w) * DT + DT - 1, (int64_t)Hi * RS * DT, kBndWork))
+        continue;
+      const float4 *a4 = reinterpret_cast<const float4 *>(acc_s + (hh * RS + w) * DT);
+      const float4 v0 = a4[0], v1 = a4[1];
+      if constexpr (sizeof(T) == 2) {
+        *reinterpret_cast<uint4 *>(gy + pix * di) =
+            make_uint4(pack_bf16x2(v0.x, v0.y), pack_bf16x2(v0.z, v0.w), pack_bf16x2(v1.x, v1.y),
+                       pack_bf16x2(v1.z, v1.w));
+      } else {
+        float4 *o = reinterpret_cast<float4 *>(gy + pix * di);
+        o[0] = v0;
+        o[1] = v1;
+      }
+    }
+  } else {
+    const int ch = tid & (DT - 1);
+    if (d0 + ch < d_in) {
+      for (int hh = 0; hh < Hi; ++hh) {
+        for (int w = tid / DT; w < Wi; w += THREADS / DT) {
+          const int pix = hh * Wi + w;
+          if (!in_bounds((ib * L + pix) * d_in + d0 + ch, p.b * L * d_in, kBndAct)) continue;
+          const float v = ACC_SMEM ? acc_s[(hh * RS + w) * DT + ch] : acc_g[pix * di + ch];
+          Elem<T>::store(gy, pix * di + ch, v);
+        }
       }
     }
   }
