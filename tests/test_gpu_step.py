@@ -46,6 +46,26 @@ def test_step_misaligned_state_and_no_gate(ssm):
     assert rel_err(y, y_ref) <= 1e-4 and rel_err(st, st_ref) <= 1e-5
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_step_state_16_but_not_32_byte_aligned(ssm, dtype):
+    """N = 16 with a state 16- but not 32-byte aligned: the one-thread-per-channel
+    kernel needs 32-byte vectors, so the four-lanes-per-channel kernel runs."""
+    dt = "bf16" if dtype == torch.bfloat16 else "fp32"
+    inp = step_inputs(3, 45, 16, dt, seed=21)
+    g = to_cuda(inp)
+    n = inp["state"].numel()
+    raw = torch.empty(n + 16, device="cuda")
+    base = (raw.data_ptr() // 4) % 8                      # floats past a 32-byte boundary
+    off = (4 - base) % 8                                  # land 16 bytes past one
+    st = raw[off:off + n].view(inp["state"].shape)
+    assert st.data_ptr() % 32 == 16
+    st.copy_(g["state"])
+    y = gpu_step(ssm, g, st)
+    y_ref, st_ref = oracle.state_update(inp["state"], inp["x"], inp["dt"], inp["A"], inp["B"],
+                                        inp["C"], D=inp["D"], z=inp["z"], dt_bias=inp["dt_bias"])
+    assert rel_err(y, y_ref) <= TOL[dtype] and rel_err(st, st_ref) <= 1e-5
+
+
 def test_decode_workload_steps_1_10_1000(ssm):
     w = WORKLOADS["mamba-decode-step"]
     d = w.dims
@@ -138,6 +158,26 @@ def test_conv_step_shapes(ssm, dtype, b, d_in, N, d_conv):
     assert rel_err(y, y_ref) <= TOL[dtype]
     assert rel_err(st, st_ref) <= 1e-5
     np.testing.assert_array_equal(to64(cs), cs_ref)      # the window only moves stored values
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_conv_step_window_not_vector_aligned(ssm, dtype):
+    """d_conv = 4 with the window one element off a vector boundary: the
+    one-thread-per-channel kernel reads and writes it tap by tap."""
+    dt = "bf16" if dtype == torch.bfloat16 else "fp32"
+    inp = step_inputs(2, 33, 16, dt, seed=31)
+    c = conv_inputs(2, 33, 4, dt, seed=32)
+    g, gc = to_cuda(inp), to_cuda(c)
+    st = g["state"].clone()
+    n = c["conv_state"].numel()
+    raw = torch.empty(n + 1, dtype=gc["conv_state"].dtype, device="cuda")
+    cs = raw[1:1 + n].view(c["conv_state"].shape)
+    assert cs.data_ptr() % (4 * cs.element_size()) != 0
+    cs.copy_(gc["conv_state"])
+    y = gpu_conv_step(ssm, g, gc, cs, st)
+    y_ref, st_ref, cs_ref = oracle_conv_then_step(inp, c, c["conv_state"], inp["state"])
+    assert rel_err(y, y_ref) <= TOL[dtype] and rel_err(st, st_ref) <= 1e-5
+    np.testing.assert_array_equal(to64(cs), cs_ref)
 
 
 def test_conv_step_no_bias_no_gate_misaligned(ssm):
