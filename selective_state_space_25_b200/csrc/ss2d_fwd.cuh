@@ -321,9 +321,6 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
       gg[j] = __fmul2_rn(c2, P);
     }
     const Aff2 mine{P, Q};
-    __syncthreads();  // staged rows consumed
-    if (c + 1 < nchunks) prefetch(K, c + 1);
-    else if (K < 3) prefetch(K + 1, 0);
 
     // ---- 2. inclusive scan over the warp's segments (lanes cp, cp + 4, ...)
     Aff2 inc = mine;
@@ -343,7 +340,9 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     exc.b.y = __shfl_up_sync(0xffffffffu, inc.b.y, 4);
     if (sl == 0) exc = Aff2{make_float2(1.0f, 1.0f), make_float2(0.0f, 0.0f)};
     if (sl == Cfg::SPW - 1) agg[warp * Cfg::PAIRS + cp] = make_float4(inc.a.x, inc.a.y, inc.b.x, inc.b.y);
-    __syncthreads();
+    __syncthreads();  // warp totals visible; every thread is done with the staged rows
+    if (c + 1 < nchunks) prefetch(K, c + 1);
+    else if (K < 3) prefetch(K + 1, 0);
 
     // ---- 3. incoming state: previous chunk's carry, earlier warps, earlier segments
     float2 h = make_float2(carry[cq * DT + 2 * cp], carry[cq * DT + 2 * cp + 1]);
