@@ -37,10 +37,10 @@
  *     reported by the call that launched.  A fault while a kernel runs is a
  *     CUDA error of the stream, reported by the next call that synchronises
  *     it (ssm_check_device_errors() does).
- *   - Calls allocate nothing and never synchronise, so they can be captured
- *     in a CUDA graph; make the first call of each kind and d_state outside
- *     any capture (it sets the kernel's shared-memory attribute once per
- *     device).
+ *   - Calls allocate nothing and never synchronise.  Those that take their
+ *     scratch from the caller can be captured in a CUDA graph; make the
+ *     first call of each kind and d_state outside any capture (it sets the
+ *     kernel's shared-memory attribute once per device).
  *   - A non-OK status leaves a message in ssm_last_error() (per thread).
  *   - Outputs must not alias inputs unless stated.
  *   - dtype: SSM_F32 or SSM_BF16 applies to every activation-sized tensor of
@@ -294,11 +294,9 @@ size_t ss2d_scan_fwd_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_
  * the process exits.  Limit: b * H * W * d_in * 4 bytes (the value
  * ss2d_scan_fwd_workspace_bytes returns) must not exceed 16 MiB, else
  * SSM_ERR_WORKSPACE; images whose accumulator fits in shared memory need
- * none of it.  A call made outside a stream capture looks the array's
- * device address up (cudaGetSymbolAddress, the device current) and caches
- * it per device, so a device reset leaves no stale address behind; a call
- * made while the stream is being captured uses the cached address, so make
- * one call on each device before capturing (else SSM_ERR_CUDA).  All calls
+ * none of it.  The array's device address is looked up with
+ * cudaGetSymbolAddress (the device current) and cached per device; a lookup
+ * made after a device reset replaces the cached address.  All calls
  * on a device share the one array, which keeps the last call's contents
  * (nothing needs clearing: every call overwrites the part it reads); calls
  * whose kernels overlap on the GPU race on it.

@@ -981,11 +981,11 @@ namespace {
 
 // Device address of the scratch array on the current device.  In host code
 // the array's name is only a host-side stand-in, so the address is looked up
-// with cudaGetSymbolAddress (that device current).  Calls outside a stream
-// capture look it up every time (cheap next to the launch; a device reset,
-// which reloads the module, cannot leave a stale address behind) and cache
-// it per device; a call made while `st` is being captured uses the cached
-// address, so the first call on a device must come before any capture.
+// with cudaGetSymbolAddress (that device current) and cached per device.
+// While `st` is not being captured the lookup is made on every call (cheap
+// next to the launch; a device reset, which reloads the module, cannot leave
+// a stale address behind); while it is, no lookup is made and the cached
+// address is used.
 ssm_status noalloc_scratch(cudaStream_t st, float **out) {
   static std::mutex mu;
   static float *ptr[64] = {};
@@ -1008,8 +1008,8 @@ ssm_status noalloc_scratch(cudaStream_t st, float **out) {
     ptr[dev] = static_cast<float *>(addr);
   } else if (!ptr[dev]) {
     return fail(SSM_ERR_CUDA,
-                "ss2d_scan_fwd_noalloc: first call on this device made during a stream "
-                "capture; make one call before capturing");
+                "ss2d_scan_fwd_noalloc: no device address cached for this device while "
+                "the stream is being captured");
   }
   *out = ptr[dev];
   return ok();
