@@ -18,14 +18,14 @@
 //           every TT-step chunk in the caller's workspace (skipped when the
 //           forward already saved them there: states_saved);
 //   pass 2  walks the chunks backwards.  Per chunk: recompute the states
-//           from the saved start into shared memory (with each thread's
-//           partial C.h); dC_t = sum over channels of g_t h_t as a column
-//           pass over those states; the adjoint, which overwrites each
-//           state row with lam_t and leaves each thread's partial sums of
-//           lam B and A lam a h_{t-1}; dB_t = sum over channels of
-//           lam_t delta_t u_t as a second column pass; and a pass per
-//           (step, channel) that adds the G partials and writes du, ddelta
-//           and dz.
+//           from the saved start into registers, writing each thread's
+//           partial C.h and its terms g_t h_t of dC_t as shared rows;
+//           dC_t = the sum of those rows over the channels (a column pass);
+//           the adjoint, taking h_{t-1} from registers, which writes the
+//           terms lam_t delta_t u_t of dB_t into the rows and leaves each
+//           thread's partial sums of lam B and A lam a h_{t-1}; dB_t as a
+//           second column sum; and a pass per (step, channel) that adds the
+//           G partials and writes du, ddelta and dz.
 // A chunk's inputs are copied into shared memory one chunk ahead (cp.async)
 // when they are 16-byte aligned.  Nothing in the per-step loops crosses
 // lanes, so each step's critical
@@ -323,6 +323,22 @@ __global__ void __launch_bounds__(128, 3) scan_bwd_kernel(BwdParams p) {
     return yp;
   };
 
+  // the same, also handing back g_t of this thread's channel
+  auto fwd_step_g = [&](int t, float &gt) -> float {
+    const float4 q = sQ[t * PROW + ch];
+    const float dl = q.x, du = q.y;
+    gt = q.z;
+    float bv[NPT], cv[NPT];
+    load_bc<NPT>(sBC + 2 * (t * N + g * NPT), bv, cv);
+    float yp = 0.0f;
+#pragma unroll
+    for (int j = 0; j < NPT; ++j) {
+      h[j] = fmaf(ex2_approx(dl * A2[j]), h[j], du * bv[j]);
+      yp = fmaf(h[j], cv[j], yp);
+    }
+    return yp;
+  };
+
   // ---------------- pass 1: chunk-start states, forwards (unless saved)
   const int n_pass1 = p.states_saved ? 0 : nC;
 #pragma unroll
@@ -361,17 +377,18 @@ __global__ void __launch_bounds__(128, 3) scan_bwd_kernel(BwdParams p) {
   const float pD = (d0 + pch < d_in && p.D) ? p.D[d0 + pch] : 0.0f;
   float Dacc = 0.0f, bias_acc = 0.0f;
 
-  // one adjoint step; hp = h_{t-1} (this thread's states before step t)
+  // one adjoint step; hp = h_{t-1} (this thread's states before step t).
+  // The chunk's row t receives lam_t delta_t u_t, this channel's terms of dB_t.
   auto adj_step_h = [&](int t, const float (&hp)[NPT]) {
     const float4 qv = sQ[t * PROW + ch];
-    const float gt = qv.z, dl = qv.x;
+    const float gt = qv.z, dl = qv.x, du = qv.y;
     float bv[NPT], cv[NPT], lt[NPT];
     load_bc<NPT>(sBC + 2 * (t * N + g * NPT), bv, cv);
     float S1 = 0.0f, S2 = 0.0f;
 #pragma unroll
     for (int j = 0; j < NPT; ++j) {
       lam[j] = fmaf(gt, cv[j], lam[j]);
-      lt[j] = lam[j];
+      lt[j] = lam[j] * du;
       const float la = lam[j] * ex2_approx(dl * A2[j]);
       const float q = la * hp[j];
       S2 = fmaf(Av[j], q, S2);
@@ -383,21 +400,9 @@ __global__ void __launch_bounds__(128, 3) scan_bwd_kernel(BwdParams p) {
     sP1[t * NT + tid] = S1;
     sP2[t * NT + tid] = S2;
   };
-  // the same with h_{t-1} read back from the chunk's state rows
-  auto adj_step = [&](int t, const float (&hs)[NPT]) {
-    float hp[NPT];
-    if (t > 0) {
-      load_vec<NPT>(sH + (t - 1) * HROW + tid * NPT, hp);
-    } else {
-#pragma unroll
-      for (int j = 0; j < NPT; ++j) hp[j] = hs[j];
-    }
-    adj_step_h(t, hp);
-  };
-
-  // sum over the CTA's channels of w[t][ch] X[t][ch][n] for every (t, n) of
-  // the chunk, X the state rows; added to out (b, L, N) rows t0 .. t0+nT-1
-  auto column_pass = [&](bool use_g, float *out, int64_t t0, int nT) {
+  // sum over the CTA's channels of the chunk's rows X[t][ch][n] for every
+  // (t, n); added to out (b, L, N) rows t0 .. t0+nT-1
+  auto column_pass = [&](float *out, int64_t t0, int nT) {
     for (int o = tid; o < TT * G; o += NT) {
       const int t = o / G, gi = o - (o / G) * G;
       float acc[NPT];
@@ -406,12 +411,10 @@ __global__ void __launch_bounds__(128, 3) scan_bwd_kernel(BwdParams p) {
       const float *xs = sH + t * HROW + gi * NPT;
 #pragma unroll 8
       for (int cc = 0; cc < DT; ++cc) {
-        const float *qw = reinterpret_cast<const float *>(sQ + t * PROW + cc);
-        const float w = use_g ? qw[2] : qw[1];
         float x[NPT];
         load_vec<NPT>(xs + cc * G * NPT, x);
 #pragma unroll
-        for (int j = 0; j < NPT; ++j) acc[j] = fmaf(w, x[j], acc[j]);
+        for (int j = 0; j < NPT; ++j) acc[j] += x[j];
       }
       if (t < nT && in_bounds((ib * L + t0 + t) * N + gi * NPT + NPT - 1, p.b * L * N, kBndBC)) {
         float *dst = out + (ib * L + t0 + t) * N + gi * NPT;
@@ -448,39 +451,36 @@ __global__ void __launch_bounds__(128, 3) scan_bwd_kernel(BwdParams p) {
     const int64_t t0 = (int64_t)c * TT;
     __syncthreads();
 
-    // recompute the chunk's states and the partial pre-gate outputs; a full
-    // chunk also keeps them in registers for the adjoint
+    // recompute the chunk's states (kept in registers for the adjoint) and
+    // the partial pre-gate outputs; row t of the chunk receives g_t h_t, this
+    // channel's terms of dC_t.  A chunk past the end of the sequence runs
+    // identity steps there (delta, delta u and g are staged as 0), so every
+    // chunk takes the same unrolled path; outputs stop at nT.
     float hreg[TT][NPT];
 #pragma unroll
     for (int j = 0; j < NPT; ++j) h[j] = hs[j];
-    if (nT == TT) {
 #pragma unroll
-      for (int t = 0; t < TT; ++t) {
-        sPy[t * NT + tid] = fwd_step(t);
-        store_vec<NPT>(sH + t * HROW + tid * NPT, h);
+    for (int t = 0; t < TT; ++t) {
+      float gt;
+      sPy[t * NT + tid] = fwd_step_g(t, gt);
+      float pc[NPT];
 #pragma unroll
-        for (int j = 0; j < NPT; ++j) hreg[t][j] = h[j];
+      for (int j = 0; j < NPT; ++j) {
+        hreg[t][j] = h[j];
+        pc[j] = gt * h[j];
       }
-    } else {
-      for (int t = 0; t < nT; ++t) {
-        sPy[t * NT + tid] = fwd_step(t);
-        store_vec<NPT>(sH + t * HROW + tid * NPT, h);
-      }
+      store_vec<NPT>(sH + t * HROW + tid * NPT, pc);
     }
     __syncthreads();
-    column_pass(true, p.dC, t0, nT);  // dC_t = sum_ch g_t h_t
+    column_pass(p.dC, t0, nT);  // dC_t = sum_ch g_t h_t
     __syncthreads();
 
-    // the adjoint through the chunk (state rows become adjoint rows)
-    if (nT == TT) {
+    // the adjoint through the chunk (rows become lam_t delta_t u_t)
 #pragma unroll
-      for (int t = TT - 1; t >= 1; --t) adj_step_h(t, hreg[t - 1]);
-      adj_step_h(0, hs);
-    } else {
-      for (int t = nT - 1; t >= 0; --t) adj_step(t, hs);
-    }
+    for (int t = TT - 1; t >= 1; --t) adj_step_h(t, hreg[t - 1]);
+    adj_step_h(0, hs);
     __syncthreads();
-    column_pass(false, p.dB, t0, nT);  // dB_t = sum_ch lam_t delta_t u_t
+    column_pass(p.dB, t0, nT);  // dB_t = sum_ch lam_t delta_t u_t
 
     // per (step, channel): add the partials, write du, ddelta, dz
     for (int i = tid; i < TT * DT; i += NT) {
