@@ -74,11 +74,10 @@ struct BwdCfg {
   static constexpr int RAW_ACT = TT * DT, RAW_BC = TT * N;
   static constexpr int RAW_BYTES = ((4 * RAW_ACT + 2 * RAW_BC) * (int)sizeof(T) + 15) / 16 * 16;
   static constexpr int OFF_F = 2 * RAW_BYTES / 4;  // first float after the raw tiles
-  // planes: {delta, delta u, g, -} as one 16-byte entry, then u, the dz
-  // factor and softplus' (one float each)
+  // planes: {delta, delta u, g, u} as one 16-byte entry, then the dz factor
+  // and softplus' (one float each)
   static constexpr int OFF_Q = OFF_F;
-  static constexpr int OFF_U = OFF_Q + 4 * PL;
-  static constexpr int OFF_DZF = OFF_U + PL;
+  static constexpr int OFF_DZF = OFF_Q + 4 * PL;
   static constexpr int OFF_SPG = OFF_DZF + PL;
   static constexpr int OFF_BC = (OFF_SPG + PL + 3) / 4 * 4;  // {B, C} pairs [t][n]
   static constexpr int OFF_P1 = OFF_BC + 2 * TT * N;     // partial sum_n lam B      [t][thread]
@@ -172,7 +171,7 @@ __global__ void __launch_bounds__(128, 3) scan_bwd_kernel(BwdParams p) {
   extern __shared__ float4 bwd_smem4[];
   float *sm = reinterpret_cast<float *>(bwd_smem4);
   float4 *sQ = reinterpret_cast<float4 *>(sm + Cfg::OFF_Q);
-  float *sU = sm + Cfg::OFF_U, *sDzf = sm + Cfg::OFF_DZF, *sSpg = sm + Cfg::OFF_SPG;
+  float *sDzf = sm + Cfg::OFF_DZF, *sSpg = sm + Cfg::OFF_SPG;
   float *sBC = sm + Cfg::OFF_BC;
   float *sP1 = sm + Cfg::OFF_P1, *sP2 = sm + Cfg::OFF_P2, *sPy = sm + Cfg::OFF_PY;
   float *sH = sm + Cfg::OFF_H;
@@ -277,8 +276,7 @@ __global__ void __launch_bounds__(128, 3) scan_bwd_kernel(BwdParams p) {
         }
       }
       const int s = t * PROW + cc;
-      sQ[s] = make_float4(dl, dl * uu, gg, 0.0f);
-      sU[s] = uu;
+      sQ[s] = make_float4(dl, dl * uu, gg, uu);
       if (full) {
         sDzf[s] = dzf;
         sSpg[s] = spg;
@@ -491,7 +489,7 @@ __global__ void __launch_bounds__(128, 3) scan_bwd_kernel(BwdParams p) {
       const float S2 = sum_partials<G>(sP2 + t * NT + pch * G, pch);
       const float yp = sum_partials<G>(sPy + t * NT + pch * G, pch);
       const float4 qv = sQ[s];
-      const float gt = qv.z, dl = qv.x, uu = sU[s];
+      const float gt = qv.z, dl = qv.x, uu = qv.w;
       const float ddt = fmaf(uu, S1, S2) * sSpg[s];
       if (t < nT && dd < d_in && in_bounds((ib * L + t0 + t) * d_in + dd, p.b * L * d_in, kBndAct)) {
         const int64_t at = (ib * L + t0 + t) * d_in + dd;
