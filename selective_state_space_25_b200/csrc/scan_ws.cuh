@@ -83,7 +83,9 @@ template <typename T, int N, int NS, int TC, int H, int P, bool HAS_Z, bool SAVE
           int DT_ = 32>
 __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P, DT_>::THREADS)
     scan_ws_kernel(ScanParams p) {
-  static_assert(!(SUMMARY && SAVE), "the summary pass saves no states");
+  // SUMMARY && SAVE is the states pass of the backward: one block from h0,
+  // no outputs, the chunk-start states saved; a plain SUMMARY is the split
+  // scan's summary of each block from h = 0.
   using K = WsScan<T, N, NS, TC, H, P, DT_>;
   constexpr int DT = K::DT, G = K::G, NP2 = K::NP2, R = K::R, TCP = K::TCP;
   extern __shared__ __align__(16) unsigned char smem[];
@@ -125,11 +127,12 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P, DT_>::THREADS)
       A2[k] = d_ok && in_bounds(d * N + n + 1, n_par, kBndParam)
                   ? make_float2(p.A[d * N + n] * kLog2e, p.A[d * N + n + 1] * kLog2e)
                   : make_float2(0.0f, 0.0f);
-      // the summary starts every block from zero; the scan starts block 0
-      // from h0 and block k > 0 from the carry the carry pass left
+      // the summary starts every block from zero; the scan (and the states
+      // pass) starts block 0 from h0 and block k > 0 from the carry the
+      // carry pass left
       const float *h0 = blk == 0 ? p.h0 + (ib * d_in + d) * N + n
                                  : p.blk_state + (blk_row + d) * N + n;
-      const bool from = d_ok && !SUMMARY && (blk > 0 || p.h0) &&
+      const bool from = d_ok && (!SUMMARY || SAVE) && (blk > 0 || p.h0) &&
                         (blk == 0 ? in_bounds((ib * d_in + d) * N + n + 1, n_state, kBndState)
                                   : in_bounds((blk_row + d) * N + n + 1, n_blk, kBndChunk));
       h[k] = from ? make_float2(h0[0], h0[1]) : make_float2(0.0f, 0.0f);
@@ -212,7 +215,9 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P, DT_>::THREADS)
       slot = slot == R - 1 ? 0 : slot + 1;
       __syncthreads();  // partials of this chunk written; next chunk's pre-pass done
     }
-    if constexpr (SUMMARY) {  // the block's map h -> P h + Q
+    if constexpr (SUMMARY && SAVE) {
+      // the states pass keeps nothing but the saved states
+    } else if constexpr (SUMMARY) {  // the block's map h -> P h + Q
       if (d_ok && in_bounds((blk_row + d) * N + g * NS + NS - 1, n_blk, kBndChunk)) {
         float *q = p.blk_state + (blk_row + d) * N + g * NS;
         float *pd = p.blk_decay + (blk_row + d) * N + g * NS;

@@ -469,8 +469,24 @@ ssm_status launch_bwd_cfg(const ssm::BwdParams &p, cudaStream_t st) {
 }
 
 template <typename T, int N>
-ssm_status launch_bwd(const ssm::BwdParams &p, bool async, cudaStream_t st) {
+ssm_status launch_bwd(const ssm::BwdParams &p, bool async, bool fwd_states, cudaStream_t st) {
   constexpr int NPT = N < 4 ? N : SSM_BWD_NPT;
+  if constexpr (ws_states(N) > 0) {
+    if (fwd_states && !p.states_saved) {
+      // the chunk-start states come from the forward kernel's states pass
+      // (no C, gate or output), written where the backward's own first
+      // pass would write them; the backward then starts from them
+      ssm::ScanParams f{p.u, p.delta, p.A, p.B, p.C, nullptr, nullptr, p.dt_bias, p.h0,
+                        nullptr, nullptr, p.b, p.L, p.d_in, p.softplus, p.chunk_h};
+      if (ssm_status s = launch_scan_ws_pass<T, N, false, true, true>(f, 1, st)) return s;
+      ssm::BwdParams q = p;
+      q.states_saved = 1;
+      if constexpr (ssm::bwd_async_ok<T, N, NPT>()) {
+        if (async) return launch_bwd_cfg<T, N, NPT, true>(q, st);
+      }
+      return launch_bwd_cfg<T, N, NPT, false>(q, st);
+    }
+  }
   if constexpr (ssm::bwd_async_ok<T, N, NPT>()) {
     if (async) return launch_bwd_cfg<T, N, NPT, true>(p, st);
   }
@@ -478,15 +494,16 @@ ssm_status launch_bwd(const ssm::BwdParams &p, bool async, cudaStream_t st) {
 }
 
 template <typename T>
-ssm_status dispatch_bwd_n(const ssm::BwdParams &p, int64_t N, bool async, cudaStream_t st) {
+ssm_status dispatch_bwd_n(const ssm::BwdParams &p, int64_t N, bool async, bool fwd_states,
+                          cudaStream_t st) {
   switch (N) {
-    case 1: return launch_bwd<T, 1>(p, async, st);
-    case 2: return launch_bwd<T, 2>(p, async, st);
-    case 4: return launch_bwd<T, 4>(p, async, st);
-    case 8: return launch_bwd<T, 8>(p, async, st);
-    case 16: return launch_bwd<T, 16>(p, async, st);
-    case 32: return launch_bwd<T, 32>(p, async, st);
-    case 64: return launch_bwd<T, 64>(p, async, st);
+    case 1: return launch_bwd<T, 1>(p, async, fwd_states, st);
+    case 2: return launch_bwd<T, 2>(p, async, fwd_states, st);
+    case 4: return launch_bwd<T, 4>(p, async, fwd_states, st);
+    case 8: return launch_bwd<T, 8>(p, async, fwd_states, st);
+    case 16: return launch_bwd<T, 16>(p, async, fwd_states, st);
+    case 32: return launch_bwd<T, 32>(p, async, fwd_states, st);
+    case 64: return launch_bwd<T, 64>(p, async, fwd_states, st);
   }
   return fail(SSM_ERR_UNSUPPORTED, "ssm_scan_bwd: d_state %lld not compiled", (long long)N);
 }
@@ -720,8 +737,12 @@ ssm_status scan_bwd_impl(const char *what, const void *u, const void *delta, con
   // the raw-tile prefetch copies 16-byte groups straight from the inputs
   const bool async = (d_in * (int64_t)es) % 16 == 0 && aligned(u, 16) && aligned(delta, 16) &&
                      aligned(dout, 16) && aligned(B, 16) && aligned(C, 16) && (!z || aligned(z, 16));
-  if (dtype == SSM_BF16) return dispatch_bwd_n<__nv_bfloat16>(p, d_state, async, st);
-  return dispatch_bwd_n<float>(p, d_state, async, st);
+  // the forward kernel's states pass needs its own 16-byte staging of u, delta, B
+  const bool fwd_states = (d_in * (int64_t)es) % 16 == 0 && aligned(u, 16) &&
+                          aligned(delta, 16) && aligned(B, 16) && b <= 65535;
+  if (dtype == SSM_BF16)
+    return dispatch_bwd_n<__nv_bfloat16>(p, d_state, async, fwd_states, st);
+  return dispatch_bwd_n<float>(p, d_state, async, fwd_states, st);
 }
 
 }  // namespace
