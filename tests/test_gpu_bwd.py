@@ -57,8 +57,12 @@ def _compare(got, ref, dtype, names=None):
 @pytest.mark.parametrize("b,L,d_in,N", [
     (2, 64, 32, 16), (1, 97, 40, 16), (2, 33, 8, 4), (1, 50, 130, 1), (2, 17, 64, 2),
     (1, 70, 20, 8), (1, 45, 24, 32), (1, 31, 12, 64), (3, 1, 16, 16), (1, 300, 48, 16),
+    (1, 50, 36, 16),
 ])
 def test_bwd_shapes(ssm, dtype, b, L, d_in, N):
+    """d_state 8, 16, 32 with 16-byte rows (d_in a multiple of 8 in bf16, of
+    4 in fp32) take the forward kernel's states pass; the rest (d_in 20 or 36
+    in bf16, other d_state) the backward kernel's own first pass."""
     dt = "bf16" if dtype == torch.bfloat16 else "fp32"
     inp = scan_inputs(b, L, d_in, N, dt, seed=b * 7 + L + d_in + N)
     dout = _dout(b, L, d_in, dtype, seed=L)
