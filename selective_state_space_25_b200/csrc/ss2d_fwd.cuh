@@ -359,7 +359,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     // ---- 4. replay, accumulate y at the visited pixels
 #pragma unroll
     for (int j = 0; j < TS; ++j) {
-      if (lb + j < Li &&
+      if (ok0 && lb + j < Li &&
           (ACC_SMEM ? in_bounds(rows[j] * DT + 2 * cp + 1, (int64_t)Hi * RS * DT, kBndWork)
                     : in_bounds((ib * L + rows[j]) * d_in + d0 + 2 * cp + (ok1 ? 1 : 0),
                                 p.b * L * d_in, kBndWork))) {
@@ -371,7 +371,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
             *d2 = yv;
           else
             *d2 = __fadd2_rn(*d2, yv);
-        } else if (ok0) {
+        } else {
           dst[0] = K == 0 ? yv.x : dst[0] + yv.x;
           if (ok1) dst[1] = K == 0 ? yv.y : dst[1] + yv.y;
         }

@@ -58,13 +58,15 @@ def main():
         for k in ("du", "ddelta", "dB", "dC", "dA"):
             check(f"backward {k} saved={saved}", gr[k], ref[k], 2e-2 if k in ("du", "ddelta") else 2e-4)
     # SS2D: shared-memory and workspace accumulators, both orders
-    for (H, W, order) in [(7, 9, "cross"), (5, 6, "snake"), (80, 81, "cross")]:
-        inp = ss2d_inputs(1, H, W, 16, 1, "bf16", seed=H + W)
+    # (d_in 13: a partial last channel group, its last pair inactive)
+    for (H, W, order, d_in) in [(7, 9, "cross", 16), (5, 6, "snake", 16), (80, 81, "cross", 16),
+                                (7, 9, "snake", 13), (80, 81, "cross", 13), (80, 81, "snake", 13)]:
+        inp = ss2d_inputs(1, H, W, d_in, 1, "bf16", seed=H + W + d_in)
         g = to_cuda(inp)
         y = S.ss2d_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], H, W, D=g["D"], order=order)
         y_ref = oracle.ss2d_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], H, W,
                                  D=inp["D"], order=order)
-        check(f"ss2d {H}x{W} {order}", y, y_ref, 2e-2)
+        check(f"ss2d {H}x{W} {order} d_in {d_in}", y, y_ref, 2e-2)
     xs = S.ss2d_cross_scan(torch.randn(1, 35, 8).cuda(), 5, 7)
     S.ss2d_cross_merge(xs, 5, 7)
     S.check_device_errors()
