@@ -102,6 +102,23 @@ def test_ss2d_workspace_odd_channels_or_4_byte_aligned(ssm, dtype, order, d_in, 
     assert rel_err(y, ref) <= TOL[dtype]
 
 
+@pytest.mark.parametrize("order", ["cross", "snake"])
+@pytest.mark.parametrize("H,W,smem", [(128, 49, True), (64, 98, False)])
+def test_ss2d_shared_accumulator_limit(ssm, order, H, W, smem):
+    """The shared accumulator holds H (W rounded up to odd) pixels of 8 fp32
+    channels, at most 6272: 128 x 49 fills it exactly; 64 x 98 has as many
+    pixels but pads to 64 x 99, so it takes the workspace."""
+    need = ssm.ss2d_scan_fwd_workspace_bytes(1, H, W, 16, 1)
+    assert (need == 0) == smem
+    inp = ss2d_inputs(1, H, W, 16, 1, "bf16", seed=H + W, with_dt_bias=True)
+    g = to_cuda(inp)
+    y = ssm.ss2d_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], H, W, D=g["D"],
+                          dt_bias=g["dt_bias"], order=order)
+    ref = oracle.ss2d_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], H, W,
+                           D=inp["D"], dt_bias=inp["dt_bias"], order=order)
+    assert rel_err(y, ref) <= 2e-2
+
+
 def test_ss2d_equals_composition_of_gpu_scans(ssm):
     """Fused SS2D == CrossScan, four 1-D scans, CrossMerge, all on the GPU."""
     b, H, W, d_in = 2, 12, 10, 16
