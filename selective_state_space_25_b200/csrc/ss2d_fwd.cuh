@@ -195,6 +195,8 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
   // caller's workspace only for even d_in and an 8-byte aligned workspace
   const bool acc_pairs =
       ACC_SMEM || ((d_in & 1) == 0 && (reinterpret_cast<uintptr_t>(p.acc_global) & 7) == 0);
+  // every channel of the tile exists and is accumulated as pairs (CTA-uniform)
+  const bool whole_tile = d0 + DT <= d_in && acc_pairs;
 
   const int nchunks = (Li + LC - 1) / LC;
 
@@ -291,7 +293,6 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
 #pragma unroll
     for (int j = 0; j < TS; ++j) {
       const int row = seg * TS + j;
-      const bool valid = lb + j < Li;
       rows[j] = tR[row];
       float2 dv, uv, bc;
       if constexpr (sizeof(T) == 2) {
@@ -306,12 +307,14 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
       if constexpr (BC_ASYNC) {
         bc = make_float2(Elem<T>::load(tB, row), Elem<T>::load(tC, row));
       } else {
-        bc = valid ? make_float2(Elem<T>::load(Bk, lb + j), Elem<T>::load(Ck, lb + j))
-                   : make_float2(0.0f, 0.0f);
+        bc = lb + j < Li ? make_float2(Elem<T>::load(Bk, lb + j), Elem<T>::load(Ck, lb + j))
+                         : make_float2(0.0f, 0.0f);
       }
+      // Steps past the end (last chunk only) run on zero-filled rows; they
+      // come after every real step, so they reach no stored output: the scan
+      // is causal and the carry out of a direction's last chunk is dropped.
       float2 e = __fadd2_rn(dv, bias);
       if (p.delta_softplus) e = softplus2_f32(e);
-      if (!valid) e = make_float2(0.0f, 0.0f);  // identity step past the end
       const float2 x = __fmul2_rn(e, A2);
       const float2 a = A_POLY ? exp2_poly2(x) : exp2_sfu2(x);
       Q = __ffma2_rn(a, Q, __fmul2_rn(__fmul2_rn(e, uv), make_float2(bc.x, bc.x)));
@@ -356,24 +359,43 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     }
     h = __ffma2_rn(exc.a, h, exc.b);
 
-    // ---- 4. replay, accumulate y at the visited pixels
+    // ---- 4. replay, accumulate y at the visited pixels.  A whole chunk of a
+    // whole channel tile (all but a direction's last chunk, all but a ragged
+    // last tile) needs no per-step checks.
+    if (whole_tile && l0 + LC <= Li) {
 #pragma unroll
-    for (int j = 0; j < TS; ++j) {
-      if (ok0 && lb + j < Li &&
-          (ACC_SMEM ? in_bounds(rows[j] * DT + 2 * cp + 1, (int64_t)Hi * RS * DT, kBndWork)
-                    : in_bounds((ib * L + rows[j]) * d_in + d0 + 2 * cp + (ok1 ? 1 : 0),
-                                p.b * L * d_in, kBndWork))) {
+      for (int j = 0; j < TS; ++j) {
+        if (!(ACC_SMEM ? in_bounds(rows[j] * DT + 2 * cp + 1, (int64_t)Hi * RS * DT, kBndWork)
+                       : in_bounds((ib * L + rows[j]) * d_in + d0 + 2 * cp + 1, p.b * L * d_in,
+                                   kBndWork)))
+          continue;
         const float2 yv = __ffma2_rn(gg[j], h, yl[j]);
-        float *dst = ACC_SMEM ? acc_s + rows[j] * DT + 2 * cp : acc_g + rows[j] * di + 2 * cp;
-        if (ok1 && acc_pairs) {
-          float2 *d2 = reinterpret_cast<float2 *>(dst);
-          if constexpr (K == 0)
-            *d2 = yv;
-          else
-            *d2 = __fadd2_rn(*d2, yv);
-        } else {
-          dst[0] = K == 0 ? yv.x : dst[0] + yv.x;
-          if (ok1) dst[1] = K == 0 ? yv.y : dst[1] + yv.y;
+        float2 *d2 = reinterpret_cast<float2 *>(ACC_SMEM ? acc_s + rows[j] * DT + 2 * cp
+                                                         : acc_g + rows[j] * di + 2 * cp);
+        if constexpr (K == 0)
+          *d2 = yv;
+        else
+          *d2 = __fadd2_rn(*d2, yv);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < TS; ++j) {
+        if (ok0 && lb + j < Li &&
+            (ACC_SMEM ? in_bounds(rows[j] * DT + 2 * cp + 1, (int64_t)Hi * RS * DT, kBndWork)
+                      : in_bounds((ib * L + rows[j]) * d_in + d0 + 2 * cp + (ok1 ? 1 : 0),
+                                  p.b * L * d_in, kBndWork))) {
+          const float2 yv = __ffma2_rn(gg[j], h, yl[j]);
+          float *dst = ACC_SMEM ? acc_s + rows[j] * DT + 2 * cp : acc_g + rows[j] * di + 2 * cp;
+          if (ok1 && acc_pairs) {
+            float2 *d2 = reinterpret_cast<float2 *>(dst);
+            if constexpr (K == 0)
+              *d2 = yv;
+            else
+              *d2 = __fadd2_rn(*d2, yv);
+          } else {
+            dst[0] = K == 0 ? yv.x : dst[0] + yv.x;
+            if (ok1) dst[1] = K == 0 ? yv.y : dst[1] + yv.y;
+          }
         }
       }
     }
