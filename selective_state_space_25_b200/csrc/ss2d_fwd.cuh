@@ -69,9 +69,10 @@ struct Ss2dParams {
 // of LC = 8 WARPS TS steps:
 //   1. the chunk's delta rows and the u rows of the pixels it visits (16
 //      bytes = 8 bf16 channels each) are copied global -> shared with
-//      cp.async, one chunk ahead, and the accumulator row each step lands on
-//      is worked out once per step for all channels; B / C values likewise
-//      when they are 16-byte aligned, else read directly;
+//      cp.async, one chunk ahead, each warp the rows of its own segments,
+//      and the accumulator row each step lands on is worked out once per
+//      step for all channels; B / C values likewise when they are 16-byte
+//      aligned, else read directly;
 //   2. thread (segment s, channel pair cp) takes TS consecutive steps of its
 //      two channels: delta = softplus(dt + bias), dA = exp2(delta A log2 e)
 //      (FMA-pipe polynomial or SFU), delta u B, C and D u go to registers,
@@ -79,6 +80,9 @@ struct Ss2dParams {
 //   3. a shuffle scan over the warp's 8 segments and a pass over the warps'
 //      totals give each segment its incoming state, the carry of the previous
 //      chunk included (the operator is (a, b) o (a', b') = (a a', a' b + b'));
+//      the exchange of the warps' totals is the chunk's one CTA barrier: the
+//      staged rows are warp-private, and the barrier also orders every
+//      accumulator update of a chunk before those of the next;
 //   4. the segment replays its steps, h = dA h + delta u B, and adds
 //      y = C h + D u into the accumulator at the pixel each step visits.
 // TS is odd so the 8 segments of a warp hit distinct bank groups in the
@@ -86,12 +90,16 @@ struct Ss2dParams {
 // row stride RS = W rounded up to odd, so both row- and column-major runs
 // spread over the banks.
 // ---------------------------------------------------------------------------
-template <typename T, int TS, int WARPS>
+template <typename T, int TS, int WARPS, bool ACC_SMEM = true>
 struct Ss2dCfg {
   static constexpr int DT = 8, PAIRS = 4, SPW = 8;
   static constexpr int THREADS = 32 * WARPS;
   static constexpr int S = SPW * WARPS;       // segments per chunk
+  static constexpr int RW = SPW * TS;         // steps (staged rows) per warp
   static constexpr int LC = S * TS;           // steps per chunk
+  // accumulator row of a step: 16-bit in shared memory (H RS <= 6272), else
+  // the pixel index
+  using RowT = typename std::conditional<ACC_SMEM, unsigned short, int>::type;
   static constexpr int ESZ = sizeof(T);
   static constexpr int ROWB = DT * ESZ;       // bytes of one staged row (8 channels)
   static constexpr int GRAN_PER_ROW = ROWB / 16;
@@ -101,13 +109,14 @@ struct Ss2dCfg {
   static constexpr int OFF_U = OFF_D + LC * ROWB;
   static constexpr int OFF_B = OFF_U + LC * ROWB;
   static constexpr int OFF_C = OFF_B + (LC + BC_PAD) * ESZ;
-  static constexpr int OFF_AGG = (OFF_C + (LC + BC_PAD) * ESZ + 15) / 16 * 16;  // float4 [WARPS][PAIRS]
-  static constexpr int OFF_CARRY = OFF_AGG + WARPS * PAIRS * 16;              // float [2][8]
-  static constexpr int OFF_ROW = OFF_CARRY + 64;   // int [LC]: accumulator row of each step
-  static constexpr int OFF_ACC = (OFF_ROW + LC * 4 + 15) / 16 * 16;           // float [L][8]
+  static constexpr int OFF_AGG = (OFF_C + (LC + BC_PAD) * ESZ + 15) / 16 * 16;  // float4 [2][WARPS][PAIRS]
+  static constexpr int OFF_CARRY = OFF_AGG + 2 * WARPS * PAIRS * 16;          // float [2][8]
+  static constexpr int OFF_ROW = OFF_CARRY + 64;   // RowT [LC]: accumulator row of each step
+  static constexpr int OFF_ACC = (OFF_ROW + LC * (int)sizeof(RowT) + 15) / 16 * 16;  // float [L][8]
   static constexpr int AUX_BYTES = OFF_ACC;
   static_assert(TS % 2 == 1, "TS odd keeps the warp's segments on distinct bank groups");
-  static_assert(ROWB % 16 == 0 && (LC * ESZ) % 16 == 0, "16-byte staging");
+  static_assert(ROWB % 16 == 0 && (RW * ESZ) % 16 == 0, "16-byte staging of a warp's rows");
+  static_assert(RW % BC_VEC == 0, "a warp's B / C rows are whole 16-byte granules");
 };
 
 struct Aff2 {
@@ -156,8 +165,9 @@ template <typename T, int TS, int WARPS, bool ACC_SMEM, bool A_POLY, bool ROW_AS
           bool BC_ASYNC, int ORDER>
 __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     ss2d_n1_kernel(Ss2dParams p) {
-  using Cfg = Ss2dCfg<T, TS, WARPS>;
-  constexpr int THREADS = Cfg::THREADS, LC = Cfg::LC, DT = Cfg::DT;
+  using Cfg = Ss2dCfg<T, TS, WARPS, ACC_SMEM>;
+  constexpr int THREADS = Cfg::THREADS, LC = Cfg::LC, DT = Cfg::DT, RW = Cfg::RW;
+  using RowT = typename Cfg::RowT;
   extern __shared__ __align__(16) unsigned char smem[];
   T *tD = reinterpret_cast<T *>(smem + Cfg::OFF_D);
   T *tU = reinterpret_cast<T *>(smem + Cfg::OFF_U);
@@ -165,7 +175,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
   T *tC = reinterpret_cast<T *>(smem + Cfg::OFF_C);
   float4 *agg = reinterpret_cast<float4 *>(smem + Cfg::OFF_AGG);
   float *carry = reinterpret_cast<float *>(smem + Cfg::OFF_CARRY);
-  int *tR = reinterpret_cast<int *>(smem + Cfg::OFF_ROW);
+  RowT *tR = reinterpret_cast<RowT *>(smem + Cfg::OFF_ROW);
   float *acc_s = reinterpret_cast<float *>(smem + Cfg::OFF_ACC);
 
   const int tid = threadIdx.x;
@@ -200,32 +210,63 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
 
   const int nchunks = (Li + LC - 1) / LC;
 
-  // stage the delta / u rows (and B / C) of chunk c of direction k
+  // stage the delta / u rows (and B / C) of this warp's steps of chunk c of
+  // direction k: rows w0 .. w0 + RW - 1
+  const int w0 = warp * RW;
+  constexpr int NRI = (RW + 31) / 32;  // rows per lane
+  int pq[NRI], pr[NRI], dq = 0, dr = 0;
   auto prefetch = [&](int k, int c) {
     const int l0 = c * LC;
     const T *dk = gdt + (int64_t)k * L * d_in;  // delta rows of direction k
     if constexpr (ROW_ASYNC) {
-      for (int r = tid; r < LC * Cfg::GRAN_PER_ROW; r += THREADS) {
-        const int row = r / Cfg::GRAN_PER_ROW, part = r - row * Cfg::GRAN_PER_ROW;
+      // lane rows w0 + lane + 32 i; their image positions are kept as
+      // (q, r) = divmod(ll, D) and moved by LC steps per chunk, so only a
+      // direction's first chunk divides
+      const bool odd = (k & 1) != 0, rev = k >= 2;
+      const int D = odd ? Hi : Wi;
+      if (c == 0) {
+        dq = div_small(LC, D, odd ? invH : invW);
+        dr = LC - dq * D;
+      }
+#pragma unroll
+      for (int i = 0; i < NRI; ++i) {
+        const int rl = lane + 32 * i;
+        if (rl >= RW) break;
+        const int row = w0 + rl;
         const int l = l0 + row;
-        int hh = 0, ww = 0;
-        if (l < Li) ss2d_pos<ORDER>(k, l, Hi, Wi, invH, invW, hh, ww);
+        if (c == 0) {  // rows past the end keep meaningless (q, r): they stay past it
+          const int ll = rev ? Li - 1 - l : l;
+          pq[i] = div_small(ll, D, odd ? invH : invW);
+          pr[i] = ll - pq[i] * D;
+        } else if (!rev) {
+          pr[i] += dr;
+          pq[i] += dq;
+          if (pr[i] >= D) { pr[i] -= D; ++pq[i]; }
+        } else {
+          pr[i] -= dr;
+          pq[i] -= dq;
+          if (pr[i] < 0) { pr[i] += D; --pq[i]; }
+        }
+        const int q = pq[i], rr = pr[i];
+        const bool flip = ORDER == kOrderSnake && (q & 1);
+        const int hh = odd ? (flip ? Hi - 1 - rr : rr) : q;
+        const int ww = odd ? q : (flip ? Wi - 1 - rr : rr);
         const int pix0 = hh * Wi + ww;
-        const int po0 = part * (16 / Cfg::ESZ);
         const bool ok =
             l < Li &&
-            in_bounds((ib * L + pix0) * d_in + d0 + po0 + 16 / Cfg::ESZ - 1, p.b * L * d_in, kBndAct) &&
-            in_bounds(((ib * 4 + k) * L + l) * d_in + d0 + po0 + 16 / Cfg::ESZ - 1,
-                      p.b * 4 * L * d_in, kBndAct);
+            in_bounds((ib * L + pix0) * d_in + d0 + DT - 1, p.b * L * d_in, kBndAct) &&
+            in_bounds(((ib * 4 + k) * L + l) * d_in + d0 + DT - 1, p.b * 4 * L * d_in, kBndAct);
         const int pix = ok ? pix0 : 0;
-        if (part == 0) tR[row] = ACC_SMEM ? (ok ? hh * RS + ww : 0) : pix;
-        const int so = row * DT + part * (16 / Cfg::ESZ);
-        const int po = part * (16 / Cfg::ESZ);
-        cp_async16(tD + so, dk + (ok ? l * di : 0) + po, ok ? 16 : 0);
-        cp_async16(tU + so, gu + pix * di + po, ok ? 16 : 0);
+        tR[row] = (RowT)(ACC_SMEM ? (ok ? hh * RS + ww : 0) : pix);
+#pragma unroll
+        for (int part = 0; part < Cfg::GRAN_PER_ROW; ++part) {
+          const int po = part * (16 / Cfg::ESZ);
+          cp_async16(tD + row * DT + po, dk + (ok ? l * di : 0) + po, ok ? 16 : 0);
+          cp_async16(tU + row * DT + po, gu + pix * di + po, ok ? 16 : 0);
+        }
       }
     } else {
-      for (int r = tid; r < LC * DT; r += THREADS) {
+      for (int r = w0 * DT + lane; r < (w0 + RW) * DT; r += 32) {
         const int row = r / DT, ch = r - row * DT;
         const int l = l0 + row;
         int hh = 0, ww = 0;
@@ -235,13 +276,13 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
                         in_bounds((ib * L + pix0) * d_in + d0 + ch, p.b * L * d_in, kBndAct) &&
                         in_bounds(((ib * 4 + k) * L + l) * d_in + d0 + ch, p.b * 4 * L * d_in, kBndAct);
         const int pix = ok ? pix0 : 0;
-        if (ch == 0) tR[row] = ACC_SMEM ? (ok ? hh * RS + ww : 0) : pix;
+        if (ch == 0) tR[row] = (RowT)(ACC_SMEM ? (ok ? hh * RS + ww : 0) : pix);
         tD[r] = ok ? dk[l * di + ch] : T(0.0f);
         tU[r] = ok ? gu[pix * di + ch] : T(0.0f);
       }
     }
     if constexpr (BC_ASYNC) {
-      for (int r = tid; r < LC / Cfg::BC_VEC; r += THREADS) {
+      for (int r = w0 / Cfg::BC_VEC + lane; r < (w0 + RW) / Cfg::BC_VEC; r += 32) {
         const int l = l0 + r * Cfg::BC_VEC;
         const int rem = Li - l;
         int bytes = rem <= 0 ? 0 : (rem >= Cfg::BC_VEC ? 16 : rem * Cfg::ESZ);
@@ -281,7 +322,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     [[maybe_unused]] const T *Bk = gB + (int64_t)K * L;
     [[maybe_unused]] const T *Ck = gC + (int64_t)K * L;
     cp_async_wait<0>();
-    __syncthreads();  // staged rows of this chunk visible
+    __syncwarp();  // this warp's staged rows visible to all its lanes
 
     // ---- 1. this segment's steps into registers
     const int lb = l0 + seg * TS;
@@ -342,17 +383,20 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     exc.b.x = __shfl_up_sync(0xffffffffu, inc.b.x, 4);
     exc.b.y = __shfl_up_sync(0xffffffffu, inc.b.y, 4);
     if (sl == 0) exc = Aff2{make_float2(1.0f, 1.0f), make_float2(0.0f, 0.0f)};
-    if (sl == Cfg::SPW - 1) agg[warp * Cfg::PAIRS + cp] = make_float4(inc.a.x, inc.a.y, inc.b.x, inc.b.y);
-    __syncthreads();  // warp totals visible; every thread is done with the staged rows
+    if (sl == Cfg::SPW - 1)
+      agg[(cq * WARPS + warp) * Cfg::PAIRS + cp] = make_float4(inc.a.x, inc.a.y, inc.b.x, inc.b.y);
+    // the warp is done with its staged rows (the scan above took every lane's
+    // steps): stage its rows of the next chunk
     if (c + 1 < nchunks) prefetch(K, c + 1);
     else if (K < 3) prefetch(K + 1, 0);
+    __syncthreads();  // warp totals visible
 
     // ---- 3. incoming state: previous chunk's carry, earlier warps, earlier segments
     float2 h = make_float2(carry[cq * DT + 2 * cp], carry[cq * DT + 2 * cp + 1]);
     {  // all warp totals are loaded at once; earlier warps' maps applied in order
       float4 g4[WARPS - 1];
 #pragma unroll
-      for (int w = 0; w < WARPS - 1; ++w) g4[w] = agg[w * Cfg::PAIRS + cp];
+      for (int w = 0; w < WARPS - 1; ++w) g4[w] = agg[(cq * WARPS + w) * Cfg::PAIRS + cp];
 #pragma unroll
       for (int w = 0; w < WARPS - 1; ++w)
         if (w < warp) h = __ffma2_rn(make_float2(g4[w].x, g4[w].y), h, make_float2(g4[w].z, g4[w].w));
@@ -400,7 +444,6 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
       }
     }
     const bool last = c == nchunks - 1;
-    if (last) __syncthreads();  // the next direction's updates touch the same pixels
     if (warp == WARPS - 1 && sl == Cfg::SPW - 1) {  // the next direction starts from h = 0
       const float2 hend = __ffma2_rn(P, h, Q);  // the state after the chunk
       carry[(cq ^ 1) * DT + 2 * cp] = last ? 0.0f : hend.x;

@@ -404,7 +404,7 @@ int64_t ss2d_acc_pixels(int64_t H, int64_t W) { return H * (W | 1); }
 
 template <typename T, bool ACC_SMEM, bool ROW_ASYNC, bool BC_ASYNC, int ORDER>
 ssm_status launch_ss2d_cfg(const ssm::Ss2dParams &p, cudaStream_t st) {
-  using Cfg = ssm::Ss2dCfg<T, SSM_SS2D_TS, SSM_SS2D_WARPS>;
+  using Cfg = ssm::Ss2dCfg<T, SSM_SS2D_TS, SSM_SS2D_WARPS, ACC_SMEM>;
   constexpr auto k = ssm::ss2d_n1_kernel<T, SSM_SS2D_TS, SSM_SS2D_WARPS, ACC_SMEM,
                                          SSM_SS2D_APOLY != 0, ROW_ASYNC, BC_ASYNC, ORDER>;
   const int smem =
