@@ -1099,6 +1099,7 @@ int ssm_debug_bounds_enabled(void) {
 
 }  // extern "C"
 
+#ifdef SSM_DEBUG_BOUNDS
 namespace {
 // One check whose index is one past its one-element range: recorded and
 // skipped in the debug-bounds build (nothing is read or written).
@@ -1106,6 +1107,7 @@ __global__ void bounds_self_test_kernel(float *never_written) {
   if (ssm::in_bounds(1, 1, ssm::kBndSelfTest)) never_written[0] = 0.0f;
 }
 }  // namespace
+#endif
 
 extern "C" {
 
