@@ -68,6 +68,32 @@ def test_ss2d_no_softplus_no_D(ssm):
     assert rel_err(y, oracle_ss2d(inp, 9, 13, softplus=False)) <= 1e-4
 
 
+@pytest.mark.parametrize("order", ["cross", "snake"])
+@pytest.mark.parametrize("dtype,b,H,W,d_in", [
+    (torch.float32, 2, 7, 9, 16),     # one partial chunk, shared accumulator
+    (torch.bfloat16, 1, 13, 11, 13),  # odd d_in: plain staging, ragged channel tile
+    (torch.bfloat16, 1, 80, 81, 16),  # workspace accumulator, 21 chunks, the last partial
+])
+def test_ss2d_steps_past_the_end_cannot_leak(ssm, order, dtype, b, H, W, d_in):
+    """The kernel runs whole chunks, and the steps past the end of a direction
+    (zero-filled rows) are not forced to identity.  With the softplus off and
+    dt_bias = -4 their decay is exp(4) > 1, so their composed maps overflow to
+    inf and nan in fp32; the real steps, which all come before them, must not
+    see that."""
+    dt = "bf16" if dtype == torch.bfloat16 else "fp32"
+    inp = ss2d_inputs(b, H, W, d_in, 1, dt, seed=H * 31 + W, with_dt_bias=True)
+    inp["dt_bias"] = torch.full_like(inp["dt_bias"], -4.0)
+    # real steps: delta + dt_bias = |delta| + 0.1 > 0, a decaying state
+    inp["delta"] = (inp["delta"].float().abs() + 4.1).to(inp["delta"].dtype)
+    g = to_cuda(inp)
+    y = ssm.ss2d_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], H, W, D=g["D"],
+                          dt_bias=g["dt_bias"], delta_softplus=False, order=order)
+    assert torch.isfinite(y.float()).all()
+    ref = oracle.ss2d_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], H, W,
+                           D=inp["D"], dt_bias=inp["dt_bias"], delta_softplus=False, order=order)
+    assert rel_err(y, ref) <= TOL[dtype]
+
+
 def test_ss2d_large_image_uses_workspace(ssm):
     """H W above the shared-memory accumulator limit: the fp32 accumulator lives
     in the caller's workspace."""
