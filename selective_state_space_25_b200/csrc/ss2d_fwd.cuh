@@ -310,11 +310,11 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     }
   }
 
-  // one chunk of direction K (index arithmetic specialised per direction)
-  // chunk q = k nchunks + c reads the carry in buffer q & 1 and leaves the
-  // next one in the other buffer, so consecutive chunks need no barrier
-  // between them (their pixels differ); a direction's last chunk ends with
-  // one, since the next direction revisits every pixel.
+  // one chunk of direction K (index arithmetic specialised per direction).
+  // Chunk q = k nchunks + c reads the carry and the warp totals in buffer
+  // q & 1 and leaves the next carry in the other buffer.  Its one CTA barrier
+  // (after the warp totals) also orders every accumulator update of the
+  // previous chunk before its own, the next direction's first chunk included.
   auto chunk = [&](auto kc, int c) {
     constexpr int K = decltype(kc)::value;
     const int l0 = c * LC;
