@@ -112,6 +112,27 @@ def test_ss2d_validation(kw, status):
     assert ss2d(**kw) == status
 
 
+BIG_WS = FAKE + (1 << 44)  # far from every input range, never dereferenced
+
+
+@pytest.mark.parametrize("kw", [
+    dict(b=1, H=2048, W=2048, d_in=8),     # H W = 2^22: per-image offsets are 32-bit
+    dict(b=1, H=1024, W=1024, d_in=2048),  # H W d_in = 2^31
+    dict(b=70000, H=4, W=5, d_in=8),       # grid.y limit
+])
+def test_ss2d_size_limits(kw):
+    need = S.ss2d_scan_fwd_workspace_bytes(kw["b"], kw["H"], kw["W"], kw["d_in"], 1)
+    assert need != ctypes.c_size_t(-1).value
+    assert ss2d(ws=BIG_WS if need else None, ws_bytes=need, **kw) == S.SSM_ERR_UNSUPPORTED
+    assert S.last_error() != ""
+
+
+def test_ss2d_unknown_order():
+    st = L.ss2d_scan_fwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 1, FAKE + 8192, 2, 4, 5, 8,
+                            1, 7, S.SSM_BF16, None, 0, None)
+    assert st == S.SSM_ERR_UNSUPPORTED and "order" in S.last_error()
+
+
 def step(**kw):
     a = dict(state=FAKE + 65536, x=FAKE, dt=FAKE, A=FAKE, B=FAKE, C=FAKE, D=None, z=None,
              dt_bias=None, sp=1, y=FAKE + 4096, b=2, d_in=16, N=16, dtype=S.SSM_BF16, stream=None)
