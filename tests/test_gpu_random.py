@@ -29,7 +29,7 @@ def _dtype(r):
     return r.choice([("bf16", torch.bfloat16), ("fp32", torch.float32)])
 
 
-@pytest.mark.parametrize("seed", _seeds(24, 11))
+@pytest.mark.parametrize("seed", _seeds(200, 11))
 def test_random_scan_forward(ssm, seed):
     r = random.Random(seed)
     b, L, d_in, N = r.randint(1, 3), r.randint(1, 300), r.randint(1, 96), r.choice(STATES)
@@ -54,7 +54,7 @@ def test_random_scan_forward(ssm, seed):
     assert rel_err(hl, h_ref) <= 1e-4, what
 
 
-@pytest.mark.parametrize("seed", _seeds(16, 12))
+@pytest.mark.parametrize("seed", _seeds(120, 12))
 def test_random_scan_backward(ssm, seed):
     r = random.Random(seed)
     b, L, d_in, N = r.randint(1, 2), r.randint(1, 120), r.randint(1, 48), r.choice(STATES)
@@ -85,7 +85,7 @@ def test_random_scan_backward(ssm, seed):
         assert rel_err(got[k], ref[k]) <= tol, (k,) + what
 
 
-@pytest.mark.parametrize("seed", _seeds(16, 13))
+@pytest.mark.parametrize("seed", _seeds(160, 13))
 def test_random_ss2d(ssm, seed):
     r = random.Random(seed)
     b, H, W, d_in = r.randint(1, 2), r.randint(1, 40), r.randint(1, 40), r.randint(1, 40)
@@ -106,7 +106,7 @@ def test_random_ss2d(ssm, seed):
     assert rel_err(y, ref) <= TOL[dtype], (b, H, W, d_in, dt, order, softplus)
 
 
-@pytest.mark.parametrize("seed", _seeds(16, 14))
+@pytest.mark.parametrize("seed", _seeds(160, 14))
 def test_random_decode_steps(ssm, seed):
     r = random.Random(seed)
     b, d_in, N = r.randint(1, 4), r.randint(1, 300), r.choice(STATES)
