@@ -241,8 +241,9 @@ ssm_status ssm_scan_bwd_saved(const void *u, const void *delta, const float *A,
  *   D, dt_bias    device fp32 (4 d_in), nullable
  *   workspace     device, >= ss2d_scan_fwd_workspace_bytes(...) bytes; may be
  *                 NULL when that is 0.  Contents on entry are ignored.
- * d_state must be 1 (the SS2D setting of VMamba), H * W below 2^22 pixels
- * and H * W * d_in below 2^31; other values return SSM_ERR_UNSUPPORTED.
+ * d_state must be 1 (the SS2D setting of VMamba), H * W below 2^22 pixels,
+ * H * W * d_in below 2^31 and b at most 65535; other values return
+ * SSM_ERR_UNSUPPORTED.
  */
 ssm_status ss2d_scan_fwd(const void *u, const void *delta, const float *A,
                          const void *B, const void *C, const float *D,
