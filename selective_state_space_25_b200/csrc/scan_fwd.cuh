@@ -32,8 +32,8 @@ struct ScanParams {
   // Sequence blocks of the split scan (scan_ws.cuh): grid z-index k covers
   // steps [k Lb, min(L, (k + 1) Lb)); Lb = 0 means one block.  blk_decay and
   // blk_state are (b, nblk, d_in, N) fp32: the summary pass leaves each
-  // block's decay product and its end state from zero there, the carry pass
-  // turns blk_state[k] (k >= 1) into the state block k starts from.
+  // block's decay product and its end state from zero there, and the carry
+  // pass overwrites blk_decay[k] with the state block k + 1 starts from.
   int64_t Lb = 0;
   float *blk_decay = nullptr;
   float *blk_state = nullptr;

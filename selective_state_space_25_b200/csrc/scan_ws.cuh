@@ -128,13 +128,13 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P, DT_>::THREADS)
                   ? make_float2(p.A[d * N + n] * kLog2e, p.A[d * N + n + 1] * kLog2e)
                   : make_float2(0.0f, 0.0f);
       // the summary starts every block from zero; the scan (and the states
-      // pass) starts block 0 from h0 and block k > 0 from the carry the
-      // carry pass left
+      // pass) starts block 0 from h0 and block k > 0 from the state the
+      // carry pass left in blk_decay[k - 1]
       const float *h0 = blk == 0 ? p.h0 + (ib * d_in + d) * N + n
-                                 : p.blk_state + (blk_row + d) * N + n;
+                                 : p.blk_decay + (blk_row - d_in + d) * N + n;
       const bool from = d_ok && (!SUMMARY || SAVE) && (blk > 0 || p.h0) &&
                         (blk == 0 ? in_bounds((ib * d_in + d) * N + n + 1, n_state, kBndState)
-                                  : in_bounds((blk_row + d) * N + n + 1, n_blk, kBndChunk));
+                                  : in_bounds((blk_row - d_in + d) * N + n + 1, n_blk, kBndChunk));
       h[k] = from ? make_float2(h0[0], h0[1]) : make_float2(0.0f, 0.0f);
     }
     float dsum = 0.0f;  // sum of delta over the block (summary pass)
@@ -437,24 +437,63 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P, DT_>::THREADS)
   cp_async_wait<0>();  // only empty groups can remain
 }
 
-// Carry pass of the split scan: per chain (batch, channel, state), the block
-// maps composed in order from h0, blk_state[k] (k >= 1) overwritten with the
-// state block k starts from (block k's own end state is read before that).
-__global__ void scan_carry_kernel(const float *h0, const float *blk_decay, float *blk_state,
-                                  int64_t b, int64_t nblk, int64_t d_in, int N) {
-  const int64_t q = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;  // (batch, channel, state)
-  const int64_t per = d_in * N;
-  if (q >= b * per) return;
-  if (!in_bounds((q / per * nblk + nblk - 1) * per + q % per, b * nblk * per, kBndChunk)) return;
-  const int64_t ib = q / per, r = q - ib * per;
-  float h = h0 ? h0[q] : 0.0f;
-  float qn = blk_state[(ib * nblk) * per + r];
-  for (int64_t k = 0; k + 1 < nblk; ++k) {
-    const int64_t i = (ib * nblk + k) * per + r;
-    const float qk = qn;
-    qn = blk_state[i + per];
-    h = fmaf(blk_decay[i], h, qk);
-    blk_state[i + per] = h;
+// Carry pass of the split scan, a parallel scan over the blocks.  Chain
+// (batch i, column r = channel N + state) has the block maps
+// h -> P_k h + Q_k (P_k = blk_decay[k], Q_k = blk_state[k], k < nblk - 1);
+// composed in order with (a, b) o (a', b') = (a a', a b' + b) and applied to
+// h0, they give the state each block starts from.  A CTA owns 32 chains;
+// 32-block tiles of P and Q are read row by row (coalesced) into shared
+// memory, each warp scans 4 chains across the tile with shuffles (lane =
+// block), and the state leaving a tile carries into the next.  The state
+// block k + 1 starts from overwrites P_k, which the tile has already read.
+constexpr int kCarryThreads = 256;
+__global__ void __launch_bounds__(kCarryThreads) scan_carry_kernel(const float *h0, float *blk_decay,
+                                                                   const float *blk_state, int64_t b,
+                                                                   int64_t nblk, int64_t d_in, int N) {
+  constexpr int TILE = 32, WARPS = kCarryThreads / 32, CPW = TILE / WARPS;  // chains per warp
+  __shared__ float sP[TILE][TILE + 1], sQ[TILE][TILE + 1];
+  const int64_t per = d_in * N, nmaps = nblk - 1;
+  const int64_t ib = blockIdx.y, r0 = (int64_t)blockIdx.x * TILE;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t col = r0 + lane;  // this lane's chain in the row loads and stores
+  float carry[CPW];               // state entering the tile, chains warp CPW + c
+#pragma unroll
+  for (int c = 0; c < CPW; ++c) {
+    const int64_t r = r0 + warp * CPW + c;
+    carry[c] = (h0 && r < per && in_bounds(ib * per + r, b * per, kBndState)) ? h0[ib * per + r]
+                                                                              : 0.0f;
+  }
+  for (int64_t k0 = 0; k0 < nmaps; k0 += TILE) {
+    __syncthreads();  // the previous tile's results are stored
+    for (int rr = warp; rr < TILE; rr += WARPS) {
+      const int64_t k = k0 + rr, i = (ib * nblk + k) * per + col;
+      const bool ok = k < nmaps && col < per && in_bounds(i, b * nblk * per, kBndChunk);
+      sP[rr][lane] = ok ? blk_decay[i] : 1.0f;  // identity maps past the last block
+      sQ[rr][lane] = ok ? blk_state[i] : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int c = 0; c < CPW; ++c) {
+      const int cc = warp * CPW + c;
+      float a = sP[lane][cc], q = sQ[lane][cc];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {  // inclusive: maps k0 .. k0 + lane
+        const float pa = __shfl_up_sync(0xffffffffu, a, off);
+        const float pq = __shfl_up_sync(0xffffffffu, q, off);
+        if (lane >= off) {
+          q = fmaf(a, pq, q);
+          a *= pa;
+        }
+      }
+      const float h = fmaf(a, carry[c], q);  // the state after block k0 + lane
+      carry[c] = __shfl_sync(0xffffffffu, h, 31);
+      sP[lane][cc] = h;
+    }
+    __syncthreads();
+    for (int rr = warp; rr < TILE; rr += WARPS) {
+      const int64_t k = k0 + rr, i = (ib * nblk + k) * per + col;
+      if (k < nmaps && col < per && in_bounds(i, b * nblk * per, kBndChunk)) blk_decay[i] = sP[rr][lane];
+    }
   }
 }
 

@@ -208,8 +208,8 @@ int device_sms() {
 // about four CTAs per SM, each block a whole number of chunks and at least
 // four chunks long.  nblk = 1: one pass.  Depends on the sizes only, so
 // ssm_scan_fwd_workspace_bytes and the launch agree.  Measured on B200
-// (b = 1, L = 16384, N = 16, bf16): d_in = 256 575 -> 94 us, d_in = 1536
-// 575 -> 321 us; at d_in = 4096 (128 CTAs) one pass is faster (577 against
+// (b = 1, L = 16384, N = 16, bf16): d_in = 256 575 -> 85 us, d_in = 1536
+// 575 -> 328 us; at d_in = 4096 (128 CTAs) one pass is faster (577 against
 // 754 us), hence the half-the-SMs threshold.
 struct SplitPlan {
   int64_t nblk = 1, Lb = 0;
@@ -248,9 +248,9 @@ ssm_status launch_scan_ws(const ssm::ScanParams &p, cudaStream_t st) {
   // split scan: block summaries, the carry pass, then every block at once
   const unsigned nblk = (unsigned)((p.L + p.Lb - 1) / p.Lb);
   if (ssm_status s = launch_scan_ws_pass<T, N, false, false, true>(p, nblk - 1, st)) return s;
-  const int64_t chains = p.b * p.d_in * N;
-  ssm::scan_carry_kernel<<<(unsigned)((chains + 255) / 256), 256, 0, st>>>(
-      p.h0, p.blk_decay, p.blk_state, p.b, nblk, p.d_in, N);
+  const int64_t chains = p.d_in * N;  // per batch
+  ssm::scan_carry_kernel<<<dim3((unsigned)((chains + 31) / 32), (unsigned)p.b), ssm::kCarryThreads,
+                           0, st>>>(p.h0, p.blk_decay, p.blk_state, p.b, nblk, p.d_in, N);
   if (ssm_status s = check_launch("ssm_scan_fwd")) return s;
   return launch_scan_ws_pass<T, N, HAS_Z, SAVE, false>(p, nblk, st);
 }

@@ -181,12 +181,15 @@ def test_mamba14b_long_workload_sampled(ssm):
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("b,L,d_in,N", [
     (1, 3000, 64, 16), (2, 777, 32, 8), (1, 1000, 32, 32), (1, 257, 32, 16), (3, 4100, 40, 16),
+    (1, 16384, 8, 16),  # 128 blocks: four 32-block tiles of the carry scan
+    (2, 10000, 16, 8),  # 63 blocks of 160 steps: a ragged second tile
 ])
 def test_split_scan(ssm, dtype, b, L, d_in, N):
     """Few channels and a long sequence: the sequence is cut into blocks whose
-    maps are summarised, composed from h0 block after block and replayed in
-    parallel (the chunked associative scan with a carry).  The blocks' last
-    one is ragged in every case."""
+    maps are summarised, composed from h0 (a warp-shuffle scan over the
+    blocks, 32 at a time, each tile carrying into the next) and replayed in
+    parallel.  The blocks' last one is ragged in every case but the first
+    of the two long ones."""
     dt = "bf16" if dtype == torch.bfloat16 else "fp32"
     need = ssm.ssm_scan_fwd_workspace_bytes(b, L, d_in, N)
     if d_in % 8 == 0:
