@@ -205,12 +205,14 @@ int device_sms() {
 
 // Split of the sequence into blocks (scan_ws.cuh, split scan) for problems
 // whose b * ceil(d_in / 32) CTAs would leave more than half of the SMs idle:
-// about four CTAs per SM, each block a whole number of chunks and at least
-// four chunks long.  nblk = 1: one pass.  Depends on the sizes only, so
+// at most four CTAs per SM (two whole waves of the two a scan-pass SM holds),
+// each block a whole number of chunks and at least four chunks long.
+// nblk = 1: one pass.  Depends on the sizes only, so
 // ssm_scan_fwd_workspace_bytes and the launch agree.  Measured on B200
-// (b = 1, L = 16384, N = 16, bf16): d_in = 256 575 -> 85 us, d_in = 1536
-// 575 -> 328 us; at d_in = 4096 (128 CTAs) one pass is faster (577 against
-// 754 us), hence the half-the-SMs threshold.
+// (b = 1, L = 16384, N = 16, bf16): d_in = 256 575 -> 80 us, d_in = 1536
+// 575 -> 320 us (329 us when the block count rounded up, a third wave);
+// at d_in = 4096 (128 CTAs) one pass is faster (577 against 754 us), hence
+// the half-the-SMs threshold.
 struct SplitPlan {
   int64_t nblk = 1, Lb = 0;
 };
@@ -220,7 +222,7 @@ SplitPlan split_plan(int64_t b, int64_t L, int64_t d_in, int64_t N) {
   const int64_t sms = device_sms();
   const int64_t ctas = b * ((d_in + 31) / 32);
   if (2 * ctas > sms) return sp;
-  int64_t nblk = (4 * sms + ctas - 1) / ctas;
+  int64_t nblk = 4 * sms / ctas;  // two whole waves of two CTAs per SM
   const int64_t by_len = L / (4 * SSM_WS_TC);
   if (nblk > by_len) nblk = by_len;
   if (nblk > 4096) nblk = 4096;
