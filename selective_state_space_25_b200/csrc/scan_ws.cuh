@@ -440,8 +440,8 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P, DT_>::THREADS)
 // Carry pass of the split scan, a parallel scan over the blocks.  Chain
 // (batch i, column r = channel N + state) has the block maps
 // h -> P_k h + Q_k (P_k = blk_decay[k], Q_k = blk_state[k], k < nblk - 1);
-// composed in order with (a, b) o (a', b') = (a a', a b' + b) and applied to
-// h0, they give the state each block starts from.  A CTA owns 32 chains;
+// composed in order with (a, b) o (a', b') = (a a', a' b + b'), (a, b) the
+// earlier map, and applied to h0, they give the state each block starts from.  A CTA owns 32 chains;
 // 32-block tiles of P and Q are read row by row (coalesced) into shared
 // memory, each warp scans 4 chains across the tile with shuffles (lane =
 // block), and the state leaving a tile carries into the next.  The state
@@ -478,6 +478,7 @@ __global__ void __launch_bounds__(kCarryThreads) scan_carry_kernel(const float *
       float a = sP[lane][cc], q = sQ[lane][cc];
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {  // inclusive: maps k0 .. k0 + lane
+        // (pa, pq) composes the off earlier maps; (a, q) this lane's so far
         const float pa = __shfl_up_sync(0xffffffffu, a, off);
         const float pq = __shfl_up_sync(0xffffffffu, q, off);
         if (lane >= off) {
@@ -492,7 +493,8 @@ __global__ void __launch_bounds__(kCarryThreads) scan_carry_kernel(const float *
     __syncthreads();
     for (int rr = warp; rr < TILE; rr += WARPS) {
       const int64_t k = k0 + rr, i = (ib * nblk + k) * per + col;
-      if (k < nmaps && col < per && in_bounds(i, b * nblk * per, kBndChunk)) blk_decay[i] = sP[rr][lane];
+      if (k < nmaps && col < per && in_bounds(i, b * nblk * per, kBndChunk))
+        blk_decay[i] = sP[rr][lane];
     }
   }
 }
