@@ -77,6 +77,9 @@ def test_workspace_query():
     # (b, blocks, d_in, N) arrays (block decays and block states)
     ws = S.ssm_scan_fwd_workspace_bytes(1, 16384, 64, 16)
     assert ws > 0 and ws % (2 * 64 * 16 * 4) == 0
+    # 48 CTAs of 32 channels on 148 SMs: 12 blocks (576 CTAs, two whole waves
+    # of two per SM), not 13 (624, a third wave)
+    assert S.ssm_scan_fwd_workspace_bytes(1, 16384, 1536, 16) == 2 * 12 * 1536 * 16 * 4
     assert S.ssm_scan_fwd_workspace_bytes(1, 200, 64, 16) == 0       # too short to split
     assert S.ssm_scan_fwd_workspace_bytes(1, 16384, 64, 64) == 0     # d_state 64: one pass
     assert S.ssm_scan_fwd_workspace_bytes(1, 16384, 60, 16) == 0     # d_in not a multiple of 8
