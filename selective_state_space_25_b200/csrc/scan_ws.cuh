@@ -116,6 +116,10 @@ __global__ void __launch_bounds__(WsScan<T, N, NS, TC, H, P, DT_>::THREADS)
 
   if (tid < K::SCAN_THREADS) {
     // =================================================== scan warps
+    // the split scan's last pass is launched while the carry pass finishes:
+    // the helpers stage inputs meanwhile, the scan warps wait for the block
+    // start states
+    grid_dependency_wait();
     const int c = tid % DT;  // channel
     const int g = tid / DT;  // state group
     const int64_t d = d0 + c;
@@ -456,6 +460,8 @@ __global__ void __launch_bounds__(kCarryThreads) scan_carry_kernel(const float *
   const int64_t ib = blockIdx.y, r0 = (int64_t)blockIdx.x * TILE;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t col = r0 + lane;  // this lane's chain in the row loads and stores
+  grid_dependents_launch();       // the scan pass may start staging its inputs
+  grid_dependency_wait();         // the summary pass's maps are written
   float carry[CPW];               // state entering the tile, chains warp CPW + c
 #pragma unroll
   for (int c = 0; c < CPW; ++c) {

@@ -224,4 +224,17 @@ template <int N> __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
 }
 
+// ------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while
+// the kernel before it in the stream still runs: the earlier one lets it
+// launch (grid_dependents_launch), and it waits for the earlier grids to
+// finish with their writes visible (grid_dependency_wait) before reading
+// what they produce.  Without such a launch the wait returns at once.
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 }  // namespace ssm

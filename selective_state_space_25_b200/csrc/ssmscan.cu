@@ -82,6 +82,31 @@ ssm_status check_launch(const char *what) {
   return ok();
 }
 
+// Launch with programmatic stream serialization: the kernel may start once
+// every block of the previous kernel in the stream has called
+// grid_dependents_launch (or exited), and calls grid_dependency_wait before
+// it reads that kernel's results.
+template <typename... KArgs, typename... Args>
+ssm_status launch_dependent(void (*kernel)(KArgs...), dim3 grid, int threads, int smem,
+                            cudaStream_t st, const char *what, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3((unsigned)threads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(SSM_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
+  }
+  return ok();
+}
+
 // Opt a kernel into > 48 KB of dynamic shared memory once per device.
 template <auto Kernel>
 ssm_status ensure_smem(int bytes, const char *what) {
@@ -131,10 +156,13 @@ constexpr int fast_npt(int n, int want, int dt) {
 
 template <auto Kernel>
 ssm_status launch_fast_kernel(const ssm::ScanParams &p, dim3 grid, int threads, int smem,
-                              cudaStream_t st) {
+                              cudaStream_t st, bool dependent = false) {
   if (ssm_status s = ensure_smem<Kernel>(smem, "ssm_scan_fwd")) return s;
-  Kernel<<<grid, threads, smem, st>>>(p);
-  return check_launch("ssm_scan_fwd");
+  if (!dependent) {
+    Kernel<<<grid, threads, smem, st>>>(p);
+    return check_launch("ssm_scan_fwd");
+  }
+  return launch_dependent(Kernel, grid, threads, smem, st, "ssm_scan_fwd", p);
 }
 
 template <typename T, int N, bool HAS_Z, int WANT_NPT>
@@ -209,8 +237,8 @@ int device_sms() {
 // each block a whole number of chunks and at least four chunks long.
 // nblk = 1: one pass.  Depends on the sizes only, so
 // ssm_scan_fwd_workspace_bytes and the launch agree.  Measured on B200
-// (b = 1, L = 16384, N = 16, bf16): d_in = 256 575 -> 80 us, d_in = 1536
-// 575 -> 320 us (329 us when the block count rounded up, a third wave);
+// (b = 1, L = 16384, N = 16, bf16): d_in = 256 575 -> 74 us, d_in = 1536
+// 575 -> 313 us (329 us when the block count rounded up, a third wave);
 // at d_in = 4096 (128 CTAs) one pass is faster (577 against 754 us), hence
 // the half-the-SMs threshold.
 struct SplitPlan {
@@ -235,13 +263,14 @@ SplitPlan split_plan(int64_t b, int64_t L, int64_t d_in, int64_t N) {
 }
 
 template <typename T, int N, bool HAS_Z, bool SAVE, bool SUMMARY>
-ssm_status launch_scan_ws_pass(const ssm::ScanParams &p, unsigned nz, cudaStream_t st) {
+ssm_status launch_scan_ws_pass(const ssm::ScanParams &p, unsigned nz, cudaStream_t st,
+                               bool dependent = false) {
   constexpr int NS = ws_states(N);
   using Cfg = ssm::WsScan<T, N, NS, SSM_WS_TC, SSM_WS_HELPERS, SSM_WS_AHEAD>;
   constexpr auto k = ssm::scan_ws_kernel<T, N, NS, SSM_WS_TC, SSM_WS_HELPERS, SSM_WS_AHEAD,
                                          HAS_Z, SAVE, SUMMARY>;
   const dim3 grid((unsigned)((p.d_in + Cfg::DT - 1) / Cfg::DT), (unsigned)p.b, nz);
-  return launch_fast_kernel<k>(p, grid, Cfg::THREADS, Cfg::SMEM, st);
+  return launch_fast_kernel<k>(p, grid, Cfg::THREADS, Cfg::SMEM, st, dependent);
 }
 
 template <typename T, int N, bool HAS_Z, bool SAVE>
@@ -250,11 +279,15 @@ ssm_status launch_scan_ws(const ssm::ScanParams &p, cudaStream_t st) {
   // split scan: block summaries, the carry pass, then every block at once
   const unsigned nblk = (unsigned)((p.L + p.Lb - 1) / p.Lb);
   if (ssm_status s = launch_scan_ws_pass<T, N, false, false, true>(p, nblk - 1, st)) return s;
+  // the carry and scan passes start while the pass before each finishes
   const int64_t chains = p.d_in * N;  // per batch
-  ssm::scan_carry_kernel<<<dim3((unsigned)((chains + 31) / 32), (unsigned)p.b), ssm::kCarryThreads,
-                           0, st>>>(p.h0, p.blk_decay, p.blk_state, p.b, nblk, p.d_in, N);
-  if (ssm_status s = check_launch("ssm_scan_fwd")) return s;
-  return launch_scan_ws_pass<T, N, HAS_Z, SAVE, false>(p, nblk, st);
+  if (ssm_status s = launch_dependent(ssm::scan_carry_kernel,
+                                      dim3((unsigned)((chains + 31) / 32), (unsigned)p.b),
+                                      ssm::kCarryThreads, 0, st, "ssm_scan_fwd", p.h0, p.blk_decay,
+                                      (const float *)p.blk_state, p.b, (int64_t)nblk, p.d_in,
+                                      (int)N))
+    return s;
+  return launch_scan_ws_pass<T, N, HAS_Z, SAVE, false>(p, nblk, st, true);
 }
 
 template <typename T, int N>
