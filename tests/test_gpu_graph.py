@@ -85,3 +85,34 @@ def test_scan_fwd_bwd_and_ss2d_in_a_graph(ssm):
             assert torch.allclose(out[k], ref[k], rtol=1e-5, atol=1e-6)
         else:
             assert torch.equal(out[k], ref[k]), k
+
+
+def test_split_scan_in_a_graph(ssm):
+    """The split scan (few channels, long sequence: summary, carry and scan
+    passes, the last two launched to start while the pass before finishes)
+    captured in a graph replays bit for bit."""
+    b, L, d_in, N = 1, 4096, 64, 16
+    need = ssm.ssm_scan_fwd_workspace_bytes(b, L, d_in, N)
+    assert need > 0, "this shape should take the split scan"
+    g = to_cuda(scan_inputs(b, L, d_in, N, "bf16", seed=9, with_h0=True))
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(g["u"])
+    hl = torch.empty(b, d_in, N, device="cuda")
+
+    def work():
+        ssm.ssm_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], D=g["D"], z=g["z"],
+                         dt_bias=g["dt_bias"], h0=g["h0"], h_last=hl, y=y, workspace=ws)
+
+    work()
+    torch.cuda.synchronize()
+    y_e, hl_e = y.clone(), hl.clone()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        work()
+    y.zero_()
+    hl.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_e) and torch.equal(hl, hl_e)
