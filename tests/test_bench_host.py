@@ -46,6 +46,19 @@ def test_sfu_ceiling():
     assert 0.25 < t_hbm / t_sfu < 0.4
 
 
+def test_launches_per_step():
+    """The gpu_launches claim: one kernel per step, two for the backward that
+    runs the states pass first, three for a scan that takes the split scan."""
+    W = WORKLOADS
+    assert bench.launches_per_step(W["mamba1.4b-long-scan"]) == 1
+    assert bench.launches_per_step(W["mamba1.4b-long-scan"], split=True) == 3
+    assert bench.launches_per_step(W["vmamba-ss2d"], split=True) == 1
+    assert bench.launches_per_step(W["mamba-decode-step"]) == 1
+    assert bench.launches_per_step(W["mamba130m-scan-bwd"]) == 2
+    assert bench.launches_per_step(W["mamba130m-scan-bwd-saved"]) == 1
+    assert set(bench.STEP_PARTS) == {"scan", "scan_bwd"}
+
+
 def test_traffic_is_null_when_kernels_changed(tmp_path, monkeypatch):
     f = tmp_path / "traffic.json"
     f.write_text(json.dumps({"w": {"dram_bytes_per_launch": 123, "source_hash": "stale"}}))
