@@ -240,7 +240,16 @@ ssm_status ssm_scan_bwd_saved(const void *u, const void *delta, const float *A,
  *   B, C          device, (b, 4, H W, d_state), dtype
  *   D, dt_bias    device fp32 (4 d_in), nullable
  *   workspace     device, >= ss2d_scan_fwd_workspace_bytes(...) bytes; may be
- *                 NULL when that is 0.  Contents on entry are ignored.
+ *                 NULL when that is 0.  Contents on entry are ignored.  With
+ *                 ss2d_scan_fwd_fast_workspace_bytes(...) bytes or more the
+ *                 call may take the direction split (below); with less it
+ *                 runs the single-kernel path.  Same results either way.
+ * Batches too small to fill the GPU (b * ceil(d_in / 8) tiles at most half
+ * the SMs, accumulator in shared memory) take the direction split when the
+ * workspace allows: one CTA per (tile, direction), each storing its
+ * direction's fp32 outputs in the workspace, then a second kernel that sums
+ * them k0 + k1 + k2 + k3 and rounds once -- the single kernel's arithmetic in
+ * its order, so the results are bit-identical.
  * d_state must be 1 (the SS2D setting of VMamba), H * W below 2^22 pixels,
  * H * W * d_in below 2^31 and b at most 65535; other values return
  * SSM_ERR_UNSUPPORTED.
@@ -280,6 +289,16 @@ ssm_status ss2d_scan_fwd_ex(const void *u, const void *delta, const float *A,
  */
 size_t ss2d_scan_fwd_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_in,
                                      int64_t d_state);
+
+/*
+ * Bytes of device workspace with which ss2d_scan_fwd takes its fastest path
+ * for this problem: 4 * b * H * W * d_in fp32 (the direction split's four
+ * slices) when the direction split applies, else the same value as
+ * ss2d_scan_fwd_workspace_bytes.  Never less than that minimum; (size_t)-1
+ * for invalid sizes.
+ */
+size_t ss2d_scan_fwd_fast_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_in,
+                                          int64_t d_state);
 
 /*
  * ss2d_scan_fwd without a workspace, for callers that cannot allocate device

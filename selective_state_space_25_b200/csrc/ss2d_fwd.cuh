@@ -161,8 +161,13 @@ __device__ __forceinline__ void ss2d_pos(int k, int l, int H, int W, float invH,
 // and 16-byte aligned u, delta); otherwise with plain bounds-checked loads.
 // BC_ASYNC: B / C staged with cp.async (needs H W a multiple of 16 / sizeof(T)
 // and 16-byte aligned B, C); otherwise read from global memory per step.
+// DSPLIT (shared accumulator only): the CTA runs direction blockIdx.z alone
+// and stores that direction's fp32 outputs, pixel-major, in slice z of the
+// caller's workspace (4, b, H W, d_in); ss2d_merge4_kernel then sums the four
+// slices k0 + k1 + k2 + k3 and rounds once -- the fused kernel's operations
+// in its order, for grids too small to fill the GPU one CTA per tile.
 template <typename T, int TS, int WARPS, bool ACC_SMEM, bool A_POLY, bool ROW_ASYNC,
-          bool BC_ASYNC, int ORDER>
+          bool BC_ASYNC, int ORDER, bool DSPLIT = false>
 __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     ss2d_n1_kernel(Ss2dParams p) {
   using Cfg = Ss2dCfg<T, TS, WARPS, ACC_SMEM>;
@@ -209,6 +214,8 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
   const bool whole_tile = d0 + DT <= d_in && acc_pairs;
 
   const int nchunks = (Li + LC - 1) / LC;
+  static_assert(!DSPLIT || ACC_SMEM, "the direction split keeps its accumulator in shared memory");
+  const int kz = DSPLIT ? (int)blockIdx.z : 0;  // the direction (DSPLIT), else the first one
 
   // stage the delta / u rows (and B / C) of this warp's steps of chunk c of
   // direction k: rows w0 .. w0 + RW - 1
@@ -296,8 +303,10 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     cp_async_commit();
   };
 
-  if (tid < DT) carry[tid] = 0.0f;  // the first direction starts from h = 0 (buffer 0)
-  prefetch(0, 0);
+  // the first direction starts from h = 0: buffer 0, or with DSPLIT buffer
+  // (kz nchunks) & 1, so both are cleared
+  if (tid < 2 * DT) carry[tid] = 0.0f;
+  prefetch(kz, 0);
   float2 A2 = make_float2(0.0f, 0.0f), bias = A2;
   // the skip term of all four directions, (sum_k D_k) u, is added once, with
   // direction 0's outputs
@@ -317,6 +326,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
   // previous chunk before its own, the next direction's first chunk included.
   auto chunk = [&](auto kc, int c) {
     constexpr int K = decltype(kc)::value;
+    constexpr bool FIRST = K == 0 || DSPLIT;  // this CTA's first direction stores, later ones add
     const int l0 = c * LC;
     const int cq = (K * nchunks + c) & 1;
     [[maybe_unused]] const T *Bk = gB + (int64_t)K * L;
@@ -388,7 +398,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     // the warp is done with its staged rows (the scan above took every lane's
     // steps): stage its rows of the next chunk
     if (c + 1 < nchunks) prefetch(K, c + 1);
-    else if (K < 3) prefetch(K + 1, 0);
+    else if (!DSPLIT && K < 3) prefetch(K + 1, 0);
     __syncthreads();  // warp totals visible
 
     // ---- 3. incoming state: previous chunk's carry, earlier warps, earlier segments
@@ -416,7 +426,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
         const float2 yv = __ffma2_rn(gg[j], h, yl[j]);
         float2 *d2 = reinterpret_cast<float2 *>(ACC_SMEM ? acc_s + rows[j] * DT + 2 * cp
                                                          : acc_g + rows[j] * di + 2 * cp);
-        if constexpr (K == 0)
+        if constexpr (FIRST)
           *d2 = yv;
         else
           *d2 = __fadd2_rn(*d2, yv);
@@ -432,13 +442,13 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
           float *dst = ACC_SMEM ? acc_s + rows[j] * DT + 2 * cp : acc_g + rows[j] * di + 2 * cp;
           if (ok1 && acc_pairs) {
             float2 *d2 = reinterpret_cast<float2 *>(dst);
-            if constexpr (K == 0)
+            if constexpr (FIRST)
               *d2 = yv;
             else
               *d2 = __fadd2_rn(*d2, yv);
           } else {
-            dst[0] = K == 0 ? yv.x : dst[0] + yv.x;
-            if (ok1) dst[1] = K == 0 ? yv.y : dst[1] + yv.y;
+            dst[0] = FIRST ? yv.x : dst[0] + yv.x;
+            if (ok1) dst[1] = FIRST ? yv.y : dst[1] + yv.y;
           }
         }
       }
@@ -451,7 +461,7 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     }
   };
 
-  for (int k = 0; k < 4; ++k) {
+  for (int k = kz; k < (DSPLIT ? kz + 1 : 4); ++k) {
     const int64_t pk0 = k * d_in + dA;  // parameter rows of (direction, channel pair)
     A2 = make_float2(ok0 ? p.A[pk0] * kLog2e : 0.0f, ok1 ? p.A[pk0 + 1] * kLog2e : 0.0f);
     bias = make_float2((ok0 && p.dt_bias) ? p.dt_bias[pk0] : 0.0f,
@@ -466,6 +476,39 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
     }
   }
   __syncthreads();
+
+  if constexpr (DSPLIT) {
+    // ---- this direction's fp32 outputs, pixel-major, into workspace slice kz
+    float *part = p.acc_global + ((int64_t)kz * p.b + ib) * L * d_in + d0;
+    const int64_t n_part = 4 * p.b * L * d_in;
+    if (d0 + DT <= d_in && (d_in & 3) == 0 && (reinterpret_cast<uintptr_t>(p.acc_global) & 15) == 0) {
+      for (int pix = tid; pix < Li; pix += THREADS) {
+        const int hh = div_small(pix, Wi, invW), w = pix - hh * Wi;
+        if (!in_bounds(((int64_t)kz * p.b + ib) * L * d_in + (int64_t)pix * d_in + d0 + DT - 1,
+                       n_part, kBndWork) ||
+            !in_bounds((int64_t)(hh * RS + w) * DT + DT - 1, (int64_t)Hi * RS * DT, kBndWork))
+          continue;
+        const float4 *a4 = reinterpret_cast<const float4 *>(acc_s + (hh * RS + w) * DT);
+        float4 *o = reinterpret_cast<float4 *>(part + (int64_t)pix * di);
+        o[0] = a4[0];
+        o[1] = a4[1];
+      }
+    } else {
+      const int ch = tid & (DT - 1);
+      if (d0 + ch < d_in) {
+        for (int hh = 0; hh < Hi; ++hh) {
+          for (int w = tid / DT; w < Wi; w += THREADS / DT) {
+            const int pix = hh * Wi + w;
+            if (!in_bounds(((int64_t)kz * p.b + ib) * L * d_in + (int64_t)pix * d_in + d0 + ch,
+                           n_part, kBndWork))
+              continue;
+            part[(int64_t)pix * di + ch] = acc_s[(hh * RS + w) * DT + ch];
+          }
+        }
+      }
+    }
+    return;
+  }
 
   // ---- round once and store.  Shared accumulator, whole 8-channel tile and
   // 16-byte aligned rows: one pixel per thread, its 8 channels as one vector;
@@ -500,6 +543,42 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
           Elem<T>::store(gy, pix * di + ch, v);
         }
       }
+    }
+  }
+}
+
+// The direction split's merge: y = ((p0 + p1) + p2) + p3 over the four fp32
+// slices (4, n) the DSPLIT kernel stored, rounded once to the activation
+// dtype.  Four elements per thread when n is a multiple of 4 and parts and y
+// are 16- and 8-byte aligned (VEC4).
+template <typename T, bool VEC4>
+__global__ void ss2d_merge4_kernel(const float *parts, T *y, int64_t n) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  if constexpr (VEC4) {
+    const float4 *p4 = reinterpret_cast<const float4 *>(parts);
+    const int64_t n4 = n / 4;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4; i += stride) {
+      if (!in_bounds(3 * n4 + i, 4 * n4, kBndWork) || !in_bounds(4 * i + 3, n, kBndAct)) continue;
+      float4 s = p4[i];
+#pragma unroll
+      for (int k = 1; k < 4; ++k) {
+        const float4 v = p4[k * n4 + i];
+        s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+      }
+      if constexpr (sizeof(T) == 2) {
+        *reinterpret_cast<uint2 *>(y + 4 * i) = make_uint2(pack_bf16x2(s.x, s.y), pack_bf16x2(s.z, s.w));
+      } else {
+        *reinterpret_cast<float4 *>(y + 4 * i) = s;
+      }
+    }
+  } else {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += stride) {
+      if (!in_bounds(3 * n + i, 4 * n, kBndWork) || !in_bounds(i, n, kBndAct)) continue;
+      float s = parts[i];
+      s += parts[n + i];
+      s += parts[2 * n + i];
+      s += parts[3 * n + i];
+      Elem<T>::store(y, i, s);
     }
   }
 }

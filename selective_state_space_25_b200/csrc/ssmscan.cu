@@ -421,6 +421,11 @@ ssm_status check_step_args(const char *what, float *ssm_state, const void *x, co
                          {"A", A, np * d_state}, {"D", D, np}, {"dt_bias", dt_bias, np}});
 }
 
+unsigned grid_for(int64_t n) {
+  const int64_t blocks = (n + 255) / 256;
+  return (unsigned)(blocks < 148 * 32 ? (blocks > 0 ? blocks : 1) : 148 * 32);
+}
+
 // ------------------------------------------------------------ SS2D launch
 // Segment length (odd), warps per CTA, and whether dA uses the FMA-pipe exp2.
 #ifndef SSM_SS2D_TS
@@ -437,52 +442,70 @@ constexpr int kSs2dDT = 8;
 constexpr int64_t kSs2dSmemPixels = 6272;
 int64_t ss2d_acc_pixels(int64_t H, int64_t W) { return H * (W | 1); }
 
-template <typename T, bool ACC_SMEM, bool ROW_ASYNC, bool BC_ASYNC, int ORDER>
+// The direction split (ss2d_fwd.cuh, DSPLIT): images whose accumulator fits
+// in shared memory and whose b * ceil(d_in / 8) CTAs would leave more than
+// half of the SMs idle run one CTA per (tile, direction) when the caller's
+// workspace holds the four fp32 direction slices (4, b, H W, d_in).
+bool ss2d_dsplit_applies(int64_t b, int64_t H, int64_t W, int64_t d_in) {
+  return ss2d_acc_pixels(H, W) <= kSs2dSmemPixels && b <= 65535 &&
+         2 * b * ((d_in + kSs2dDT - 1) / kSs2dDT) <= device_sms();
+}
+
+template <typename T, bool ACC_SMEM, bool ROW_ASYNC, bool BC_ASYNC, int ORDER, bool DSPLIT>
 ssm_status launch_ss2d_cfg(const ssm::Ss2dParams &p, cudaStream_t st) {
   using Cfg = ssm::Ss2dCfg<T, SSM_SS2D_TS, SSM_SS2D_WARPS, ACC_SMEM>;
   constexpr auto k = ssm::ss2d_n1_kernel<T, SSM_SS2D_TS, SSM_SS2D_WARPS, ACC_SMEM,
-                                         SSM_SS2D_APOLY != 0, ROW_ASYNC, BC_ASYNC, ORDER>;
+                                         SSM_SS2D_APOLY != 0, ROW_ASYNC, BC_ASYNC, ORDER, DSPLIT>;
   const int smem =
       Cfg::AUX_BYTES + (ACC_SMEM ? (int)(ss2d_acc_pixels(p.H, p.W) * kSs2dDT * sizeof(float)) : 0);
   if (ssm_status s = ensure_smem<k>(Cfg::AUX_BYTES + (int)(kSs2dSmemPixels * kSs2dDT * 4),
                                     "ss2d_scan_fwd"))
     return s;
-  const dim3 grid((unsigned)((p.d_in + kSs2dDT - 1) / kSs2dDT), (unsigned)p.b);
+  const dim3 grid((unsigned)((p.d_in + kSs2dDT - 1) / kSs2dDT), (unsigned)p.b, DSPLIT ? 4u : 1u);
   k<<<grid, Cfg::THREADS, smem, st>>>(p);
-  return check_launch("ss2d_scan_fwd");
+  if (ssm_status s = check_launch("ss2d_scan_fwd")) return s;
+  if constexpr (DSPLIT) {  // sum the four direction slices, round once
+    const int64_t n = p.b * p.H * p.W * p.d_in;
+    const bool vec4 = n % 4 == 0 && aligned(p.acc_global, 16) && aligned(p.y, 4 * sizeof(T));
+    const unsigned blocks = grid_for(vec4 ? n / 4 : n);
+    if (vec4)
+      ssm::ss2d_merge4_kernel<T, true><<<blocks, 256, 0, st>>>(p.acc_global, static_cast<T *>(p.y), n);
+    else
+      ssm::ss2d_merge4_kernel<T, false><<<blocks, 256, 0, st>>>(p.acc_global, static_cast<T *>(p.y), n);
+    return check_launch("ss2d_scan_fwd");
+  }
+  return ok();
 }
 
-template <typename T, bool ACC_SMEM, int ORDER>
+template <typename T, bool ACC_SMEM, int ORDER, bool DSPLIT = false>
 ssm_status launch_ss2d_acc(const ssm::Ss2dParams &p, bool row_async, bool bc_async,
                            cudaStream_t st) {
   if (row_async)
-    return bc_async ? launch_ss2d_cfg<T, ACC_SMEM, true, true, ORDER>(p, st)
-                    : launch_ss2d_cfg<T, ACC_SMEM, true, false, ORDER>(p, st);
-  return bc_async ? launch_ss2d_cfg<T, ACC_SMEM, false, true, ORDER>(p, st)
-                  : launch_ss2d_cfg<T, ACC_SMEM, false, false, ORDER>(p, st);
+    return bc_async ? launch_ss2d_cfg<T, ACC_SMEM, true, true, ORDER, DSPLIT>(p, st)
+                    : launch_ss2d_cfg<T, ACC_SMEM, true, false, ORDER, DSPLIT>(p, st);
+  return bc_async ? launch_ss2d_cfg<T, ACC_SMEM, false, true, ORDER, DSPLIT>(p, st)
+                  : launch_ss2d_cfg<T, ACC_SMEM, false, false, ORDER, DSPLIT>(p, st);
 }
 
 template <typename T, int ORDER>
-ssm_status launch_ss2d_order(const ssm::Ss2dParams &p, cudaStream_t st) {
+ssm_status launch_ss2d_order(const ssm::Ss2dParams &p, bool dsplit, cudaStream_t st) {
   const int64_t L = p.H * p.W;
   const size_t es = sizeof(T);
   const bool row_async = (p.d_in % kSs2dDT) == 0 && aligned(p.u, 16) && aligned(p.delta, 16);
   const bool bc_async = (L * (int64_t)es) % 16 == 0 && aligned(p.B, 16) && aligned(p.C, 16);
+  if (dsplit) return launch_ss2d_acc<T, true, ORDER, true>(p, row_async, bc_async, st);
   if (ss2d_acc_pixels(p.H, p.W) <= kSs2dSmemPixels)
     return launch_ss2d_acc<T, true, ORDER>(p, row_async, bc_async, st);
   return launch_ss2d_acc<T, false, ORDER>(p, row_async, bc_async, st);
 }
 
 template <typename T>
-ssm_status launch_ss2d(const ssm::Ss2dParams &p, ssm_ss2d_order order, cudaStream_t st) {
-  return order == SSM_SS2D_SNAKE ? launch_ss2d_order<T, ssm::kOrderSnake>(p, st)
-                                 : launch_ss2d_order<T, ssm::kOrderCross>(p, st);
+ssm_status launch_ss2d(const ssm::Ss2dParams &p, ssm_ss2d_order order, bool dsplit,
+                       cudaStream_t st) {
+  return order == SSM_SS2D_SNAKE ? launch_ss2d_order<T, ssm::kOrderSnake>(p, dsplit, st)
+                                 : launch_ss2d_order<T, ssm::kOrderCross>(p, dsplit, st);
 }
 
-unsigned grid_for(int64_t n) {
-  const int64_t blocks = (n + 255) / 256;
-  return (unsigned)(blocks < 148 * 32 ? (blocks > 0 ? blocks : 1) : 148 * 32);
-}
 
 // ------------------------------------------------------------ backward scan
 // States per thread of the backward kernel for d_state >= 4.
@@ -822,6 +845,13 @@ size_t ss2d_scan_fwd_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_
   return (size_t)(b * L * d_in) * sizeof(float);
 }
 
+size_t ss2d_scan_fwd_fast_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_in,
+                                          int64_t d_state) {
+  const size_t need = ss2d_scan_fwd_workspace_bytes(b, H, W, d_in, d_state);
+  if (need == (size_t)-1 || d_state != 1 || !ss2d_dsplit_applies(b, H, W, d_in)) return need;
+  return (size_t)(4 * b * H * W * d_in) * sizeof(float);  // overflow excluded by the check above
+}
+
 ssm_status ss2d_scan_fwd(const void *u, const void *delta, const float *A, const void *B,
                          const void *C, const float *D, const float *dt_bias, int delta_softplus,
                          void *y, int64_t b, int64_t H, int64_t W, int64_t d_in, int64_t d_state,
@@ -868,10 +898,14 @@ ssm_status ss2d_scan_fwd_ex(const void *u, const void *delta, const float *A, co
   for (const void *q : f32)
     if (q && !aligned(q, 4))
       return fail(SSM_ERR_INVALID_ARG, "ss2d_scan_fwd: fp32 pointer not 4-byte aligned");
+  // the direction split when the workspace holds its four fp32 slices
+  const size_t fast = ss2d_scan_fwd_fast_workspace_bytes(b, H, W, d_in, d_state);
+  const bool dsplit = fast > need && workspace && workspace_bytes >= fast;
+  const size_t used = dsplit ? fast : need;
   {
     const int64_t by = b * L * d_in * (int64_t)es, bk = 4 * by, bbc = b * 4 * L * d_state * (int64_t)es;
     if (ssm_status s = check_disjoint(
-            "ss2d_scan_fwd", {{"y", y, by}, {"workspace", workspace, (int64_t)need}},
+            "ss2d_scan_fwd", {{"y", y, by}, {"workspace", workspace, (int64_t)used}},
             {{"u", u, by}, {"delta", delta, bk}, {"B", B, bbc}, {"C", C, bbc},
              {"A", A, 4 * d_in * d_state * 4}, {"D", D, 4 * d_in * 4},
              {"dt_bias", dt_bias, 4 * d_in * 4}}))
@@ -881,8 +915,8 @@ ssm_status ss2d_scan_fwd_ex(const void *u, const void *delta, const float *A, co
   ssm::Ss2dParams p{u, delta, A, B, C, D, dt_bias, y, static_cast<float *>(workspace),
                     b, H, W, d_in, delta_softplus};
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype == SSM_BF16) return launch_ss2d<__nv_bfloat16>(p, order, st);
-  return launch_ss2d<float>(p, order, st);
+  if (dtype == SSM_BF16) return launch_ss2d<__nv_bfloat16>(p, order, dsplit, st);
+  return launch_ss2d<float>(p, order, dsplit, st);
 }
 
 ssm_status ssm_state_update(float *ssm_state, const void *x, const void *dt, const float *A,

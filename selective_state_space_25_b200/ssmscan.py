@@ -57,6 +57,8 @@ _lib.ssm_scan_bwd_saved.argtypes = ([_P] * 8 + [_INT] + [_P] * 11 + [_I64] * 4
 _lib.ssm_scan_bwd_saved.restype = _INT
 _lib.ss2d_scan_fwd_workspace_bytes.argtypes = [_I64] * 5
 _lib.ss2d_scan_fwd_workspace_bytes.restype = _SZ
+_lib.ss2d_scan_fwd_fast_workspace_bytes.argtypes = [_I64] * 5
+_lib.ss2d_scan_fwd_fast_workspace_bytes.restype = _SZ
 _lib.ss2d_scan_fwd.argtypes = [_P] * 7 + [_INT, _P] + [_I64] * 5 + [_INT, _P, _SZ, _P]
 _lib.ss2d_scan_fwd.restype = _INT
 _lib.ssm_state_update.argtypes = [_P] * 9 + [_INT, _P] + [_I64] * 3 + [_INT, _P]
@@ -268,11 +270,16 @@ def ss2d_scan_fwd_workspace_bytes(b: int, H: int, W: int, d_in: int, d_state: in
     return int(_lib.ss2d_scan_fwd_workspace_bytes(b, H, W, d_in, d_state))
 
 
+def ss2d_scan_fwd_fast_workspace_bytes(b: int, H: int, W: int, d_in: int, d_state: int) -> int:
+    return int(_lib.ss2d_scan_fwd_fast_workspace_bytes(b, H, W, d_in, d_state))
+
+
 def ss2d_scan_fwd(u, delta, A, B, C, H, W, D=None, dt_bias=None, delta_softplus=True, y=None,
                   workspace=None, stream=None, order="cross"):
     """SS2D forward.  u: (b, H W, d_in); delta: (b, 4, H W, d_in); A: (4 d_in, N)
     fp32; B, C: (b, 4, H W, N); D, dt_bias: (4 d_in,) fp32; order "cross" or
-    "snake".  Returns y (b, H W, d_in)."""
+    "snake".  Returns y (b, H W, d_in).  Without a ``workspace`` the binding
+    allocates the one that lets the call take its fastest path."""
     b, L, d_in = u.shape
     N = A.shape[-1]
     if L != H * W:
@@ -288,7 +295,7 @@ def ss2d_scan_fwd(u, delta, A, B, C, H, W, D=None, dt_bias=None, delta_softplus=
     if y is None:
         y = torch.empty_like(u)
     _need(y, "y", (b, L, d_in), act, dev)
-    ws_bytes = ss2d_scan_fwd_workspace_bytes(b, H, W, d_in, N)
+    ws_bytes = ss2d_scan_fwd_fast_workspace_bytes(b, H, W, d_in, N)
     if workspace is None and ws_bytes > 0:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     st = _lib.ss2d_scan_fwd_ex(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),

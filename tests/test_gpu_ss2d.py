@@ -263,3 +263,29 @@ def test_fused_ss2d_permutation_bit_exact(ssm, order, dtype, b, H, W, d_in):
                            delta_softplus=False, order=order)
     expect = torch.from_numpy(np.asarray(ref)).to(y.dtype)
     assert torch.equal(y.cpu(), expect)
+
+
+@pytest.mark.parametrize("order", ["cross", "snake"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("b,H,W,d_in", [
+    (1, 56, 56, 192),  # batch 1 of the VMamba shape: 24 tiles
+    (2, 7, 9, 24), (1, 13, 11, 13), (1, 1, 37, 16), (1, 37, 1, 16), (3, 17, 5, 40),
+])
+def test_direction_split_is_bit_identical(ssm, order, dtype, b, H, W, d_in):
+    """Small batches with the fast workspace run one CTA per (tile, direction)
+    and sum the four fp32 direction outputs in a second kernel; with no
+    workspace the same call runs the single kernel.  Same operations in the
+    same order: the outputs agree bit for bit (and with the oracle)."""
+    fast = ssm.ss2d_scan_fwd_fast_workspace_bytes(b, H, W, d_in, 1)
+    assert ssm.ss2d_scan_fwd_workspace_bytes(b, H, W, d_in, 1) == 0
+    assert fast == 4 * b * H * W * d_in * 4, "these shapes should take the direction split"
+    inp = ss2d_inputs(b, H, W, d_in, 1, dtype, seed=H * 7 + W + d_in, with_dt_bias=True)
+    g = to_cuda(inp)
+    run = lambda ws: ssm.ss2d_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], H, W,
+                                       D=g["D"], dt_bias=g["dt_bias"], order=order, workspace=ws)
+    y_split = run(torch.empty(fast, dtype=torch.uint8, device="cuda"))
+    y_one = run(torch.empty(0, dtype=torch.uint8, device="cuda"))
+    assert torch.equal(y_split, y_one)
+    ref = oracle.ss2d_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], H, W,
+                           D=inp["D"], dt_bias=inp["dt_bias"], order=order)
+    assert rel_err(y_split, ref) <= TOL[torch.bfloat16 if dtype == "bf16" else torch.float32]
