@@ -245,8 +245,8 @@ ssm_status ssm_scan_bwd_saved(const void *u, const void *delta, const float *A,
  *                 call may take the direction split (below); with less it
  *                 runs the single-kernel path.  Same results either way.
  * Batches too small to fill the GPU (b * ceil(d_in / 8) tiles at most half
- * the SMs, accumulator in shared memory) take the direction split when the
- * workspace allows: one CTA per (tile, direction), each storing its
+ * the SMs) take the direction split when the workspace allows: one CTA per
+ * (tile, direction), each storing its
  * direction's fp32 outputs in the workspace, then a second kernel that sums
  * them k0 + k1 + k2 + k3 and rounds once -- the single kernel's arithmetic in
  * its order, so the results are bit-identical.

@@ -161,11 +161,13 @@ __device__ __forceinline__ void ss2d_pos(int k, int l, int H, int W, float invH,
 // and 16-byte aligned u, delta); otherwise with plain bounds-checked loads.
 // BC_ASYNC: B / C staged with cp.async (needs H W a multiple of 16 / sizeof(T)
 // and 16-byte aligned B, C); otherwise read from global memory per step.
-// DSPLIT (shared accumulator only): the CTA runs direction blockIdx.z alone
-// and stores that direction's fp32 outputs, pixel-major, in slice z of the
-// caller's workspace (4, b, H W, d_in); ss2d_merge4_kernel then sums the four
-// slices k0 + k1 + k2 + k3 and rounds once -- the fused kernel's operations
-// in its order, for grids too small to fill the GPU one CTA per tile.
+// DSPLIT: the CTA runs direction blockIdx.z alone and leaves that
+// direction's fp32 outputs, pixel-major, in slice z of the caller's
+// workspace (4, b, H W, d_in) -- from its shared accumulator at the end, or
+// directly when the accumulator lives in the workspace; ss2d_merge4_kernel
+// then sums the four slices k0 + k1 + k2 + k3 and rounds once -- the fused
+// kernel's operations in its order, for grids too small to fill the GPU one
+// CTA per tile.
 template <typename T, int TS, int WARPS, bool ACC_SMEM, bool A_POLY, bool ROW_ASYNC,
           bool BC_ASYNC, int ORDER, bool DSPLIT = false>
 __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
@@ -205,7 +207,8 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
   const T *gC = static_cast<const T *>(p.C) + ib * 4 * L;
   T *gy = static_cast<T *>(p.y) + ib * L * d_in + d0;
 
-  float *acc_g = p.acc_global + ib * L * d_in + d0;  // this image, channel d0
+  // this image, channel d0 (with DSPLIT in the slice of direction blockIdx.z)
+  float *acc_g = p.acc_global + ((DSPLIT ? (int64_t)blockIdx.z * p.b : 0) + ib) * L * d_in + d0;
   // a channel pair is one 8-byte access: always in shared memory; in the
   // caller's workspace only for even d_in and an 8-byte aligned workspace
   const bool acc_pairs =
@@ -214,7 +217,6 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
   const bool whole_tile = d0 + DT <= d_in && acc_pairs;
 
   const int nchunks = (Li + LC - 1) / LC;
-  static_assert(!DSPLIT || ACC_SMEM, "the direction split keeps its accumulator in shared memory");
   const int kz = DSPLIT ? (int)blockIdx.z : 0;  // the direction (DSPLIT), else the first one
 
   // stage the delta / u rows (and B / C) of this warp's steps of chunk c of
@@ -477,7 +479,9 @@ __global__ void __launch_bounds__(Ss2dCfg<T, TS, WARPS>::THREADS)
   }
   __syncthreads();
 
-  if constexpr (DSPLIT) {
+  if constexpr (DSPLIT && !ACC_SMEM) {
+    return;  // the replay wrote this direction's slice
+  } else if constexpr (DSPLIT) {
     // ---- this direction's fp32 outputs, pixel-major, into workspace slice kz
     float *part = p.acc_global + ((int64_t)kz * p.b + ib) * L * d_in + d0;
     const int64_t n_part = 4 * p.b * L * d_in;

@@ -442,13 +442,12 @@ constexpr int kSs2dDT = 8;
 constexpr int64_t kSs2dSmemPixels = 6272;
 int64_t ss2d_acc_pixels(int64_t H, int64_t W) { return H * (W | 1); }
 
-// The direction split (ss2d_fwd.cuh, DSPLIT): images whose accumulator fits
-// in shared memory and whose b * ceil(d_in / 8) CTAs would leave more than
-// half of the SMs idle run one CTA per (tile, direction) when the caller's
-// workspace holds the four fp32 direction slices (4, b, H W, d_in).
-bool ss2d_dsplit_applies(int64_t b, int64_t H, int64_t W, int64_t d_in) {
-  return ss2d_acc_pixels(H, W) <= kSs2dSmemPixels && b <= 65535 &&
-         2 * b * ((d_in + kSs2dDT - 1) / kSs2dDT) <= device_sms();
+// The direction split (ss2d_fwd.cuh, DSPLIT): problems whose b * ceil(d_in / 8)
+// CTAs would leave more than half of the SMs idle run one CTA per (tile,
+// direction) when the caller's workspace holds the four fp32 direction
+// slices (4, b, H W, d_in).
+bool ss2d_dsplit_applies(int64_t b, int64_t d_in) {
+  return b <= 65535 && 2 * b * ((d_in + kSs2dDT - 1) / kSs2dDT) <= device_sms();
 }
 
 template <typename T, bool ACC_SMEM, bool ROW_ASYNC, bool BC_ASYNC, int ORDER, bool DSPLIT>
@@ -493,10 +492,11 @@ ssm_status launch_ss2d_order(const ssm::Ss2dParams &p, bool dsplit, cudaStream_t
   const size_t es = sizeof(T);
   const bool row_async = (p.d_in % kSs2dDT) == 0 && aligned(p.u, 16) && aligned(p.delta, 16);
   const bool bc_async = (L * (int64_t)es) % 16 == 0 && aligned(p.B, 16) && aligned(p.C, 16);
-  if (dsplit) return launch_ss2d_acc<T, true, ORDER, true>(p, row_async, bc_async, st);
   if (ss2d_acc_pixels(p.H, p.W) <= kSs2dSmemPixels)
-    return launch_ss2d_acc<T, true, ORDER>(p, row_async, bc_async, st);
-  return launch_ss2d_acc<T, false, ORDER>(p, row_async, bc_async, st);
+    return dsplit ? launch_ss2d_acc<T, true, ORDER, true>(p, row_async, bc_async, st)
+                  : launch_ss2d_acc<T, true, ORDER>(p, row_async, bc_async, st);
+  return dsplit ? launch_ss2d_acc<T, false, ORDER, true>(p, row_async, bc_async, st)
+                : launch_ss2d_acc<T, false, ORDER>(p, row_async, bc_async, st);
 }
 
 template <typename T>
@@ -848,7 +848,7 @@ size_t ss2d_scan_fwd_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_
 size_t ss2d_scan_fwd_fast_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_in,
                                           int64_t d_state) {
   const size_t need = ss2d_scan_fwd_workspace_bytes(b, H, W, d_in, d_state);
-  if (need == (size_t)-1 || d_state != 1 || !ss2d_dsplit_applies(b, H, W, d_in)) return need;
+  if (need == (size_t)-1 || d_state != 1 || !ss2d_dsplit_applies(b, d_in)) return need;
   return (size_t)(4 * b * H * W * d_in) * sizeof(float);  // overflow excluded by the check above
 }
 

@@ -87,11 +87,13 @@ def test_workspace_query():
     assert S.ss2d_scan_fwd_workspace_bytes(32, 56, 56, 192, 1) == 0
     big = S.ss2d_scan_fwd_workspace_bytes(2, 100, 100, 16, 1)
     assert big == 2 * 100 * 100 * 16 * 4
-    # the direction split's four fp32 slices: small batches of images whose
-    # accumulator fits in shared memory; otherwise the minimum
+    # the direction split's four fp32 slices for small batches; otherwise the
+    # minimum
     assert S.ss2d_scan_fwd_fast_workspace_bytes(1, 56, 56, 192, 1) == 4 * 56 * 56 * 192 * 4
     assert S.ss2d_scan_fwd_fast_workspace_bytes(32, 56, 56, 192, 1) == 0
-    assert S.ss2d_scan_fwd_fast_workspace_bytes(2, 100, 100, 16, 1) == big
+    assert S.ss2d_scan_fwd_fast_workspace_bytes(2, 100, 100, 16, 1) == 4 * big
+    assert S.ss2d_scan_fwd_fast_workspace_bytes(80, 100, 100, 16, 1) == \
+        S.ss2d_scan_fwd_workspace_bytes(80, 100, 100, 16, 1)
     assert L.ss2d_scan_fwd_fast_workspace_bytes(-1, 2, 2, 8, 1) == ctypes.c_size_t(-1).value
 
 
