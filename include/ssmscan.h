@@ -244,8 +244,9 @@ ssm_status ssm_scan_bwd_saved(const void *u, const void *delta, const float *A,
  *                 ss2d_scan_fwd_fast_workspace_bytes(...) bytes or more the
  *                 call may take the direction split (below); with less it
  *                 runs the single-kernel path.  Same results either way.
- * Batches too small to fill the GPU (b * ceil(d_in / 8) tiles at most half
- * the SMs) take the direction split when the workspace allows: one CTA per
+ * Images whose accumulator would live in the workspace, and batches too
+ * small to fill the GPU (b * ceil(d_in / 8) tiles at most half the SMs),
+ * take the direction split when the workspace allows: one CTA per
  * (tile, direction), each storing its
  * direction's fp32 outputs in the workspace, then a second kernel that sums
  * them k0 + k1 + k2 + k3 and rounds once -- the single kernel's arithmetic in
@@ -293,9 +294,9 @@ size_t ss2d_scan_fwd_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_
 /*
  * Bytes of device workspace with which ss2d_scan_fwd takes its fastest path
  * for this problem: 4 * b * H * W * d_in fp32 (the direction split's four
- * slices) when the direction split applies, else the same value as
- * ss2d_scan_fwd_workspace_bytes.  Never less than that minimum; (size_t)-1
- * for invalid sizes.
+ * slices) when the direction split applies (large images, small batches),
+ * else the same value as ss2d_scan_fwd_workspace_bytes.  Never less than
+ * that minimum; (size_t)-1 for invalid sizes.
  */
 size_t ss2d_scan_fwd_fast_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_in,
                                           int64_t d_state);

@@ -442,12 +442,16 @@ constexpr int kSs2dDT = 8;
 constexpr int64_t kSs2dSmemPixels = 6272;
 int64_t ss2d_acc_pixels(int64_t H, int64_t W) { return H * (W | 1); }
 
-// The direction split (ss2d_fwd.cuh, DSPLIT): problems whose b * ceil(d_in / 8)
-// CTAs would leave more than half of the SMs idle run one CTA per (tile,
+// The direction split (ss2d_fwd.cuh, DSPLIT) runs one CTA per (tile,
 // direction) when the caller's workspace holds the four fp32 direction
-// slices (4, b, H W, d_in).
-bool ss2d_dsplit_applies(int64_t b, int64_t d_in) {
-  return b <= 65535 && 2 * b * ((d_in + kSs2dDT - 1) / kSs2dDT) <= device_sms();
+// slices (4, b, H W, d_in): for images whose accumulator would live in the
+// workspace (the slices are only written, where that accumulator takes a
+// read-modify-write per direction on the replay's path: 2.7-6.5x faster at
+// 112 x 112), and for problems whose b * ceil(d_in / 8) CTAs would leave
+// more than half of the SMs idle.
+bool ss2d_dsplit_applies(int64_t b, int64_t H, int64_t W, int64_t d_in) {
+  return b <= 65535 && (ss2d_acc_pixels(H, W) > kSs2dSmemPixels ||
+                        2 * b * ((d_in + kSs2dDT - 1) / kSs2dDT) <= device_sms());
 }
 
 template <typename T, bool ACC_SMEM, bool ROW_ASYNC, bool BC_ASYNC, int ORDER, bool DSPLIT>
@@ -848,7 +852,7 @@ size_t ss2d_scan_fwd_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_
 size_t ss2d_scan_fwd_fast_workspace_bytes(int64_t b, int64_t H, int64_t W, int64_t d_in,
                                           int64_t d_state) {
   const size_t need = ss2d_scan_fwd_workspace_bytes(b, H, W, d_in, d_state);
-  if (need == (size_t)-1 || d_state != 1 || !ss2d_dsplit_applies(b, d_in)) return need;
+  if (need == (size_t)-1 || d_state != 1 || !ss2d_dsplit_applies(b, H, W, d_in)) return need;
   return (size_t)(4 * b * H * W * d_in) * sizeof(float);  // overflow excluded by the check above
 }
 

@@ -92,8 +92,10 @@ def test_workspace_query():
     assert S.ss2d_scan_fwd_fast_workspace_bytes(1, 56, 56, 192, 1) == 4 * 56 * 56 * 192 * 4
     assert S.ss2d_scan_fwd_fast_workspace_bytes(32, 56, 56, 192, 1) == 0
     assert S.ss2d_scan_fwd_fast_workspace_bytes(2, 100, 100, 16, 1) == 4 * big
+    # large images take the split at any batch; small ones only at small batch
     assert S.ss2d_scan_fwd_fast_workspace_bytes(80, 100, 100, 16, 1) == \
-        S.ss2d_scan_fwd_workspace_bytes(80, 100, 100, 16, 1)
+        4 * S.ss2d_scan_fwd_workspace_bytes(80, 100, 100, 16, 1)
+    assert S.ss2d_scan_fwd_fast_workspace_bytes(80, 56, 56, 16, 1) == 0
     assert L.ss2d_scan_fwd_fast_workspace_bytes(-1, 2, 2, 8, 1) == ctypes.c_size_t(-1).value
 
 

@@ -272,12 +272,14 @@ def test_fused_ss2d_permutation_bit_exact(ssm, order, dtype, b, H, W, d_in):
     (2, 7, 9, 24), (1, 13, 11, 13), (1, 1, 37, 16), (1, 37, 1, 16), (3, 17, 5, 40),
     (1, 100, 100, 16),  # accumulator in the workspace
     (1, 80, 81, 13),    # ... with odd d_in (channel pairs as two 4-byte accesses)
+    (80, 80, 81, 8),    # ... and a batch that fills the GPU (80 tiles)
 ])
 def test_direction_split_is_bit_identical(ssm, order, dtype, b, H, W, d_in):
-    """Small batches with the fast workspace run one CTA per (tile, direction)
-    and sum the four fp32 direction outputs in a second kernel; with the
-    minimum workspace the same call runs the single kernel.  Same operations
-    in the same order: the outputs agree bit for bit (and with the oracle)."""
+    """Small batches and large images with the fast workspace run one CTA per
+    (tile, direction) and sum the four fp32 direction outputs in a second
+    kernel; with the minimum workspace the same call runs the single kernel.
+    Same operations in the same order: the outputs agree bit for bit (and
+    with the oracle)."""
     fast = ssm.ss2d_scan_fwd_fast_workspace_bytes(b, H, W, d_in, 1)
     least = ssm.ss2d_scan_fwd_workspace_bytes(b, H, W, d_in, 1)
     assert fast == 4 * b * H * W * d_in * 4, "these shapes should take the direction split"
