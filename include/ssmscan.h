@@ -231,8 +231,9 @@ ssm_status ssm_scan_bwd_saved(const void *u, const void *delta, const float *A,
  * u[i, p_k(l), :] with its own delta/B/C (given in its scan order) and the
  * rows k*d_in .. k*d_in + d_in - 1 of A, D, dt_bias, with no gate and a zero
  * start; the output is y[i,p,d] = sum_k y_k at pixel p (fp32 sum, one
- * rounding).  The four orders are index arithmetic: no permuted copy of u
- * and no per-direction output is stored.
+ * rounding).  The four orders are index arithmetic: no permuted copy of u is
+ * stored, and per-direction outputs only by the direction split (below), in
+ * the workspace.
  *
  *   u, y          device, (b, H W, d_in), dtype
  *   delta         device, (b, 4, H W, d_in), dtype

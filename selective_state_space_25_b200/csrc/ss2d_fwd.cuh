@@ -7,8 +7,9 @@
 //   k0 row-major p = l; k1 column-major l = w H + h; k2 = k0 reversed;
 //   k3 = k1 reversed.
 // The orders are index arithmetic: u is gathered at p_k(l) when it is read
-// and each output lands at p_k(l) when it is produced; no permuted copy and
-// no per-direction output exists in memory.
+// and each output lands at p_k(l) when it is produced; no permuted copy
+// exists in memory, and per-direction outputs only in the direction split
+// (DSPLIT below), as fp32 slices of the caller's workspace.
 #pragma once
 
 #include <type_traits>
