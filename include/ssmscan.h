@@ -162,6 +162,20 @@ ssm_status ssm_scan_fwd_save(const void *u, const void *delta, const float *A,
 size_t ssm_scan_bwd_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t d_state);
 
 /*
+ * Workspace with which ssm_scan_bwd takes its fastest path: for d_state 8,
+ * 16 or 32 when b * ceil(d_in / channels per CTA) backward blocks would leave
+ * more than half of the SMs idle, the chunk states followed by the split
+ * backward's block buffers (the forward split's block decays and states, the
+ * adjoint's block maps); otherwise ssm_scan_bwd_workspace_bytes.  With that
+ * much (16-byte aligned) ssm_scan_bwd cuts the sequence into blocks: the
+ * chunk-start states from the forward's split scan, each block's adjoint map
+ * composed from dh_last by the carry scan, every block's backward at once.
+ * With less it runs unsplit; the gradients agree within rounding (sums are
+ * taken in a different order).  ssm_scan_bwd_saved always runs unsplit.
+ */
+size_t ssm_scan_bwd_fast_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t d_state);
+
+/*
  * Selective scan backward: the gradients of
  *     loss = sum dout[i,t,d] out[i,t,d] + sum dh_last[i,d,n] h_last[i,d,n]
  * for the forward of ssm_scan_fwd with the same inputs, by the chain rule

@@ -55,6 +55,12 @@ struct BwdParams {
   int softplus;
   int vec_atomics;   // dB and dC 16-byte aligned: float4 atomics
   int states_saved;  // chunk_h already holds the chunk-start states (saved by the forward)
+  // Split backward (few channels): grid z-index k walks chunks
+  // [k Cb, min(nC, (k + 1) Cb)) from the adjoint lam_in holds for it
+  // (scan_bwd_adjoint_kernel + scan_carry_kernel); Cb = 0 means one block.
+  // Needs states_saved.
+  int64_t Cb = 0;
+  const float *lam_in = nullptr;  // (b, nblk, d_in, N): block k's start at slot nblk - 2 - k
 };
 
 template <typename T, int N, int NPT_>
@@ -184,6 +190,11 @@ __global__ void __launch_bounds__(128, 3) scan_bwd_kernel(BwdParams p) {
   const bool active = d < p.d_in;
   const int64_t L = p.L, d_in = p.d_in;
   const int nC = (int)((L + TT - 1) / TT);
+  // this CTA's chunks [c_begin, c_end) (all of them without the split)
+  const int blk = (int)blockIdx.z;
+  const int nblk = p.Cb > 0 ? (int)((nC + p.Cb - 1) / p.Cb) : 1;
+  const int c_begin = p.Cb > 0 ? blk * (int)p.Cb : 0;
+  const int c_end = p.Cb > 0 && c_begin + p.Cb < nC ? c_begin + (int)p.Cb : nC;
   const T *gu = static_cast<const T *>(p.u);
   const T *gdelta = static_cast<const T *>(p.delta);
   const T *gB = static_cast<const T *>(p.B);
@@ -344,7 +355,7 @@ __global__ void __launch_bounds__(128, 3) scan_bwd_kernel(BwdParams p) {
     h[j] = (active && p.h0) ? p.h0[(ib * d_in + d) * N + g * NPT + j] : 0.0f;
   if constexpr (ASYNC) {
     // chunks 0 .. nC-2 (partial input), then the first chunk of pass 2 (full)
-    if (n_pass1 >= 2) issue(0, false, 0); else issue(nC - 1, true, (nC - 1) & 1);
+    if (n_pass1 >= 2) issue(0, false, 0); else issue(c_end - 1, true, (c_end - 1) & 1);
     cp_async_commit();
   }
   for (int c = 0; c < n_pass1; ++c) {
@@ -367,7 +378,12 @@ __global__ void __launch_bounds__(128, 3) scan_bwd_kernel(BwdParams p) {
   float lam[NPT], dAacc[NPT];
 #pragma unroll
   for (int j = 0; j < NPT; ++j) {
-    lam[j] = (active && p.dh_last) ? p.dh_last[(ib * d_in + d) * N + g * NPT + j] : 0.0f;
+    if (blk == nblk - 1) {  // the last block starts from dh_last
+      lam[j] = (active && p.dh_last) ? p.dh_last[(ib * d_in + d) * N + g * NPT + j] : 0.0f;
+    } else {  // an earlier one from the adjoint its right-hand blocks leave
+      const int64_t i = ((ib * nblk + (nblk - 2 - blk)) * d_in + d) * N + g * NPT + j;
+      lam[j] = active && in_bounds(i, p.b * nblk * d_in * N, kBndChunk) ? p.lam_in[i] : 0.0f;
+    }
     dAacc[j] = 0.0f;
   }
   // the per-(step, channel) pass keeps one channel per thread
@@ -432,15 +448,16 @@ __global__ void __launch_bounds__(128, 3) scan_bwd_kernel(BwdParams p) {
   };
 
   float hs_next[NPT];
-  if (active && chunk_ok(nC - 1)) load_vec<NPT>(my_chunk_h + (int64_t)(nC - 1) * d_in * N, hs_next);
-  for (int c = nC - 1; c >= 0; --c) {
+  if (active && chunk_ok(c_end - 1))
+    load_vec<NPT>(my_chunk_h + (int64_t)(c_end - 1) * d_in * N, hs_next);
+  for (int c = c_end - 1; c >= c_begin; --c) {
     float hs[NPT];
 #pragma unroll
     for (int j = 0; j < NPT; ++j) hs[j] = active ? hs_next[j] : 0.0f;
-    if (c > 0 && active && chunk_ok(c - 1))
+    if (c > c_begin && active && chunk_ok(c - 1))
       load_vec<NPT>(my_chunk_h + (int64_t)(c - 1) * d_in * N, hs_next);
     if constexpr (ASYNC) {
-      if (c > 0) issue(c - 1, true, (c - 1) & 1);
+      if (c > c_begin) issue(c - 1, true, (c - 1) & 1);
       cp_async_commit();
       cp_async_wait<1>();
     }
@@ -508,12 +525,72 @@ __global__ void __launch_bounds__(128, 3) scan_bwd_kernel(BwdParams p) {
 #pragma unroll
     for (int j = 0; j < NPT; ++j) {
       atomicAdd(p.dA + d * N + g * NPT + j, dAacc[j]);
-      if (p.dh0) p.dh0[(ib * d_in + d) * N + g * NPT + j] = lam[j];
+      if (p.dh0 && blk == 0) p.dh0[(ib * d_in + d) * N + g * NPT + j] = lam[j];
     }
   }
   if (d0 + pch < d_in) {
     if (p.dD) atomicAdd(p.dD + d0 + pch, Dacc);
     if (p.ddt_bias) atomicAdd(p.ddt_bias + d0 + pch, bias_acc);
+  }
+}
+
+// Adjoint summary of the split backward.  Block k >= 1 of the sequence
+// (chunks [k Cb, min(nC, (k + 1) Cb))) maps the adjoint arriving at its last
+// step, lam_in, to the one leaving its first step: lam_out = M_k lam_in + R_k
+// (per (batch, channel, state)), with M_k = prod_t exp(delta_t A) and R_k the
+// adjoint walked backwards through the block from zero, lam <- (lam + g_t C_t)
+// exp(delta_t A) -- scan_bwd_kernel's adjoint step, g_t = dout_t silu(z_t).
+// M_k and R_k go to slot nblk - 1 - k of (b, nblk, d_in, N) arrays, the order
+// in which scan_carry_kernel composes them from dh_last; the carry then leaves
+// in slot nblk - 2 - k the adjoint block k starts from.  One thread per
+// (batch, block, channel), all N states in registers, lanes over channels.
+template <typename T, int N>
+__global__ void __launch_bounds__(128) scan_bwd_adjoint_kernel(BwdParams p, float *adj_decay,
+                                                               float *adj_state) {
+  const int64_t L = p.L, d_in = p.d_in;
+  const int64_t nC = (L + kStateChunk - 1) / kStateChunk;
+  const int64_t nblk = (nC + p.Cb - 1) / p.Cb;
+  const int64_t blk = (int64_t)blockIdx.y + 1;  // blocks 1 .. nblk - 1
+  const int64_t ib = blockIdx.z;
+  const int64_t d = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (d >= d_in || blk >= nblk) return;
+  const int64_t t_begin = blk * p.Cb * kStateChunk;
+  const int64_t t_end = t_begin + p.Cb * kStateChunk < L ? t_begin + p.Cb * kStateChunk : L;
+  const T *gdelta = static_cast<const T *>(p.delta);
+  const T *gz = static_cast<const T *>(p.z);
+  const T *gdout = static_cast<const T *>(p.dout);
+  const T *gC = static_cast<const T *>(p.C);
+  float A2[N], lam[N];
+#pragma unroll
+  for (int n = 0; n < N; ++n) {
+    A2[n] = in_bounds(d * N + n, d_in * N, kBndParam) ? p.A[d * N + n] * kLog2e : 0.0f;
+    lam[n] = 0.0f;
+  }
+  const float bias = p.dt_bias ? p.dt_bias[d] : 0.0f;
+  float dsum = 0.0f;
+  for (int64_t t = t_end - 1; t >= t_begin; --t) {
+    const int64_t at = (ib * L + t) * d_in + d, ct = (ib * L + t) * N;
+    if (!in_bounds(at, p.b * L * d_in, kBndAct) || !in_bounds(ct + N - 1, p.b * L * N, kBndBC))
+      continue;
+    const float pre = Elem<T>::load(gdelta, at) + bias;
+    const float dl = p.softplus ? softplus_f32(pre) : pre;
+    const float go = Elem<T>::load(gdout, at);
+    float gt = go;
+    if (gz) {
+      const float zz = Elem<T>::load(gz, at);
+      gt = go * zz * rcp_approx(1.0f + ex2_approx(-zz * kLog2e));
+    }
+    dsum += dl;
+#pragma unroll
+    for (int n = 0; n < N; ++n)
+      lam[n] = fmaf(gt, Elem<T>::load(gC, ct + n), lam[n]) * ex2_approx(dl * A2[n]);
+  }
+  const int64_t row = ((ib * nblk + (nblk - 1 - blk)) * d_in + d) * N;
+  if (!in_bounds(row + N - 1, p.b * nblk * d_in * N, kBndChunk)) return;
+#pragma unroll
+  for (int n = 0; n < N; ++n) {
+    adj_state[row + n] = lam[n];
+    adj_decay[row + n] = ex2_approx(dsum * A2[n]);
   }
 }
 

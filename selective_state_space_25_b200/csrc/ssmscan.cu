@@ -520,14 +520,106 @@ ssm_status launch_ss2d(const ssm::Ss2dParams &p, ssm_ss2d_order order, bool dspl
 constexpr int64_t bwd_chunk(int64_t) { return ssm::BwdCfg<float, 16, 4>::TT; }
 
 template <typename T, int N, int NPT, bool ASYNC>
-ssm_status launch_bwd_cfg(const ssm::BwdParams &p, cudaStream_t st) {
+ssm_status launch_bwd_cfg(const ssm::BwdParams &p, unsigned nz, cudaStream_t st) {
   using Cfg = ssm::BwdCfg<T, N, NPT>;
   static_assert(Cfg::TT == bwd_chunk(N), "bwd_chunk must match BwdCfg");
   constexpr auto k = ssm::scan_bwd_kernel<T, N, NPT, ASYNC>;
   if (ssm_status s = ensure_smem<k>((int)Cfg::SMEM, "ssm_scan_bwd")) return s;
-  const dim3 grid((unsigned)((p.d_in + Cfg::DT - 1) / Cfg::DT), (unsigned)p.b);
+  const dim3 grid((unsigned)((p.d_in + Cfg::DT - 1) / Cfg::DT), (unsigned)p.b, nz);
   k<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(p);
   return check_launch("ssm_scan_bwd");
+}
+
+// Split backward (ssm_scan_bwd with the fast workspace, d_state 8, 16, 32):
+// when b * ceil(d_in / channels per CTA) backward CTAs would leave more than
+// half of the SMs idle, the chunks are cut into blocks -- at most two waves
+// of three CTAs per SM, each block at least four chunks.  The chunk-start
+// states come from the forward's split (when it splits) and the adjoint each
+// block starts from from scan_bwd_adjoint_kernel + scan_carry_kernel.
+struct BwdSplitPlan {
+  int64_t nblk = 1, Cb = 0;     // backward blocks of Cb chunks
+  SplitPlan fwd;                // the forward's split for the chunk-start states
+};
+int64_t bwd_channels_per_cta(int64_t N) {
+  return 128 / (N / (N < 4 ? N : SSM_BWD_NPT));
+}
+BwdSplitPlan bwd_split_plan(int64_t b, int64_t L, int64_t d_in, int64_t N) {
+  BwdSplitPlan sp;
+  if (b <= 0 || L <= 0 || d_in <= 0 || !(N == 8 || N == 16 || N == 32)) return sp;
+  const int64_t sms = device_sms();
+  const int64_t ctas = b * ((d_in + bwd_channels_per_cta(N) - 1) / bwd_channels_per_cta(N));
+  if (2 * ctas > sms) return sp;
+  const int64_t nC = (L + bwd_chunk(N) - 1) / bwd_chunk(N);
+  int64_t nblk = 6 * sms / ctas;
+  if (nblk > nC / 4) nblk = nC / 4;
+  if (nblk > 4096) nblk = 4096;
+  if (nblk < 2) return sp;
+  sp.Cb = (nC + nblk - 1) / nblk;
+  sp.nblk = (nC + sp.Cb - 1) / sp.Cb;
+  if (sp.nblk < 2) return BwdSplitPlan{};
+  sp.fwd = split_plan(b, L, d_in, N);
+  return sp;
+}
+// Extra fp32 words of the split after the chunk states: the forward split's
+// block decays and states, then the backward's adjoint maps.
+int64_t bwd_split_words(const BwdSplitPlan &sp, int64_t b, int64_t d_in, int64_t N) {
+  return 2 * b * (sp.fwd.nblk > 1 ? sp.fwd.nblk : 0) * d_in * N + 2 * b * sp.nblk * d_in * N;
+}
+
+template <typename T, int N, int NPT>
+ssm_status launch_bwd_main(const ssm::BwdParams &p, bool async, unsigned nz, cudaStream_t st) {
+  if constexpr (ssm::bwd_async_ok<T, N, NPT>()) {
+    if (async) return launch_bwd_cfg<T, N, NPT, true>(p, nz, st);
+  }
+  return launch_bwd_cfg<T, N, NPT, false>(p, nz, st);
+}
+
+template <typename T, int N>
+ssm_status launch_bwd_split(const ssm::BwdParams &p, bool async, const BwdSplitPlan &sp,
+                            float *extra, cudaStream_t st) {
+  constexpr int NPT = N < 4 ? N : SSM_BWD_NPT;
+  if constexpr (ws_states(N) > 0) {
+    // 1. chunk-start states: the forward's states pass, split like the forward
+    ssm::ScanParams f{p.u, p.delta, p.A, p.B, p.C, nullptr, nullptr, p.dt_bias, p.h0,
+                      nullptr, nullptr, p.b, p.L, p.d_in, p.softplus, p.chunk_h};
+    float *adj = extra;
+    if (sp.fwd.nblk > 1) {
+      f.Lb = sp.fwd.Lb;
+      f.blk_decay = extra;
+      f.blk_state = extra + p.b * sp.fwd.nblk * p.d_in * N;
+      adj = extra + 2 * p.b * sp.fwd.nblk * p.d_in * N;
+      const unsigned nb = (unsigned)sp.fwd.nblk;
+      if (ssm_status s = launch_scan_ws_pass<T, N, false, false, true>(f, nb - 1, st)) return s;
+      if (ssm_status s = launch_dependent(
+              ssm::scan_carry_kernel, dim3((unsigned)((p.d_in * N + 31) / 32), (unsigned)p.b),
+              ssm::kCarryThreads, 0, st, "ssm_scan_bwd", p.h0, f.blk_decay,
+              (const float *)f.blk_state, p.b, (int64_t)nb, p.d_in, (int)N))
+        return s;
+      if (ssm_status s = launch_scan_ws_pass<T, N, false, true, true>(f, nb, st, true)) return s;
+    } else if (ssm_status s = launch_scan_ws_pass<T, N, false, true, true>(f, 1, st)) {
+      return s;
+    }
+    // 2. each block's adjoint map, then the adjoint each block starts from
+    ssm::BwdParams q = p;
+    q.states_saved = 1;
+    q.Cb = sp.Cb;
+    float *adj_decay = adj, *adj_state = adj + p.b * sp.nblk * p.d_in * N;
+    ssm::scan_bwd_adjoint_kernel<T, N>
+        <<<dim3((unsigned)((p.d_in + 127) / 128), (unsigned)(sp.nblk - 1), (unsigned)p.b), 128, 0,
+           st>>>(q, adj_decay, adj_state);
+    if (ssm_status s = check_launch("ssm_scan_bwd")) return s;
+    if (ssm_status s = launch_dependent(
+            ssm::scan_carry_kernel, dim3((unsigned)((p.d_in * N + 31) / 32), (unsigned)p.b),
+            ssm::kCarryThreads, 0, st, "ssm_scan_bwd", p.dh_last, adj_decay,
+            (const float *)adj_state, p.b, sp.nblk, p.d_in, (int)N))
+      return s;
+    // 3. every block's backward at once
+    q.lam_in = adj_decay;
+    return launch_bwd_main<T, N, NPT>(q, async, (unsigned)sp.nblk, st);
+  } else {
+    (void)p; (void)async; (void)sp; (void)extra; (void)st;
+    return fail(SSM_ERR_UNSUPPORTED, "ssm_scan_bwd: no split backward for d_state %d", N);
+  }
 }
 
 template <typename T, int N>
@@ -544,15 +636,27 @@ ssm_status launch_bwd(const ssm::BwdParams &p, bool async, bool fwd_states, cuda
       ssm::BwdParams q = p;
       q.states_saved = 1;
       if constexpr (ssm::bwd_async_ok<T, N, NPT>()) {
-        if (async) return launch_bwd_cfg<T, N, NPT, true>(q, st);
+        if (async) return launch_bwd_cfg<T, N, NPT, true>(q, 1, st);
       }
-      return launch_bwd_cfg<T, N, NPT, false>(q, st);
+      return launch_bwd_cfg<T, N, NPT, false>(q, 1, st);
     }
   }
   if constexpr (ssm::bwd_async_ok<T, N, NPT>()) {
-    if (async) return launch_bwd_cfg<T, N, NPT, true>(p, st);
+    if (async) return launch_bwd_cfg<T, N, NPT, true>(p, 1, st);
   }
-  return launch_bwd_cfg<T, N, NPT, false>(p, st);
+  return launch_bwd_cfg<T, N, NPT, false>(p, 1, st);
+}
+
+template <typename T>
+ssm_status dispatch_bwd_split_n(const ssm::BwdParams &p, int64_t N, bool async,
+                                const BwdSplitPlan &sp, float *extra, cudaStream_t st) {
+  switch (N) {
+    case 8: return launch_bwd_split<T, 8>(p, async, sp, extra, st);
+    case 16: return launch_bwd_split<T, 16>(p, async, sp, extra, st);
+    case 32: return launch_bwd_split<T, 32>(p, async, sp, extra, st);
+  }
+  return fail(SSM_ERR_UNSUPPORTED, "ssm_scan_bwd: no split backward for d_state %lld",
+              (long long)N);
 }
 
 template <typename T>
@@ -714,6 +818,14 @@ size_t ssm_scan_bwd_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t 
   return (size_t)t * sizeof(float);
 }
 
+size_t ssm_scan_bwd_fast_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t d_state) {
+  const size_t need = ssm_scan_bwd_workspace_bytes(b, L, d_in, d_state);
+  if (need == (size_t)-1) return need;
+  const BwdSplitPlan sp = bwd_split_plan(b, L, d_in, d_state);
+  if (sp.nblk < 2) return need;
+  return need + (size_t)bwd_split_words(sp, b, d_in, d_state) * sizeof(float);
+}
+
 }  // extern "C"
 
 namespace {
@@ -760,9 +872,17 @@ ssm_status scan_bwd_impl(const char *what, const void *u, const void *delta, con
   for (const void *q : f32)
     if (q && !aligned(q, 4))
       return fail(SSM_ERR_INVALID_ARG, "%s: fp32 pointer not 4-byte aligned", what);
+  // the forward kernel's states pass needs its own 16-byte staging of u, delta, B
+  const bool fwd_states = (d_in * (int64_t)es) % 16 == 0 && aligned(u, 16) &&
+                          aligned(delta, 16) && aligned(B, 16) && b <= 65535;
+  // the split backward when the workspace holds its block buffers after the
+  // chunk states (ssm_scan_bwd only: the saved-states call has no workspace to spare)
+  const size_t fast = states_saved ? need : ssm_scan_bwd_fast_workspace_bytes(b, L, d_in, d_state);
+  const bool split = !states_saved && fwd_states && fast > need && workspace &&
+                     workspace_bytes >= fast && aligned(workspace, 16);
   {
     const int64_t ba = n_act * (int64_t)es, bbc = n_bc * (int64_t)es, bs = n_state * 4;
-    const int64_t bp = d_in * 4, bA = d_in * d_state * 4, bw = (int64_t)need;
+    const int64_t bp = d_in * 4, bA = d_in * d_state * 4, bw = (int64_t)(split ? fast : need);
     // the saved states are read, not written, in the split mode
     const Span ws{"workspace", states_saved ? nullptr : workspace, bw};
     const Span ws_in{"chunk_states", states_saved ? workspace : nullptr, bw};
@@ -799,9 +919,12 @@ ssm_status scan_bwd_impl(const char *what, const void *u, const void *delta, con
   // the raw-tile prefetch copies 16-byte groups straight from the inputs
   const bool async = (d_in * (int64_t)es) % 16 == 0 && aligned(u, 16) && aligned(delta, 16) &&
                      aligned(dout, 16) && aligned(B, 16) && aligned(C, 16) && (!z || aligned(z, 16));
-  // the forward kernel's states pass needs its own 16-byte staging of u, delta, B
-  const bool fwd_states = (d_in * (int64_t)es) % 16 == 0 && aligned(u, 16) &&
-                          aligned(delta, 16) && aligned(B, 16) && b <= 65535;
+  if (split) {
+    const BwdSplitPlan sp = bwd_split_plan(b, L, d_in, d_state);
+    float *extra = static_cast<float *>(workspace) + need / sizeof(float);
+    if (dtype == SSM_BF16) return dispatch_bwd_split_n<__nv_bfloat16>(p, d_state, async, sp, extra, st);
+    return dispatch_bwd_split_n<float>(p, d_state, async, sp, extra, st);
+  }
   if (dtype == SSM_BF16)
     return dispatch_bwd_n<__nv_bfloat16>(p, d_state, async, fwd_states, st);
   return dispatch_bwd_n<float>(p, d_state, async, fwd_states, st);

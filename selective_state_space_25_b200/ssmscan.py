@@ -48,6 +48,8 @@ _lib.ssm_scan_fwd.argtypes = [_P] * 8 + [_INT, _P, _P, _P] + [_I64] * 4 + [_INT,
 _lib.ssm_scan_fwd.restype = _INT
 _lib.ssm_scan_bwd_workspace_bytes.argtypes = [_I64] * 4
 _lib.ssm_scan_bwd_workspace_bytes.restype = _SZ
+_lib.ssm_scan_bwd_fast_workspace_bytes.argtypes = [_I64] * 4
+_lib.ssm_scan_bwd_fast_workspace_bytes.restype = _SZ
 _lib.ssm_scan_bwd.argtypes = [_P] * 8 + [_INT] + [_P] * 12 + [_I64] * 4 + [_INT, _P, _SZ, _P]
 _lib.ssm_scan_bwd.restype = _INT
 _lib.ssm_scan_fwd_save.argtypes = [_P] * 8 + [_INT, _P, _P, _P, _P, _SZ] + [_I64] * 4 + [_INT, _P]
@@ -202,6 +204,10 @@ def ssm_scan_bwd_workspace_bytes(b: int, L: int, d_in: int, d_state: int) -> int
     return int(_lib.ssm_scan_bwd_workspace_bytes(b, L, d_in, d_state))
 
 
+def ssm_scan_bwd_fast_workspace_bytes(b: int, L: int, d_in: int, d_state: int) -> int:
+    return int(_lib.ssm_scan_bwd_fast_workspace_bytes(b, L, d_in, d_state))
+
+
 def ssm_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_softplus=True,
                  h0=None, dh_last=None, want_dh0=False, workspace=None, stream=None, out=None,
                  states=None):
@@ -252,7 +258,7 @@ def ssm_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_so
             _ptr(states), states.numel() * states.element_size(), _stream(stream))
         _check(st, "ssm_scan_bwd_saved")
         return {k: v for k, v in g.items() if v is not None}
-    need = ssm_scan_bwd_workspace_bytes(b, L, d_in, N)
+    need = ssm_scan_bwd_fast_workspace_bytes(b, L, d_in, N)  # the fastest path's
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
     ws_bytes = workspace.numel() * workspace.element_size()

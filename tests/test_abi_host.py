@@ -230,6 +230,14 @@ def test_bwd_validation(saved, kw, status):
 
 def test_bwd_workspace_query():
     assert S.ssm_scan_bwd_workspace_bytes(8, 2048, 1536, 16) == 8 * 128 * 1536 * 16 * 4
+    # the split backward's block buffers follow the chunk states for few
+    # channels; a shape that fills the GPU runs unsplit
+    assert S.ssm_scan_bwd_fast_workspace_bytes(8, 2048, 1536, 16) == 8 * 128 * 1536 * 16 * 4
+    need = S.ssm_scan_bwd_workspace_bytes(1, 16384, 256, 16)
+    assert S.ssm_scan_bwd_fast_workspace_bytes(1, 16384, 256, 16) > need
+    assert S.ssm_scan_bwd_fast_workspace_bytes(1, 16384, 256, 4) == \
+        S.ssm_scan_bwd_workspace_bytes(1, 16384, 256, 4)      # d_state 4: no split
+    assert L.ssm_scan_bwd_fast_workspace_bytes(-1, 1, 1, 16) == ctypes.c_size_t(-1).value
     assert S.ssm_scan_bwd_workspace_bytes(1, 17, 3, 4) == 1 * 2 * 3 * 4 * 4   # ceil(17 / 16) chunks
     assert L.ssm_scan_bwd_workspace_bytes(1, 1, 1, 3) == ctypes.c_size_t(-1).value
 

@@ -209,7 +209,11 @@ def test_bwd_saved_equals_self_contained(ssm, dtype):
     ssm.ssm_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], D=g["D"], z=g["z"],
                      dt_bias=g["dt_bias"], h0=g["h0"], chunk_states=states)
     kw = dict(D=g["D"], z=g["z"], dt_bias=g["dt_bias"], dh_last=dhl, want_dh0=True)
-    full = ssm.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], dout, h0=g["h0"], **kw)
+    # the minimum workspace: the unsplit backward, the saved call's arithmetic
+    least = torch.empty(ssm.ssm_scan_bwd_workspace_bytes(b, L, d_in, N), dtype=torch.uint8,
+                        device="cuda")
+    full = ssm.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], dout, h0=g["h0"],
+                            workspace=least, **kw)
     saved = ssm.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], dout, states=states, **kw)
     for k in full:
         assert rel_err(saved[k], to64(full[k])) <= 1e-5, k
@@ -222,3 +226,41 @@ def test_fwd_save_rejects_small_buffer(ssm):
     states = torch.empty(ssm.ssm_scan_bwd_workspace_bytes(1, 40, 16, 16) // 4 - 1, device="cuda")
     with pytest.raises(ssm.SsmError, match="chunk_states"):
         ssm.ssm_scan_fwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], chunk_states=states)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("b,L,d_in,N,with_z", [
+    (1, 4096, 64, 16, True),   # 256 chunks in blocks; the forward's states pass split too
+    (2, 1000, 32, 8, True),    # ragged last chunk and block
+    (1, 777, 48, 32, False),   # no gate
+    (1, 300, 64, 16, True),    # few blocks (the forward's states unsplit)
+])
+def test_bwd_split(ssm, dtype, b, L, d_in, N, with_z):
+    """Few channels: with the fast workspace ssm_scan_bwd cuts the chunks into
+    blocks (the forward's split scan for the chunk-start states, each block's
+    adjoint map composed from dh_last by the carry scan, every block's
+    backward at once).  The gradients match the oracle and, within rounding,
+    the unsplit backward the minimum workspace runs."""
+    need = ssm.ssm_scan_bwd_workspace_bytes(b, L, d_in, N)
+    fast = ssm.ssm_scan_bwd_fast_workspace_bytes(b, L, d_in, N)
+    assert fast > need, "this shape should take the split backward"
+    dt = "bf16" if dtype == torch.bfloat16 else "fp32"
+    inp = scan_inputs(b, L, d_in, N, dt, seed=L + d_in + N, with_z=with_z)
+    dout = _dout(b, L, d_in, dtype, seed=L + 1)
+    g = torch.Generator().manual_seed(d_in + 3)
+    h0 = torch.randn(b, d_in, N, generator=g)
+    dhl = torch.randn(b, d_in, N, generator=g)
+    c = to_cuda(inp)
+
+    def run(nbytes):
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        return ssm.ssm_scan_bwd(c["u"], c["delta"], c["A"], c["B"], c["C"], dout.cuda(),
+                                D=c["D"], z=c["z"], dt_bias=c["dt_bias"], h0=h0.cuda(),
+                                dh_last=dhl.cuda(), want_dh0=True, workspace=ws)
+
+    split, one = run(fast), run(need)
+    _compare(split, _ref(inp, dout, h0, dhl), dtype)
+    # the chunk states and the adjoint reach each block by composed maps, so
+    # the two paths round differently: they agree within the parity tolerances
+    for k in one:
+        assert rel_err(split[k], one[k]) <= _tol(k, dtype), k
