@@ -171,7 +171,8 @@ size_t ssm_scan_bwd_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t 
  * chunk-start states from the forward's split scan, each block's adjoint map
  * composed from dh_last by the carry scan, every block's backward at once.
  * With less it runs unsplit; the gradients agree within rounding (sums are
- * taken in a different order).  ssm_scan_bwd_saved always runs unsplit.
+ * taken in a different order).  ssm_scan_bwd_saved runs unsplit;
+ * ssm_scan_bwd_saved_ex splits from the saved states.
  */
 size_t ssm_scan_bwd_fast_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t d_state);
 
@@ -236,6 +237,36 @@ ssm_status ssm_scan_bwd_saved(const void *u, const void *delta, const float *A,
                               int64_t b, int64_t L, int64_t d_in, int64_t d_state,
                               ssm_dtype dtype, const float *chunk_states,
                               size_t chunk_states_bytes, ssm_stream_t stream);
+
+/*
+ * ssm_scan_bwd_saved with a workspace for the split backward (few channels):
+ * given ssm_scan_bwd_saved_workspace_bytes(...) bytes or more (when that is
+ * not 0), 16-byte aligned, the chunks are cut into blocks as in
+ * ssm_scan_bwd, from the saved states (no states pass); with less, or NULL,
+ * it is ssm_scan_bwd_saved.  The two agree within rounding.
+ *
+ *   workspace     device, nullable; contents on entry are ignored.  Must be
+ *                 4-byte aligned and share no byte with any argument.
+ * Other arguments, layouts and errors as ssm_scan_bwd_saved.
+ */
+ssm_status ssm_scan_bwd_saved_ex(const void *u, const void *delta, const float *A,
+                                 const void *B, const void *C, const float *D,
+                                 const void *z, const float *dt_bias, int delta_softplus,
+                                 const void *dout, const float *dh_last,
+                                 void *du, void *ddelta, float *dA, float *dB, float *dC,
+                                 float *dD, void *dz, float *ddt_bias, float *dh0,
+                                 int64_t b, int64_t L, int64_t d_in, int64_t d_state,
+                                 ssm_dtype dtype, const float *chunk_states,
+                                 size_t chunk_states_bytes, void *workspace,
+                                 size_t workspace_bytes, ssm_stream_t stream);
+
+/*
+ * Workspace of ssm_scan_bwd_saved_ex's split: the adjoint's block maps,
+ * 2 * b * blocks * d_in * d_state fp32, when the split applies (d_state 8,
+ * 16, 32 and too few channels to fill the GPU); 0 otherwise.  (size_t)-1 for
+ * invalid sizes.
+ */
+size_t ssm_scan_bwd_saved_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t d_state);
 
 /*
  * SS2D forward on an H x W grid (pixels row-major, p = h W + w, L = H W).

@@ -579,11 +579,14 @@ ssm_status launch_bwd_split(const ssm::BwdParams &p, bool async, const BwdSplitP
                             float *extra, cudaStream_t st) {
   constexpr int NPT = N < 4 ? N : SSM_BWD_NPT;
   if constexpr (ws_states(N) > 0) {
-    // 1. chunk-start states: the forward's states pass, split like the forward
+    // 1. chunk-start states (unless saved): the forward's states pass, split
+    // like the forward
     ssm::ScanParams f{p.u, p.delta, p.A, p.B, p.C, nullptr, nullptr, p.dt_bias, p.h0,
                       nullptr, nullptr, p.b, p.L, p.d_in, p.softplus, p.chunk_h};
     float *adj = extra;
-    if (sp.fwd.nblk > 1) {
+    if (p.states_saved) {
+      // the states are there already; `extra` holds the adjoint's maps only
+    } else if (sp.fwd.nblk > 1) {
       f.Lb = sp.fwd.Lb;
       f.blk_decay = extra;
       f.blk_state = extra + p.b * sp.fwd.nblk * p.d_in * N;
@@ -837,7 +840,8 @@ ssm_status scan_bwd_impl(const char *what, const void *u, const void *delta, con
                          float *dA, float *dB, float *dC, float *dD, void *dz, float *ddt_bias,
                          float *dh0, int64_t b, int64_t L, int64_t d_in, int64_t d_state,
                          ssm_dtype dtype, void *workspace, size_t workspace_bytes,
-                         int states_saved, ssm_stream_t stream) {
+                         int states_saved, ssm_stream_t stream, void *aux = nullptr,
+                         size_t aux_bytes = 0) {
   g_last_error.clear();
   if (b < 0 || L < 0 || d_in < 0)
     return fail(SSM_ERR_INVALID_ARG, "%s: negative size (b=%lld L=%lld d_in=%lld)", what,
@@ -877,15 +881,23 @@ ssm_status scan_bwd_impl(const char *what, const void *u, const void *delta, con
                           aligned(delta, 16) && aligned(B, 16) && b <= 65535;
   // the split backward when the workspace holds its block buffers after the
   // chunk states (ssm_scan_bwd only: the saved-states call has no workspace to spare)
+  // (from saved states: when `aux` holds the adjoint's block maps)
   const size_t fast = states_saved ? need : ssm_scan_bwd_fast_workspace_bytes(b, L, d_in, d_state);
-  const bool split = !states_saved && fwd_states && fast > need && workspace &&
-                     workspace_bytes >= fast && aligned(workspace, 16);
+  const size_t aux_need = states_saved ? ssm_scan_bwd_saved_workspace_bytes(b, L, d_in, d_state) : 0;
+  const bool split = states_saved
+                         ? aux_need > 0 && aux_need != (size_t)-1 && aux && aux_bytes >= aux_need &&
+                               aligned(aux, 16)
+                         : fwd_states && fast > need && workspace && workspace_bytes >= fast &&
+                               aligned(workspace, 16);
+  if (aux && !aligned(aux, 4))
+    return fail(SSM_ERR_INVALID_ARG, "%s: workspace not 4-byte aligned", what);
   {
     const int64_t ba = n_act * (int64_t)es, bbc = n_bc * (int64_t)es, bs = n_state * 4;
     const int64_t bp = d_in * 4, bA = d_in * d_state * 4, bw = (int64_t)(split ? fast : need);
     // the saved states are read, not written, in the split mode
-    const Span ws{"workspace", states_saved ? nullptr : workspace, bw};
-    const Span ws_in{"chunk_states", states_saved ? workspace : nullptr, bw};
+    const Span ws{"workspace", states_saved ? (split ? aux : nullptr) : workspace,
+                  states_saved ? (int64_t)aux_need : bw};
+    const Span ws_in{"chunk_states", states_saved ? workspace : nullptr, (int64_t)need};
     if (ssm_status s = check_disjoint(
             what,
             {{"du", du, ba}, {"ddelta", ddelta, ba}, {"dz", z ? dz : nullptr, ba}, {"dA", dA, bA},
@@ -921,7 +933,8 @@ ssm_status scan_bwd_impl(const char *what, const void *u, const void *delta, con
                      aligned(dout, 16) && aligned(B, 16) && aligned(C, 16) && (!z || aligned(z, 16));
   if (split) {
     const BwdSplitPlan sp = bwd_split_plan(b, L, d_in, d_state);
-    float *extra = static_cast<float *>(workspace) + need / sizeof(float);
+    float *extra = states_saved ? static_cast<float *>(aux)
+                                : static_cast<float *>(workspace) + need / sizeof(float);
     if (dtype == SSM_BF16) return dispatch_bwd_split_n<__nv_bfloat16>(p, d_state, async, sp, extra, st);
     return dispatch_bwd_split_n<float>(p, d_state, async, sp, extra, st);
   }
@@ -944,6 +957,28 @@ ssm_status ssm_scan_bwd(const void *u, const void *delta, const float *A, const 
   return scan_bwd_impl("ssm_scan_bwd", u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0,
                        dout, dh_last, du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, b, L, d_in,
                        d_state, dtype, workspace, workspace_bytes, 0, stream);
+}
+
+size_t ssm_scan_bwd_saved_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t d_state) {
+  if (ssm_scan_bwd_workspace_bytes(b, L, d_in, d_state) == (size_t)-1) return (size_t)-1;
+  const BwdSplitPlan sp = bwd_split_plan(b, L, d_in, d_state);
+  if (sp.nblk < 2) return 0;
+  return (size_t)(2 * b * sp.nblk * d_in * d_state) * sizeof(float);
+}
+
+ssm_status ssm_scan_bwd_saved_ex(const void *u, const void *delta, const float *A, const void *B,
+                                 const void *C, const float *D, const void *z,
+                                 const float *dt_bias, int delta_softplus, const void *dout,
+                                 const float *dh_last, void *du, void *ddelta, float *dA,
+                                 float *dB, float *dC, float *dD, void *dz, float *ddt_bias,
+                                 float *dh0, int64_t b, int64_t L, int64_t d_in, int64_t d_state,
+                                 ssm_dtype dtype, const float *chunk_states,
+                                 size_t chunk_states_bytes, void *workspace,
+                                 size_t workspace_bytes, ssm_stream_t stream) {
+  return scan_bwd_impl("ssm_scan_bwd_saved", u, delta, A, B, C, D, z, dt_bias, delta_softplus,
+                       nullptr, dout, dh_last, du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, b, L,
+                       d_in, d_state, dtype, const_cast<float *>(chunk_states),
+                       chunk_states_bytes, 1, stream, workspace, workspace_bytes);
 }
 
 ssm_status ssm_scan_bwd_saved(const void *u, const void *delta, const float *A, const void *B,

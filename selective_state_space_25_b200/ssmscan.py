@@ -50,6 +50,8 @@ _lib.ssm_scan_bwd_workspace_bytes.argtypes = [_I64] * 4
 _lib.ssm_scan_bwd_workspace_bytes.restype = _SZ
 _lib.ssm_scan_bwd_fast_workspace_bytes.argtypes = [_I64] * 4
 _lib.ssm_scan_bwd_fast_workspace_bytes.restype = _SZ
+_lib.ssm_scan_bwd_saved_workspace_bytes.argtypes = [_I64] * 4
+_lib.ssm_scan_bwd_saved_workspace_bytes.restype = _SZ
 _lib.ssm_scan_bwd.argtypes = [_P] * 8 + [_INT] + [_P] * 12 + [_I64] * 4 + [_INT, _P, _SZ, _P]
 _lib.ssm_scan_bwd.restype = _INT
 _lib.ssm_scan_fwd_save.argtypes = [_P] * 8 + [_INT, _P, _P, _P, _P, _SZ] + [_I64] * 4 + [_INT, _P]
@@ -57,6 +59,9 @@ _lib.ssm_scan_fwd_save.restype = _INT
 _lib.ssm_scan_bwd_saved.argtypes = ([_P] * 8 + [_INT] + [_P] * 11 + [_I64] * 4
                                     + [_INT, _P, _SZ, _P])
 _lib.ssm_scan_bwd_saved.restype = _INT
+_lib.ssm_scan_bwd_saved_ex.argtypes = (_lib.ssm_scan_bwd_saved.argtypes[:-1]
+                                       + [_P, _SZ, _P])
+_lib.ssm_scan_bwd_saved_ex.restype = _INT
 _lib.ss2d_scan_fwd_workspace_bytes.argtypes = [_I64] * 5
 _lib.ss2d_scan_fwd_workspace_bytes.restype = _SZ
 _lib.ss2d_scan_fwd_fast_workspace_bytes.argtypes = [_I64] * 5
@@ -208,6 +213,10 @@ def ssm_scan_bwd_fast_workspace_bytes(b: int, L: int, d_in: int, d_state: int) -
     return int(_lib.ssm_scan_bwd_fast_workspace_bytes(b, L, d_in, d_state))
 
 
+def ssm_scan_bwd_saved_workspace_bytes(b: int, L: int, d_in: int, d_state: int) -> int:
+    return int(_lib.ssm_scan_bwd_saved_workspace_bytes(b, L, d_in, d_state))
+
+
 def ssm_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_softplus=True,
                  h0=None, dh_last=None, want_dh0=False, workspace=None, stream=None, out=None,
                  states=None):
@@ -218,7 +227,8 @@ def ssm_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_so
     (a dict returned by an earlier call with the same shapes) is refilled
     in place instead of allocating.  ``states``: the chunk_states buffer a
     forward with the same inputs filled (ssm_scan_fwd(..., chunk_states=));
-    the backward then starts from it (ssm_scan_bwd_saved) and h0 is unused."""
+    the backward then starts from it (ssm_scan_bwd_saved_ex, with ``workspace``
+    or an allocated one for its split when channels are few) and h0 is unused."""
     b, L, d_in = u.shape
     N = A.shape[1]
     dev, act, f32 = u.device, u.dtype, torch.float32
@@ -250,12 +260,17 @@ def ssm_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_so
                  ddt_bias=torch.empty(d_in, dtype=f32, device=dev),
                  dh0=torch.empty((b, d_in, N), dtype=f32, device=dev) if want_dh0 else None)
     if states is not None:
-        st = _lib.ssm_scan_bwd_saved(
+        aux = ssm_scan_bwd_saved_workspace_bytes(b, L, d_in, N)
+        if workspace is None and aux > 0:
+            workspace = torch.empty(aux, dtype=torch.uint8, device=dev)
+        st = _lib.ssm_scan_bwd_saved_ex(
             _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
             int(bool(delta_softplus)), _ptr(dout), _ptr(dh_last), _ptr(g["du"]),
             _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dD"]),
             _ptr(g["dz"]), _ptr(g["ddt_bias"]), _ptr(g["dh0"]), b, L, d_in, N, _dtype_code(u),
-            _ptr(states), states.numel() * states.element_size(), _stream(stream))
+            _ptr(states), states.numel() * states.element_size(), _ptr(workspace),
+            0 if workspace is None else workspace.numel() * workspace.element_size(),
+            _stream(stream))
         _check(st, "ssm_scan_bwd_saved")
         return {k: v for k, v in g.items() if v is not None}
     need = ssm_scan_bwd_fast_workspace_bytes(b, L, d_in, N)  # the fastest path's

@@ -57,6 +57,24 @@ def main():
                             z=g["z"], dt_bias=g["dt_bias"], states=states if saved else None)
         for k in ("du", "ddelta", "dB", "dC", "dA"):
             check(f"backward {k} saved={saved}", gr[k], ref[k], 2e-2 if k in ("du", "ddelta") else 2e-4)
+    # split backward (few channels): self-contained and from saved states;
+    # the binding allocates the split's workspace
+    inp = scan_inputs(1, 1000, 32, 8, "bf16", seed=21, with_h0=True)
+    g = to_cuda(inp)
+    assert S.ssm_scan_bwd_saved_workspace_bytes(1, 1000, 32, 8) > 0
+    states = torch.empty(S.ssm_scan_bwd_workspace_bytes(1, 1000, 32, 8) // 4, device="cuda")
+    S.ssm_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], D=g["D"], z=g["z"],
+                   dt_bias=g["dt_bias"], h0=g["h0"], chunk_states=states)
+    dout = torch.randn(1, 1000, 32, generator=torch.Generator().manual_seed(6)).to(torch.bfloat16)
+    ref = oracle.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dout,
+                                    D=inp["D"], z=inp["z"], dt_bias=inp["dt_bias"], h0=inp["h0"])
+    for saved in (False, True):
+        gr = S.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], dout.cuda(), D=g["D"],
+                            z=g["z"], dt_bias=g["dt_bias"], h0=None if saved else g["h0"],
+                            states=states if saved else None, want_dh0=True)
+        for k in ("du", "ddelta", "dB", "dC", "dA", "dh0"):
+            check(f"split backward {k} saved={saved}", gr[k], ref[k],
+                  2e-2 if k in ("du", "ddelta") else 2e-4)
     # SS2D: shared-memory and workspace accumulators, both orders
     # (d_in 13: a partial last channel group, its last pair inactive)
     for (H, W, order, d_in) in [(7, 9, "cross", 16), (5, 6, "snake", 16), (80, 81, "cross", 16),

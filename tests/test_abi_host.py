@@ -193,6 +193,13 @@ def bwd(saved=False, **kw):
              dh0=None, b=2, L=40, d_in=16, N=16, dtype=S.SSM_BF16, ws=FAKE + 65536,
              ws_bytes=1 << 20, stream=None)
     a.update(kw)
+    if saved == "ex":
+        return L.ssm_scan_bwd_saved_ex(a["u"], a["delta"], a["A"], a["B"], a["C"], a["D"],
+                                       a["z"], a["dt_bias"], a["sp"], a["dout"], a["dh_last"],
+                                       a["du"], a["ddelta"], a["dA"], a["dB"], a["dC"], a["dD"],
+                                       a["dz"], a["ddt_bias"], a["dh0"], a["b"], a["L"],
+                                       a["d_in"], a["N"], a["dtype"], a["ws"], a["ws_bytes"],
+                                       a.get("aux"), a.get("aux_bytes", 0), a["stream"])
     if saved:
         return L.ssm_scan_bwd_saved(a["u"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"],
                                     a["dt_bias"], a["sp"], a["dout"], a["dh_last"], a["du"],
@@ -205,7 +212,7 @@ def bwd(saved=False, **kw):
                           a["d_in"], a["N"], a["dtype"], a["ws"], a["ws_bytes"], a["stream"])
 
 
-@pytest.mark.parametrize("saved", [False, True])
+@pytest.mark.parametrize("saved", [False, True, "ex"])
 @pytest.mark.parametrize("kw,status", [
     (dict(b=-1), S.SSM_ERR_INVALID_ARG),
     (dict(N=12), S.SSM_ERR_UNSUPPORTED),
@@ -226,6 +233,40 @@ def test_bwd_validation(saved, kw, status):
     assert bwd(saved=saved, **kw) == status
     if status != S.SSM_OK:
         assert S.last_error() != ""
+
+
+# b=1, L=16384, d_in=256, N=16 takes the saved split: outputs and the
+# chunk states far apart, so that each case overlaps one argument only
+SAVED_SPLIT = dict(b=1, L=16384, d_in=256, N=16, du=FAKE + (1 << 40), ddelta=FAKE + (2 << 40),
+                   dout=FAKE + (3 << 40), dA=FAKE + (4 << 40), dB=FAKE + (5 << 40),
+                   dC=FAKE + (6 << 40), ws=FAKE + (7 << 40), ws_bytes=1 << 30)
+
+
+@pytest.mark.parametrize("aux,why", [
+    (FAKE + (8 << 40) + 2, "not 4-byte aligned"),
+    (FAKE + (2 << 40) + 4096, "ddelta and workspace overlap"),
+    (FAKE + (1 << 20), "overlaps the input u"),
+    (FAKE + (7 << 40) + 64, "overlaps the input chunk_states"),
+])
+def test_bwd_saved_ex_workspace_validation(aux, why):
+    assert bwd(saved="ex", aux=aux, aux_bytes=1 << 22, **SAVED_SPLIT) == S.SSM_ERR_INVALID_ARG
+    assert why in S.last_error()
+
+
+def test_bwd_saved_workspace_query():
+    # the saved split needs only the adjoint's block maps: the fast workspace
+    # less the chunk states and the forward split's block buffers
+    for shape in [(1, 16384, 256, 16), (1, 4096, 64, 16), (2, 1000, 32, 8), (1, 777, 48, 32)]:
+        sv = S.ssm_scan_bwd_saved_workspace_bytes(*shape)
+        assert sv > 0, shape
+        assert sv == (S.ssm_scan_bwd_fast_workspace_bytes(*shape)
+                      - S.ssm_scan_bwd_workspace_bytes(*shape)
+                      - S.ssm_scan_fwd_workspace_bytes(*shape)), shape
+        assert sv % (2 * shape[0] * shape[2] * shape[3] * 4) == 0, shape
+    assert S.ssm_scan_bwd_saved_workspace_bytes(8, 2048, 1536, 16) == 0   # fills the GPU
+    assert S.ssm_scan_bwd_saved_workspace_bytes(1, 16384, 256, 4) == 0    # d_state 4
+    assert S.ssm_scan_bwd_saved_workspace_bytes(1, 40, 16, 16) == 0       # too few chunks
+    assert L.ssm_scan_bwd_saved_workspace_bytes(-1, 1, 1, 16) == ctypes.c_size_t(-1).value
 
 
 def test_bwd_workspace_query():

@@ -214,7 +214,10 @@ def test_bwd_saved_equals_self_contained(ssm, dtype):
                         device="cuda")
     full = ssm.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], dout, h0=g["h0"],
                             workspace=least, **kw)
-    saved = ssm.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], dout, states=states, **kw)
+    # no workspace for the saved call: unsplit as well
+    none = torch.empty(0, dtype=torch.uint8, device="cuda")
+    saved = ssm.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], dout, states=states,
+                             workspace=none, **kw)
     for k in full:
         assert rel_err(saved[k], to64(full[k])) <= 1e-5, k
     ref = _ref(inp, dout.cpu(), inp["h0"], dhl.cpu())
@@ -233,7 +236,7 @@ def test_fwd_save_rejects_small_buffer(ssm):
     (1, 4096, 64, 16, True),   # 256 chunks in blocks; the forward's states pass split too
     (2, 1000, 32, 8, True),    # ragged last chunk and block
     (1, 777, 48, 32, False),   # no gate
-    (1, 300, 64, 16, True),    # few blocks (the forward's states unsplit)
+    (1, 300, 64, 16, True),    # few blocks
 ])
 def test_bwd_split(ssm, dtype, b, L, d_in, N, with_z):
     """Few channels: with the fast workspace ssm_scan_bwd cuts the chunks into
@@ -264,3 +267,46 @@ def test_bwd_split(ssm, dtype, b, L, d_in, N, with_z):
     # the two paths round differently: they agree within the parity tolerances
     for k in one:
         assert rel_err(split[k], one[k]) <= _tol(k, dtype), k
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("b,L,d_in,N,with_z", [
+    (1, 4096, 64, 16, True),
+    (2, 1000, 32, 8, True),    # ragged last chunk and block
+    (1, 777, 48, 32, False),
+    (2, 203, 48, 16, True),    # three blocks
+])
+def test_bwd_saved_split(ssm, dtype, b, L, d_in, N, with_z):
+    """Few channels, from the forward's saved chunk states: with
+    ssm_scan_bwd_saved_workspace_bytes of workspace the backward runs in
+    blocks (no states pass; the adjoint maps composed from dh_last), without
+    it unsplit.  Both match the oracle, and each other within rounding."""
+    aux = ssm.ssm_scan_bwd_saved_workspace_bytes(b, L, d_in, N)
+    assert aux > 0, "this shape should take the split backward"
+    dt = "bf16" if dtype == torch.bfloat16 else "fp32"
+    inp = scan_inputs(b, L, d_in, N, dt, seed=3 * L + d_in, with_z=with_z, with_h0=True)
+    dout = _dout(b, L, d_in, dtype, seed=L + 7)
+    dhl = torch.randn(b, d_in, N, generator=torch.Generator().manual_seed(N + 5))
+    c = to_cuda(inp)
+    states = torch.empty(ssm.ssm_scan_bwd_workspace_bytes(b, L, d_in, N) // 4, device="cuda")
+    ssm.ssm_scan_fwd(c["u"], c["delta"], c["A"], c["B"], c["C"], D=c["D"], z=c["z"],
+                     dt_bias=c["dt_bias"], h0=c["h0"], chunk_states=states)
+    kept = states.clone()
+
+    def run(nbytes):
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        return ssm.ssm_scan_bwd(c["u"], c["delta"], c["A"], c["B"], c["C"], dout.cuda(),
+                                D=c["D"], z=c["z"], dt_bias=c["dt_bias"], states=states,
+                                dh_last=dhl.cuda(), want_dh0=True, workspace=ws)
+
+    split, one = run(aux), run(0)
+    assert torch.equal(states, kept), "the saved states are read only"
+    _compare(split, _ref(inp, dout, inp["h0"], dhl), dtype)
+    for k in one:
+        assert rel_err(split[k], one[k]) <= _tol(k, dtype), k
+    # the binding's default allocates the split's workspace
+    dflt = ssm.ssm_scan_bwd(c["u"], c["delta"], c["A"], c["B"], c["C"], dout.cuda(), D=c["D"],
+                            z=c["z"], dt_bias=c["dt_bias"], states=states, dh_last=dhl.cuda(),
+                            want_dh0=True)
+    for k in ("du", "ddelta", "dh0"):
+        assert torch.equal(dflt[k], split[k]), k
