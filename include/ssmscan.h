@@ -167,10 +167,12 @@ size_t ssm_scan_bwd_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t 
  * more than half of the SMs idle, the chunk states followed by the split
  * backward's block buffers (the forward split's block decays and states, the
  * adjoint's block maps); otherwise ssm_scan_bwd_workspace_bytes.  With that
- * much (16-byte aligned) ssm_scan_bwd cuts the sequence into blocks: the
+ * much (16-byte aligned), when d_in times the element size is a multiple of
+ * 16 bytes and u, delta, B are 16-byte aligned (the forward kernel's
+ * staging), ssm_scan_bwd cuts the sequence into blocks: the
  * chunk-start states from the forward's split scan, each block's adjoint map
  * composed from dh_last by the carry scan, every block's backward at once.
- * With less it runs unsplit; the gradients agree within rounding (sums are
+ * Otherwise it runs unsplit; the gradients agree within rounding (sums are
  * taken in a different order).  ssm_scan_bwd_saved runs unsplit;
  * ssm_scan_bwd_saved_ex splits from the saved states.
  */

@@ -879,9 +879,9 @@ ssm_status scan_bwd_impl(const char *what, const void *u, const void *delta, con
   // the forward kernel's states pass needs its own 16-byte staging of u, delta, B
   const bool fwd_states = (d_in * (int64_t)es) % 16 == 0 && aligned(u, 16) &&
                           aligned(delta, 16) && aligned(B, 16) && b <= 65535;
-  // the split backward when the workspace holds its block buffers after the
-  // chunk states (ssm_scan_bwd only: the saved-states call has no workspace to spare)
-  // (from saved states: when `aux` holds the adjoint's block maps)
+  // the split backward: self-contained when the workspace holds its block
+  // buffers after the chunk states (and the forward kernel can write those
+  // states); from saved states when `aux` holds the adjoint's block maps
   const size_t fast = states_saved ? need : ssm_scan_bwd_fast_workspace_bytes(b, L, d_in, d_state);
   const size_t aux_need = states_saved ? ssm_scan_bwd_saved_workspace_bytes(b, L, d_in, d_state) : 0;
   const bool split = states_saved

@@ -85,6 +85,53 @@ def test_random_scan_backward(ssm, seed):
         assert rel_err(got[k], ref[k]) <= tol, (k,) + what
 
 
+@pytest.mark.parametrize("seed", _seeds(60, 15))
+def test_random_split_paths(ssm, seed):
+    """Long sequences over few channels: the split forward scan and the split
+    backward (self-contained, or from saved states), which the binding's
+    default workspaces select, on random sizes, alignments and options."""
+    r = random.Random(seed)
+    b, L, N = r.randint(1, 2), r.randint(128, 2500), r.choice((8, 16, 32))
+    d_in = r.choice([r.randint(1, 64), 8 * r.randint(1, 8)])   # the fast kernels want 8 | d_in
+    dt, dtype = _dtype(r)
+    mode = r.choice(["forward", "backward", "saved"])
+    inp = scan_inputs(b, L, d_in, N, dt, seed=seed, with_z=r.random() < 0.7,
+                      with_D=r.random() < 0.7, with_dt_bias=r.random() < 0.7,
+                      with_h0=r.random() < 0.5)
+    g = to_cuda(inp)
+    what = (b, L, d_in, N, dt, mode)
+    if mode == "forward":
+        hl = torch.empty(b, d_in, N, device="cuda")
+        y = ssm.ssm_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], D=g["D"], z=g["z"],
+                             dt_bias=g["dt_bias"], h0=g["h0"], h_last=hl)
+        y_ref, h_ref = oracle.selective_scan(inp["u"], inp["delta"], inp["A"], inp["B"],
+                                             inp["C"], D=inp["D"], z=inp["z"],
+                                             dt_bias=inp["dt_bias"], h0=inp["h0"],
+                                             return_last_state=True)
+        assert rel_err(y, y_ref) <= TOL[dtype], what
+        assert rel_err(hl, h_ref) <= 1e-4, what
+        return
+    gd = torch.Generator().manual_seed(seed + 1)
+    dout = torch.randn(b, L, d_in, generator=gd).to(dtype)
+    dhl = torch.randn(b, d_in, N, generator=gd) if r.random() < 0.5 else None
+    kw = dict(D=g["D"], z=g["z"], dt_bias=g["dt_bias"], h0=g["h0"],
+              dh_last=None if dhl is None else dhl.cuda(), want_dh0=True)
+    if mode == "saved":
+        states = torch.empty(ssm.ssm_scan_bwd_workspace_bytes(b, L, d_in, N) // 4, device="cuda")
+        ssm.ssm_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], D=g["D"], z=g["z"],
+                         dt_bias=g["dt_bias"], h0=g["h0"], chunk_states=states)
+        kw["states"] = states
+    got = ssm.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], dout.cuda(), **kw)
+    ref = oracle.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dout,
+                                    D=inp["D"], z=inp["z"], dt_bias=inp["dt_bias"],
+                                    h0=inp["h0"], dh_last=dhl)
+    for k in ref:
+        if k not in got or got[k] is None:
+            continue
+        tol = TOL[dtype] if k in ("du", "ddelta", "dz") else (1e-4 if dtype == torch.float32 else 2e-4)
+        assert rel_err(got[k], ref[k]) <= tol, (k,) + what
+
+
 @pytest.mark.parametrize("seed", _seeds(160, 13))
 def test_random_ss2d(ssm, seed):
     r = random.Random(seed)
