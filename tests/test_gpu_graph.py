@@ -116,3 +116,51 @@ def test_split_scan_in_a_graph(ssm):
     graph.replay()
     torch.cuda.synchronize()
     assert torch.equal(y, y_e) and torch.equal(hl, hl_e)
+
+
+@pytest.mark.parametrize("saved", [False, True])
+def test_split_backward_in_a_graph(ssm, saved):
+    """The split backward (few channels: the chunk states from the forward's
+    split scan or from the saved ones, the adjoint's block maps, the carry
+    scan, every block at once) captured in a graph replays the eager call:
+    the per-channel gradients bit for bit, the channel sums within rounding
+    (they are taken with atomics)."""
+    b, L, d_in, N = 1, 4096, 64, 16
+    g = to_cuda(scan_inputs(b, L, d_in, N, "bf16", seed=10, with_h0=True))
+    dout = torch.randn(b, L, d_in, device="cuda").to(torch.bfloat16)
+    dhl = torch.randn(b, d_in, N, device="cuda")
+    states = None
+    if saved:
+        states = torch.empty(ssm.ssm_scan_bwd_workspace_bytes(b, L, d_in, N) // 4, device="cuda")
+        ssm.ssm_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], D=g["D"], z=g["z"],
+                         dt_bias=g["dt_bias"], h0=g["h0"], chunk_states=states)
+        nbytes = ssm.ssm_scan_bwd_saved_workspace_bytes(b, L, d_in, N)
+        assert nbytes > 0, "this shape should take the saved split"
+    else:
+        nbytes = ssm.ssm_scan_bwd_fast_workspace_bytes(b, L, d_in, N)
+        assert nbytes > ssm.ssm_scan_bwd_workspace_bytes(b, L, d_in, N), "should split"
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    kw = dict(D=g["D"], z=g["z"], dt_bias=g["dt_bias"], dh_last=dhl, want_dh0=True,
+              workspace=ws, h0=None if saved else g["h0"], states=states)
+    ref = ssm.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], dout, **kw)
+    out = {k: torch.empty_like(v) for k, v in ref.items()}
+
+    def work():
+        ssm.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], dout, out=out, **kw)
+
+    work()
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        work()
+    for v in out.values():
+        v.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    for k in ("du", "ddelta", "dz", "dh0"):
+        assert torch.equal(out[k], ref[k]), k
+    for k in ("dA", "dB", "dC", "dD", "ddt_bias"):
+        # a sum near zero takes the rounding of its terms: measured on the scale
+        assert (out[k] - ref[k]).abs().max() <= 1e-5 * ref[k].abs().max(), k
