@@ -879,24 +879,29 @@ ssm_status scan_bwd_impl(const char *what, const void *u, const void *delta, con
   // the forward kernel's states pass needs its own 16-byte staging of u, delta, B
   const bool fwd_states = (d_in * (int64_t)es) % 16 == 0 && aligned(u, 16) &&
                           aligned(delta, 16) && aligned(B, 16) && b <= 65535;
-  // the split backward: self-contained when the workspace holds its block
-  // buffers after the chunk states (and the forward kernel can write those
-  // states); from saved states when `aux` holds the adjoint's block maps
-  const size_t fast = states_saved ? need : ssm_scan_bwd_fast_workspace_bytes(b, L, d_in, d_state);
-  const size_t aux_need = states_saved ? ssm_scan_bwd_saved_workspace_bytes(b, L, d_in, d_state) : 0;
-  const bool split = states_saved
-                         ? aux_need > 0 && aux_need != (size_t)-1 && aux && aux_bytes >= aux_need &&
-                               aligned(aux, 16)
-                         : fwd_states && fast > need && workspace && workspace_bytes >= fast &&
-                               aligned(workspace, 16);
+  // The split backward.  Self-contained: when the workspace holds its block
+  // buffers after the chunk states and the forward kernel can write those
+  // states.  From saved states: when `aux` holds the adjoint's block maps.
+  // `used` is the scratch the call writes (the workspace, or `aux`).
+  bool split;
+  size_t used;
+  if (states_saved) {
+    const size_t aux_need = ssm_scan_bwd_saved_workspace_bytes(b, L, d_in, d_state);
+    split = aux_need > 0 && aux && aux_bytes >= aux_need && aligned(aux, 16);
+    used = split ? aux_need : 0;
+  } else {
+    const size_t fast = ssm_scan_bwd_fast_workspace_bytes(b, L, d_in, d_state);
+    split = fwd_states && fast > need && workspace && workspace_bytes >= fast &&
+            aligned(workspace, 16);
+    used = split ? fast : need;
+  }
   if (aux && !aligned(aux, 4))
     return fail(SSM_ERR_INVALID_ARG, "%s: workspace not 4-byte aligned", what);
   {
     const int64_t ba = n_act * (int64_t)es, bbc = n_bc * (int64_t)es, bs = n_state * 4;
-    const int64_t bp = d_in * 4, bA = d_in * d_state * 4, bw = (int64_t)(split ? fast : need);
-    // the saved states are read, not written, in the split mode
-    const Span ws{"workspace", states_saved ? (split ? aux : nullptr) : workspace,
-                  states_saved ? (int64_t)aux_need : bw};
+    const int64_t bp = d_in * 4, bA = d_in * d_state * 4;
+    const Span ws{"workspace", states_saved ? aux : workspace, (int64_t)used};
+    // from saved states the caller's `workspace` is the chunk states, read only
     const Span ws_in{"chunk_states", states_saved ? workspace : nullptr, (int64_t)need};
     if (ssm_status s = check_disjoint(
             what,
