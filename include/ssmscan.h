@@ -22,7 +22,8 @@
  *   ssm_scan_bwd      the gradients of ssm_scan_fwd by the reverse-time
  *                     adjoint of its recurrence (same passages);
  *                     ssm_scan_fwd_save / ssm_scan_bwd_saved split it as a
- *                     training step does (the forward keeps chunk states).
+ *                     training step does (the forward keeps chunk states;
+ *                     ssm_scan_bwd_saved_ex adds scratch for few channels).
  *   ssm_conv_state_update  the same step with the depthwise causal-conv1d
  *                     step of Mamba.step() in front of it (roll conv_state
  *                     left, append x, sum conv_state * weight + bias, SiLU).
