@@ -23,7 +23,8 @@
  *                     adjoint of its recurrence (same passages);
  *                     ssm_scan_fwd_save / ssm_scan_bwd_saved split it as a
  *                     training step does (the forward keeps chunk states;
- *                     ssm_scan_bwd_saved_ex adds scratch for few channels).
+ *                     ssm_scan_fwd_save_ex and ssm_scan_bwd_saved_ex add
+ *                     scratch for few channels).
  *   ssm_conv_state_update  the same step with the depthwise causal-conv1d
  *                     step of Mamba.step() in front of it (roll conv_state
  *                     left, append x, sum conv_state * weight + bias, SiLU).
@@ -145,7 +146,7 @@ ssm_status ssm_scan_fwd(const void *u, const void *delta, const float *A,
  * following ssm_scan_bwd_saved with the same inputs starts from these
  * states instead of walking the sequence forwards again (the saved chunk
  * states the backward of a training step keeps from its forward).  Every
- * other argument as for ssm_scan_fwd.
+ * other argument as for ssm_scan_fwd.  It runs in one pass (no workspace).
  */
 ssm_status ssm_scan_fwd_save(const void *u, const void *delta, const float *A,
                              const void *B, const void *C, const float *D,
@@ -154,6 +155,26 @@ ssm_status ssm_scan_fwd_save(const void *u, const void *delta, const float *A,
                              float *chunk_states, size_t chunk_states_bytes,
                              int64_t b, int64_t L, int64_t d_in, int64_t d_state,
                              ssm_dtype dtype, ssm_stream_t stream);
+
+/*
+ * ssm_scan_fwd_save with a workspace for the split scan (few channels):
+ * given ssm_scan_fwd_workspace_bytes(...) bytes or more (when that is not
+ * 0), 16-byte aligned, the sequence is cut into blocks as in ssm_scan_fwd
+ * (summary, carry and scan passes; the scan pass writes y, h_last and the
+ * chunk states); with less, or NULL, it is ssm_scan_fwd_save.  The two
+ * agree within rounding (the block start states are composed maps).
+ *
+ *   workspace     device, nullable; contents on entry are ignored.  Must be
+ *                 4-byte aligned and share no byte with any argument.
+ */
+ssm_status ssm_scan_fwd_save_ex(const void *u, const void *delta, const float *A,
+                                const void *B, const void *C, const float *D,
+                                const void *z, const float *dt_bias, int delta_softplus,
+                                const float *h0, float *h_last, void *y,
+                                float *chunk_states, size_t chunk_states_bytes,
+                                int64_t b, int64_t L, int64_t d_in, int64_t d_state,
+                                ssm_dtype dtype, void *workspace, size_t workspace_bytes,
+                                ssm_stream_t stream);
 
 /*
  * Workspace of ssm_scan_bwd: the state at the start of every 16-step chunk

@@ -721,13 +721,21 @@ ssm_status scan_fwd_impl(const void *u, const void *delta, const float *A, const
       !mul_ok(n_bc, d_state, &n_bc) || !mul_ok(b, d_in, &n_state) ||
       !mul_ok(n_state, d_state, &n_state) || n_act > INT64_MAX / 4)
     return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd: sizes overflow int64");
-  // the forward that saves chunk states always runs in one pass (no workspace)
-  const size_t need = chunk_h ? 0 : ssm_scan_fwd_workspace_bytes(b, L, d_in, d_state);
+  // The split scan's workspace: the plain forward requires it; the forward
+  // that saves chunk states takes the split only when given one (16-byte
+  // aligned) and otherwise runs in one pass.
+  const size_t split_bytes = ssm_scan_fwd_workspace_bytes(b, L, d_in, d_state);
+  const size_t need = chunk_h ? 0 : split_bytes;
   if (workspace_bytes < need || (need > 0 && !workspace))
     return fail(SSM_ERR_WORKSPACE, "ssm_scan_fwd: workspace %zu bytes < %zu needed",
                 workspace_bytes, need);
   if (need > 0 && !aligned(workspace, 16))
     return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd: workspace not 16-byte aligned");
+  if (chunk_h && workspace && !aligned(workspace, 4))
+    return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd_save: workspace not 4-byte aligned");
+  const bool split = split_bytes > 0 && split_bytes != (size_t)-1 &&
+                     (!chunk_h || (workspace && workspace_bytes >= split_bytes &&
+                                   aligned(workspace, 16)));
   if (b == 0 || d_in == 0) return ok();
   if (!A) return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd: A is NULL");
   if (L > 0 && (!u || !delta || !B || !C || !y))
@@ -747,7 +755,7 @@ ssm_status scan_fwd_impl(const void *u, const void *delta, const float *A, const
     if (ssm_status s = check_disjoint(
             "ssm_scan_fwd",
             {{"y", y, ba}, {"h_last", h_last, bs}, {"chunk_states", chunk_h, nc},
-             {"workspace", need > 0 ? workspace : nullptr, (int64_t)need}},
+             {"workspace", split ? workspace : nullptr, split ? (int64_t)split_bytes : 0}},
             {{"u", u, ba}, {"delta", delta, ba}, {"z", z, ba}, {"B", B, bbc}, {"C", C, bbc},
              {"A", A, d_in * d_state * 4}, {"D", D, d_in * 4}, {"dt_bias", dt_bias, d_in * 4},
              {"h0", h0, bs}},
@@ -765,7 +773,7 @@ ssm_status scan_fwd_impl(const void *u, const void *delta, const float *A, const
 
   ssm::ScanParams p{u, delta, A, B, C, D, z, dt_bias, h0, h_last, y, b, L, d_in, delta_softplus,
                     chunk_h};
-  if (!chunk_h && need > 0) {  // the split scan (its plan is the one need was sized for)
+  if (split) {  // the split scan (its plan is the one split_bytes was sized for)
     const SplitPlan sp = split_plan(b, L, d_in, d_state);
     p.Lb = sp.Lb;
     p.blk_decay = static_cast<float *>(workspace);
@@ -791,12 +799,13 @@ ssm_status ssm_scan_fwd(const void *u, const void *delta, const float *A, const 
                        d_in, d_state, dtype, workspace, workspace_bytes, nullptr, stream);
 }
 
-ssm_status ssm_scan_fwd_save(const void *u, const void *delta, const float *A, const void *B,
-                             const void *C, const float *D, const void *z, const float *dt_bias,
-                             int delta_softplus, const float *h0, float *h_last, void *y,
-                             float *chunk_states, size_t chunk_states_bytes, int64_t b,
-                             int64_t L, int64_t d_in, int64_t d_state, ssm_dtype dtype,
-                             ssm_stream_t stream) {
+ssm_status ssm_scan_fwd_save_ex(const void *u, const void *delta, const float *A,
+                                const void *B, const void *C, const float *D, const void *z,
+                                const float *dt_bias, int delta_softplus, const float *h0,
+                                float *h_last, void *y, float *chunk_states,
+                                size_t chunk_states_bytes, int64_t b, int64_t L, int64_t d_in,
+                                int64_t d_state, ssm_dtype dtype, void *workspace,
+                                size_t workspace_bytes, ssm_stream_t stream) {
   g_last_error.clear();
   const size_t need = ssm_scan_bwd_workspace_bytes(b, L, d_in, d_state);
   if (need == (size_t)-1)
@@ -806,9 +815,22 @@ ssm_status ssm_scan_fwd_save(const void *u, const void *delta, const float *A, c
                 chunk_states_bytes, need);
   if (chunk_states && !aligned(chunk_states, 16))
     return fail(SSM_ERR_INVALID_ARG, "ssm_scan_fwd_save: chunk_states not 16-byte aligned");
+  if (need == 0)  // no chunk starts (b, L or d_in of 0): a plain forward
+    return scan_fwd_impl(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, h_last, y, b, L,
+                         d_in, d_state, dtype, nullptr, 0, nullptr, stream);
   return scan_fwd_impl(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, h_last, y, b, L,
-                       d_in, d_state, dtype, nullptr, 0, need > 0 ? chunk_states : nullptr,
-                       stream);
+                       d_in, d_state, dtype, workspace, workspace_bytes, chunk_states, stream);
+}
+
+ssm_status ssm_scan_fwd_save(const void *u, const void *delta, const float *A, const void *B,
+                             const void *C, const float *D, const void *z, const float *dt_bias,
+                             int delta_softplus, const float *h0, float *h_last, void *y,
+                             float *chunk_states, size_t chunk_states_bytes, int64_t b,
+                             int64_t L, int64_t d_in, int64_t d_state, ssm_dtype dtype,
+                             ssm_stream_t stream) {
+  return ssm_scan_fwd_save_ex(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, h_last, y,
+                              chunk_states, chunk_states_bytes, b, L, d_in, d_state, dtype,
+                              nullptr, 0, stream);
 }
 
 size_t ssm_scan_bwd_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t d_state) {

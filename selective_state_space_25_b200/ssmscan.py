@@ -56,6 +56,8 @@ _lib.ssm_scan_bwd.argtypes = [_P] * 8 + [_INT] + [_P] * 12 + [_I64] * 4 + [_INT,
 _lib.ssm_scan_bwd.restype = _INT
 _lib.ssm_scan_fwd_save.argtypes = [_P] * 8 + [_INT, _P, _P, _P, _P, _SZ] + [_I64] * 4 + [_INT, _P]
 _lib.ssm_scan_fwd_save.restype = _INT
+_lib.ssm_scan_fwd_save_ex.argtypes = _lib.ssm_scan_fwd_save.argtypes[:-1] + [_P, _SZ, _P]
+_lib.ssm_scan_fwd_save_ex.restype = _INT
 _lib.ssm_scan_bwd_saved.argtypes = ([_P] * 8 + [_INT] + [_P] * 11 + [_I64] * 4
                                     + [_INT, _P, _SZ, _P])
 _lib.ssm_scan_bwd_saved.restype = _INT
@@ -165,7 +167,9 @@ def ssm_scan_fwd(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus
     A: (d_in, N) fp32; B, C: (b, L, N); D, dt_bias: (d_in,) fp32; h0, h_last:
     (b, d_in, N) fp32.  Returns y (b, L, d_in).  With ``chunk_states`` (a
     device buffer of ssm_scan_bwd_workspace_bytes(...) bytes) the forward
-    also saves the chunk-start states for ssm_scan_bwd(..., states=...)."""
+    also saves the chunk-start states for ssm_scan_bwd(..., states=...).
+    Unless ``workspace`` is given, the split scan's workspace
+    (ssm_scan_fwd_workspace_bytes) is allocated when it is not 0."""
     if u.dim() != 3:
         raise ValueError("u must be (b, L, d_in)")
     b, L, d_in = u.shape
@@ -185,17 +189,18 @@ def ssm_scan_fwd(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus
     if y is None:
         y = torch.empty_like(u)
     _need(y, "y", (b, L, d_in), act, dev)
-    if chunk_states is not None:
-        st = _lib.ssm_scan_fwd_save(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
-                                    _ptr(z), _ptr(dt_bias), int(bool(delta_softplus)), _ptr(h0),
-                                    _ptr(h_last), _ptr(y), _ptr(chunk_states),
-                                    chunk_states.numel() * chunk_states.element_size(),
-                                    b, L, d_in, N, _dtype_code(u), _stream(stream))
-        _check(st, "ssm_scan_fwd_save")
-        return y
     ws_bytes = ssm_scan_fwd_workspace_bytes(b, L, d_in, N)
     if workspace is None and ws_bytes > 0:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    if chunk_states is not None:
+        st = _lib.ssm_scan_fwd_save_ex(
+            _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
+            int(bool(delta_softplus)), _ptr(h0), _ptr(h_last), _ptr(y), _ptr(chunk_states),
+            chunk_states.numel() * chunk_states.element_size(), b, L, d_in, N, _dtype_code(u),
+            _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
+            _stream(stream))
+        _check(st, "ssm_scan_fwd_save")
+        return y
     st = _lib.ssm_scan_fwd(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
                            _ptr(dt_bias), int(bool(delta_softplus)), _ptr(h0), _ptr(h_last),
                            _ptr(y), b, L, d_in, N, _dtype_code(u), _ptr(workspace),

@@ -295,6 +295,25 @@ def test_fwd_save_validation():
     assert L.ssm_scan_fwd_save(*args(None, 0, b=0)) == S.SSM_OK
 
 
+@pytest.mark.parametrize("ws,why", [
+    (FAKE + (8 << 40) + 2, "not 4-byte aligned"),
+    (FAKE + 4096, "overlaps the input u"),
+    (FAKE + (2 << 40) + 4096, "y and workspace overlap"),
+    (FAKE + (3 << 40) + 64, "chunk_states and workspace overlap"),
+])
+def test_fwd_save_ex_workspace_validation(ws, why):
+    # b=1, L=4096, d_in=64, N=16 takes the split scan when given its workspace
+    b, Ls, d, N = 1, 4096, 64, 16
+    nbytes = S.ssm_scan_fwd_workspace_bytes(b, Ls, d, N)
+    assert nbytes > 0
+    st = L.ssm_scan_fwd_save_ex(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 1, None, None,
+                                FAKE + (2 << 40), FAKE + (3 << 40),
+                                S.ssm_scan_bwd_workspace_bytes(b, Ls, d, N), b, Ls, d, N,
+                                S.SSM_BF16, ws, nbytes, None)
+    assert st == S.SSM_ERR_INVALID_ARG
+    assert why in S.last_error()
+
+
 def test_split_scan_needs_its_workspace():
     need = S.ssm_scan_fwd_workspace_bytes(1, 4096, 64, 16)
     assert need > 0

@@ -166,24 +166,42 @@ def test_bwd_mamba130m_workload_sampled(ssm):
 
 # ------------------------------------ forward-saved chunk states (training split)
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("b,L,d_in,N", [(2, 100, 32, 16), (1, 33, 20, 4), (2, 48, 16, 1),
-                                        (1, 70, 24, 8), (1, 16, 8, 64)])
-def test_fwd_save_states_match_oracle_prefix_scans(ssm, dtype, b, L, d_in, N):
+@pytest.mark.parametrize("b,L,d_in,N,split", [
+    (2, 100, 32, 16, False), (1, 33, 20, 4, False), (2, 48, 16, 1, False), (1, 70, 24, 8, False),
+    (1, 16, 8, 64, False),
+    (1, 1000, 32, 8, True),    # split scan: 7 blocks of 160 steps, the last ragged
+    (2, 2100, 64, 16, True),   # 14 blocks, two batches
+    (1, 1300, 48, 32, True),
+])
+def test_fwd_save_states_match_oracle_prefix_scans(ssm, dtype, b, L, d_in, N, split):
     """Saved state c is the state after the first 16 c steps: the oracle's
-    h_last of the scan over that prefix (chunk 0 is h0)."""
+    h_last of the scan over that prefix (chunk 0 is h0).  Few channels over a
+    long sequence take the split scan (the binding allocates its workspace):
+    the scan pass of every block writes its chunks' states."""
+    assert (ssm.ssm_scan_fwd_workspace_bytes(b, L, d_in, N) > 0) == split
     dt = "bf16" if dtype == torch.bfloat16 else "fp32"
     inp = scan_inputs(b, L, d_in, N, dt, seed=L + N, with_h0=True)
     g = to_cuda(inp)
     nbytes = ssm.ssm_scan_bwd_workspace_bytes(b, L, d_in, N)
     states = torch.empty(nbytes // 4, device="cuda")
+    hl = torch.empty(b, d_in, N, device="cuda")
     y = ssm.ssm_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], D=g["D"], z=g["z"],
-                         dt_bias=g["dt_bias"], h0=g["h0"], chunk_states=states)
-    y_ref = oracle.selective_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"],
-                                  z=inp["z"], dt_bias=inp["dt_bias"], h0=inp["h0"])
+                         dt_bias=g["dt_bias"], h0=g["h0"], h_last=hl, chunk_states=states)
+    y_ref, h_ref = oracle.selective_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"],
+                                         D=inp["D"], z=inp["z"], dt_bias=inp["dt_bias"],
+                                         h0=inp["h0"], return_last_state=True)
     assert rel_err(y, y_ref) <= TOL[dtype]
+    assert rel_err(hl, h_ref) <= 1e-4
     nC = (L + 15) // 16
     got = states.view(b, nC, d_in, N)
-    for c in range(nC):
+    if split:  # the one-pass forward (no workspace) saves the same states within rounding
+        one = torch.empty_like(states)
+        y1 = ssm.ssm_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], D=g["D"], z=g["z"],
+                              dt_bias=g["dt_bias"], h0=g["h0"], chunk_states=one,
+                              workspace=torch.empty(0, dtype=torch.uint8, device="cuda"))
+        assert rel_err(states, to64(one)) <= 1e-4
+        assert rel_err(y, to64(y1)) <= TOL[dtype]
+    for c in range(0, nC, 1 if nC <= 40 else 5):
         if c == 0:
             ref = to64(inp["h0"])
         else:
