@@ -542,55 +542,139 @@ __global__ void __launch_bounds__(128, 3) scan_bwd_kernel(BwdParams p) {
 // exp(delta_t A) -- scan_bwd_kernel's adjoint step, g_t = dout_t silu(z_t).
 // M_k and R_k go to slot nblk - 1 - k of (b, nblk, d_in, N) arrays, the order
 // in which scan_carry_kernel composes them from dh_last; the carry then leaves
-// in slot nblk - 2 - k the adjoint block k starts from.  One thread per
-// (batch, block, channel), all N states in registers, lanes over channels.
-template <typename T, int N>
+// in slot nblk - 2 - k the adjoint block k starts from.
+// kAdjG threads per (batch, block, channel), N / kAdjG states each, so a CTA
+// of 128 threads covers kAdjChannels channels.  The walk is one dependent
+// chain per state and needs only the step's inputs, so they are staged in
+// shared memory by chunk (delta, dout, z rows of the CTA's channels and the
+// C row), two chunks ahead in a three-slot ring: with ASYNC by cp.async (the
+// rows are whole 16-byte groups: d_in times the element size a multiple of
+// 16 and 16-byte aligned inputs), else by plain loads before each chunk.
+constexpr int kAdjG = 4, kAdjChannels = 128 / kAdjG;
+template <typename T, int N, bool ASYNC>
 __global__ void __launch_bounds__(128) scan_bwd_adjoint_kernel(BwdParams p, float *adj_decay,
                                                                float *adj_state) {
+  constexpr int NA = N / kAdjG, CH = kAdjChannels, TT = kStateChunk, R = 3;
+  constexpr int VEC = 16 / (int)sizeof(T);          // elements per 16-byte group
+  constexpr int ROW_G = CH / VEC, C_G = N / VEC;    // groups per channel row, per C row
+  static_assert(N % kAdjG == 0 && NA >= 1, "states per thread");
+  static_assert(CH % VEC == 0 && N % VEC == 0, "whole 16-byte groups");
+  __shared__ __align__(16) T sD[R][TT][CH], sG[R][TT][CH], sZ[R][TT][CH], sC[R][TT][N];
   const int64_t L = p.L, d_in = p.d_in;
-  const int64_t nC = (L + kStateChunk - 1) / kStateChunk;
+  const int64_t nC = (L + TT - 1) / TT;
   const int64_t nblk = (nC + p.Cb - 1) / p.Cb;
   const int64_t blk = (int64_t)blockIdx.y + 1;  // blocks 1 .. nblk - 1
+  if (blk >= nblk) return;                        // the whole CTA
   const int64_t ib = blockIdx.z;
-  const int64_t d = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (d >= d_in || blk >= nblk) return;
-  const int64_t t_begin = blk * p.Cb * kStateChunk;
-  const int64_t t_end = t_begin + p.Cb * kStateChunk < L ? t_begin + p.Cb * kStateChunk : L;
+  const int tid = threadIdx.x, j = tid % kAdjG, cc = tid / kAdjG;
+  const int64_t d0 = (int64_t)blockIdx.x * CH, d = d0 + cc;
+  const bool active = d < d_in;
+  const int64_t c_begin = blk * p.Cb, c_end = c_begin + p.Cb < nC ? c_begin + p.Cb : nC;
+  const int nch = (int)(c_end - c_begin);
   const T *gdelta = static_cast<const T *>(p.delta);
   const T *gz = static_cast<const T *>(p.z);
   const T *gdout = static_cast<const T *>(p.dout);
   const T *gC = static_cast<const T *>(p.C);
-  float A2[N], lam[N];
-#pragma unroll
-  for (int n = 0; n < N; ++n) {
-    A2[n] = in_bounds(d * N + n, d_in * N, kBndParam) ? p.A[d * N + n] * kLog2e : 0.0f;
-    lam[n] = 0.0f;
-  }
-  const float bias = p.dt_bias ? p.dt_bias[d] : 0.0f;
-  float dsum = 0.0f;
-  for (int64_t t = t_end - 1; t >= t_begin; --t) {
-    const int64_t at = (ib * L + t) * d_in + d, ct = (ib * L + t) * N;
-    if (!in_bounds(at, p.b * L * d_in, kBndAct) || !in_bounds(ct + N - 1, p.b * L * N, kBndBC))
-      continue;
-    const float pre = Elem<T>::load(gdelta, at) + bias;
-    const float dl = p.softplus ? softplus_f32(pre) : pre;
-    const float go = Elem<T>::load(gdout, at);
-    float gt = go;
-    if (gz) {
-      const float zz = Elem<T>::load(gz, at);
-      gt = go * zz * rcp_approx(1.0f + ex2_approx(-zz * kLog2e));
+  const int64_t n_act = p.b * L * d_in, n_bc = p.b * L * N;
+
+  // stage chunk c into ring slot `slot` (rows past L and channels past d_in
+  // are zero)
+  auto stage = [&](int64_t c, int slot) {
+    const int64_t t0 = c * TT;
+    if constexpr (ASYNC) {
+      for (int q = tid; q < 3 * TT * ROW_G; q += 128) {
+        const int which = q / (TT * ROW_G), rem = q - which * TT * ROW_G;
+        const int i = rem / ROW_G, g = rem - i * ROW_G;
+        const int64_t at = (ib * L + t0 + i) * d_in + d0 + g * VEC;
+        const bool ok = (which != 2 || gz) && t0 + i < L && d0 + g * VEC < d_in &&
+                        in_bounds(at + VEC - 1, n_act, kBndAct);
+        const T *src = which == 0 ? gdelta : which == 1 ? gdout : (gz ? gz : gdelta);
+        T *dst = which == 0 ? &sD[slot][i][g * VEC] : which == 1 ? &sG[slot][i][g * VEC]
+                                                               : &sZ[slot][i][g * VEC];
+        cp_async16(dst, src + (ok ? at : 0), ok ? 16 : 0);
+      }
+      for (int q = tid; q < TT * C_G; q += 128) {
+        const int i = q / C_G, g = q - i * C_G;
+        const int64_t ct = (ib * L + t0 + i) * N + g * VEC;
+        const bool ok = t0 + i < L && in_bounds(ct + VEC - 1, n_bc, kBndBC);
+        cp_async16(&sC[slot][i][g * VEC], gC + (ok ? ct : 0), ok ? 16 : 0);
+      }
+      cp_async_commit();
+    } else {
+      for (int q = tid; q < 3 * TT * CH; q += 128) {
+        const int which = q / (TT * CH), rem = q - which * TT * CH;
+        const int i = rem / CH, e = rem - i * CH;
+        const int64_t at = (ib * L + t0 + i) * d_in + d0 + e;
+        const T *src = which == 0 ? gdelta : which == 1 ? gdout : gz;
+        const bool ok = src && t0 + i < L && d0 + e < d_in && in_bounds(at, n_act, kBndAct);
+        T *dst = which == 0 ? &sD[slot][i][e] : which == 1 ? &sG[slot][i][e] : &sZ[slot][i][e];
+        *dst = ok ? src[at] : T(0.0f);
+      }
+      for (int q = tid; q < TT * N; q += 128) {
+        const int i = q / N, n = q - i * N;
+        const int64_t ct = (ib * L + t0 + i) * N + n;
+        const bool ok = t0 + i < L && in_bounds(ct, n_bc, kBndBC);
+        sC[slot][i][n] = ok ? gC[ct] : T(0.0f);
+      }
     }
-    dsum += dl;
+  };
+
+  float A2[NA], lam[NA];
 #pragma unroll
-    for (int n = 0; n < N; ++n)
-      lam[n] = fmaf(gt, Elem<T>::load(gC, ct + n), lam[n]) * ex2_approx(dl * A2[n]);
+  for (int k = 0; k < NA; ++k) {
+    const int64_t n = j * NA + k;
+    A2[k] = active && in_bounds(d * N + n, d_in * N, kBndParam) ? p.A[d * N + n] * kLog2e : 0.0f;
+    lam[k] = 0.0f;
   }
-  const int64_t row = ((ib * nblk + (nblk - 1 - blk)) * d_in + d) * N;
-  if (!in_bounds(row + N - 1, p.b * nblk * d_in * N, kBndChunk)) return;
+  const float bias = active && p.dt_bias ? p.dt_bias[d] : 0.0f;
+  float dsum = 0.0f;
+
+  // chunks from the block's last backwards: chunk c_end - 1 - i in slot i % R
+  if constexpr (ASYNC) {
+    stage(c_end - 1, 0);
+    if (nch > 1) stage(c_end - 2, 1);
+    else cp_async_commit();
+  }
+  for (int i = 0; i < nch; ++i) {
+    const int64_t c = c_end - 1 - i;
+    const int slot = i % R;
+    if constexpr (ASYNC) {
+      if (i + 2 < nch) stage(c - 2, (i + 2) % R);
+      else cp_async_commit();
+      cp_async_wait<2>();  // chunk c has landed (this thread's copies)
+    } else {
+      stage(c, slot);
+    }
+    __syncthreads();  // every thread's copies of chunk c are visible
+    if (active) {
+      const int64_t t0 = c * TT;
+      const int tc = (int)(L - t0 < TT ? L - t0 : TT);
+      for (int s = tc - 1; s >= 0; --s) {
+        const float pre = Elem<T>::load(&sD[slot][s][0], cc) + bias;
+        const float dl = p.softplus ? softplus_f32(pre) : pre;
+        const float go = Elem<T>::load(&sG[slot][s][0], cc);
+        float gt = go;
+        if (gz) {
+          const float zz = Elem<T>::load(&sZ[slot][s][0], cc);
+          gt = go * zz * rcp_approx(1.0f + ex2_approx(-zz * kLog2e));
+        }
+        dsum += dl;
 #pragma unroll
-  for (int n = 0; n < N; ++n) {
-    adj_state[row + n] = lam[n];
-    adj_decay[row + n] = ex2_approx(dsum * A2[n]);
+        for (int k = 0; k < NA; ++k)
+          lam[k] = fmaf(gt, Elem<T>::load(&sC[slot][s][0], j * NA + k), lam[k]) *
+                   ex2_approx(dl * A2[k]);
+      }
+    }
+    __syncthreads();  // slot i % R is refilled at iteration i + 1
+  }
+  if constexpr (ASYNC) cp_async_wait<0>();  // only empty groups can remain
+
+  const int64_t row = ((ib * nblk + (nblk - 1 - blk)) * d_in + d) * N + j * NA;
+  if (!active || !in_bounds(row + NA - 1, p.b * nblk * d_in * N, kBndChunk)) return;
+#pragma unroll
+  for (int k = 0; k < NA; ++k) {
+    adj_state[row + k] = lam[k];
+    adj_decay[row + k] = ex2_approx(dsum * A2[k]);
   }
 }
 

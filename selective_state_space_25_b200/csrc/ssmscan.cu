@@ -607,9 +607,12 @@ ssm_status launch_bwd_split(const ssm::BwdParams &p, bool async, const BwdSplitP
     q.states_saved = 1;
     q.Cb = sp.Cb;
     float *adj_decay = adj, *adj_state = adj + p.b * sp.nblk * p.d_in * N;
-    ssm::scan_bwd_adjoint_kernel<T, N>
-        <<<dim3((unsigned)((p.d_in + 127) / 128), (unsigned)(sp.nblk - 1), (unsigned)p.b), 128, 0,
-           st>>>(q, adj_decay, adj_state);
+    const dim3 agrid((unsigned)((p.d_in + ssm::kAdjChannels - 1) / ssm::kAdjChannels),
+                     (unsigned)(sp.nblk - 1), (unsigned)p.b);
+    if (async)
+      ssm::scan_bwd_adjoint_kernel<T, N, true><<<agrid, 128, 0, st>>>(q, adj_decay, adj_state);
+    else
+      ssm::scan_bwd_adjoint_kernel<T, N, false><<<agrid, 128, 0, st>>>(q, adj_decay, adj_state);
     if (ssm_status s = check_launch("ssm_scan_bwd")) return s;
     if (ssm_status s = launch_dependent(
             ssm::scan_carry_kernel, dim3((unsigned)((p.d_in * N + 31) / 32), (unsigned)p.b),
