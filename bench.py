@@ -137,20 +137,29 @@ KERNEL_KNOBS = {"scan": ("SSM_SCAN_", "SSM_WS_"), "ss2d": ("SSM_SS2D_",),
                 "scan_bwd_saved": ("SSM_BWD_",)}
 
 
-def launches_per_step(w, split: bool = False) -> int:
-    """Kernels of this repository one step launches.  The backward without
-    saved states runs the forward kernel's states pass (which writes the
-    chunk-start states) and then the backward for d_state 8, 16 and 32 with
-    16-byte aligned inputs, as the bench's are; a scan with few enough
-    channels for the split scan (split: the library asks for a workspace)
-    runs its summary, carry and scan passes; every other workload is one
-    launch (the named scan workloads are too wide for the split scan)."""
+def launches_per_step(w, split: bool = False, bwd_split: bool = False) -> int:
+    """Kernels of this repository one step launches (the bench's inputs are
+    16-byte aligned).  A scan with few enough channels for the split scan
+    (split: the library asks for a workspace) runs its summary, carry and scan
+    passes.  The backward without saved states runs the forward kernel's
+    states pass (which writes the chunk-start states; split like the scan
+    when `split`) and then the backward, for d_state 8, 16 and 32.  A split
+    backward (bwd_split: the library asks for the block buffers) adds the
+    adjoint block maps and their carry before it.  Every other workload is one
+    launch; the named workloads are too wide for either split."""
+    n = 1
     if w.kind == "scan_bwd" and w.dims["N"] in (8, 16, 32):
-        return 2
-    return 3 if w.kind == "scan" and split else 1
+        n = 1 + (3 if split else 1)
+    elif w.kind == "scan" and split:
+        n = 3
+    if bwd_split and w.kind in ("scan_bwd", "scan_bwd_saved"):
+        n += 2
+    return n
 
 
 STEP_PARTS = {"scan_bwd": "the states pass and the backward together (one step)",
+              "scan_bwd_saved": "the adjoint block maps, their carry and the backward together "
+                                "(one step)",
               "scan": "the summary, carry and scan passes together (one step)"}
 
 
@@ -251,10 +260,14 @@ def build_step(S, w, dev_in):
     import torch
     d = w.dims
     g = dev_in
+    # scratch a default call would allocate, allocated once outside the timing
+    scratch = lambda nbytes: (torch.empty(nbytes, dtype=torch.uint8, device=g["u"].device)
+                              if nbytes > 0 else None)
     if w.kind == "scan":
         y = torch.empty_like(g["u"])
+        ws = scratch(S.ssm_scan_fwd_workspace_bytes(d["b"], d["L"], d["d_in"], d["N"]))
         fn = lambda: S.ssm_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], D=g["D"], z=g["z"],
-                                    dt_bias=g["dt_bias"], y=y)
+                                    dt_bias=g["dt_bias"], y=y, workspace=ws)
         return fn, y
     if w.kind == "ss2d":
         y = torch.empty_like(g["u"])
@@ -268,15 +281,17 @@ def build_step(S, w, dev_in):
                              dtype=torch.float32, device=g["u"].device)
         S.ssm_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], D=g["D"], z=g["z"],
                        dt_bias=g["dt_bias"], chunk_states=states)
+        aux = scratch(S.ssm_scan_bwd_saved_workspace_bytes(d["b"], d["L"], d["d_in"], d["N"]))
         out = S.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["dout"], D=g["D"],
-                             z=g["z"], dt_bias=g["dt_bias"], states=states)
+                             z=g["z"], dt_bias=g["dt_bias"], states=states, workspace=aux)
         fn = lambda: S.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["dout"], D=g["D"],
-                                    z=g["z"], dt_bias=g["dt_bias"], states=states, out=out)
+                                    z=g["z"], dt_bias=g["dt_bias"], states=states, out=out,
+                                    workspace=aux)
         return fn, list(out.values())
     if w.kind == "scan_bwd":
         out = S.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["dout"], D=g["D"],
                              z=g["z"], dt_bias=g["dt_bias"])
-        ws = torch.empty(S.ssm_scan_bwd_workspace_bytes(d["b"], d["L"], d["d_in"], d["N"]),
+        ws = torch.empty(S.ssm_scan_bwd_fast_workspace_bytes(d["b"], d["L"], d["d_in"], d["N"]),
                          dtype=torch.uint8, device=g["u"].device)
         fn = lambda: S.ssm_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["dout"], D=g["D"],
                                     z=g["z"], dt_bias=g["dt_bias"], workspace=ws, out=out)
@@ -447,9 +462,13 @@ def run_ours(args, w):
     dev_in = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in host.items()}
     step, y = build_step(S, w, dev_in)
     d = w.dims
-    split = w.kind == "scan" and S.ssm_scan_fwd_workspace_bytes(d["b"], d["L"], d["d_in"],
-                                                                 d["N"]) > 0
-    nk = launches_per_step(w, split)
+    dims = (d["b"], d["L"], d["d_in"], d["N"]) if "L" in d else None
+    split = bool(dims) and w.kind in ("scan", "scan_bwd") and S.ssm_scan_fwd_workspace_bytes(*dims) > 0
+    bwd_split = bool(dims) and (
+        (w.kind == "scan_bwd" and S.ssm_scan_bwd_fast_workspace_bytes(*dims)
+         > S.ssm_scan_bwd_workspace_bytes(*dims)) or
+        (w.kind == "scan_bwd_saved" and S.ssm_scan_bwd_saved_workspace_bytes(*dims) > 0))
+    nk = launches_per_step(w, split, bwd_split)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 

@@ -48,7 +48,9 @@ def test_sfu_ceiling():
 
 def test_launches_per_step():
     """The gpu_launches claim: one kernel per step, two for the backward that
-    runs the states pass first, three for a scan that takes the split scan."""
+    runs the states pass first, three for a scan that takes the split scan;
+    the split backward adds the adjoint maps and their carry (and its states
+    pass may be the split scan's three passes)."""
     W = WORKLOADS
     assert bench.launches_per_step(W["mamba1.4b-long-scan"]) == 1
     assert bench.launches_per_step(W["mamba1.4b-long-scan"], split=True) == 3
@@ -56,7 +58,10 @@ def test_launches_per_step():
     assert bench.launches_per_step(W["mamba-decode-step"]) == 1
     assert bench.launches_per_step(W["mamba130m-scan-bwd"]) == 2
     assert bench.launches_per_step(W["mamba130m-scan-bwd-saved"]) == 1
-    assert set(bench.STEP_PARTS) == {"scan", "scan_bwd"}
+    assert bench.launches_per_step(W["mamba130m-scan-bwd-saved"], bwd_split=True) == 3
+    assert bench.launches_per_step(W["mamba130m-scan-bwd"], bwd_split=True) == 4
+    assert bench.launches_per_step(W["mamba130m-scan-bwd"], split=True, bwd_split=True) == 6
+    assert set(bench.STEP_PARTS) == {"scan", "scan_bwd", "scan_bwd_saved"}
 
 
 def test_traffic_is_null_when_kernels_changed(tmp_path, monkeypatch):
