@@ -157,6 +157,21 @@ def launches_per_step(w, split: bool = False, bwd_split: bool = False) -> int:
     return n
 
 
+def split_flags(S, w):
+    """(split, bwd_split) of launches_per_step from the library's workspace
+    queries for the workload's sizes: whether the scan (or the backward's
+    states pass) takes the split scan, and whether the backward splits."""
+    d = w.dims
+    if "L" not in d:
+        return False, False
+    dims = (d["b"], d["L"], d["d_in"], d["N"])
+    split = w.kind in ("scan", "scan_bwd") and S.ssm_scan_fwd_workspace_bytes(*dims) > 0
+    bwd_split = ((w.kind == "scan_bwd" and S.ssm_scan_bwd_fast_workspace_bytes(*dims)
+                  > S.ssm_scan_bwd_workspace_bytes(*dims)) or
+                 (w.kind == "scan_bwd_saved" and S.ssm_scan_bwd_saved_workspace_bytes(*dims) > 0))
+    return split, bwd_split
+
+
 STEP_PARTS = {"scan_bwd": "the states pass and the backward together (one step)",
               "scan_bwd_saved": "the adjoint block maps, their carry and the backward together "
                                 "(one step)",
@@ -462,13 +477,7 @@ def run_ours(args, w):
     dev_in = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in host.items()}
     step, y = build_step(S, w, dev_in)
     d = w.dims
-    dims = (d["b"], d["L"], d["d_in"], d["N"]) if "L" in d else None
-    split = bool(dims) and w.kind in ("scan", "scan_bwd") and S.ssm_scan_fwd_workspace_bytes(*dims) > 0
-    bwd_split = bool(dims) and (
-        (w.kind == "scan_bwd" and S.ssm_scan_bwd_fast_workspace_bytes(*dims)
-         > S.ssm_scan_bwd_workspace_bytes(*dims)) or
-        (w.kind == "scan_bwd_saved" and S.ssm_scan_bwd_saved_workspace_bytes(*dims) > 0))
-    nk = launches_per_step(w, split, bwd_split)
+    nk = launches_per_step(w, *split_flags(S, w))
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 

@@ -64,6 +64,27 @@ def test_launches_per_step():
     assert set(bench.STEP_PARTS) == {"scan", "scan_bwd", "scan_bwd_saved"}
 
 
+def test_split_flags_from_the_library_queries():
+    """The named workloads take no split; the saved-state and self-contained
+    backward overridden to few channels over a long sequence do (and the
+    latter's states pass takes the split scan), which is what a profiling run
+    with --override measures."""
+    import dataclasses
+    from selective_state_space_25_b200 import ssmscan as S
+    for w in WORKLOADS.values():
+        assert bench.split_flags(S, w) == (False, False), w.name
+    few = dict(b=1, L=16384, d_in=256, N=16)
+    saved = dataclasses.replace(WORKLOADS["mamba130m-scan-bwd-saved"], dims=few)
+    bwd = dataclasses.replace(WORKLOADS["mamba130m-scan-bwd"], dims=few)
+    scan = dataclasses.replace(WORKLOADS["mamba130m-scan"], dims=few)
+    assert bench.split_flags(S, saved) == (False, True)
+    assert bench.split_flags(S, bwd) == (True, True)
+    assert bench.split_flags(S, scan) == (True, False)
+    assert bench.launches_per_step(saved, *bench.split_flags(S, saved)) == 3
+    assert bench.launches_per_step(bwd, *bench.split_flags(S, bwd)) == 6
+    assert bench.launches_per_step(scan, *bench.split_flags(S, scan)) == 3
+
+
 def test_traffic_is_null_when_kernels_changed(tmp_path, monkeypatch):
     f = tmp_path / "traffic.json"
     f.write_text(json.dumps({"w": {"dram_bytes_per_launch": 123, "source_hash": "stale"}}))
