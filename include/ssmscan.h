@@ -100,9 +100,11 @@ typedef enum {
  * into blocks scanned in parallel: every block's map h -> P h + Q is stored
  * in the workspace, a carry pass turns the maps into each block's start
  * state, and a replay writes y.  The workspace then holds two fp32 arrays
- * (b, nblk, d_in, d_state) (the block decays P, then the block states Q and
- * carries); nblk depends on the device's SM count, so query it on the device
- * that runs the scan.  Returns (size_t)-1 for invalid sizes.
+ * (b, nblk, d_in, d_state): the block decays P (which the carry pass
+ * overwrites with the state each next block starts from), then the block
+ * states Q; nblk depends on the device's SM count, so query it on the device
+ * that runs the scan.  ssm_scan_fwd_save_ex takes the same workspace (there
+ * it is optional).  Returns (size_t)-1 for invalid sizes.
  */
 size_t ssm_scan_fwd_workspace_bytes(int64_t b, int64_t L, int64_t d_in, int64_t d_state);
 
